@@ -1,0 +1,275 @@
+"""CPU oracle for the GShard top-2 (top-k) MoE layer forward.  TEST INFRASTRUCTURE.
+
+This file exists to check the CUDA path, never to serve it.  Only `tests/`,
+`__graft_entry__.smoke()` and `bench.py`'s CPU-baseline / reference arm may
+import it; the library under `gshard_top_gating_b200/` never does, and it shares
+no code, table or helper with it.
+
+Everything is plain numpy in float64 (inputs given in fp32 or bf16 are upcast
+exactly).  A library matmul or cumulative sum serves as a step where the
+definition is a plain matrix product or count; there is no blocking, fusion or
+reordering beyond that.
+
+Sources (the web pages this method is taken from):
+
+[gist]  "GShard (Expert Parallelism)", learn card, "In plain words": experts sit
+        in per-device buffers, tokens go out to them and come back; capacity
+        factors bound each expert's load.
+[note]  "GShard: Scaling Giant Models with Conditional Computation and Automatic
+        Sharding", paper note, summary paragraph: top-2 gating with
+        softmax-normalised top-2 weights; auxiliary load-balance loss
+        N * sum_j f_j * P_j plus a z-loss; tokens beyond an expert's capacity
+        (set by capacity_factor) are dropped.
+[blog]  "GShard: Scaling Giant Neural Networks with Conditional Computation",
+        section "Mixture-of-Experts Implementation": G(x) = Softmax(x . W_g),
+        top-k with k = 2 typical, the "Expert Capacity" paragraph; section "Core
+        Components", "Expert Networks": each expert is a Transformer-style
+        feed-forward network.
+
+Readings where the pages are silent (each one is listed in the design notes):
+ * N in N*sum f_j P_j is the number of experts E; f_j is the fraction of tokens
+   whose FIRST choice is j, counted before capacity; P_j is the mean over tokens
+   of the full softmax probability of expert j.
+ * z-loss = mean over tokens of logsumexp(logits)^2, unweighted.
+ * The normalised top-k weights are g_r = p_{e_r} / sum_{r'<k} p_{e_r'}.
+ * Capacity C = ceil(capacity_factor * k * S / E), evaluated in double.
+ * Slots are handed out rank-major: all first choices in token order, then all
+   second choices, and so on; an assignment whose expert is full is dropped and
+   contributes zero; the surviving weights are not renormalised.
+ * Top-k selects on the fp32 logits, ties to the lower expert index.
+ * The expert FFN is relu(x W1[e]) W2[e] with no biases.
+ * An empty batch (S = 0) has l_aux = z = 0.
+
+Pins: every function here is checked in tests/test_oracle_pins.py against hand
+examples, closed forms, library routines, brute force and invariants.
+"""
+from __future__ import annotations
+
+import math
+from types import SimpleNamespace
+
+import numpy as np
+
+__all__ = [
+    "capacity", "gate_logits", "softmax_stats", "top_k", "normalized_gates",
+    "assign_slots", "expert_ffn", "dispatch", "combine", "aux_losses",
+    "route", "forward", "outputs_for_tokens",
+]
+
+
+def _f64(a) -> np.ndarray:
+    """Exact upcast of a numpy array or torch tensor (fp32 / bf16 / f64) to float64."""
+    if hasattr(a, "detach"):          # torch tensor (bf16 has no numpy dtype)
+        import torch
+        a = a.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+def capacity(S: int, E: int, k: int, cf: float) -> int:
+    """Expert capacity C = ceil(cf * k * S / E).
+
+    [note] summary: over-capacity tokens are dropped, "governed by
+    capacity_factor"; [blog] "Expert Capacity": each expert processes at most a
+    fixed number of tokens per batch.  The formula itself is the reading above.
+    """
+    return int(math.ceil(cf * k * S / E))
+
+
+def gate_logits(x, Wg, bias=None) -> np.ndarray:
+    """Gating logits l = x . W_g (+ b), returned as float32 [S, E].
+
+    [blog] "Mixture-of-Experts Implementation", G(x) = Softmax(x . W_g): the
+    product is taken in float64 and rounded once to float32; a per-expert bias,
+    when given, is added in float32 after that rounding.
+    """
+    l = (_f64(x) @ _f64(Wg)).astype(np.float32)
+    if bias is not None:
+        l = (l + np.asarray(_f64(bias), dtype=np.float32)).astype(np.float32)
+    return l
+
+
+def softmax_stats(logits):
+    """Softmax probabilities p[S,E] and log-sum-exp lse[S] of the logits, float64.
+
+    [blog] "Mixture-of-Experts Implementation": G(x) = Softmax(x . W_g).
+    """
+    l = _f64(logits)
+    if l.shape[0] == 0:
+        return np.zeros_like(l), np.zeros(0)
+    mx = l.max(axis=1, keepdims=True)
+    ex = np.exp(l - mx)
+    s = ex.sum(axis=1, keepdims=True)
+    p = ex / s
+    lse = (mx + np.log(s))[:, 0]
+    return p, lse
+
+
+def top_k(logits, k: int) -> np.ndarray:
+    """Expert ids [S, k] int32: the k largest logits per token, best first.
+
+    [note] "top-2"; [blog] "top-k experts (typically k=2)".  Selection is on
+    the logits (order-equivalent to the probabilities); ties go to the lower
+    expert index (np.argmax returns the first maximum).
+    """
+    l = np.array(logits, dtype=np.float32, copy=True)
+    assert np.all(np.isfinite(l)), "logits must be finite"
+    S = l.shape[0]
+    ids = np.zeros((S, k), dtype=np.int32)
+    rows = np.arange(S)
+    for r in range(k):
+        j = np.argmax(l, axis=1) if S else np.zeros(0, dtype=np.int64)
+        ids[:, r] = j
+        l[rows, j] = -np.inf
+    return ids
+
+
+def normalized_gates(p, ids) -> np.ndarray:
+    """Gate weights g[S, k] = p[t, e_r] / sum_{r'} p[t, e_r'] (float64).
+
+    [note] "softmax-normalised top-2 weights".
+    """
+    p = _f64(p)
+    sel = np.take_along_axis(p, ids.astype(np.int64), axis=1)
+    return sel / sel.sum(axis=1, keepdims=True)
+
+
+def assign_slots(ids, E: int, C: int):
+    """Capacity-limited slot assignment.
+
+    Returns slot[S, k] int32 (-1 where dropped) and cnt[E] int64 (demand, before
+    capacity).  Rank-major order: for r = 0..k-1 and tokens in order, the
+    position of (t, r) at expert e is the number of earlier assignments to e;
+    it is kept iff that position is below C.  [note] summary (dropping beyond
+    capacity), [blog] "Expert Capacity".
+    """
+    ids = np.asarray(ids)
+    S, k = ids.shape
+    slot = np.full((S, k), -1, dtype=np.int32)
+    cnt = np.zeros(E, dtype=np.int64)
+    experts = np.arange(E)
+    for r in range(k):
+        onehot = (ids[:, r][:, None] == experts[None, :]).astype(np.int64)   # [S, E]
+        earlier = np.cumsum(onehot, axis=0) - onehot                            # same-rank, earlier tokens
+        pos = cnt[ids[:, r]] + earlier[np.arange(S), ids[:, r]]
+        slot[:, r] = np.where(pos < C, pos, -1)
+        cnt += onehot.sum(axis=0)
+    return slot, cnt
+
+
+def expert_ffn(rows, W1e, W2e) -> np.ndarray:
+    """One expert's two-layer ReLU feed-forward network: relu(rows W1e) W2e.
+
+    [blog] "Core Components", "Expert Networks" (Transformer-style FFN, no
+    biases by the reading above).
+    """
+    h = np.maximum(_f64(rows) @ _f64(W1e), 0.0)
+    return h @ _f64(W2e)
+
+
+def dispatch(x, ids, slot, E: int, C: int) -> np.ndarray:
+    """Per-expert capacity buffers xbuf[E, C, M]: xbuf[e_r, slot_r] = x[t] for kept (t, r).
+
+    [gist] "In plain words": tokens are sent to the experts' buffers (on one
+    device the all-to-all becomes this permutation).  Unused rows are zero.
+    """
+    x = _f64(x)
+    S, M = x.shape
+    xbuf = np.zeros((E, C, M))
+    for r in range(ids.shape[1]):
+        keep = slot[:, r] >= 0
+        xbuf[ids[keep, r], slot[keep, r]] = x[keep]
+    return xbuf
+
+
+def combine(ybuf, ids, gates, slot) -> np.ndarray:
+    """Gate-weighted combine y[t] = sum_{r kept} g_r * ybuf[e_r, slot_r].
+
+    [gist] "In plain words" (results are returned to their tokens); the
+    weighting by the normalised gates follows [note].  Dropped assignments
+    contribute zero and the kept weights are not renormalised.
+    """
+    S, k = ids.shape
+    y = np.zeros((S, ybuf.shape[2]))
+    for r in range(k):
+        keep = slot[:, r] >= 0
+        y[keep] += gates[keep, r][:, None] * ybuf[ids[keep, r], slot[keep, r]]
+    return y
+
+
+def aux_losses(p, ids, lse, E: int):
+    """Auxiliary load-balance loss l_aux = E * sum_j f_j P_j and z-loss mean(lse^2).
+
+    [note] summary: "N * sum_j f_j * P_j plus a z-loss" (readings of N, f_j,
+    P_j and the z-loss above).  Returns (l_aux, z, f, P) as floats / float64.
+    """
+    p = _f64(p)
+    S = p.shape[0]
+    if S == 0:
+        return 0.0, 0.0, np.zeros(E), np.zeros(E)
+    P = p.sum(axis=0) / S
+    f = np.bincount(np.asarray(ids)[:, 0], minlength=E).astype(np.float64) / S
+    l_aux = float(E * np.sum(f * P))
+    z = float(np.sum(_f64(lse) ** 2) / S)
+    return l_aux, z, f, P
+
+
+def route(logits, k: int, cf: float):
+    """Routing of given fp32 logits: everything between the gate GEMM and dispatch.
+
+    Returns a namespace with p, lse, ids, gates, C, slot, cnt, n, l_aux, z.
+    """
+    logits = np.asarray(logits, dtype=np.float32)
+    S, E = logits.shape
+    C = capacity(S, E, k, cf)
+    p, lse = softmax_stats(logits)
+    ids = top_k(logits, k)
+    g = normalized_gates(p, ids) if S else np.zeros((0, k))
+    slot, cnt = assign_slots(ids, E, C)
+    l_aux, z, f, P = aux_losses(p, ids, lse, E)
+    return SimpleNamespace(p=p, lse=lse, ids=ids, gates=g, C=C, slot=slot, cnt=cnt,
+                           n=np.minimum(cnt, C), l_aux=l_aux, z=z, f=f, P=P)
+
+
+def forward(x, Wg, bias, W1, W2, k: int, cf: float):
+    """The whole layer forward on the CPU (small cases).
+
+    Returns the `route` namespace plus logits and the output y[S, M] (float64).
+    """
+    logits = gate_logits(x, Wg, bias)
+    rt = route(logits, k, cf)
+    S, E = logits.shape
+    C = rt.C
+    W1 = _f64(W1)
+    W2 = _f64(W2)
+    xbuf = dispatch(x, rt.ids, rt.slot, E, C)
+    ybuf = np.zeros_like(xbuf)
+    for e in range(E):
+        n = int(rt.n[e])
+        if n:
+            ybuf[e, :n] = expert_ffn(xbuf[e, :n], W1[e], W2[e])
+    rt.logits = logits
+    rt.y = combine(ybuf, rt.ids, rt.gates, rt.slot)
+    return rt
+
+
+def outputs_for_tokens(tokens, x_rows, ids, gates, slot, expert_weights):
+    """Layer outputs y[tokens] for a sample of tokens, given the full routing.
+
+    Because xbuf[e_r, slot_r] holds x[t] itself, y[t] = sum_{r kept} g_r *
+    FFN_{e_r}(x[t]) depends only on x[t] and the routing of t.  `x_rows[i]` is
+    x[tokens[i]]; `expert_weights(e)` returns (W1[e], W2[e]).  Experts are
+    visited one at a time so only one expert's weights are held.
+    """
+    tokens = np.asarray(tokens, dtype=np.int64)
+    xr = _f64(x_rows)
+    y = np.zeros((len(tokens), xr.shape[1]))
+    sid = ids[tokens]
+    sg = _f64(gates)[tokens]
+    ss = slot[tokens]
+    for e in np.unique(sid[ss >= 0]):
+        W1e, W2e = expert_weights(int(e))
+        for r in range(ids.shape[1]):
+            sel = np.nonzero((sid[:, r] == e) & (ss[:, r] >= 0))[0]
+            if len(sel):
+                y[sel] += sg[sel, r][:, None] * expert_ffn(xr[sel], W1e, W2e)
+    return y
