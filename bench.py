@@ -1,0 +1,361 @@
+"""Benchmark of the GShard MoE layer forward on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload mid]
+
+A step is one whole layer forward (router, capacity scan, dispatch, two grouped
+expert GEMMs, combine, losses) over one batch of synthetic tokens already
+resident in HBM.  The default workload is the mid configuration (S=8192
+tokens, M=1024, H=4096, E=32, top-2, capacity factor 2.0, bf16).  L2 is flushed
+(a 256 MB write) before every timed step and each step is timed with CUDA
+events on the launching stream; the sum over the K steps is the timed region.
+
+With N > 1 (launched by torch.distributed.run) every rank runs an independent
+replica of the layer on its own GPU and batch (the forward has no exchange on
+one GPU); the slowest rank's time gives the job throughput ("scaling": "weak").
+
+--impl reference times the CPU oracle (the plain float64 restatement of the
+method) on a bounded token sample of the same workload; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gshard_top_gating_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+STAGES = ("router", "scan", "dispatch", "ffn1", "ffn2", "combine")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+def dist_setup(n):
+    if n <= 1 or "RANK" not in os.environ:
+        return 0, 1, 0
+    import torch.distributed as dist
+    from datetime import timedelta
+    rank = int(os.environ["RANK"])
+    world = int(os.environ["WORLD_SIZE"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    cs = os.path.join(ROOT, "gshard_top_gating_b200", "csrc")
+    for f in sorted(os.listdir(cs)):
+        with open(os.path.join(cs, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """dram bytes per launch of `kernel` from the committed ncu summary, if it is current."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(workload, {}).get(kernel)
+    if not ent or ent.get("source_hash") != source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def algorithmic(w, A, n_active):
+    """Algorithmic bytes / flops per launch of each stage (A kept assignments)."""
+    s = 2 if w.act == "bf16" else 4
+    S, M, H, E, k = w.S, w.M, w.H, w.E, w.k
+    return {
+        "router": ("hbm", S * M * s + 4 * M * E + S * E * 4 + S * k * 12),
+        "scan": ("hbm", 0),
+        "dispatch": ("hbm", (S + A) * M * s),
+        "ffn1": ("tensor", 2.0 * A * M * H),
+        "ffn2": ("tensor", 2.0 * A * M * H),
+        "combine": ("hbm", (A + S) * M * s + S * k * 12),
+    }
+
+
+def run_ours(args, rank, world, local):
+    w = WORKLOADS[args.workload]
+    from gshard_top_gating_b200 import _lib as L
+    from gshard_top_gating_b200.layer import MoeLayer
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    x, Wg, b, W1, W2 = make_inputs(w, device=dev)
+    layer = MoeLayer(w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b, W1, W2)
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MB > L2
+
+    for _ in range(args.warmup):
+        layer(x, out=y)
+    torch.cuda.synchronize()
+    _, _, slot, cnt = layer.routing(w.S)
+    C = layer.capacity(w.S)
+    n_e = torch.clamp(cnt.long(), max=C)
+    A = int(n_e.sum().item())
+    n_active = int((n_e > 0).sum().item())
+
+    # ---- timed region: K forwards, L2 flushed before each, device time per step
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            layer(x, out=y)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    value = world * w.S * args.steps / (total_ms / 1e3)
+
+    # ---- per-stage device times (events recorded by the library on the same stream)
+    L.moe_set_profiling(layer.h, True)
+    per_stage = [[] for _ in STAGES]
+    for i in range(args.steps):
+        flush.zero_()
+        layer(x, out=y)
+        for j, t in enumerate(L.moe_get_stage_times(layer.h)):
+            per_stage[j].append(t)
+    L.moe_set_profiling(layer.h, False)
+    stage_ms = {n: statistics.mean(v) for n, v in zip(STAGES, per_stage)}
+
+    # ---- end to end through the C ABI with host buffers (copies inside the timed region)
+    xh = x.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    for _ in range(2):
+        layer.forward_host(xh, yh)
+    torch.cuda.synchronize()
+    e_s = torch.cuda.Event(enable_timing=True)
+    e_e = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e_s.record(stream)
+    for _ in range(args.steps):
+        layer.forward_host(xh, yh)
+    e_e.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), world)
+    nbytes = x.numel() * x.element_size()
+
+    pk, pk_kind = peaks()
+    algo = algorithmic(w, A, n_active)
+    dom = max(stage_ms, key=lambda n: stage_ms[n])
+    bound, work = algo[dom]
+    t = stage_ms[dom] / 1e3
+    if bound == "tensor":
+        achieved, peak, unit = work / t / 1e12, pk["bf16_tflops"], "TFLOP/s"
+    else:
+        achieved, peak, unit = work / t / 1e9, pk["hbm_gbs"], "GB/s"
+    roof = {"bound": bound, "kernel": dom, "achieved": round(achieved, 2), "peak": peak,
+            "unit": unit, "frac": round(achieved / peak, 4), "traffic": ncu_traffic(dom, w.name),
+            "peak_source": pk_kind}
+    stages = {}
+    for n in STAGES:
+        b_, wk = algo[n]
+        tt = stage_ms[n] / 1e3
+        if b_ == "tensor":
+            stages[n] = {"ms": round(stage_ms[n], 4), "TFLOP/s": round(wk / tt / 1e12, 1),
+                         "frac_of_peak": round(wk / tt / 1e12 / pk["bf16_tflops"], 4)}
+        else:
+            stages[n] = {"ms": round(stage_ms[n], 4), "GB/s": round(wk / tt / 1e9, 1),
+                         "frac_of_peak": round(wk / tt / 1e9 / pk["hbm_gbs"], 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_tokens, x, Wg, b, W1, W2)
+
+    line = {
+        "metric": "MoE-layer tokens/sec on 1 B200; FFN % of bf16 TC peak; dispatch/combine HBM GB/s",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.act, "data": "synthetic",
+        "config": {"workload": f"{w.name} (S={w.S}, M={w.M}, H={w.H}, E={w.E}, k={w.k}, cf={w.cf})",
+                   "S": w.S, "M": w.M, "H": w.H, "E": w.E, "k": w.k, "capacity_factor": w.cf,
+                   "C": C, "kept_assignments": A, "active_experts": n_active,
+                   "l2": "flushed before every timed step (256 MB write)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": roof, "stages": stages,
+        "e2e": {"value": round(world * w.S * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes},
+        "gpu_launches": args.steps * L.moe_kernels_per_forward(layer.h, w.S),
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+    }
+    layer.close()
+    return line
+
+
+def _oracle_sample(w, ntok, x, Wg, b, W1, W2):
+    """Inputs of a bounded sample of the workload: the first ntok tokens, all experts."""
+    xs = x[:ntok].cpu()
+    return xs, Wg.cpu(), None if b is None else b.cpu(), W1.cpu(), W2.cpu()
+
+
+def cpu_baseline(w, ntok, x, Wg, b, W1, W2, threads=None):
+    import oracle as O
+    xs, Wgc, bc, W1c, W2c = _oracle_sample(w, ntok, x, Wg, b, W1, W2)
+    cores = torch.get_num_threads() if threads is None else threads
+    t0 = time.perf_counter()
+    O.forward(xs, Wgc, bc, W1c, W2c, w.k, w.cf)
+    dt = time.perf_counter() - t0
+    return {"value": round(ntok / dt, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {ntok} of {w.S} tokens of the {w.name} workload (same M, H, E, k, cf; "
+                      f"C scaled to the sample), full float64 oracle forward, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    w = WORKLOADS[args.workload]
+    if rank != 0:
+        return None
+    ntok = args.cpu_tokens
+    x, Wg, b, W1, W2 = make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
+    import oracle as O
+    xs, Wgc, bc, W1c, W2c = _oracle_sample(w, ntok, x, Wg, b, W1, W2)
+    del x, W1, W2
+    for _ in range(args.warmup if args.warmup < 1 else 1):
+        O.forward(xs, Wgc, bc, W1c, W2c, w.k, w.cf)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        O.forward(xs, Wgc, bc, W1c, W2c, w.k, w.cf)
+        times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    v = round(ntok * args.steps / tot, 2)
+    return {
+        "impl": "reference",
+        "metric": "MoE-layer tokens/sec on 1 B200; FFN % of bf16 TC peak; dispatch/combine HBM GB/s",
+        "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * tot / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name} (S={w.S}, M={w.M}, H={w.H}, E={w.E}, k={w.k}, cf={w.cf})",
+                   "S": w.S, "M": w.M, "H": w.H, "E": w.E, "k": w.k, "capacity_factor": w.cf},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": torch.get_num_threads(),
+                         "kind": "oracle",
+                         "sample": f"first {ntok} of {w.S} tokens per step (same M, H, E, k, cf)"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="mid")
+    ap.add_argument("--cpu-tokens", type=int, default=512)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "ours" and args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_ours(args, rank, world, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,163 @@
+"""ctypes binding of the C ABI in include/moe.h (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does nothing
+but turn tensors into pointers, streams into handles and non-OK status codes
+into MoeError.  All computation happens in the CUDA library; there is no other
+path: if the shared library is missing the import fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgshard_moe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_OOM, MOE_ERR_STATE, \
+    MOE_ERR_TIMEOUT = range(7)
+MOE_F32, MOE_BF16 = 0, 1
+MOE_NUM_STAGES = 6
+STAGES = ("router", "scan", "dispatch", "ffn1", "ffn2", "combine")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {msg} (status {status})")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"CUDA library {LIB_PATH} is missing: build it with "
+            "`python -m gshard_top_gating_b200.build` (there is no fallback path)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, I32, D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+    sig = {
+        "moe_create": [ctypes.POINTER(P), I64, I64, I64, I32, I32, D, ctypes.c_int, P, P, P, P],
+        "moe_forward": [P, I64, P, P, P],
+        "moe_forward_host": [P, I64, P, P, P],
+        "moe_aux_loss": [P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float), P],
+        "moe_destroy": [P],
+        "moe_check": [P, P],
+        "moe_get_logits": [P, P, P],
+        "moe_get_routing": [P, P, P, P, P, P],
+        "moe_route_from_logits": [P, I64, P, P],
+        "moe_get_capacity": [P, I64, ctypes.POINTER(I64)],
+        "moe_set_profiling": [P, I32],
+        "moe_get_stage_times": [P, ctypes.POINTER(ctypes.c_float), I32],
+        "moe_selftest_wait_timeout": [I32, P],
+    }
+    for name, args in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    lib.moe_kernels_per_forward.argtypes = [P, I64]
+    lib.moe_kernels_per_forward.restype = I32
+    lib.moe_status_string.argtypes = [ctypes.c_int]
+    lib.moe_status_string.restype = ctypes.c_char_p
+    lib.moe_stage_name.argtypes = [I32]
+    lib.moe_stage_name.restype = ctypes.c_char_p
+    return lib
+
+
+lib = _load()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != MOE_OK:
+        raise MoeError(fn, status, lib.moe_status_string(status).decode())
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def moe_status_string(status: int) -> str:
+    return lib.moe_status_string(status).decode()
+
+
+def moe_stage_name(stage: int) -> str:
+    return lib.moe_stage_name(stage).decode()
+
+
+def moe_create(S_max, M, H, E, k, capacity_factor, act, Wg, gate_bias, W1, W2) -> int:
+    h = ctypes.c_void_p()
+    dt = MOE_BF16 if act in ("bf16", torch.bfloat16, MOE_BF16) else MOE_F32
+    _check("moe_create", lib.moe_create(ctypes.byref(h), S_max, M, H, E, k, float(capacity_factor),
+                                        dt, _ptr(Wg), _ptr(gate_bias), _ptr(W1), _ptr(W2)))
+    return h.value
+
+
+def moe_forward(h, S, x, y, stream=None) -> None:
+    _check("moe_forward", lib.moe_forward(h, S, _ptr(x), _ptr(y), _stream(stream)))
+
+
+def moe_forward_host(h, S, x_host, y_host, stream=None) -> None:
+    _check("moe_forward_host", lib.moe_forward_host(h, S, _ptr(x_host), _ptr(y_host), _stream(stream)))
+
+
+def moe_aux_loss(h, stream=None):
+    a, z = ctypes.c_float(), ctypes.c_float()
+    _check("moe_aux_loss", lib.moe_aux_loss(h, ctypes.byref(a), ctypes.byref(z), _stream(stream)))
+    return a.value, z.value
+
+
+def moe_destroy(h) -> None:
+    _check("moe_destroy", lib.moe_destroy(h))
+
+
+def moe_check(h, stream=None) -> None:
+    _check("moe_check", lib.moe_check(h, _stream(stream)))
+
+
+def moe_get_logits(h, logits, stream=None) -> None:
+    _check("moe_get_logits", lib.moe_get_logits(h, _ptr(logits), _stream(stream)))
+
+
+def moe_get_routing(h, eidx=None, gate=None, slot=None, cnt=None, stream=None) -> None:
+    _check("moe_get_routing", lib.moe_get_routing(h, _ptr(eidx), _ptr(gate), _ptr(slot), _ptr(cnt),
+                                                  _stream(stream)))
+
+
+def moe_route_from_logits(h, S, logits, stream=None) -> None:
+    _check("moe_route_from_logits", lib.moe_route_from_logits(h, S, _ptr(logits), _stream(stream)))
+
+
+def moe_get_capacity(h, S) -> int:
+    c = ctypes.c_int64()
+    _check("moe_get_capacity", lib.moe_get_capacity(h, S, ctypes.byref(c)))
+    return c.value
+
+
+def moe_set_profiling(h, enable: bool) -> None:
+    _check("moe_set_profiling", lib.moe_set_profiling(h, 1 if enable else 0))
+
+
+def moe_get_stage_times(h):
+    buf = (ctypes.c_float * MOE_NUM_STAGES)()
+    _check("moe_get_stage_times", lib.moe_get_stage_times(h, buf, MOE_NUM_STAGES))
+    return list(buf)
+
+
+def moe_kernels_per_forward(h, S) -> int:
+    return int(lib.moe_kernels_per_forward(h, S))
+
+
+def moe_selftest_wait_timeout(limit_us: int, stream=None) -> int:
+    """Returns the raw status (MOE_ERR_TIMEOUT when the bounded wait works)."""
+    return int(lib.moe_selftest_wait_timeout(limit_us, _stream(stream)))

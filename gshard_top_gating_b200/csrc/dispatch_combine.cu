@@ -1,0 +1,190 @@
+// dispatch_combine.cu -- token -> expert-buffer dispatch and gate-weighted combine.
+//
+// On several devices the tokens travel to their experts by an all-to-all and
+// come back by a second one ("GShard (Expert Parallelism)", "In plain words").
+// On one GPU both become permutations in HBM:
+//   dispatch: xbuf[e_r, slot_r] = x[t] for every kept choice (t, r)
+//   combine : y[t] = sum_{r kept} g_r * ybuf[e_r, slot_r]   (r ascending, fp32)
+// A dropped choice contributes nothing and the kept gates are not renormalised
+// ("GShard: Scaling Giant Models ...", paper-note summary: over-capacity tokens
+// are dropped).  Both kernels are token-centric (one warp per token), read and
+// write whole rows in 16-byte vectors, and need no atomics, so the result does
+// not depend on scheduling.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) dispatch_kernel(const T* __restrict__ x, int S, int M,
+                                                            int E, int k, int C, int64_t Cbuf,
+                                                            int nchunk, Routing R,
+                                                            T* __restrict__ xbuf) {
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * kThreads) >> 5;
+  const int nv = (int)((int64_t)M * sizeof(T) / 16);
+  for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < S; t += warps) {
+    int e = 0, s = -1;
+    if (lane < k) {
+      e = R.eidx[(int64_t)t * k + lane];
+      const int c = t / kChunk;
+      int pos = 0x7fffffff;
+      if (e >= 0 && e < E) {
+        pos = R.off[((int64_t)lane * nchunk + c) * E + e] + R.lrank[(int64_t)t * k + lane];
+      } else {
+        atomicOr(R.err, DEVERR_BOUNDS);
+      }
+      s = (pos < C && pos < Cbuf) ? pos : -1;
+      R.slot[(int64_t)t * k + lane] = s;
+    }
+    if (x == nullptr) continue;                // slot-only pass (routing without data)
+    const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)t * M);
+    uint4* dst[kMaxK];
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) {
+      const int er = __shfl_sync(0xffffffffu, e, r);
+      const int sr = __shfl_sync(0xffffffffu, s, r);
+      dst[r] = (r < k && sr >= 0) ? reinterpret_cast<uint4*>(xbuf + ((int64_t)er * Cbuf + sr) * M)
+                                  : nullptr;
+    }
+    for (int v0 = lane; v0 < nv; v0 += 32 * kUnroll) {
+      uint4 val[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (v0 + 32 * u < nv) val[u] = ld_nc_v4(src + v0 + 32 * u);
+#pragma unroll
+      for (int r = 0; r < kMaxK; ++r) {
+        if (dst[r] == nullptr) continue;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+          if (v0 + 32 * u < nv) dst[r][v0 + 32 * u] = val[u];
+      }
+    }
+  }
+}
+
+template <typename T>
+struct Vec;
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void load_fma(float (&a)[8], const uint4& u, float g) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      a[2 * q] = fmaf(g, bf16lo(w[q]), a[2 * q]);
+      a[2 * q + 1] = fmaf(g, bf16hi(w[q]), a[2 * q + 1]);
+    }
+  }
+  __device__ static uint4 pack(const float (&a)[8]) {
+    return make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                      pack_bf16x2(a[6], a[7]));
+  }
+};
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ static void load_fma(float (&a)[8], const uint4& u, float g) {
+    a[0] = fmaf(g, __uint_as_float(u.x), a[0]);
+    a[1] = fmaf(g, __uint_as_float(u.y), a[1]);
+    a[2] = fmaf(g, __uint_as_float(u.z), a[2]);
+    a[3] = fmaf(g, __uint_as_float(u.w), a[3]);
+  }
+  __device__ static uint4 pack(const float (&a)[8]) {
+    return make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
+                      __float_as_uint(a[3]));
+  }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) combine_kernel(const T* __restrict__ ybuf, int S, int M,
+                                                           int k, int64_t Cbuf, Routing R,
+                                                           T* __restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * kThreads) >> 5;
+  const int nv = (int)((int64_t)M * sizeof(T) / 16);
+  for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < S; t += warps) {
+    int e = 0, s = -1;
+    float g = 0.f;
+    if (lane < k) {
+      e = R.eidx[(int64_t)t * k + lane];
+      s = R.slot[(int64_t)t * k + lane];
+      g = R.gate[(int64_t)t * k + lane];
+    }
+    const uint4* srcs[kMaxK];
+    float gr[kMaxK];
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) {
+      const int er = __shfl_sync(0xffffffffu, e, r);
+      const int sr = __shfl_sync(0xffffffffu, s, r);
+      gr[r] = __shfl_sync(0xffffffffu, g, r);
+      srcs[r] = (r < k && sr >= 0)
+                    ? reinterpret_cast<const uint4*>(ybuf + ((int64_t)er * Cbuf + sr) * M)
+                    : nullptr;
+    }
+    uint4* dst = reinterpret_cast<uint4*>(y + (int64_t)t * M);
+    for (int v0 = lane; v0 < nv; v0 += 32 * 2) {
+      float acc[2][8];
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[u][q] = 0.f;
+#pragma unroll
+      for (int r = 0; r < kMaxK; ++r) {
+        if (srcs[r] == nullptr) continue;
+        uint4 val[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+          if (v0 + 32 * u < nv) val[u] = ld_nc_v4(srcs[r] + v0 + 32 * u);
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+          if (v0 + 32 * u < nv) Vec<T>::load_fma(acc[u], val[u], gr[r]);
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        if (v0 + 32 * u < nv) dst[v0 + 32 * u] = Vec<T>::pack(acc[u]);
+    }
+  }
+}
+
+int grid_for(int S) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int want = (S + (kThreads / 32) - 1) / (kThreads / 32);
+  return want < sms * 8 ? want : sms * 8;
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const void* x, bool bf16, int S, int M, int E, int k, int C,
+                            int64_t Cbuf, const Routing& R, void* xbuf, cudaStream_t st) {
+  const int nchunk = (S + kChunk - 1) / kChunk;
+  const int grid = grid_for(S);
+  if (bf16)
+    dispatch_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(
+        (const __nv_bfloat16*)x, S, M, E, k, C, Cbuf, nchunk, R, (__nv_bfloat16*)xbuf);
+  else
+    dispatch_kernel<float><<<grid, kThreads, 0, st>>>((const float*)x, S, M, E, k, C, Cbuf, nchunk,
+                                                      R, (float*)xbuf);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const void* ybuf, bool bf16, int S, int M, int k, int64_t Cbuf,
+                           const Routing& R, void* y, cudaStream_t st) {
+  const int grid = grid_for(S);
+  if (bf16)
+    combine_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>((const __nv_bfloat16*)ybuf, S, M, k,
+                                                             Cbuf, R, (__nv_bfloat16*)y);
+  else
+    combine_kernel<float><<<grid, kThreads, 0, st>>>((const float*)ybuf, S, M, k, Cbuf, R,
+                                                     (float*)y);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,361 @@
+// ffn_tc.cu -- grouped expert GEMM on 5th-generation tensor cores (tcgen05), bf16 in, fp32 accumulate.
+//
+// Each expert is a two-layer ReLU feed-forward network ("GShard: Scaling Giant
+// Neural Networks with Conditional Computation", "Core Components", "Expert
+// Networks"); on one GPU all experts' GEMMs run in one persistent launch:
+//
+//   D[e, :n_e, :] = act( A[e, :n_e, :] . B[e] )      A [E*Cbuf, K], B [E*K, N], D [E*Cbuf, N]
+//
+// with n_e (kept rows of expert e) read on the device, so the host never waits
+// for the routing.  FFN1: A = xbuf, B = W1 ([M, H] per expert, H contiguous),
+// act = ReLU.  FFN2: A = hbuf, B = W2 ([H, M] per expert), act = identity.
+//
+// Design (one CTA per SM, 192 threads):
+//   warp 0     TMA producer: A tile 128x64 (K-major, 128B swizzle) and B tile
+//              64xBN (N contiguous = "MN-major" operand, 128B swizzle) per stage
+//   warp 1     TMEM allocator + single-thread tcgen05.mma issuer (M=128, N=BN, K=16)
+//   warps 2-5  epilogue: tcgen05.ld 32 lanes x 32 columns, fp32 -> bf16 (+ReLU),
+//              predicated 16-byte stores of rows < n_e
+// The fp32 accumulator lives in TMEM, double buffered (2*BN columns) so the
+// epilogue of one tile overlaps the main loop of the next.  Tiles are ordered
+// (expert, n-tile, m-tile) with m fastest, so the CTAs working at the same time
+// share one weight column strip through L2.  All waits are bounded.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128, BK = 64;
+constexpr int kThreads = 192;
+constexpr uint32_t A_BYTES = BM * BK * 2;   // 16 KB
+
+template <int BN>
+struct Cfg {
+  static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr uint32_t B_BYTES = BK * BN * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  // 1 KB alignment slack + stages + 512 B of barriers + misc words and the tile tables
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 512 + 16 + 4 * (3 * kMaxExperts + 1);
+};
+
+// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: version 1 at bit 46,
+// layout type 2 = SWIZZLE_128B at bits 61-63).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: D fp32, A bf16 (K-major), B bf16 (MN-major), M=128, N=BN.
+template <int BN>
+__device__ __forceinline__ uint32_t idesc_bf16() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(BN >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+
+// Walks this CTA's tiles in the global order (expert, n-tile, m-tile).
+struct TileIter {
+  const int* tile_pre;   // smem [E+1]: first tile of each expert
+  const int* mtiles;     // smem [E]
+  int E, NT, e;
+  __device__ bool decode(int tile, int& ex, int& mt, int& nt) {
+    if (tile >= tile_pre[E]) return false;
+    while (tile >= tile_pre[e + 1]) ++e;
+    const int local = tile - tile_pre[e];
+    const int m_e = mtiles[e];
+    nt = local / m_e;
+    mt = local - nt * m_e;
+    ex = e;
+    return true;
+  }
+};
+
+template <int BN, bool RELU>
+__global__ void __launch_bounds__(kThreads, 1)
+    ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  __nv_bfloat16* __restrict__ D, const int32_t* __restrict__ nexp, int E,
+                  int64_t Cbuf, int K, int N, unsigned* err, uint64_t limit_ns) {
+  using C = Cfg<BN>;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;                 // 1024-aligned for swizzle
+  unsigned char* gbase = smem_raw + (base - raw_base);
+  const uint32_t bar0 = base + C::STAGES * C::STAGE_BYTES;
+  // barriers: full[S], empty[S], tfull[2], tempty[2], done
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 2 + a); };
+  const uint32_t done_bar = bar0 + 8u * (2 * C::STAGES + 4);
+  unsigned char* misc = gbase + C::STAGES * C::STAGE_BYTES + 512;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  int* tile_pre = reinterpret_cast<int*>(misc + 16);                 // [E+1]
+  int* mtiles = tile_pre + (kMaxExperts + 1);                        // [E]
+  int* nrows = mtiles + kMaxExperts;                                 // [E]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NT = N / BN;
+  const int KB = K / BK;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 128);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 2) {
+    // tile prefix over experts (warp-parallel scan, ceil(E/32) experts per lane)
+    const int per = (E + 31) / 32;
+    const int e0 = lane * per;
+    int sum = 0;
+    for (int e = e0; e < min(E, e0 + per); ++e) {
+      const int n = nexp[e];
+      const int m = (n + BM - 1) / BM;
+      nrows[e] = n;
+      mtiles[e] = m;
+      sum += m * NT;
+    }
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    int run = inc - sum;
+    for (int e = e0; e < min(E, e0 + per); ++e) {
+      tile_pre[e] = run;
+      run += mtiles[e] * NT;
+    }
+    if (lane == 31) tile_pre[E] = inc;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      TileIter it{tile_pre, mtiles, E, NT, 0};
+      int s = 0;
+      uint32_t ph = 0, issued = 0, issued_par = 0;
+      bool ok = true;
+      int e, mt, nt;
+      for (int tile = blockIdx.x; ok && it.decode(tile, e, mt, nt); tile += gridDim.x) {
+        const int rowA = (int)(e * Cbuf + mt * BM);
+        const int rowB = e * K;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (*abort_flag || !mbar_wait(empty_bar(s), ph ^ 1u, err, limit_ns)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const uint32_t sa = base + s * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(full_bar(s), C::STAGE_BYTES);
+          tma_load_2d(sa, &tmA, full_bar(s), kb * BK, rowA);
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j)
+            tma_load_2d(sa + A_BYTES + j * 8192u, &tmB, full_bar(s), nt * BN + j * 64, rowB + kb * BK);
+          issued |= 1u << s;
+          issued_par = (issued_par & ~(1u << s)) | (ph << s);
+          if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {   // let copies in flight land before the CTA exits
+        for (int q = 0; q < C::STAGES; ++q)
+          if ((issued >> q) & 1u) mbar_wait(full_bar(q), (issued_par >> q) & 1u, err, limit_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      TileIter it{tile_pre, mtiles, E, NT, 0};
+      const uint32_t idesc = idesc_bf16<BN>();
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int e, mt, nt, i = 0;
+      for (int tile = blockIdx.x; ok && it.decode(tile, e, mt, nt); tile += gridDim.x, ++i) {
+        const int acc = i & 1;
+        const uint32_t aph = (i >> 1) & 1;
+        if (*abort_flag || !mbar_wait(tempty_bar(acc), aph ^ 1u, err, limit_ns)) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (*abort_flag || !mbar_wait(full_bar(s), ph, err, limit_ns)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base + s * C::STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = desc_sw128(sa + kk * 32u, 16u, 1024u);
+            const uint64_t bd = desc_sw128(sb + kk * 2048u, 8192u, 1024u);
+            tc_mma_f16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          }
+          tc_commit(empty_bar(s));
+          if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (ok) tc_commit(tfull_bar(acc));
+      }
+      if (!ok) {   // let issued MMAs finish before TMEM is released
+        tc_commit(done_bar);
+        mbar_wait(done_bar, 0, err, limit_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;                     // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    TileIter it{tile_pre, mtiles, E, NT, 0};
+    int e, mt, nt, i = 0;
+    for (int tile = blockIdx.x; it.decode(tile, e, mt, nt); tile += gridDim.x, ++i) {
+      const int acc = i & 1;
+      const uint32_t aph = (i >> 1) & 1;
+      if (*abort_flag || !mbar_wait(tfull_bar(acc), aph, err, limit_ns)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int grow = mt * BM + row;
+      const bool valid = grow < nrows[e];
+      __nv_bfloat16* dst = D + ((int64_t)e * Cbuf + grow) * N + (int64_t)nt * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c * 32, r);
+        tmem_ld_wait();
+        if (valid) {
+          uint32_t p[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float a = __uint_as_float(r[2 * j]), b = __uint_as_float(r[2 * j + 1]);
+            if (RELU) {
+              a = fmaxf(a, 0.f);
+              b = fmaxf(b, 0.f);
+            }
+            p[j] = pack_bf16x2(a, b);
+          }
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) d4[j] = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+bool encode_2d(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_in,
+               uint32_t box_out) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_in, box_out};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, bool RELU>
+cudaError_t launch_t(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint64_t limit_ns,
+                     int num_sms, cudaStream_t st) {
+  auto kern = ffn_tc_kernel<BN, RELU>;
+  const size_t smem = Cfg<BN>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<num_sms, kThreads, smem, st>>>(p.tmA, p.tmB, (__nv_bfloat16*)p.D, nexp, p.E, p.Cbuf, p.K,
+                                        p.N, err, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool make_gemm_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, int64_t Cbuf, int K,
+                    int N, bool relu) {
+  p.E = E;
+  p.Cbuf = Cbuf;
+  p.K = K;
+  p.N = N;
+  p.D = D;
+  p.relu = relu;
+  p.BN = (N % 256 == 0) ? 256 : (N % 128 == 0 ? 128 : 64);
+  if (K % BK || N % 64) return false;
+  if (!encode_2d(&p.tmA, A, (uint64_t)K, (uint64_t)E * Cbuf, BK, BM)) return false;
+  if (!encode_2d(&p.tmB, B, (uint64_t)N, (uint64_t)E * K, 64, BK)) return false;
+  return true;
+}
+
+cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* err,
+                            uint64_t wait_limit_ns, int num_sms, cudaStream_t st) {
+  switch (p.BN) {
+    case 256:
+      return p.relu ? launch_t<256, true>(p, nexp, err, wait_limit_ns, num_sms, st)
+                    : launch_t<256, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+    case 128:
+      return p.relu ? launch_t<128, true>(p, nexp, err, wait_limit_ns, num_sms, st)
+                    : launch_t<128, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+    default:
+      return p.relu ? launch_t<64, true>(p, nexp, err, wait_limit_ns, num_sms, st)
+                    : launch_t<64, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+  }
+}
+
+}  // namespace moe

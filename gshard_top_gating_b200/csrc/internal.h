@@ -1,0 +1,62 @@
+// internal.h -- host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kMaxExperts = 256;
+constexpr int kMaxK = 8;
+constexpr int kChunk = 64;          // tokens per router CTA (= scan chunk)
+
+// Device tables of one forward (all owned by the handle's workspace).
+struct Routing {
+  float* logits;     // [S, E]   fp32 logits as routed (bias included)
+  int32_t* eidx;     // [S, k]   expert of each choice, best first
+  float* gate;       // [S, k]   normalised gate weight
+  int32_t* lrank;    // [S, k]   rank of (t, r) among same-expert rank-r choices in t's chunk
+  int32_t* slot;     // [S, k]   slot in the expert's buffer, -1 if dropped
+  int32_t* hist;     // [k, nchunk, E] rank-r choices of each expert per chunk
+  int32_t* off;      // [k, nchunk, E] exclusive rank-major prefix of hist per expert
+  int32_t* cnt;      // [E] demand per expert (before capacity)
+  int32_t* nexp;     // [E] kept rows per expert = min(cnt, C)
+  float* psum;       // [nchunk, E] per-chunk sum of softmax probabilities
+  float* lse2;       // [nchunk]    per-chunk sum of lse^2
+  float* losses;     // [2]  l_aux, z
+  unsigned* err;     // device error word
+};
+
+// router.cu
+cudaError_t launch_router(const void* x, bool x_bf16, const float* Wg, const float* bias, int S,
+                          int M, int E, int k, const Routing& R, cudaStream_t st);
+cudaError_t launch_route_logits(const float* logits, int S, int E, int k, const Routing& R,
+                                cudaStream_t st);
+// scan.cu
+cudaError_t launch_scan(int S, int E, int k, int C, int64_t Cbuf, const Routing& R, cudaStream_t st);
+// dispatch_combine.cu
+cudaError_t launch_dispatch(const void* x, bool bf16, int S, int M, int E, int k, int C,
+                            int64_t Cbuf, const Routing& R, void* xbuf, cudaStream_t st);
+cudaError_t launch_combine(const void* ybuf, bool bf16, int S, int M, int k, int64_t Cbuf,
+                           const Routing& R, void* y, cudaStream_t st);
+// ffn_simt.cu  (fp32 activations)
+cudaError_t launch_ffn_f32(const float* A, const float* B, float* D, const int32_t* nexp, int E,
+                           int64_t Cbuf, int K, int N, bool relu, cudaStream_t st);
+// ffn_tc.cu  (bf16 activations, tcgen05)
+struct GemmPlan {
+  CUtensorMap tmA;   // [E*Cbuf, K] bf16, box {64, 128}, 128B swizzle
+  CUtensorMap tmB;   // [E*K, N]    bf16, box {64, 64},  128B swizzle
+  void* D;           // [E*Cbuf, N] bf16
+  int E, K, N, BN;
+  int64_t Cbuf;
+  bool relu;
+};
+bool make_gemm_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, int64_t Cbuf, int K,
+                    int N, bool relu);
+cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* err,
+                            uint64_t wait_limit_ns, int num_sms, cudaStream_t st);
+// selftest.cu
+cudaError_t launch_wait_selftest(unsigned* flag, unsigned* err, uint64_t limit_ns, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,393 @@
+// moe_api.cu -- the C ABI (include/moe.h): handle, workspace, launch sequence.
+//
+// One forward enqueues six kernels on the caller's stream and never waits on
+// the host:
+//   router  (gate GEMM, softmax, top-k, gates, loss partials, chunk tables)
+//   scan    (rank-major capacity offsets per expert, kept counts, losses)
+//   dispatch(slots, x rows -> per-expert buffers)
+//   ffn1    (grouped relu(xbuf W1))      ffn2 (grouped hbuf W2)
+//   combine (gate-weighted sum back to token order)
+// The data-dependent per-expert counts stay on the device: the grouped GEMMs
+// read them there.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "internal.h"
+
+using namespace moe;
+
+struct moe_layer {
+  int64_t S_max, M, H;
+  int32_t E, k;
+  double cf;
+  moe_dtype act;
+  const float* Wg;
+  const float* bias;
+  const void* W1;
+  const void* W2;
+  int64_t Cbuf;          // rows per expert in xbuf / hbuf / ybuf
+  int device, num_sms;
+  size_t ws_bytes;
+  void* ws;              // the one device allocation
+  Routing R;
+  void* xbuf;
+  void* hbuf;
+  void* ybuf;
+  void* xstage;          // moe_forward_host staging
+  void* ystage;
+  GemmPlan plan1, plan2;
+  int64_t last_S;
+  bool have_forward;
+  bool profiling;
+  cudaEvent_t ev[MOE_NUM_STAGES + 1];
+  bool have_events;
+  uint64_t wait_limit_ns;
+};
+
+namespace {
+
+size_t act_bytes(moe_dtype a) { return a == MOE_BF16 ? 2 : 4; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  if (e == cudaErrorMemoryAllocation) return MOE_ERR_OOM;
+  return MOE_ERR_CUDA;
+}
+
+// C = ceil(capacity_factor * k * S / E), evaluated in double left to right.
+int64_t capacity_of(double cf, int k, int64_t S, int E) {
+  const double c = ceil(cf * (double)k * (double)S / (double)E);
+  if (!(c < 2147483647.0)) return 2147483647;
+  return (int64_t)c;
+}
+
+struct Carver {
+  char* base;
+  size_t off = 0;
+  template <typename T>
+  T* take(size_t n) {
+    off = (off + 255) & ~(size_t)255;
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += n * sizeof(T);
+    return p;
+  }
+};
+
+// Lays out the workspace; with base == nullptr only measures it.
+size_t carve(moe_layer* h, char* base) {
+  Carver c{base};
+  const int64_t S = h->S_max, E = h->E, k = h->k;
+  const int64_t nchunk = (S + kChunk - 1) / kChunk;
+  const size_t as = act_bytes(h->act);
+  Routing& R = h->R;
+  R.logits = c.take<float>(S * E);
+  R.eidx = c.take<int32_t>(S * k);
+  R.gate = c.take<float>(S * k);
+  R.lrank = c.take<int32_t>(S * k);
+  R.slot = c.take<int32_t>(S * k);
+  R.hist = c.take<int32_t>(k * nchunk * E);
+  R.off = c.take<int32_t>(k * nchunk * E);
+  R.cnt = c.take<int32_t>(E);
+  R.nexp = c.take<int32_t>(E);
+  R.psum = c.take<float>(nchunk * E);
+  R.lse2 = c.take<float>(nchunk);
+  R.losses = c.take<float>(2);
+  R.err = c.take<unsigned>(1);
+  h->xbuf = c.take<char>((size_t)E * h->Cbuf * h->M * as);
+  h->hbuf = c.take<char>((size_t)E * h->Cbuf * h->H * as);
+  h->ybuf = c.take<char>((size_t)E * h->Cbuf * h->M * as);
+  h->xstage = c.take<char>((size_t)S * h->M * as);
+  h->ystage = c.take<char>((size_t)S * h->M * as);
+  return c.off + 256;
+}
+
+moe_status read_device_error(moe_handle h, cudaStream_t st) {
+  unsigned e = 0;
+  cudaError_t ce = cudaMemcpyAsync(&e, h->R.err, sizeof(unsigned), cudaMemcpyDeviceToHost, st);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+  if (ce != cudaSuccess) return from_cuda(ce);
+  if (e) {
+    cudaMemsetAsync(h->R.err, 0, sizeof(unsigned), st);
+    cudaStreamSynchronize(st);
+    return (e & DEVERR_TIMEOUT) ? MOE_ERR_TIMEOUT : MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+#define MOE_TRY(call)                            \
+  do {                                           \
+    cudaError_t _e = (call);                     \
+    if (_e != cudaSuccess) return from_cuda(_e); \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_OOM: return "out of device memory";
+    case MOE_ERR_STATE: return "call out of order";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* moe_stage_name(int32_t s) {
+  static const char* names[MOE_NUM_STAGES] = {"router", "scan", "dispatch", "ffn1", "ffn2", "combine"};
+  return (s >= 0 && s < MOE_NUM_STAGES) ? names[s] : "?";
+}
+
+moe_status moe_create(moe_handle* out, int64_t S_max, int64_t M, int64_t H, int32_t E, int32_t k,
+                      double capacity_factor, moe_dtype act, const float* Wg, const float* bias,
+                      const void* W1, const void* W2) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (S_max < 1 || M < 64 || H < 64 || (M % 64) || (H % 64) || E < 1 || k < 1 || k > E)
+    return MOE_ERR_INVALID_ARG;
+  if (!(capacity_factor > 0.0) || !isfinite(capacity_factor)) return MOE_ERR_INVALID_ARG;
+  if (act != MOE_F32 && act != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (!Wg || !W1 || !W2 || !aligned(Wg, 4) || !aligned(W1, 16) || !aligned(W2, 16) ||
+      (bias && !aligned(bias, 4)))
+    return MOE_ERR_INVALID_ARG;
+  if (E > kMaxExperts || k > kMaxK) return MOE_ERR_UNSUPPORTED;
+  if (S_max > (int64_t)1 << 30 || M > (1 << 16) || H > (1 << 16)) return MOE_ERR_UNSUPPORTED;
+
+  moe_layer* h = new (std::nothrow) moe_layer();
+  if (!h) return MOE_ERR_OOM;
+  h->S_max = S_max;
+  h->M = M;
+  h->H = H;
+  h->E = E;
+  h->k = k;
+  h->cf = capacity_factor;
+  h->act = act;
+  h->Wg = Wg;
+  h->bias = bias;
+  h->W1 = W1;
+  h->W2 = W2;
+  const int64_t C = capacity_of(capacity_factor, k, S_max, E);
+  h->Cbuf = C < S_max ? C : S_max;
+  h->wait_limit_ns = 2000000000ull;   // 2 s per wait: far above any legitimate wait
+  cudaError_t ce = cudaGetDevice(&h->device);
+  if (ce == cudaSuccess)
+    ce = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+  if (ce != cudaSuccess) {
+    delete h;
+    return from_cuda(ce);
+  }
+  h->ws_bytes = carve(h, nullptr);
+  ce = cudaMalloc(&h->ws, h->ws_bytes);
+  if (ce != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return from_cuda(ce);
+  }
+  carve(h, static_cast<char*>(h->ws));
+  ce = cudaMemset(h->R.err, 0, sizeof(unsigned));
+  if (ce == cudaSuccess) ce = cudaMemset(h->R.losses, 0, 2 * sizeof(float));
+  if (ce != cudaSuccess) {
+    cudaFree(h->ws);
+    delete h;
+    return from_cuda(ce);
+  }
+  if (act == MOE_BF16) {
+    const bool ok1 = make_gemm_plan(h->plan1, h->xbuf, W1, h->hbuf, E, h->Cbuf, (int)M, (int)H, true);
+    const bool ok2 = make_gemm_plan(h->plan2, h->hbuf, W2, h->ybuf, E, h->Cbuf, (int)H, (int)M, false);
+    if (!ok1 || !ok2) {
+      cudaFree(h->ws);
+      delete h;
+      return MOE_ERR_CUDA;
+    }
+  }
+  *out = h;
+  return MOE_OK;
+}
+
+moe_status moe_destroy(moe_handle h) {
+  if (!h) return MOE_OK;
+  cudaError_t ce = cudaDeviceSynchronize();
+  if (h->have_events)
+    for (auto& e : h->ev) cudaEventDestroy(e);
+  cudaError_t fe = cudaFree(h->ws);
+  delete h;
+  if (ce != cudaSuccess) return from_cuda(ce);
+  return from_cuda(fe);
+}
+
+moe_status moe_get_capacity(moe_handle h, int64_t S, int64_t* C_out) {
+  if (!h || !C_out || S < 0) return MOE_ERR_INVALID_ARG;
+  *C_out = capacity_of(h->cf, h->k, S, h->E);
+  return MOE_OK;
+}
+
+int32_t moe_kernels_per_forward(moe_handle h, int64_t S) {
+  if (!h || S <= 0) return 0;
+  return 6;
+}
+
+moe_status moe_forward(moe_handle h, int64_t S, const void* x, void* y, void* stream) {
+  if (!h || S < 0 || S > h->S_max) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (S > 0 && (!x || !y || !aligned(x, 16) || !aligned(y, 16))) return MOE_ERR_INVALID_ARG;
+  h->last_S = S;
+  h->have_forward = true;
+  if (S == 0) {
+    MOE_TRY(cudaMemsetAsync(h->R.losses, 0, 2 * sizeof(float), st));
+    return MOE_OK;
+  }
+  const bool bf16 = h->act == MOE_BF16;
+  const int C = (int)capacity_of(h->cf, h->k, S, h->E);
+  const int iS = (int)S, iM = (int)h->M, iH = (int)h->H;
+  const Routing& R = h->R;
+  const bool prof = h->profiling && h->have_events;
+  auto mark = [&](int i) -> cudaError_t { return prof ? cudaEventRecord(h->ev[i], st) : cudaSuccess; };
+
+  MOE_TRY(mark(0));
+  MOE_TRY(launch_router(x, bf16, h->Wg, h->bias, iS, iM, h->E, h->k, R, st));
+  MOE_TRY(mark(1));
+  MOE_TRY(launch_scan(iS, h->E, h->k, C, h->Cbuf, R, st));
+  MOE_TRY(mark(2));
+  MOE_TRY(launch_dispatch(x, bf16, iS, iM, h->E, h->k, C, h->Cbuf, R, h->xbuf, st));
+  MOE_TRY(mark(3));
+  if (bf16) {
+    MOE_TRY(launch_ffn_bf16(h->plan1, R.nexp, R.err, h->wait_limit_ns, h->num_sms, st));
+    MOE_TRY(mark(4));
+    MOE_TRY(launch_ffn_bf16(h->plan2, R.nexp, R.err, h->wait_limit_ns, h->num_sms, st));
+  } else {
+    MOE_TRY(launch_ffn_f32((const float*)h->xbuf, (const float*)h->W1, (float*)h->hbuf, R.nexp,
+                           h->E, h->Cbuf, iM, iH, true, st));
+    MOE_TRY(mark(4));
+    MOE_TRY(launch_ffn_f32((const float*)h->hbuf, (const float*)h->W2, (float*)h->ybuf, R.nexp,
+                           h->E, h->Cbuf, iH, iM, false, st));
+  }
+  MOE_TRY(mark(5));
+  MOE_TRY(launch_combine(h->ybuf, bf16, iS, iM, h->k, h->Cbuf, R, y, st));
+  MOE_TRY(mark(6));
+  return MOE_OK;
+}
+
+moe_status moe_forward_host(moe_handle h, int64_t S, const void* x_host, void* y_host, void* stream) {
+  if (!h || S < 0 || S > h->S_max) return MOE_ERR_INVALID_ARG;
+  if (S > 0 && (!x_host || !y_host)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)S * h->M * act_bytes(h->act);
+  if (S > 0) MOE_TRY(cudaMemcpyAsync(h->xstage, x_host, bytes, cudaMemcpyHostToDevice, st));
+  moe_status s = moe_forward(h, S, h->xstage, h->ystage, stream);
+  if (s != MOE_OK) return s;
+  if (S > 0) MOE_TRY(cudaMemcpyAsync(y_host, h->ystage, bytes, cudaMemcpyDeviceToHost, st));
+  return MOE_OK;
+}
+
+moe_status moe_aux_loss(moe_handle h, float* l_aux, float* z_loss, void* stream) {
+  if (!h || !l_aux || !z_loss) return MOE_ERR_INVALID_ARG;
+  if (!h->have_forward) return MOE_ERR_STATE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float v[2] = {0.f, 0.f};
+  MOE_TRY(cudaMemcpyAsync(v, h->R.losses, sizeof(v), cudaMemcpyDeviceToHost, st));
+  moe_status s = read_device_error(h, st);   // synchronises
+  if (s != MOE_OK) return s;
+  *l_aux = v[0];
+  *z_loss = v[1];
+  return MOE_OK;
+}
+
+moe_status moe_check(moe_handle h, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  return read_device_error(h, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_get_logits(moe_handle h, float* logits, void* stream) {
+  if (!h || !logits) return MOE_ERR_INVALID_ARG;
+  if (!h->have_forward) return MOE_ERR_STATE;
+  if (h->last_S == 0) return MOE_OK;
+  MOE_TRY(cudaMemcpyAsync(logits, h->R.logits, (size_t)h->last_S * h->E * sizeof(float),
+                          cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_get_routing(moe_handle h, int32_t* eidx, float* gate, int32_t* slot, int32_t* cnt,
+                           void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (!h->have_forward) return MOE_ERR_STATE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n = (size_t)h->last_S * h->k;
+  if (n) {
+    if (eidx) MOE_TRY(cudaMemcpyAsync(eidx, h->R.eidx, n * 4, cudaMemcpyDeviceToDevice, st));
+    if (gate) MOE_TRY(cudaMemcpyAsync(gate, h->R.gate, n * 4, cudaMemcpyDeviceToDevice, st));
+    if (slot) MOE_TRY(cudaMemcpyAsync(slot, h->R.slot, n * 4, cudaMemcpyDeviceToDevice, st));
+  }
+  if (cnt) {
+    if (h->last_S == 0)
+      MOE_TRY(cudaMemsetAsync(cnt, 0, (size_t)h->E * 4, st));
+    else
+      MOE_TRY(cudaMemcpyAsync(cnt, h->R.cnt, (size_t)h->E * 4, cudaMemcpyDeviceToDevice, st));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_route_from_logits(moe_handle h, int64_t S, const float* logits, void* stream) {
+  if (!h || S < 0 || S > h->S_max) return MOE_ERR_INVALID_ARG;
+  if (S > 0 && (!logits || !aligned(logits, 4))) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_S = S;
+  h->have_forward = true;
+  if (S == 0) {
+    MOE_TRY(cudaMemsetAsync(h->R.losses, 0, 2 * sizeof(float), st));
+    return MOE_OK;
+  }
+  const int C = (int)capacity_of(h->cf, h->k, S, h->E);
+  MOE_TRY(launch_route_logits(logits, (int)S, h->E, h->k, h->R, st));
+  MOE_TRY(launch_scan((int)S, h->E, h->k, C, h->Cbuf, h->R, st));
+  // slot pass of the dispatch kernel without moving any row
+  MOE_TRY(launch_dispatch(nullptr, h->act == MOE_BF16, (int)S, (int)h->M, h->E, h->k, C, h->Cbuf,
+                          h->R, h->xbuf, st));
+  return MOE_OK;
+}
+
+moe_status moe_set_profiling(moe_handle h, int32_t enable) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (enable && !h->have_events) {
+    for (auto& e : h->ev) MOE_TRY(cudaEventCreate(&e));
+    h->have_events = true;
+  }
+  h->profiling = enable != 0;
+  return MOE_OK;
+}
+
+moe_status moe_get_stage_times(moe_handle h, float* ms, int32_t n) {
+  if (!h || !ms || n < MOE_NUM_STAGES) return MOE_ERR_INVALID_ARG;
+  if (!h->profiling || !h->have_events || !h->have_forward || h->last_S == 0) return MOE_ERR_STATE;
+  MOE_TRY(cudaEventSynchronize(h->ev[MOE_NUM_STAGES]));
+  for (int i = 0; i < MOE_NUM_STAGES; ++i) MOE_TRY(cudaEventElapsedTime(&ms[i], h->ev[i], h->ev[i + 1]));
+  return MOE_OK;
+}
+
+moe_status moe_selftest_wait_timeout(int32_t limit_us, void* stream) {
+  if (limit_us < 0 || limit_us > 10000000) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned* buf = nullptr;
+  MOE_TRY(cudaMalloc(&buf, 2 * sizeof(unsigned)));
+  unsigned host[2] = {0, 0};
+  cudaError_t ce = cudaMemsetAsync(buf, 0, 2 * sizeof(unsigned), st);
+  if (ce == cudaSuccess) ce = launch_wait_selftest(buf, buf + 1, (uint64_t)limit_us * 1000ull, st);
+  if (ce == cudaSuccess) ce = cudaMemcpyAsync(host, buf, sizeof(host), cudaMemcpyDeviceToHost, st);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+  cudaFree(buf);
+  if (ce != cudaSuccess) return from_cuda(ce);
+  if (host[0] == 2u && (host[1] & DEVERR_TIMEOUT)) return MOE_ERR_TIMEOUT;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,118 @@
+// scan.cu -- capacity scan (rank-major slot offsets per expert) and loss finalize.
+//
+// Capacity: each expert takes at most C = ceil(capacity_factor * k * S / E)
+// assignments and the rest are dropped ("GShard: Scaling Giant Models with
+// Conditional Computation and Automatic Sharding", paper-note summary; "GShard:
+// Scaling Giant Neural Networks with Conditional Computation", "Expert Capacity").
+// Order: all first choices in token order, then all second choices, ...  The
+// router leaves hist[r][chunk][e] (rank-r choices of expert e in a chunk of 64
+// tokens); for each expert the exclusive prefix over (r, chunk) in that
+// lexicographic order is the position of the chunk's first such choice.
+//
+// Losses ("GShard: Scaling Giant Models ...", paper-note summary: load-balance
+// loss N * sum_j f_j P_j plus a z-loss): l_aux = E * sum_j f_j P_j with
+// f_j = (first choices of j) / S and P_j = (sum_t p_tj) / S; z = sum_t lse_t^2 / S.
+// Partials are summed in a fixed order in double, so results are deterministic.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < (kThreads / 32) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kThreads / 32) warp_sums[lane] = w;   // inclusive over warps
+  }
+  __syncthreads();
+  total = warp_sums[kThreads / 32 - 1];
+  const int before = warp ? warp_sums[warp - 1] : 0;
+  return before + x - v;
+}
+
+__device__ __forceinline__ double block_sum_f64(double v, double* sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) sm[warp] = v;
+  __syncthreads();
+  double s = 0.0;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) s += sm[w];
+  __syncthreads();
+  return s;
+}
+
+__global__ void __launch_bounds__(kThreads) scan_kernel(int S, int E, int k, int C, int Cbuf,
+                                                        int nchunk, Routing R) {
+  __shared__ int warp_sums[kThreads / 32];
+  __shared__ double dsum[kThreads / 32];
+  const int tid = threadIdx.x;
+  if (blockIdx.x < (unsigned)E) {
+    const int e = blockIdx.x;
+    const int L = k * nchunk;                 // entries (r, chunk), r-major
+    const int seg = (L + kThreads - 1) / kThreads;
+    const int a = min(L, tid * seg), b = min(L, a + seg);
+    int local = 0;
+    for (int q = a; q < b; ++q) local += R.hist[(int64_t)q * E + e];
+    int total;
+    int run = block_exclusive_scan(local, warp_sums, total);
+    for (int q = a; q < b; ++q) {
+      R.off[(int64_t)q * E + e] = run;
+      run += R.hist[(int64_t)q * E + e];
+    }
+    if (tid == 0) {
+      R.cnt[e] = total;
+      R.nexp[e] = min(total, min(C, Cbuf));   // Cbuf bounds the buffers even on bad input
+    }
+    return;
+  }
+  // block E: auxiliary losses
+  double term = 0.0;
+  for (int j = tid; j < E; j += kThreads) {
+    double P = 0.0;
+    long long f = 0;
+    for (int c = 0; c < nchunk; ++c) {
+      P += (double)R.psum[(int64_t)c * E + j];
+      f += R.hist[(int64_t)c * E + j];          // rank 0 rows of hist
+    }
+    term += (double)f * P;
+  }
+  const double fp = block_sum_f64(term, dsum);
+  double zl = 0.0;
+  for (int c = tid; c < nchunk; c += kThreads) zl += (double)R.lse2[c];
+  const double zs = block_sum_f64(zl, dsum);
+  if (tid == 0) {
+    const double Sd = (double)S;
+    R.losses[0] = (float)((double)E * fp / (Sd * Sd));
+    R.losses[1] = (float)(zs / Sd);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_scan(int S, int E, int k, int C, int64_t Cbuf, const Routing& R, cudaStream_t st) {
+  const int nchunk = (S + kChunk - 1) / kChunk;
+  const int cb = Cbuf < 0x7fffffff ? (int)Cbuf : 0x7fffffff;
+  scan_kernel<<<E + 1, kThreads, 0, st>>>(S, E, k, C, cb, nchunk, R);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -139,8 +139,9 @@ def normal(shape, std: float, seed: int, tid: int, dtype: torch.dtype,
         n *= int(s)
     out = torch.empty(n, dtype=dtype, device=device)
     key = _key(seed, tid)
-    for a in range(0, n, _CHUNK):
-        b = min(n, a + _CHUNK)
+    chunk = _CHUNK if out.device.type == "cpu" else _CHUNK * 16
+    for a in range(0, n, chunk):
+        b = min(n, a + chunk)
         idx = torch.arange(a + index_offset, b + index_offset, dtype=torch.int64, device=device)
         z = _irwin_hall(idx, key) * std
         out[a:b] = z.to(torch.float32).to(dtype)

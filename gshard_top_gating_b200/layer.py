@@ -1,0 +1,75 @@
+"""MoeLayer: an owning wrapper around one C-ABI handle (marshalling only).
+
+    layer = MoeLayer(S_max, M, H, E, k, cf, Wg, bias, W1, W2)   # device tensors
+    y = layer(x)                                                 # moe_forward
+    l_aux, z = layer.aux_loss()                                  # moe_aux_loss
+
+The tensors passed in are borrowed by the C library; this object keeps Python
+references to them so they outlive the handle.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib as L
+
+
+class MoeLayer:
+    def __init__(self, S_max, M, H, E, k, capacity_factor, Wg, gate_bias, W1, W2):
+        act = W1.dtype
+        if act not in (torch.float32, torch.bfloat16):
+            raise TypeError("expert weights must be float32 or bfloat16")
+        for t in (Wg, W1, W2) + ((gate_bias,) if gate_bias is not None else ()):
+            if not (t.is_cuda and t.is_contiguous()):
+                raise ValueError("weights must be contiguous CUDA tensors")
+        if Wg.dtype != torch.float32 or (gate_bias is not None and gate_bias.dtype != torch.float32):
+            raise TypeError("gate weights and bias are float32")
+        self.S_max, self.M, self.H, self.E, self.k = S_max, M, H, E, k
+        self.cf = capacity_factor
+        self.act = act
+        self._keep = (Wg, gate_bias, W1, W2)
+        self.h = L.moe_create(S_max, M, H, E, k, capacity_factor, act, Wg, gate_bias, W1, W2)
+
+    def __call__(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        if x.dtype != self.act or not x.is_contiguous() or x.dim() != 2 or x.shape[1] != self.M:
+            raise ValueError("x must be a contiguous [S, M] tensor of the activation dtype")
+        S = x.shape[0]
+        y = out if out is not None else torch.empty_like(x)
+        L.moe_forward(self.h, S, x, y, stream)
+        return y
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None) -> None:
+        L.moe_forward_host(self.h, x_host.shape[0], x_host, y_host, stream)
+
+    def aux_loss(self, stream=None):
+        return L.moe_aux_loss(self.h, stream)
+
+    def capacity(self, S: int) -> int:
+        return L.moe_get_capacity(self.h, S)
+
+    def logits(self, S: int, stream=None) -> torch.Tensor:
+        out = torch.empty(S, self.E, dtype=torch.float32, device="cuda")
+        L.moe_get_logits(self.h, out, stream)
+        return out
+
+    def routing(self, S: int, stream=None):
+        eidx = torch.empty(S, self.k, dtype=torch.int32, device="cuda")
+        gate = torch.empty(S, self.k, dtype=torch.float32, device="cuda")
+        slot = torch.empty(S, self.k, dtype=torch.int32, device="cuda")
+        cnt = torch.empty(self.E, dtype=torch.int32, device="cuda")
+        L.moe_get_routing(self.h, eidx, gate, slot, cnt, stream)
+        return eidx, gate, slot, cnt
+
+    def route_from_logits(self, logits: torch.Tensor, stream=None) -> None:
+        L.moe_route_from_logits(self.h, logits.shape[0], logits, stream)
+
+    def close(self) -> None:
+        if getattr(self, "h", None):
+            L.moe_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,184 @@
+/*
+ * moe.h -- C ABI of a single-GPU GShard Mixture-of-Experts layer forward (B200, sm_100a).
+ *
+ * The layer (sources: "GShard: Scaling Giant Neural Networks with Conditional
+ * Computation", section "Mixture-of-Experts Implementation" and its "Expert
+ * Capacity" paragraph; "GShard: Scaling Giant Models with Conditional
+ * Computation and Automatic Sharding", paper-note summary paragraph; "GShard
+ * (Expert Parallelism)", "In plain words"):
+ *
+ *   logits  l = x . W_g (+ b)                         fp32, [S, E]
+ *   p       = Softmax(l);  lse = logsumexp(l)          per token
+ *   e_0..e_{k-1} = the k largest logits, ties to the lower expert index
+ *   g_r     = p[e_r] / sum_{r'} p[e_r']                "softmax-normalised top-k weights"
+ *   C       = ceil(capacity_factor * k * S / E)        expert capacity
+ *   slots   : rank-major -- all first choices in token order, then all second
+ *             choices, ...; an assignment at position >= C of its expert is
+ *             dropped (contributes zero, no renormalisation)
+ *   xbuf[e, slot] = x[t]                               dispatch (on-device all-to-all)
+ *   ybuf[e, :n_e] = relu(xbuf[e, :n_e] W1[e]) W2[e]    expert feed-forward networks
+ *   y[t]    = sum_{r kept} g_r ybuf[e_r, slot_r]        combine (second all-to-all)
+ *   l_aux   = E * sum_j f_j P_j,  z = mean_t lse_t^2   auxiliary losses
+ *
+ * with f_j = fraction of tokens whose first choice is j (before capacity) and
+ * P_j = mean_t p[t, j].
+ *
+ * Conventions for every entry point:
+ *  - Every pointer argument named *_dev or documented "device" is a CUDA device
+ *    pointer on the current device, 16-byte aligned.  Host pointers are named so.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    All work is enqueued asynchronously on it unless stated otherwise.
+ *  - Errors are returned as moe_status; nothing aborts or throws across the ABI.
+ *    An asynchronous device fault or a device-side wait that timed out surfaces
+ *    on the next synchronising call (moe_aux_loss, moe_check) as MOE_ERR_CUDA or
+ *    MOE_ERR_TIMEOUT.
+ *  - A handle may be used by one host thread / one stream at a time.
+ */
+#ifndef GSHARD_MOE_H
+#define GSHARD_MOE_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* a null, misaligned or out-of-range argument */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid but outside what this build handles (e.g. E > 256) */
+  MOE_ERR_CUDA = 3,          /* a CUDA runtime / driver call failed, or a device fault */
+  MOE_ERR_OOM = 4,           /* device workspace allocation failed */
+  MOE_ERR_STATE = 5,         /* call out of order (e.g. aux loss before any forward) */
+  MOE_ERR_TIMEOUT = 6        /* a device-side bounded wait gave up */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+typedef struct moe_layer* moe_handle;
+
+/* Stage indices of moe_get_stage_times. */
+enum { MOE_STAGE_ROUTER = 0, MOE_STAGE_SCAN = 1, MOE_STAGE_DISPATCH = 2, MOE_STAGE_FFN1 = 3,
+       MOE_STAGE_FFN2 = 4, MOE_STAGE_COMBINE = 5, MOE_NUM_STAGES = 6 };
+
+/*
+ * moe_create -- build a layer handle and allocate its device workspace.
+ *
+ * S_max            largest token count a forward will be given (>= 1).
+ * M, H             model and expert-hidden widths; multiples of 64.
+ * E, k             number of experts and choices per token, 1 <= k <= E <= 256.
+ * capacity_factor  > 0 and finite; C = ceil(capacity_factor * k * S / E) per forward.
+ * act              dtype of x, W1, W2 and y (MOE_F32 or MOE_BF16).  Gating is fp32.
+ * Wg_dev           [M, E] fp32 row-major gate weights (E contiguous).
+ * gate_bias_dev    [E] fp32 added to the logits before the softmax, or NULL.
+ * W1_dev           [E, M, H] act, row-major (H contiguous): first expert layer.
+ * W2_dev           [E, H, M] act, row-major (M contiguous): second expert layer.
+ *
+ * Ownership: the weights and bias are BORROWED -- the caller keeps them alive
+ * and unchanged until moe_destroy.  The handle owns its workspace (per-expert
+ * buffers [E, min(C(S_max), S_max), M|H], routing tables and loss partials),
+ * allocated here with one cudaMalloc; no later call allocates device memory.
+ * Must be called with the target device current.  On error *out is NULL.
+ */
+MOE_API moe_status moe_create(moe_handle* out, int64_t S_max, int64_t M, int64_t H, int32_t E, int32_t k,
+                      double capacity_factor, moe_dtype act, const float* Wg_dev,
+                      const float* gate_bias_dev, const void* W1_dev, const void* W2_dev);
+
+/*
+ * moe_forward -- one layer forward of S tokens (0 <= S <= S_max), enqueued on `stream`.
+ *
+ * x_dev  [S, M] act, row-major (read only).     y_dev  [S, M] act, fully overwritten.
+ * A token whose k assignments were all dropped gets y = 0.  S = 0 enqueues no
+ * kernel and sets l_aux = z = 0.  No host synchronisation, no allocation.
+ */
+MOE_API moe_status moe_forward(moe_handle h, int64_t S, const void* x_dev, void* y_dev, void* stream);
+
+/*
+ * moe_forward_host -- the same forward from and to HOST memory: copies x_host
+ * ([S, M] act) into the handle's device staging buffer, runs moe_forward and
+ * copies y back into y_host ([S, M] act), all enqueued on `stream`.  The host
+ * buffers must stay valid until the stream reaches this point; page-locked
+ * (pinned) buffers make the copies asynchronous.
+ */
+MOE_API moe_status moe_forward_host(moe_handle h, int64_t S, const void* x_host, void* y_host, void* stream);
+
+/*
+ * moe_aux_loss -- the auxiliary losses of the last forward, to host floats.
+ * l_aux = E * sum_j f_j P_j ("N * sum_j f_j * P_j", paper-note summary, N read
+ * as E); z = mean_t logsumexp(l_t)^2.  The caller applies loss weights.
+ * Synchronises `stream`; returns MOE_ERR_STATE before the first forward and
+ * reports pending device errors (MOE_ERR_CUDA / MOE_ERR_TIMEOUT).
+ */
+MOE_API moe_status moe_aux_loss(moe_handle h, float* l_aux_host, float* z_loss_host, void* stream);
+
+/* moe_destroy -- free the workspace (synchronises the device).  NULL is accepted. */
+MOE_API moe_status moe_destroy(moe_handle h);
+
+/*
+ * moe_check -- synchronise `stream` and report a pending device error from any
+ * earlier call on this handle (MOE_ERR_TIMEOUT, MOE_ERR_CUDA), clearing it.
+ */
+MOE_API moe_status moe_check(moe_handle h, void* stream);
+
+/* ---- inspection (device-to-device copies on `stream`, valid after a forward) ---- */
+
+/* logits_dev [S, E] fp32: the logits the routing used (bias included). */
+MOE_API moe_status moe_get_logits(moe_handle h, float* logits_dev, void* stream);
+
+/*
+ * Routing of the last forward / route call: eidx_dev [S, k] int32 expert ids
+ * (best first), gate_dev [S, k] fp32 normalised gates, slot_dev [S, k] int32
+ * slot within the expert or -1 if dropped, cnt_dev [E] int32 demand per expert
+ * before capacity.  Any pointer may be NULL to skip it.
+ */
+MOE_API moe_status moe_get_routing(moe_handle h, int32_t* eidx_dev, float* gate_dev, int32_t* slot_dev,
+                           int32_t* cnt_dev, void* stream);
+
+/*
+ * moe_route_from_logits -- run only the routing steps (softmax, top-k, gates,
+ * loss partials, capacity scan, slot assignment) on given fp32 logits
+ * [S, E] (as they enter the softmax, bias included).  Results are read with
+ * moe_get_routing / moe_aux_loss.  Expert buffers are not touched.
+ */
+MOE_API moe_status moe_route_from_logits(moe_handle h, int64_t S, const float* logits_dev, void* stream);
+
+/* Capacity C this handle uses for S tokens (host arithmetic, no device work). */
+MOE_API moe_status moe_get_capacity(moe_handle h, int64_t S, int64_t* C_out);
+
+/*
+ * Per-stage timing.  With profiling on, moe_forward records CUDA events on its
+ * stream between its kernels; moe_get_stage_times synchronises and writes the
+ * last forward's per-stage milliseconds (MOE_NUM_STAGES values, order of the
+ * MOE_STAGE_* enum) to ms_host.
+ */
+MOE_API moe_status moe_set_profiling(moe_handle h, int32_t enable);
+MOE_API moe_status moe_get_stage_times(moe_handle h, float* ms_host, int32_t n);
+
+/* Number of kernels one moe_forward of S tokens launches. */
+MOE_API int32_t moe_kernels_per_forward(moe_handle h, int64_t S);
+
+/*
+ * moe_selftest_wait_timeout -- launch a kernel whose bounded wait is made to run
+ * out (it waits for a device flag that nothing sets, with a limit of
+ * limit_us microseconds) and return what the host reads back: MOE_ERR_TIMEOUT
+ * when the bound works.  Leaves the context usable.  Synchronises `stream`.
+ */
+MOE_API moe_status moe_selftest_wait_timeout(int32_t limit_us, void* stream);
+
+/* Static description of a status code (never NULL). */
+MOE_API const char* moe_status_string(moe_status s);
+
+/* Name of a MOE_STAGE_* index ("router", "scan", ...), or "?" */
+MOE_API const char* moe_stage_name(int32_t stage);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GSHARD_MOE_H */

@@ -1,0 +1,40 @@
+"""The five benchmark workloads at full size, in the launch configuration the bench times (GPU).
+
+Routing is compared in full (every token, bit-exact given the GPU's logits);
+logits and layer outputs on seeded token samples the oracle computes one by
+one (every output row depends only on its own token once the routing is
+fixed); losses against the oracle both on the GPU's logits and on its own.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gshard_top_gating_b200.inputs import WORKLOADS
+from tests import gpu_helpers as G
+
+pytestmark = pytest.mark.gpu
+
+SAMPLES = {"tiny": None, "mid": 768, "skewed": 768, "large": 384, "wide": 48}
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_workload_full_size(name):
+    w = WORKLOADS[name]
+    run = G.build(w)
+    out = G.forward(run)
+    rt = G.check_routing(run, out)
+    n = SAMPLES[name]
+    if n is None:
+        tokens = np.arange(w.S)
+    else:
+        rng = np.random.default_rng(2024)
+        tokens = np.unique(np.concatenate([[0, w.S - 1], rng.choice(w.S, n, replace=False)]))
+    G.check_logits(run, out, tokens)
+    G.check_outputs(run, out, rt, tokens)
+    G.check_losses_own_logits(run, out)
+    # capacity invariants at full size
+    n_e = np.minimum(rt.cnt, rt.C)
+    assert np.all(n_e <= rt.C) and (out.slot >= 0).sum() == n_e.sum()
+    run.layer.close()
+    del run
+    torch.cuda.empty_cache()
