@@ -114,12 +114,19 @@ def dist_setup(n):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """Slowest rank's value (every rank calls this at the same point)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, steps: int, max_total_ms: float, world: int) -> float:
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's timed region."""
+    return world * tokens_per_rank * steps / (max_total_ms / 1e3)
 
 
 def barrier(world):
@@ -201,7 +208,7 @@ def run_ours(args, rank, world, local):
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
-    value = world * w.S * args.steps / (total_ms / 1e3)
+    value = job_throughput(w.S, args.steps, total_ms, world)
 
     # ---- per-stage device times (events recorded by the library on the same stream)
     L.moe_set_profiling(layer.h, True)
@@ -269,7 +276,7 @@ def run_ours(args, rank, world, local):
                    "l2": "flushed before every timed step (256 MB write)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roof, "stages": stages,
-        "e2e": {"value": round(world * w.S * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(job_throughput(w.S, args.steps, e2e_ms, world), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes},
         "gpu_launches": args.steps * L.moe_kernels_per_forward(layer.h, w.S),
         "clocks": clk.summary(),
