@@ -49,6 +49,7 @@ def _load() -> ctypes.CDLL:
         "moe_set_profiling": [P, I32],
         "moe_get_stage_times": [P, ctypes.POINTER(ctypes.c_float), I32],
         "moe_selftest_wait_timeout": [I32, P],
+        "moe_assign_slots_noalloc": [I64, I32, I32, I64, P, P, P, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -161,3 +162,9 @@ def moe_kernels_per_forward(h, S) -> int:
 def moe_selftest_wait_timeout(limit_us: int, stream=None) -> int:
     """Returns the raw status (MOE_ERR_TIMEOUT when the bounded wait works)."""
     return int(lib.moe_selftest_wait_timeout(limit_us, _stream(stream)))
+
+
+def moe_assign_slots_noalloc(S, E, k, C, eidx, slot, cnt, stream=None) -> None:
+    """Capacity slots from expert ids with no device allocation (see include/moe.h)."""
+    _check("moe_assign_slots_noalloc",
+           lib.moe_assign_slots_noalloc(S, E, k, C, _ptr(eidx), _ptr(slot), _ptr(cnt), _stream(stream)))

@@ -171,6 +171,37 @@ MOE_API int32_t moe_kernels_per_forward(moe_handle h, int64_t S);
  */
 MOE_API moe_status moe_selftest_wait_timeout(int32_t limit_us, void* stream);
 
+/*
+ * moe_assign_slots_noalloc -- the capacity slot assignment, with no device allocation.
+ * (The pages have no counterpart: this is an interface for callers of this library.)
+ *
+ * For callers that cannot call cudaMalloc.  Examples: a serving process whose
+ * memory pool already holds nearly all of HBM, or a runtime where every device
+ * allocation must go through its own allocator.  It applies the layer's
+ * capacity rule to expert ids the caller already has; the caller passes all
+ * inputs and outputs.
+ *
+ * S tokens (>= 0), E experts (1..256), k choices (1..min(E, 8)), capacity C (>= 0).
+ * eidx_dev  [S, k] int32 expert ids, best choice first (input).
+ * slot_dev  [S, k] int32 output: for r = 0..k-1 and tokens in order, an
+ *           assignment takes the next free slot of its expert while fewer than C
+ *           are taken, else -1 (dropped); ids outside [0, E) get -1.
+ * cnt_dev   [E] int32 output: assignments per expert before capacity.
+ *
+ * Scratch lives in one fixed 8 MiB device array inside the library, which
+ * every GPU that loads the library holds until the process exits.  The call
+ * needs round256(4*S*k) + 2*round256(4*k*ceil(S/64)*E) bytes of it and
+ * returns MOE_ERR_UNSUPPORTED, with no device work, when that exceeds 8 MiB.
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  Every call shares the array and leaves its contents behind, so
+ * calls whose work overlaps on the GPU (other streams, other host threads)
+ * race.  Enqueued on `stream`; no host synchronisation.
+ */
+MOE_API moe_status moe_assign_slots_noalloc(int64_t S, int32_t E, int32_t k, int64_t C,
+                                            const int32_t* eidx_dev, int32_t* slot_dev,
+                                            int32_t* cnt_dev, void* stream);
+
 /* Static description of a status code (never NULL). */
 MOE_API const char* moe_status_string(moe_status s);
 
