@@ -50,7 +50,7 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+    """nvidia-smi clock / throttle samples, each stamped with the host's monotonic clock."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -65,10 +65,13 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            t0 = time.monotonic()
+            while not self.rows and time.monotonic() - t0 < 10.0:
+                time.sleep(0.05)
         except OSError:
             self.proc = None
         return self
@@ -77,7 +80,7 @@ class ClockSampler:
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) >= 9:
-                self.rows.append(parts)
+                self.rows.append((time.monotonic(), parts))
 
     def __exit__(self, *a):
         if self.proc:
@@ -87,16 +90,29 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
-        if not self.rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+    def count(self, t0, t1):
+        return sum(1 for t, _ in self.rows if t0 <= t <= t1)
+
+    def summary(self, t0, t1, window):
+        rows = [r for t, r in self.rows if t0 <= t <= t1]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0,
+                    "window": window}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [v for v in (num(r[1]) for r in rows) if v is not None]
+        mx = [v for v in (num(r[2]) for r in rows) if v is not None]
+        pw = [v for v in (num(r[3]) for r in rows) if v is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i] == "Active"})
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(self.rows)}
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "reasons": reasons, "samples": len(rows), "window": window}
 
 
 def dist_setup(n):
@@ -135,24 +151,25 @@ def barrier(world):
         dist.barrier()
 
 
-def source_hash() -> str:
+def source_hash(files) -> str:
+    """Hash of the given files under the library's csrc/ (the kernel a counter was taken on)."""
     h = hashlib.sha256()
     cs = os.path.join(ROOT, "gshard_top_gating_b200", "csrc")
-    for f in sorted(os.listdir(cs)):
+    for f in sorted(files):
         with open(os.path.join(cs, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel: str, workload: str):
-    """dram bytes per launch of `kernel` from the committed ncu summary, if it is current."""
+    """DRAM bytes per launch of `kernel` from the committed ncu record, while its sources are unchanged."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     ent = d.get(workload, {}).get(kernel)
-    if not ent or ent.get("source_hash") != source_hash():
+    if not ent or ent.get("source_hash") != source_hash(ent.get("sources", [])):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -195,16 +212,18 @@ def run_ours(args, rank, world, local):
     # ---- timed region: K forwards, L2 flushed before each, device time per step
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    with ClockSampler(local) as clk:
-        barrier(world)
-        torch.cuda.synchronize()
-        for i in range(args.steps):
-            flush.zero_()
-            starts[i].record(stream)
-            layer(x, out=y)
-            ends[i].record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
+    clk = ClockSampler(local).__enter__()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_begin = time.monotonic()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        layer(x, out=y)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    t_end = time.monotonic()
+    barrier(world)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
@@ -238,6 +257,21 @@ def run_ours(args, rank, world, local):
     e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), world)
     nbytes = x.numel() * x.element_size()
 
+    # clocks: the timed region itself when it held enough samples, else a soak of
+    # the same forward right after it (the timed region was too short to sample)
+    if clk.count(t_begin, t_end) >= 3:
+        clocks = clk.summary(t_begin, t_end, "timed region")
+    else:
+        s0 = time.monotonic()
+        while time.monotonic() - s0 < 1.5:
+            for _ in range(20):
+                flush.zero_()
+                layer(x, out=y)
+            torch.cuda.synchronize()
+        clocks = clk.summary(s0, time.monotonic(),
+                             "1.5 s soak of the same step right after the timed region")
+    clk.__exit__()
+
     pk, pk_kind = peaks()
     algo = algorithmic(w, A, n_active)
     dom = max(stage_ms, key=lambda n: stage_ms[n])
@@ -263,7 +297,7 @@ def run_ours(args, rank, world, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, args.cpu_tokens, x, Wg, b, W1, W2)
+        cpu = cpu_baseline(w, args.cpu_budget, x, Wg, b, W1, W2)
 
     line = {
         "metric": "MoE-layer tokens/sec on 1 B200; FFN % of bf16 TC peak; dispatch/combine HBM GB/s",
@@ -279,47 +313,67 @@ def run_ours(args, rank, world, local):
         "e2e": {"value": round(job_throughput(w.S, args.steps, e2e_ms, world), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes},
         "gpu_launches": args.steps * L.moe_kernels_per_forward(layer.h, w.S),
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "cpu_baseline": cpu,
     }
     layer.close()
     return line
 
 
-def _oracle_sample(w, ntok, x, Wg, b, W1, W2):
-    """Inputs of a bounded sample of the workload: the first ntok tokens, all experts."""
-    xs = x[:ntok].cpu()
-    return xs, Wg.cpu(), None if b is None else b.cpu(), W1.cpu(), W2.cpu()
+def _oracle_inputs(w, x, Wg, b, W1, W2):
+    """Host float64 copies of the workload's inputs (the oracle's input form)."""
+    import numpy as np
+    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+    return (f64(x), f64(Wg), None if b is None else f64(b), f64(W1), f64(W2))
 
 
-def cpu_baseline(w, ntok, x, Wg, b, W1, W2, threads=None):
-    import oracle as O
-    xs, Wgc, bc, W1c, W2c = _oracle_sample(w, ntok, x, Wg, b, W1, W2)
-    cores = torch.get_num_threads() if threads is None else threads
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d["num_threads"] for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _oracle_step(O, w, inp, ntok):
+    xs, Wg, b, W1, W2 = inp
     t0 = time.perf_counter()
-    O.forward(xs, Wgc, bc, W1c, W2c, w.k, w.cf)
-    dt = time.perf_counter() - t0
-    return {"value": round(ntok / dt, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+    O.forward(xs[:ntok], Wg, b, W1, W2, w.k, w.cf)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, budget_s, x, Wg, b, W1, W2):
+    """The oracle as it stands, timed on the host cores on a bounded token sample."""
+    import oracle as O
+    inp = _oracle_inputs(w, x, Wg, b, W1, W2)
+    probe = min(w.S, 256)
+    c = _oracle_step(O, w, inp, probe) / probe                 # seconds per token
+    ntok = int(max(64, min(w.S, budget_s / max(c, 1e-9))))
+    dt = _oracle_step(O, w, inp, ntok)
+    return {"value": round(ntok / dt, 2), "unit": "tokens/s", "cores": _blas_threads(),
+            "kind": "oracle",
             "sample": f"first {ntok} of {w.S} tokens of the {w.name} workload (same M, H, E, k, cf; "
-                      f"C scaled to the sample), full float64 oracle forward, {dt:.1f} s"}
+                      f"C scaled to the sample); float64 oracle forward, {dt:.1f} s; weights "
+                      f"converted to float64 once, outside the timing"}
 
 
 def run_reference(args, rank, world):
     w = WORKLOADS[args.workload]
     if rank != 0:
         return None
-    ntok = args.cpu_tokens
-    x, Wg, b, W1, W2 = make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
     import oracle as O
-    xs, Wgc, bc, W1c, W2c = _oracle_sample(w, ntok, x, Wg, b, W1, W2)
-    del x, W1, W2
-    for _ in range(args.warmup if args.warmup < 1 else 1):
-        O.forward(xs, Wgc, bc, W1c, W2c, w.k, w.cf)
-    times = []
-    for _ in range(args.steps):
-        t0 = time.perf_counter()
-        O.forward(xs, Wgc, bc, W1c, W2c, w.k, w.cf)
-        times.append(time.perf_counter() - t0)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = _oracle_inputs(w, *make_inputs(w, device=dev))
+    torch.cuda.empty_cache() if dev == "cuda" else None
+    probe = min(w.S, 256)
+    c = _oracle_step(O, w, inp, probe) / probe
+    # per-step sample sized so the whole run stays near args.ref_budget seconds
+    per_step = args.ref_budget / max(1, args.steps + args.warmup)
+    ntok = int(max(64, min(w.S, per_step / max(c, 1e-9))))
+    for _ in range(args.warmup):
+        _oracle_step(O, w, inp, ntok)
+    times = [_oracle_step(O, w, inp, ntok) for _ in range(args.steps)]
     tot = sum(times)
     v = round(ntok * args.steps / tot, 2)
     return {
@@ -331,9 +385,9 @@ def run_reference(args, rank, world):
         "data": "synthetic",
         "config": {"workload": f"{w.name} (S={w.S}, M={w.M}, H={w.H}, E={w.E}, k={w.k}, cf={w.cf})",
                    "S": w.S, "M": w.M, "H": w.H, "E": w.E, "k": w.k, "capacity_factor": w.cf},
-        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": torch.get_num_threads(),
-                         "kind": "oracle",
-                         "sample": f"first {ntok} of {w.S} tokens per step (same M, H, E, k, cf)"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+                         "sample": f"first {ntok} of {w.S} tokens per step (same M, H, E, k, cf; "
+                                   f"C scaled to the sample); float64 oracle forward"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -341,21 +395,28 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(WORKLOADS), default="mid")
-    ap.add_argument("--cpu-tokens", type=int, default=512)
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle work for the CPU baseline sample")
+    ap.add_argument("--ref-budget", type=float, default=120.0,
+                    help="seconds of oracle work for the whole --impl reference run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.impl == "ours" and args.warmup < 3:
         args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
     rank, world, local = dist_setup(args.gpus)
     try:
-        if args.impl == "reference":
-            line = run_reference(args, rank, world)
-        else:
-            line = run_ours(args, rank, world, local)
+        line = run_ours(args, rank, world, local)
         if rank == 0 and line is not None:
             print(json.dumps(line), flush=True)
     finally:

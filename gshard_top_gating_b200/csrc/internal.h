@@ -33,6 +33,13 @@ cudaError_t launch_router(const void* x, bool x_bf16, const float* Wg, const flo
                           int M, int E, int k, const Routing& R, cudaStream_t st);
 cudaError_t launch_route_logits(const float* logits, int S, int E, int k, const Routing& R,
                                 cudaStream_t st);
+// router_tc.cu  (bf16 tokens: gate GEMM on tcgen05 with a bf16x3 split of W_g)
+int router_tc_pad(int E);
+cudaError_t split_gate_weights(const float* Wg, int M, int E, void* out3, cudaStream_t st);
+bool make_router_wmap(CUtensorMap* tm, const void* wsplit, int M, int E);
+bool make_router_xmap(CUtensorMap* tm, const void* x, int S, int M);
+cudaError_t launch_router_tc(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias, int S,
+                             int M, int E, int k, const Routing& R, uint64_t limit_ns, cudaStream_t st);
 // scan.cu
 cudaError_t launch_scan(int S, int E, int k, int C, int64_t Cbuf, const Routing& R, cudaStream_t st);
 // dispatch_combine.cu

@@ -41,6 +41,10 @@ struct moe_layer {
   void* xstage;          // moe_forward_host staging
   void* ystage;
   GemmPlan plan1, plan2;
+  void* wsplit;          // bf16 tokens: W_g split into three bf16 parts [3][EP][M]
+  CUtensorMap wmap, xmap;
+  const void* xmap_ptr;  // x pointer / S the cached xmap describes
+  int64_t xmap_S;
   int64_t last_S;
   bool have_forward;
   bool profiling;
@@ -105,6 +109,7 @@ size_t carve(moe_layer* h, char* base) {
   h->ybuf = c.take<char>((size_t)E * h->Cbuf * h->M * as);
   h->xstage = c.take<char>((size_t)S * h->M * as);
   h->ystage = c.take<char>((size_t)S * h->M * as);
+  h->wsplit = h->act == MOE_BF16 ? c.take<char>((size_t)3 * router_tc_pad(h->E) * h->M * 2) : nullptr;
   return c.off + 256;
 }
 
@@ -205,7 +210,10 @@ moe_status moe_create(moe_handle* out, int64_t S_max, int64_t M, int64_t H, int3
   if (act == MOE_BF16) {
     const bool ok1 = make_gemm_plan(h->plan1, h->xbuf, W1, h->hbuf, E, h->Cbuf, (int)M, (int)H, true);
     const bool ok2 = make_gemm_plan(h->plan2, h->hbuf, W2, h->ybuf, E, h->Cbuf, (int)H, (int)M, false);
-    if (!ok1 || !ok2) {
+    ce = split_gate_weights(Wg, (int)M, E, h->wsplit, 0);
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(0);
+    const bool ok3 = ce == cudaSuccess && make_router_wmap(&h->wmap, h->wsplit, (int)M, E);
+    if (!ok1 || !ok2 || !ok3) {
       cudaFree(h->ws);
       delete h;
       return MOE_ERR_CUDA;
@@ -255,7 +263,16 @@ moe_status moe_forward(moe_handle h, int64_t S, const void* x, void* y, void* st
   auto mark = [&](int i) -> cudaError_t { return prof ? cudaEventRecord(h->ev[i], st) : cudaSuccess; };
 
   MOE_TRY(mark(0));
-  MOE_TRY(launch_router(x, bf16, h->Wg, h->bias, iS, iM, h->E, h->k, R, st));
+  if (bf16) {
+    if (h->xmap_ptr != x || h->xmap_S != S) {
+      if (!make_router_xmap(&h->xmap, x, iS, iM)) return MOE_ERR_CUDA;
+      h->xmap_ptr = x;
+      h->xmap_S = S;
+    }
+    MOE_TRY(launch_router_tc(h->xmap, h->wmap, h->bias, iS, iM, h->E, h->k, R, h->wait_limit_ns, st));
+  } else {
+    MOE_TRY(launch_router(x, bf16, h->Wg, h->bias, iS, iM, h->E, h->k, R, st));
+  }
   MOE_TRY(mark(1));
   MOE_TRY(launch_scan(iS, h->E, h->k, C, h->Cbuf, R, st));
   MOE_TRY(mark(2));

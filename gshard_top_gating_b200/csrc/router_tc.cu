@@ -1,0 +1,483 @@
+// router_tc.cu -- gate GEMM on tcgen05 tensor cores for bf16 tokens, then softmax, top-k,
+// normalised gates and the per-chunk tables of the capacity scan.
+//
+// Gating: G(x) = Softmax(x . W_g) ("GShard: Scaling Giant Neural Networks with
+// Conditional Computation", "Mixture-of-Experts Implementation"), top-k experts
+// with "softmax-normalised top-2 weights" ("GShard: Scaling Giant Models with
+// Conditional Computation and Automatic Sharding", paper-note summary).
+//
+// Precision.  The gate GEMM is fp32 in the method.  A bf16 token is exact in
+// bf16, and W_g is split once, at create time, into three bf16 parts
+// W_g = hi + mid + lo (about 24 significant bits, the bf16x3 scheme of Henry,
+// Tang and Heinecke, "Leveraging the bfloat16 artificial intelligence datatype
+// for higher-precision computations", ARITH 2019).  The three products
+// x.hi + x.mid + x.lo accumulate in an fp32 TMEM accumulator.  The tensor
+// core's fp32 accumulation does not round to nearest, and over a long K its
+// rounding error builds up coherently, so K is cut into segments of
+// kSegBlocks*64: each segment accumulates from zero and the epilogue warps add
+// it into a second TMEM region with ordinary round-to-nearest fp32 adds.  The
+// logits so carry fp32-level error at tensor-core speed.
+//
+// One CTA = 128 tokens x EP experts (E padded to 32/64/128/256), 192 threads:
+// warp 0 TMA producer (x tile 128x64 + three W_g parts EPx64 per stage, K-major,
+// 128B swizzle), warp 1 TMEM owner and single-thread MMA issuer, warps 2-5 the
+// epilogue with one token row per thread.  The epilogue reads the accumulator
+// three times (max and top-k; sum of exponentials; probabilities), keeps the
+// top-k in registers with ties to the lower expert index, and writes the same
+// per-64-token chunk tables (probability sums, lse^2 sums, rank-r histograms,
+// local ranks) as the CUDA-core router.
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128, BK = 64;
+constexpr int kThreads = 192;
+constexpr uint32_t A_BYTES = BM * BK * 2;
+constexpr int kSegBlocks = 8;      // k-blocks (of 64) accumulated before each fp32 round-to-nearest add
+
+template <int EP>
+struct RCfg {
+  static constexpr uint32_t PART_BYTES = EP * BK * 2;            // one W_g part, EP x 64 bf16
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + 3 * PART_BYTES;
+  static constexpr int STAGES = (EP == 256) ? 2 : (EP == 128 ? 3 : (EP == 64 ? 5 : 7));
+  static constexpr uint32_t TMEM_COLS = 2 * EP;        // accumulator + running sum
+  // epilogue scratch reuses the stage buffers: P [128][EP] f32, sel [128][8] i32,
+  // lse2 [128] f32, hist [2][8][EP] i32
+  static constexpr uint32_t P_OFF = 0;
+  static constexpr uint32_t SEL_OFF = P_OFF + 128 * EP * 4;
+  static constexpr uint32_t L_OFF = SEL_OFF + 128 * kMaxK * 4;
+  static constexpr uint32_t H_OFF = L_OFF + 128 * 4;
+  static constexpr uint32_t EPI_END = H_OFF + 2 * kMaxK * EP * 4;
+  static_assert(EPI_END <= STAGES * STAGE_BYTES, "epilogue scratch must fit in the stage buffers");
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + 16;
+};
+
+__device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         (1ull << 46) | (2ull << 61);
+}
+
+// kind::f16, D fp32, A bf16 K-major, B bf16 K-major, M=128, N=EP
+template <int EP>
+__device__ __forceinline__ uint32_t idesc_router() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(EP >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void named_sync_epi() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+template <int EP>
+__global__ void __launch_bounds__(kThreads, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const float* __restrict__ bias, int S, int M, int E, int k, int nchunk,
+                     Routing R, uint64_t limit_ns) {
+  using C = RCfg<EP>;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;
+  unsigned char* gbase = smem_raw + (base - raw_base);
+  const uint32_t bar0 = base + C::STAGES * C::STAGE_BYTES;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  const uint32_t tfull_bar = bar0 + 8u * (2 * C::STAGES);      // a K-segment is accumulated
+  const uint32_t done_bar = bar0 + 8u * (2 * C::STAGES + 1);
+  const uint32_t tempty_bar = bar0 + 8u * (2 * C::STAGES + 2);   // the epilogue took the segment
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + C::STAGES * C::STAGE_BYTES + 256);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::STAGES * C::STAGE_BYTES + 260);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, tok0 = tile * BM;
+  const int KB = M / BK;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(tfull_bar, 1);
+    mbar_init(done_bar, 1);
+    mbar_init(tempty_bar, 128);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, issued = 0, issued_par = 0;
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (*abort_flag || !mbar_wait(empty_bar(s), ph ^ 1u, R.err, limit_ns)) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        const uint32_t sa = base + s * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(full_bar(s), C::STAGE_BYTES);
+        tma_load_2d(sa, &tmX, full_bar(s), kb * BK, tok0);
+#pragma unroll
+        for (int part = 0; part < 3; ++part)
+          tma_load_2d(sa + A_BYTES + part * C::PART_BYTES, &tmW, full_bar(s), kb * BK, part * EP);
+        issued |= 1u << s;
+        issued_par = (issued_par & ~(1u << s)) | (ph << s);
+        if (++s == C::STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (!ok)
+        for (int q = 0; q < C::STAGES; ++q)
+          if ((issued >> q) & 1u) mbar_wait(full_bar(q), (issued_par >> q) & 1u, R.err, limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_router<EP>();
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb) {
+        const int seg = kb / kSegBlocks;
+        const bool seg_first = (kb % kSegBlocks) == 0;
+        const bool seg_last = (kb % kSegBlocks) == kSegBlocks - 1 || kb == KB - 1;
+        if (seg_first) {   // the epilogue must have taken the previous segment
+          if (*abort_flag || !mbar_wait(tempty_bar, (seg & 1) ^ 1u, R.err, limit_ns)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        if (*abort_flag || !mbar_wait(full_bar(s), ph, R.err, limit_ns)) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = base + s * C::STAGE_BYTES;
+#pragma unroll
+        for (int part = 2; part >= 0; --part) {       // smallest part first
+          const uint32_t sb = sa + A_BYTES + part * C::PART_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_f16(tmem_base, desc_kmajor_sw128(sa + kk * 32u), desc_kmajor_sw128(sb + kk * 32u),
+                       idesc, !(seg_first && kk == 0 && part == 2));
+        }
+        tc_commit(empty_bar(s));
+        if (seg_last) tc_commit(tfull_bar);
+        if (++s == C::STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (!ok) {
+        tc_commit(done_bar);
+        mbar_wait(done_bar, 0, R.err, limit_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue: one token per thread
+    const int q = warp & 3;
+    const int row = q * 32 + lane;              // token row within the tile (= TMEM lane)
+    const int et = threadIdx.x - 64;            // 0..127 epilogue thread index
+    const int tok = tok0 + row;
+    const bool live = tok < S;
+    float* Ps = reinterpret_cast<float*>(gbase + C::P_OFF);
+    int32_t* sel = reinterpret_cast<int32_t*>(gbase + C::SEL_OFF);
+    float* Ls = reinterpret_cast<float*>(gbase + C::L_OFF);
+    int32_t* Hs = reinterpret_cast<int32_t*>(gbase + C::H_OFF);
+    const uint32_t tlane = tmem_base + ((uint32_t)(q * 32) << 16);
+    // fold the K-segments: sum (columns EP..2EP) += segment accumulator (columns 0..EP)
+    const int nseg = (KB + kSegBlocks - 1) / kSegBlocks;
+    bool ok = true;
+    for (int seg = 0; seg < nseg; ++seg) {
+      if (*abort_flag || !mbar_wait(tfull_bar, seg & 1, R.err, limit_ns)) {
+        *abort_flag = 1;
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (nseg > 1) {
+#pragma unroll 1
+        for (int c = 0; c < EP / 32; ++c) {
+          uint32_t a[32], b[32];
+          tmem_ld_32x32b_x32(tlane + c * 32, a);
+          if (seg > 0) tmem_ld_32x32b_x32(tlane + EP + c * 32, b);
+          tmem_ld_wait();
+          if (seg > 0) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) + __uint_as_float(b[i]));
+          }
+          tmem_st_32x32b_x32(tlane + EP + c * 32, a);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar);
+    }
+    tc_fence_after();
+    const uint32_t taddr = tlane + (nseg > 1 ? EP : 0);    // final logits (before bias)
+
+    float bv[kMaxK];
+    int bj[kMaxK];
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) {
+      bv[r] = -INFINITY;
+      bj[r] = 0x7fffffff;
+    }
+    float mx = -INFINITY;
+    // pass A: logits out, max, top-k (insertion in ascending expert order keeps ties stable)
+#pragma unroll 1
+    for (int c = 0; c < EP / 32; ++c) {
+      uint32_t u[32];
+      tmem_ld_32x32b_x32(taddr + c * 32, u);
+      tmem_ld_wait();
+      if (ok && live) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int j = c * 32 + i;
+          if (j < E) {
+            float v = __uint_as_float(u[i]);
+            if (bias) v += __ldg(bias + j);
+            R.logits[(int64_t)tok * E + j] = v;
+            mx = fmaxf(mx, v);
+            if (v > bv[kMaxK - 1]) {
+              bv[kMaxK - 1] = v;
+              bj[kMaxK - 1] = j;
+#pragma unroll
+              for (int r = kMaxK - 1; r > 0; --r) {
+                if (bv[r] > bv[r - 1]) {
+                  const float tv = bv[r];
+                  bv[r] = bv[r - 1];
+                  bv[r - 1] = tv;
+                  const int tj = bj[r];
+                  bj[r] = bj[r - 1];
+                  bj[r - 1] = tj;
+                }
+              }
+            }
+          }
+        }
+      }
+    }
+    // pass B: sum of exponentials
+    float s = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < EP / 32; ++c) {
+      uint32_t u[32];
+      tmem_ld_32x32b_x32(taddr + c * 32, u);
+      tmem_ld_wait();
+      if (ok && live) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int j = c * 32 + i;
+          if (j < E) {
+            float v = __uint_as_float(u[i]);
+            if (bias) v += __ldg(bias + j);
+            s += expf(v - mx);
+          }
+        }
+      }
+    }
+    const float inv = (ok && live) ? 1.f / s : 0.f;
+    // pass C: probabilities into smem for the per-chunk column sums
+#pragma unroll 1
+    for (int c = 0; c < EP / 32; ++c) {
+      uint32_t u[32];
+      tmem_ld_32x32b_x32(taddr + c * 32, u);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int j = c * 32 + i;
+        float p = 0.f;
+        if (ok && live && j < E) {
+          float v = __uint_as_float(u[i]);
+          if (bias) v += __ldg(bias + j);
+          p = expf(v - mx) * inv;
+        }
+        Ps[row * EP + ((j + row) & (EP - 1))] = p;     // rotated columns: no bank conflicts
+      }
+    }
+    if (ok && live) {
+      const float lse = mx + logf(s);
+      Ls[row] = lse * lse;
+      float gs = 0.f, gr[kMaxK];
+#pragma unroll
+      for (int r = 0; r < kMaxK; ++r) {
+        gr[r] = (r < k) ? expf(bv[r] - bv[0]) : 0.f;
+        gs += gr[r];
+      }
+      const float ginv = 1.f / gs;
+#pragma unroll
+      for (int r = 0; r < kMaxK; ++r) {
+        if (r < k) {
+          int j = bj[r];
+          if (j >= E) {                        // only for non-finite logits
+            atomicOr(R.err, DEVERR_BOUNDS);
+            j = 0;
+          }
+          R.eidx[(int64_t)tok * k + r] = j;
+          R.gate[(int64_t)tok * k + r] = gr[r] * ginv;
+          sel[row * kMaxK + r] = j;
+        }
+      }
+    } else {
+      Ls[row] = 0.f;
+    }
+    for (int i = et; i < 2 * kMaxK * EP; i += 128) Hs[i] = 0;
+    tc_fence_before();
+    named_sync_epi();
+
+    // per-chunk column sums of p (two 64-token chunks per tile), fixed order
+    const int chunk0 = tile * 2;
+    for (int cc = 0; cc < 2; ++cc) {
+      const int chunk = chunk0 + cc;
+      if (chunk >= nchunk) break;
+      for (int j = et; j < E; j += 128) {
+        float acc = 0.f;
+        for (int rr = cc * 64; rr < cc * 64 + 64; ++rr) acc += Ps[rr * EP + ((j + rr) & (EP - 1))];
+        R.psum[(int64_t)chunk * E + j] = acc;
+      }
+      if (et == 0) {
+        float acc = 0.f;
+        for (int rr = cc * 64; rr < cc * 64 + 64; ++rr) acc += Ls[rr];
+        R.lse2[chunk] = acc;
+      }
+    }
+    // local ranks within each 64-token chunk and rank-r histograms
+    const int ntile = min(BM, S - tok0);
+    for (int idx = et; idx < ntile * k; idx += 128) {
+      const int t = idx / k, r = idx - t * k;
+      const int e = sel[t * kMaxK + r];
+      const int cbeg = (t >> 6) << 6;
+      int c = 0;
+      for (int u = cbeg; u < t; ++u) c += (sel[u * kMaxK + r] == e);
+      R.lrank[(int64_t)(tok0 + t) * k + r] = c;
+      atomicAdd(&Hs[((t >> 6) * kMaxK + r) * EP + e], 1);
+    }
+    named_sync_epi();
+    for (int cc = 0; cc < 2; ++cc) {
+      const int chunk = chunk0 + cc;
+      if (chunk >= nchunk) break;
+      for (int idx = et; idx < k * E; idx += 128) {
+        const int r = idx / E, e = idx - r * E;
+        R.hist[((int64_t)r * nchunk + chunk) * E + e] = Hs[(cc * kMaxK + r) * EP + e];
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// W_g [M, E] fp32 -> three bf16 parts, each [EP, M] (K contiguous), rows >= E zero.
+__global__ void split_gate_kernel(const float* __restrict__ Wg, int M, int E, int EP,
+                                  __nv_bfloat16* __restrict__ out) {
+  const int64_t n = (int64_t)EP * M;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int j = (int)(i / M), m = (int)(i - (int64_t)j * M);
+    const float w = j < E ? Wg[(int64_t)m * E + j] : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+    out[i] = hi;
+    out[n + i] = mid;
+    out[2 * n + i] = lo;
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+bool encode_kmajor(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_out) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, box_out};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EP>
+cudaError_t launch_t(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias, int S, int M,
+                     int E, int k, const Routing& R, uint64_t limit_ns, cudaStream_t st) {
+  auto kern = router_tc_kernel<EP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)RCfg<EP>::SMEM);
+  if (e != cudaSuccess) return e;
+  const int nchunk = (S + kChunk - 1) / kChunk;
+  kern<<<(S + BM - 1) / BM, kThreads, RCfg<EP>::SMEM, st>>>(tmX, tmW, bias, S, M, E, k, nchunk, R,
+                                                            limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int router_tc_pad(int E) { return E <= 32 ? 32 : (E <= 64 ? 64 : (E <= 128 ? 128 : 256)); }
+
+cudaError_t split_gate_weights(const float* Wg, int M, int E, void* out3, cudaStream_t st) {
+  const int EP = router_tc_pad(E);
+  const int64_t n = (int64_t)EP * M;
+  const int grid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  split_gate_kernel<<<grid, 256, 0, st>>>(Wg, M, E, EP, (__nv_bfloat16*)out3);
+  return cudaGetLastError();
+}
+
+bool make_router_wmap(CUtensorMap* tm, const void* wsplit, int M, int E) {
+  const int EP = router_tc_pad(E);
+  return encode_kmajor(tm, wsplit, (uint64_t)M, (uint64_t)3 * EP, (uint32_t)EP);
+}
+
+bool make_router_xmap(CUtensorMap* tm, const void* x, int S, int M) {
+  return encode_kmajor(tm, x, (uint64_t)M, (uint64_t)S, (uint32_t)BM);
+}
+
+cudaError_t launch_router_tc(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias, int S,
+                             int M, int E, int k, const Routing& R, uint64_t limit_ns, cudaStream_t st) {
+  switch (router_tc_pad(E)) {
+    case 32: return launch_t<32>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);
+    case 64: return launch_t<64>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);
+    case 128: return launch_t<128>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);
+    default: return launch_t<256>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);
+  }
+}
+
+}  // namespace moe

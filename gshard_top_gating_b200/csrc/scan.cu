@@ -84,14 +84,30 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(int S, int E, int k, int
     }
     return;
   }
-  // block E: auxiliary losses
+  // block E: auxiliary losses.  G threads share each expert column j, thread
+  // (j, g) summing chunks g, g+G, ...; the G partials are then added in order.
+  __shared__ double part_P[kThreads];
+  __shared__ long long part_f[kThreads];
+  const int G = E >= kThreads ? 1 : kThreads / E;
+  if (tid < E * G) {
+    const int j = tid % E, g = tid / E;
+    double P = 0.0;
+    long long f = 0;
+    for (int c = g; c < nchunk; c += G) {
+      P += (double)R.psum[(int64_t)c * E + j];
+      f += R.hist[(int64_t)c * E + j];          // rank-0 plane of hist: first choices
+    }
+    part_P[tid] = P;
+    part_f[tid] = f;
+  }
+  __syncthreads();
   double term = 0.0;
   for (int j = tid; j < E; j += kThreads) {
     double P = 0.0;
     long long f = 0;
-    for (int c = 0; c < nchunk; ++c) {
-      P += (double)R.psum[(int64_t)c * E + j];
-      f += R.hist[(int64_t)c * E + j];          // rank 0 rows of hist
+    for (int g = 0; g < G; ++g) {
+      P += part_P[g * E + j];
+      f += part_f[g * E + j];
     }
     term += (double)f * P;
   }

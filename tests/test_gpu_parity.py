@@ -39,6 +39,9 @@ BF16_SHAPES = [
     (129, 128, 128, 1, 1, 1.0),       # E=1: dense FFN
     (70, 128, 256, 5, 5, 1.0),        # k = E
     (1, 128, 256, 8, 2, 1.25),
+    (300, 128, 128, 200, 8, 1.25),    # router: E padded to 256, top-8
+    (200, 192, 128, 100, 3, 1.0),     # router: E padded to 128
+    (333, 64, 64, 33, 2, 1.0),        # router: E padded to 64
 ]
 
 

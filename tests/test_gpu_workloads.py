@@ -29,9 +29,11 @@ def test_workload_full_size(name):
     else:
         rng = np.random.default_rng(2024)
         tokens = np.unique(np.concatenate([[0, w.S - 1], rng.choice(w.S, n, replace=False)]))
-    G.check_logits(run, out, tokens)
-    G.check_outputs(run, out, rt, tokens)
+    e_logits = G.check_logits(run, out, tokens)
+    e_y = G.check_outputs(run, out, rt, tokens)
     G.check_losses_own_logits(run, out)
+    print(f"\n{name}: logits rel err {e_logits:.3e}, output rel err {e_y:.3e}, "
+          f"dropped {(out.slot < 0).mean():.4f}, l_aux {out.l_aux:.6f}, z {out.z:.6f}")
     # capacity invariants at full size
     n_e = np.minimum(rt.cnt, rt.C)
     assert np.all(n_e <= rt.C) and (out.slot >= 0).sum() == n_e.sum()
