@@ -20,15 +20,25 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads) dispatch_kernel(const T* __restrict__ x, int S, int M,
-                                                            int E, int k, int C, int64_t Cbuf,
-                                                            int nchunk, Routing R,
-                                                            T* __restrict__ xbuf) {
+// One warp per token.  The first slice of the token's row is loaded before the
+// slot lookups (which depend on two chained table reads), so the row's memory
+// latency overlaps them.
+template <typename T, int KM>
+__global__ void __launch_bounds__(kThreads, 4) dispatch_kernel(const T* __restrict__ x, int S, int M,
+                                                               int E, int k, int C, int64_t Cbuf,
+                                                               int nchunk, Routing R,
+                                                               T* __restrict__ xbuf) {
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * kThreads) >> 5;
   const int nv = (int)((int64_t)M * sizeof(T) / 16);
   for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < S; t += warps) {
+    const uint4* src = x ? reinterpret_cast<const uint4*>(x + (int64_t)t * M) : nullptr;
+    uint4 first[kUnroll];
+    if (src) {
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (lane + 32 * u < nv) first[u] = ld_nc_v4(src + lane + 32 * u);
+    }
     int e = 0, s = -1;
     if (lane < k) {
       e = R.eidx[(int64_t)t * k + lane];
@@ -42,11 +52,10 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(const T* __restrict_
       s = (pos < C && pos < Cbuf) ? pos : -1;
       R.slot[(int64_t)t * k + lane] = s;
     }
-    if (x == nullptr) continue;                // slot-only pass (routing without data)
-    const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)t * M);
-    uint4* dst[kMaxK];
+    if (src == nullptr) continue;              // slot-only pass (routing without data)
+    uint4* dst[KM];
 #pragma unroll
-    for (int r = 0; r < kMaxK; ++r) {
+    for (int r = 0; r < KM; ++r) {
       const int er = __shfl_sync(0xffffffffu, e, r);
       const int sr = __shfl_sync(0xffffffffu, s, r);
       dst[r] = (r < k && sr >= 0) ? reinterpret_cast<uint4*>(xbuf + ((int64_t)er * Cbuf + sr) * M)
@@ -55,10 +64,12 @@ __global__ void __launch_bounds__(kThreads) dispatch_kernel(const T* __restrict_
     for (int v0 = lane; v0 < nv; v0 += 32 * kUnroll) {
       uint4 val[kUnroll];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
-        if (v0 + 32 * u < nv) val[u] = ld_nc_v4(src + v0 + 32 * u);
+      for (int u = 0; u < kUnroll; ++u) {
+        if (v0 == lane) val[u] = first[u];
+        else if (v0 + 32 * u < nv) val[u] = ld_nc_v4(src + v0 + 32 * u);
+      }
 #pragma unroll
-      for (int r = 0; r < kMaxK; ++r) {
+      for (int r = 0; r < KM; ++r) {
         if (dst[r] == nullptr) continue;
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u)
@@ -101,13 +112,14 @@ struct Vec<float> {
   }
 };
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads) combine_kernel(const T* __restrict__ ybuf, int S, int M,
-                                                           int k, int64_t Cbuf, Routing R,
-                                                           T* __restrict__ y) {
+template <typename T, int KM>
+__global__ void __launch_bounds__(kThreads, KM >= 8 ? 3 : 4) combine_kernel(const T* __restrict__ ybuf, int S, int M,
+                                                              int k, int64_t Cbuf, Routing R,
+                                                              T* __restrict__ y) {
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * kThreads) >> 5;
   const int nv = (int)((int64_t)M * sizeof(T) / 16);
+  constexpr int U = KM >= 4 ? 1 : 2;          // 16-byte vectors per lane per step
   for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < S; t += warps) {
     int e = 0, s = -1;
     float g = 0.f;
@@ -116,10 +128,10 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const T* __restrict__
       s = R.slot[(int64_t)t * k + lane];
       g = R.gate[(int64_t)t * k + lane];
     }
-    const uint4* srcs[kMaxK];
-    float gr[kMaxK];
+    const uint4* srcs[KM];
+    float gr[KM];
 #pragma unroll
-    for (int r = 0; r < kMaxK; ++r) {
+    for (int r = 0; r < KM; ++r) {
       const int er = __shfl_sync(0xffffffffu, e, r);
       const int sr = __shfl_sync(0xffffffffu, s, r);
       gr[r] = __shfl_sync(0xffffffffu, g, r);
@@ -128,25 +140,26 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const T* __restrict__
                     : nullptr;
     }
     uint4* dst = reinterpret_cast<uint4*>(y + (int64_t)t * M);
-    for (int v0 = lane; v0 < nv; v0 += 32 * 2) {
-      float acc[2][8];
+    for (int v0 = lane; v0 < nv; v0 += 32 * U) {
+      float acc[U][8];
 #pragma unroll
-      for (int u = 0; u < 2; ++u)
+      for (int u = 0; u < U; ++u)
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[u][q] = 0.f;
+      // all k rows' loads first, then the fixed-order fp32 sum
+      uint4 val[KM][U];
 #pragma unroll
-      for (int r = 0; r < kMaxK; ++r) {
-        if (srcs[r] == nullptr) continue;
-        uint4 val[2];
+      for (int r = 0; r < KM; ++r)
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
-          if (v0 + 32 * u < nv) val[u] = ld_nc_v4(srcs[r] + v0 + 32 * u);
+        for (int u = 0; u < U; ++u)
+          if (srcs[r] != nullptr && v0 + 32 * u < nv) val[r][u] = ld_nc_v4(srcs[r] + v0 + 32 * u);
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
-          if (v0 + 32 * u < nv) Vec<T>::load_fma(acc[u], val[u], gr[r]);
-      }
+      for (int r = 0; r < KM; ++r)
 #pragma unroll
-      for (int u = 0; u < 2; ++u)
+        for (int u = 0; u < U; ++u)
+          if (srcs[r] != nullptr && v0 + 32 * u < nv) Vec<T>::load_fma(acc[u], val[r][u], gr[r]);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
         if (v0 + 32 * u < nv) dst[v0 + 32 * u] = Vec<T>::pack(acc[u]);
     }
   }
@@ -156,8 +169,39 @@ int grid_for(int S) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int want = (S + (kThreads / 32) - 1) / (kThreads / 32);
-  return want < sms * 8 ? want : sms * 8;
+  const int want = (S + (kThreads / 32) - 1) / (kThreads / 32);   // one warp per token
+  return want < sms * 4 ? want : sms * 4;                          // 4 CTAs per SM resident
+}
+
+template <typename T, int KM>
+void dispatch_t(const void* x, int S, int M, int E, int k, int C, int64_t Cbuf, int nchunk,
+                const Routing& R, void* xbuf, int grid, cudaStream_t st) {
+  dispatch_kernel<T, KM><<<grid, kThreads, 0, st>>>((const T*)x, S, M, E, k, C, Cbuf, nchunk, R,
+                                                    (T*)xbuf);
+}
+
+template <typename T, int KM>
+void combine_t(const void* ybuf, int S, int M, int k, int64_t Cbuf, const Routing& R, void* y,
+               int grid, cudaStream_t st) {
+  combine_kernel<T, KM><<<grid, kThreads, 0, st>>>((const T*)ybuf, S, M, k, Cbuf, R, (T*)y);
+}
+
+template <typename T>
+void dispatch_k(int k, const void* x, int S, int M, int E, int C, int64_t Cbuf, int nchunk,
+                const Routing& R, void* xbuf, int grid, cudaStream_t st) {
+  if (k <= 1) dispatch_t<T, 1>(x, S, M, E, k, C, Cbuf, nchunk, R, xbuf, grid, st);
+  else if (k <= 2) dispatch_t<T, 2>(x, S, M, E, k, C, Cbuf, nchunk, R, xbuf, grid, st);
+  else if (k <= 4) dispatch_t<T, 4>(x, S, M, E, k, C, Cbuf, nchunk, R, xbuf, grid, st);
+  else dispatch_t<T, 8>(x, S, M, E, k, C, Cbuf, nchunk, R, xbuf, grid, st);
+}
+
+template <typename T>
+void combine_k(int k, const void* ybuf, int S, int M, int64_t Cbuf, const Routing& R, void* y,
+               int grid, cudaStream_t st) {
+  if (k <= 1) combine_t<T, 1>(ybuf, S, M, k, Cbuf, R, y, grid, st);
+  else if (k <= 2) combine_t<T, 2>(ybuf, S, M, k, Cbuf, R, y, grid, st);
+  else if (k <= 4) combine_t<T, 4>(ybuf, S, M, k, Cbuf, R, y, grid, st);
+  else combine_t<T, 8>(ybuf, S, M, k, Cbuf, R, y, grid, st);
 }
 
 }  // namespace
@@ -167,11 +211,9 @@ cudaError_t launch_dispatch(const void* x, bool bf16, int S, int M, int E, int k
   const int nchunk = (S + kChunk - 1) / kChunk;
   const int grid = grid_for(S);
   if (bf16)
-    dispatch_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(
-        (const __nv_bfloat16*)x, S, M, E, k, C, Cbuf, nchunk, R, (__nv_bfloat16*)xbuf);
+    dispatch_k<__nv_bfloat16>(k, x, S, M, E, C, Cbuf, nchunk, R, xbuf, grid, st);
   else
-    dispatch_kernel<float><<<grid, kThreads, 0, st>>>((const float*)x, S, M, E, k, C, Cbuf, nchunk,
-                                                      R, (float*)xbuf);
+    dispatch_k<float>(k, x, S, M, E, C, Cbuf, nchunk, R, xbuf, grid, st);
   return cudaGetLastError();
 }
 
@@ -179,11 +221,9 @@ cudaError_t launch_combine(const void* ybuf, bool bf16, int S, int M, int k, int
                            const Routing& R, void* y, cudaStream_t st) {
   const int grid = grid_for(S);
   if (bf16)
-    combine_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>((const __nv_bfloat16*)ybuf, S, M, k,
-                                                             Cbuf, R, (__nv_bfloat16*)y);
+    combine_k<__nv_bfloat16>(k, ybuf, S, M, Cbuf, R, y, grid, st);
   else
-    combine_kernel<float><<<grid, kThreads, 0, st>>>((const float*)ybuf, S, M, k, Cbuf, R,
-                                                     (float*)y);
+    combine_k<float>(k, ybuf, S, M, Cbuf, R, y, grid, st);
   return cudaGetLastError();
 }
 

@@ -37,7 +37,7 @@ cudaError_t launch_route_logits(const float* logits, int S, int E, int k, const 
 int router_tc_pad(int E);
 cudaError_t split_gate_weights(const float* Wg, int M, int E, void* out3, cudaStream_t st);
 bool make_router_wmap(CUtensorMap* tm, const void* wsplit, int M, int E);
-bool make_router_xmap(CUtensorMap* tm, const void* x, int S, int M);
+bool make_router_xmap(CUtensorMap* tm, const void* x, int S, int M, int E);
 cudaError_t launch_router_tc(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias, int S,
                              int M, int E, int k, const Routing& R, uint64_t limit_ns, cudaStream_t st);
 // scan.cu

@@ -265,7 +265,7 @@ moe_status moe_forward(moe_handle h, int64_t S, const void* x, void* y, void* st
   MOE_TRY(mark(0));
   if (bf16) {
     if (h->xmap_ptr != x || h->xmap_S != S) {
-      if (!make_router_xmap(&h->xmap, x, iS, iM)) return MOE_ERR_CUDA;
+      if (!make_router_xmap(&h->xmap, x, iS, iM, h->E)) return MOE_ERR_CUDA;
       h->xmap_ptr = x;
       h->xmap_S = S;
     }

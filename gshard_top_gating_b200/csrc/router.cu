@@ -17,6 +17,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "route_token.cuh"
 
 namespace moe {
 
@@ -40,15 +41,14 @@ struct __align__(16) GemmSmem {
 
 // Route the 8 tokens of this warp whose logits are in acc[t][i] (expert lane+32i).
 template <int RE>
-__device__ __forceinline__ void route_warp(float (&acc)[8][RE], int tok0, int chunk, int S,
-                                           int E, int k, const float* __restrict__ bias,
-                                           bool write_logits, const Routing& R, EpiSmem& es) {
+__device__ __forceinline__ void route_warp(float (&acc)[8][RE], int tok0, int S, int E, int k,
+                                           const float* __restrict__ bias, bool write_logits,
+                                           const Routing& R, EpiSmem& es) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float psum[RE];
 #pragma unroll
   for (int i = 0; i < RE; ++i) psum[i] = 0.f;
   float lse2 = 0.f;
-
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
     const int tl = warp * 8 + t;
@@ -58,88 +58,9 @@ __device__ __forceinline__ void route_warp(float (&acc)[8][RE], int tok0, int ch
 #pragma unroll
     for (int i = 0; i < RE; ++i) {
       const int j = lane + 32 * i;
-      float a = acc[t][i];
-      if (j < E) {
-        if (bias) a += __ldg(bias + j);
-        if (write_logits) R.logits[(int64_t)tok * E + j] = a;
-      } else {
-        a = -INFINITY;
-      }
-      v[i] = a;
+      v[i] = (j < E) ? acc[t][i] + (bias ? __ldg(bias + j) : 0.f) : -INFINITY;
     }
-    // softmax statistics
-    float mx = v[0];
-#pragma unroll
-    for (int i = 1; i < RE; ++i) mx = fmaxf(mx, v[i]);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float ex[RE], s = 0.f;
-#pragma unroll
-    for (int i = 0; i < RE; ++i) {
-      ex[i] = (lane + 32 * i < E) ? expf(v[i] - mx) : 0.f;
-      s += ex[i];
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    const float inv = 1.f / s;
-#pragma unroll
-    for (int i = 0; i < RE; ++i) psum[i] += ex[i] * inv;
-    const float lse = mx + logf(s);
-    lse2 += lse * lse;
-
-    // top-k on the logits, ties -> lower expert index
-    unsigned taken = 0;
-    int er[kMaxK];
-    float lr[kMaxK];
-#pragma unroll
-    for (int r = 0; r < kMaxK; ++r) {
-      er[r] = 0;
-      lr[r] = 0.f;
-      if (r < k) {
-        float bv = -INFINITY;
-        int bj = 0x7fffffff;
-#pragma unroll
-        for (int i = 0; i < RE; ++i) {
-          const int j = lane + 32 * i;
-          if (j < E && !((taken >> i) & 1u) && (v[i] > bv || bj == 0x7fffffff)) {
-            bv = v[i];
-            bj = j;
-          }
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-          const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-          if (ov > bv || (ov == bv && oj < bj)) {
-            bv = ov;
-            bj = oj;
-          }
-        }
-        if (bj >= E) {                  // only for non-finite logits
-          if (lane == 0) atomicOr(R.err, DEVERR_BOUNDS);
-          bj = 0;
-        }
-        if ((bj & 31) == lane) taken |= 1u << (bj >> 5);
-        er[r] = bj;
-        lr[r] = bv;
-      }
-    }
-    // normalised gates g_r = exp(l_r - l_0) / sum_r' exp(l_r' - l_0)
-    float gs = 0.f, gr[kMaxK];
-#pragma unroll
-    for (int r = 0; r < kMaxK; ++r) {
-      gr[r] = (r < k) ? expf(lr[r] - lr[0]) : 0.f;
-      gs += gr[r];
-    }
-    const float ginv = 1.f / gs;
-#pragma unroll
-    for (int r = 0; r < kMaxK; ++r) {
-      if (r < k && lane == r) {
-        R.eidx[(int64_t)tok * k + r] = er[r];
-        R.gate[(int64_t)tok * k + r] = gr[r] * ginv;
-      }
-      if (r < k && lane == 0) es.sel[tl][r] = er[r];
-    }
+    route_token<RE>(v, tok, E, k, write_logits, R, psum, lse2, es.sel[tl]);
   }
 #pragma unroll
   for (int i = 0; i < RE; ++i) es.red[warp][lane + 32 * i] = psum[i];
@@ -251,7 +172,7 @@ __global__ void __launch_bounds__(kThreads) router_kernel(const TX* __restrict__
       }
     }
   }
-  route_warp<RE>(acc, tok0, chunk, S, E, k, bias, true, R, es);
+  route_warp<RE>(acc, tok0, S, E, k, bias, true, R, es);
   chunk_tables<RE>(tok0, chunk, nchunk, S, E, k, R, es);
 }
 
@@ -275,7 +196,7 @@ __global__ void __launch_bounds__(kThreads) route_logits_kernel(const float* __r
     }
   }
   __syncthreads();
-  route_warp<RE>(acc, tok0, chunk, S, E, k, nullptr, true, R, es);
+  route_warp<RE>(acc, tok0, S, E, k, nullptr, true, R, es);
   chunk_tables<RE>(tok0, chunk, nchunk, S, E, k, R, es);
 }
 

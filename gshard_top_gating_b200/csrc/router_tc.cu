@@ -18,42 +18,53 @@
 // it into a second TMEM region with ordinary round-to-nearest fp32 adds.  The
 // logits so carry fp32-level error at tensor-core speed.
 //
-// One CTA = 128 tokens x EP experts (E padded to 32/64/128/256), 192 threads:
+// One CTA = 128 tokens x EP experts (E padded to 32/64/128/256), 256 threads:
 // warp 0 TMA producer (x tile 128x64 + three W_g parts EPx64 per stage, K-major,
-// 128B swizzle), warp 1 TMEM owner and single-thread MMA issuer, warps 2-5 the
-// epilogue with one token row per thread.  The epilogue reads the accumulator
-// three times (max and top-k; sum of exponentials; probabilities), keeps the
-// top-k in registers with ties to the lower expert index, and writes the same
-// per-64-token chunk tables (probability sums, lse^2 sums, rank-r histograms,
-// local ranks) as the CUDA-core router.
+// 128B swizzle), warp 1 TMEM owner and single-thread MMA issuer, warps 2-5 fold
+// the K-segments (one token row per thread, as TMEM lanes dictate) and leave the
+// final logits tile in shared memory.  Then all eight warps route warp-per-token
+// (lanes over experts, shuffle max / sum / argmax, ties to the lower index) and
+// write the same per-64-token chunk tables (probability sums, lse^2 sums,
+// rank-r histograms, local ranks) as the CUDA-core router.
 #include <cudaTypedefs.h>
 #include <math.h>
 
 #include "common.cuh"
 #include "internal.h"
+#include "route_token.cuh"
 
 namespace moe {
 
 namespace {
 
 constexpr int BM = 128, BK = 64;
-constexpr int kThreads = 192;
+constexpr int kThreads = 512;   // 16 warps: all route; warps 0/1/2-5 also load / issue / fold
 constexpr uint32_t A_BYTES = BM * BK * 2;
+constexpr int kPrefetchX = 12;     // L2 prefetch distance of the token tiles, k-blocks
 constexpr int kSegBlocks = 8;      // k-blocks (of 64) accumulated before each fp32 round-to-nearest add
 
 template <int EP>
 struct RCfg {
-  static constexpr uint32_t PART_BYTES = EP * BK * 2;            // one W_g part, EP x 64 bf16
+  // tokens per CTA: 64 for small E (twice the CTAs stream x; the MMA keeps M=128
+  // and its upper 64 accumulator rows are ignored), 128 otherwise
+  static constexpr int TT = EP <= 64 ? 64 : 128;
+  static constexpr int NCH = TT / kChunk;                       // 64-token chunks per CTA
+  static constexpr uint32_t X_BYTES = TT * BK * 2;              // bytes TMA writes into the A tile
+  static constexpr uint32_t PART_BYTES = EP * BK * 2;           // one W_g part, EP x 64 bf16
   static constexpr uint32_t STAGE_BYTES = A_BYTES + 3 * PART_BYTES;
+  static constexpr uint32_t TX_BYTES = X_BYTES + 3 * PART_BYTES;
   static constexpr int STAGES = (EP == 256) ? 2 : (EP == 128 ? 3 : (EP == 64 ? 5 : 7));
   static constexpr uint32_t TMEM_COLS = 2 * EP;        // accumulator + running sum
-  // epilogue scratch reuses the stage buffers: P [128][EP] f32, sel [128][8] i32,
-  // lse2 [128] f32, hist [2][8][EP] i32
-  static constexpr uint32_t P_OFF = 0;
-  static constexpr uint32_t SEL_OFF = P_OFF + 128 * EP * 4;
-  static constexpr uint32_t L_OFF = SEL_OFF + 128 * kMaxK * 4;
-  static constexpr uint32_t H_OFF = L_OFF + 128 * 4;
-  static constexpr uint32_t EPI_END = H_OFF + 2 * kMaxK * EP * 4;
+  // epilogue scratch reuses the stage buffers: logits L [TT][EP+1] f32 (padded row),
+  // per-warp probability sums red [16][EP] f32, per-warp lse^2 [16], sel [TT][8] i32,
+  // hist [NCH][8][EP] i32
+  static constexpr uint32_t LD = EP + 1;
+  static constexpr uint32_t L_OFF = 0;
+  static constexpr uint32_t RED_OFF = L_OFF + TT * LD * 4;
+  static constexpr uint32_t LSE_OFF = RED_OFF + 16 * EP * 4;
+  static constexpr uint32_t SEL_OFF = LSE_OFF + 16 * 4;
+  static constexpr uint32_t H_OFF = SEL_OFF + TT * kMaxK * 4;
+  static constexpr uint32_t EPI_END = H_OFF + NCH * kMaxK * EP * 4;
   static_assert(EPI_END <= STAGES * STAGE_BYTES, "epilogue scratch must fit in the stage buffers");
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + 16;
 };
@@ -67,10 +78,6 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
 template <int EP>
 __device__ __forceinline__ uint32_t idesc_router() {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(EP >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-}
-
-__device__ __forceinline__ void named_sync_epi() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
 template <int EP>
@@ -93,7 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::STAGES * C::STAGE_BYTES + 260);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x, tok0 = tile * BM;
+  const int tile = blockIdx.x, tok0 = tile * C::TT;
   const int KB = M / BK;
 
   if (warp == 0 && lane == 0) {
@@ -103,7 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(tfull_bar, 1);
     mbar_init(done_bar, 1);
-    mbar_init(tempty_bar, 128);
+    mbar_init(tempty_bar, C::TT);            // one arrival per token row
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     tma_prefetch_desc(&tmX);
@@ -123,14 +130,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_par = 0;
       bool ok = true;
+      // x streams from DRAM once: prefetch it into L2 kPrefetchX k-blocks ahead
+      for (int kb = 0; kb < KB && kb < kPrefetchX; ++kb) tma_prefetch_l2_2d(&tmX, kb * BK, tok0);
       for (int kb = 0; kb < KB; ++kb) {
+        if (kb + kPrefetchX < KB) tma_prefetch_l2_2d(&tmX, (kb + kPrefetchX) * BK, tok0);
         if (*abort_flag || !mbar_wait(empty_bar(s), ph ^ 1u, R.err, limit_ns)) {
           *abort_flag = 1;
           ok = false;
           break;
         }
         const uint32_t sa = base + s * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(full_bar(s), C::STAGE_BYTES);
+        mbar_arrive_expect_tx(full_bar(s), C::TX_BYTES);
         tma_load_2d(sa, &tmX, full_bar(s), kb * BK, tok0);
 #pragma unroll
         for (int part = 0; part < 3; ++part)
@@ -193,19 +203,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------ epilogue: one token per thread
+  } else if (warp < 6 && (warp & 3) < C::TT / 32) {
+    // ------------------------------------------------------------ fold K-segments (warps 2-5)
     const int q = warp & 3;
     const int row = q * 32 + lane;              // token row within the tile (= TMEM lane)
-    const int et = threadIdx.x - 64;            // 0..127 epilogue thread index
-    const int tok = tok0 + row;
-    const bool live = tok < S;
-    float* Ps = reinterpret_cast<float*>(gbase + C::P_OFF);
-    int32_t* sel = reinterpret_cast<int32_t*>(gbase + C::SEL_OFF);
-    float* Ls = reinterpret_cast<float*>(gbase + C::L_OFF);
-    int32_t* Hs = reinterpret_cast<int32_t*>(gbase + C::H_OFF);
     const uint32_t tlane = tmem_base + ((uint32_t)(q * 32) << 16);
-    // fold the K-segments: sum (columns EP..2EP) += segment accumulator (columns 0..EP)
+    float* Ls = reinterpret_cast<float*>(gbase + C::L_OFF);
     const int nseg = (KB + kSegBlocks - 1) / kSegBlocks;
     bool ok = true;
     for (int seg = 0; seg < nseg; ++seg) {
@@ -215,156 +218,101 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      if (nseg > 1) {
+      const bool last = seg == nseg - 1;
 #pragma unroll 1
-        for (int c = 0; c < EP / 32; ++c) {
-          uint32_t a[32], b[32];
-          tmem_ld_32x32b_x32(tlane + c * 32, a);
-          if (seg > 0) tmem_ld_32x32b_x32(tlane + EP + c * 32, b);
-          tmem_ld_wait();
-          if (seg > 0) {
+      for (int c = 0; c < EP / 32; ++c) {
+        uint32_t a[32], b[32];
+        tmem_ld_32x32b_x32(tlane + c * 32, a);
+        if (seg > 0) tmem_ld_32x32b_x32(tlane + EP + c * 32, b);
+        tmem_ld_wait();
+        if (seg > 0) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) + __uint_as_float(b[i]));
+          for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) + __uint_as_float(b[i]));
+        }
+        if (last) {          // final logits (+ bias) into the shared tile
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int j = c * 32 + i;
+            Ls[row * C::LD + j] = __uint_as_float(a[i]) + ((bias && j < E) ? __ldg(bias + j) : 0.f);
           }
+        } else {
           tmem_st_32x32b_x32(tlane + EP + c * 32, a);
         }
-        tmem_st_wait();
       }
+      if (!last) tmem_st_wait();
       tc_fence_before();
       mbar_arrive(tempty_bar);
     }
-    tc_fence_after();
-    const uint32_t taddr = tlane + (nseg > 1 ? EP : 0);    // final logits (before bias)
+    if (!ok)
+      for (int c = 0; c < EP; ++c) Ls[row * C::LD + c] = 0.f;
+  }
 
-    float bv[kMaxK];
-    int bj[kMaxK];
+  // ------------------------------------------------------------ route, all 8 warps
+  __syncthreads();
+  {
+    float* Ls = reinterpret_cast<float*>(gbase + C::L_OFF);
+    float* red = reinterpret_cast<float*>(gbase + C::RED_OFF);
+    float* lse_w = reinterpret_cast<float*>(gbase + C::LSE_OFF);
+    int32_t* sel = reinterpret_cast<int32_t*>(gbase + C::SEL_OFF);
+    int32_t* Hs = reinterpret_cast<int32_t*>(gbase + C::H_OFF);
+    constexpr int RE = EP / 32;
+    constexpr int TPW = C::TT / 16;                         // tokens per warp (4 or 8)
+    constexpr int WPC = 16 / C::NCH;                        // warps per 64-token chunk
+    const int tid = threadIdx.x;
+    const bool good = !*abort_flag;
+    float psum[RE];
 #pragma unroll
-    for (int r = 0; r < kMaxK; ++r) {
-      bv[r] = -INFINITY;
-      bj[r] = 0x7fffffff;
-    }
-    float mx = -INFINITY;
-    // pass A: logits out, max, top-k (insertion in ascending expert order keeps ties stable)
-#pragma unroll 1
-    for (int c = 0; c < EP / 32; ++c) {
-      uint32_t u[32];
-      tmem_ld_32x32b_x32(taddr + c * 32, u);
-      tmem_ld_wait();
-      if (ok && live) {
+    for (int i = 0; i < RE; ++i) psum[i] = 0.f;
+    float lse2 = 0.f;
+    const int ntile = good ? min(C::TT, S - tok0) : 0;
+    for (int t = warp * TPW; t < warp * TPW + TPW && t < ntile; t += 2) {   // two tokens in flight
+      if (t + 1 < ntile) {
+        float v[2][RE];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int j = c * 32 + i;
-          if (j < E) {
-            float v = __uint_as_float(u[i]);
-            if (bias) v += __ldg(bias + j);
-            R.logits[(int64_t)tok * E + j] = v;
-            mx = fmaxf(mx, v);
-            if (v > bv[kMaxK - 1]) {
-              bv[kMaxK - 1] = v;
-              bj[kMaxK - 1] = j;
+        for (int n = 0; n < 2; ++n)
 #pragma unroll
-              for (int r = kMaxK - 1; r > 0; --r) {
-                if (bv[r] > bv[r - 1]) {
-                  const float tv = bv[r];
-                  bv[r] = bv[r - 1];
-                  bv[r - 1] = tv;
-                  const int tj = bj[r];
-                  bj[r] = bj[r - 1];
-                  bj[r - 1] = tj;
-                }
-              }
-            }
+          for (int i = 0; i < RE; ++i) {
+            const int j = lane + 32 * i;
+            v[n][i] = j < E ? Ls[(t + n) * C::LD + j] : -INFINITY;
           }
+        const int64_t tk[2] = {tok0 + t, tok0 + t + 1};
+        int32_t* const rows[2] = {sel + t * kMaxK, sel + (t + 1) * kMaxK};
+        route_tokens<RE, 2>(v, tk, E, k, true, R, psum, lse2, rows);
+      } else {
+        float v[RE];
+#pragma unroll
+        for (int i = 0; i < RE; ++i) {
+          const int j = lane + 32 * i;
+          v[i] = j < E ? Ls[t * C::LD + j] : -INFINITY;
         }
+        route_token<RE>(v, tok0 + t, E, k, true, R, psum, lse2, sel + t * kMaxK);
       }
     }
-    // pass B: sum of exponentials
-    float s = 0.f;
-#pragma unroll 1
-    for (int c = 0; c < EP / 32; ++c) {
-      uint32_t u[32];
-      tmem_ld_32x32b_x32(taddr + c * 32, u);
-      tmem_ld_wait();
-      if (ok && live) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int j = c * 32 + i;
-          if (j < E) {
-            float v = __uint_as_float(u[i]);
-            if (bias) v += __ldg(bias + j);
-            s += expf(v - mx);
-          }
-        }
-      }
-    }
-    const float inv = (ok && live) ? 1.f / s : 0.f;
-    // pass C: probabilities into smem for the per-chunk column sums
-#pragma unroll 1
-    for (int c = 0; c < EP / 32; ++c) {
-      uint32_t u[32];
-      tmem_ld_32x32b_x32(taddr + c * 32, u);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int j = c * 32 + i;
-        float p = 0.f;
-        if (ok && live && j < E) {
-          float v = __uint_as_float(u[i]);
-          if (bias) v += __ldg(bias + j);
-          p = expf(v - mx) * inv;
-        }
-        Ps[row * EP + ((j + row) & (EP - 1))] = p;     // rotated columns: no bank conflicts
-      }
-    }
-    if (ok && live) {
-      const float lse = mx + logf(s);
-      Ls[row] = lse * lse;
-      float gs = 0.f, gr[kMaxK];
-#pragma unroll
-      for (int r = 0; r < kMaxK; ++r) {
-        gr[r] = (r < k) ? expf(bv[r] - bv[0]) : 0.f;
-        gs += gr[r];
-      }
-      const float ginv = 1.f / gs;
-#pragma unroll
-      for (int r = 0; r < kMaxK; ++r) {
-        if (r < k) {
-          int j = bj[r];
-          if (j >= E) {                        // only for non-finite logits
-            atomicOr(R.err, DEVERR_BOUNDS);
-            j = 0;
-          }
-          R.eidx[(int64_t)tok * k + r] = j;
-          R.gate[(int64_t)tok * k + r] = gr[r] * ginv;
-          sel[row * kMaxK + r] = j;
-        }
-      }
-    } else {
-      Ls[row] = 0.f;
-    }
-    for (int i = et; i < 2 * kMaxK * EP; i += 128) Hs[i] = 0;
-    tc_fence_before();
-    named_sync_epi();
-
-    // per-chunk column sums of p (two 64-token chunks per tile), fixed order
-    const int chunk0 = tile * 2;
-    for (int cc = 0; cc < 2; ++cc) {
+    for (int i = 0; i < RE; ++i) red[warp * EP + lane + 32 * i] = psum[i];
+    if (lane == 0) lse_w[warp] = lse2;
+    for (int i = tid; i < C::NCH * kMaxK * EP; i += kThreads) Hs[i] = 0;
+    __syncthreads();
+    // per-chunk probability and lse^2 sums, warps of a chunk added in order
+    const int chunk0 = tile * C::NCH;
+    for (int cc = 0; cc < C::NCH; ++cc) {
       const int chunk = chunk0 + cc;
       if (chunk >= nchunk) break;
-      for (int j = et; j < E; j += 128) {
+      for (int j = tid; j < E; j += kThreads) {
         float acc = 0.f;
-        for (int rr = cc * 64; rr < cc * 64 + 64; ++rr) acc += Ps[rr * EP + ((j + rr) & (EP - 1))];
+#pragma unroll
+        for (int w = 0; w < WPC; ++w) acc += red[(cc * WPC + w) * EP + j];
         R.psum[(int64_t)chunk * E + j] = acc;
       }
-      if (et == 0) {
+      if (tid == 0) {
         float acc = 0.f;
-        for (int rr = cc * 64; rr < cc * 64 + 64; ++rr) acc += Ls[rr];
+#pragma unroll
+        for (int w = 0; w < WPC; ++w) acc += lse_w[cc * WPC + w];
         R.lse2[chunk] = acc;
       }
     }
     // local ranks within each 64-token chunk and rank-r histograms
-    const int ntile = min(BM, S - tok0);
-    for (int idx = et; idx < ntile * k; idx += 128) {
+    for (int idx = tid; idx < ntile * k; idx += kThreads) {
       const int t = idx / k, r = idx - t * k;
       const int e = sel[t * kMaxK + r];
       const int cbeg = (t >> 6) << 6;
@@ -373,11 +321,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       R.lrank[(int64_t)(tok0 + t) * k + r] = c;
       atomicAdd(&Hs[((t >> 6) * kMaxK + r) * EP + e], 1);
     }
-    named_sync_epi();
-    for (int cc = 0; cc < 2; ++cc) {
+    __syncthreads();
+    for (int cc = 0; cc < C::NCH; ++cc) {
       const int chunk = chunk0 + cc;
       if (chunk >= nchunk) break;
-      for (int idx = et; idx < k * E; idx += 128) {
+      for (int idx = tid; idx < k * E; idx += kThreads) {
         const int r = idx / E, e = idx - r * E;
         R.hist[((int64_t)r * nchunk + chunk) * E + e] = Hs[(cc * kMaxK + r) * EP + e];
       }
@@ -444,8 +392,8 @@ cudaError_t launch_t(const CUtensorMap& tmX, const CUtensorMap& tmW, const float
                                        (int)RCfg<EP>::SMEM);
   if (e != cudaSuccess) return e;
   const int nchunk = (S + kChunk - 1) / kChunk;
-  kern<<<(S + BM - 1) / BM, kThreads, RCfg<EP>::SMEM, st>>>(tmX, tmW, bias, S, M, E, k, nchunk, R,
-                                                            limit_ns);
+  kern<<<(S + RCfg<EP>::TT - 1) / RCfg<EP>::TT, kThreads, RCfg<EP>::SMEM, st>>>(
+      tmX, tmW, bias, S, M, E, k, nchunk, R, limit_ns);
   return cudaGetLastError();
 }
 
@@ -466,8 +414,9 @@ bool make_router_wmap(CUtensorMap* tm, const void* wsplit, int M, int E) {
   return encode_kmajor(tm, wsplit, (uint64_t)M, (uint64_t)3 * EP, (uint32_t)EP);
 }
 
-bool make_router_xmap(CUtensorMap* tm, const void* x, int S, int M) {
-  return encode_kmajor(tm, x, (uint64_t)M, (uint64_t)S, (uint32_t)BM);
+bool make_router_xmap(CUtensorMap* tm, const void* x, int S, int M, int E) {
+  const int TT = router_tc_pad(E) <= 64 ? 64 : 128;      // = RCfg<EP>::TT
+  return encode_kmajor(tm, x, (uint64_t)M, (uint64_t)S, (uint32_t)TT);
 }
 
 cudaError_t launch_router_tc(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias, int S,
