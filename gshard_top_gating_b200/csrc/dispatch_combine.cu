@@ -31,13 +31,19 @@ __global__ void __launch_bounds__(kThreads, 4) dispatch_kernel(const T* __restri
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * kThreads) >> 5;
   const int nv = (int)((int64_t)M * sizeof(T) / 16);
+  pdl_trigger();
+  bool waited = false;
   for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < S; t += warps) {
     const uint4* src = x ? reinterpret_cast<const uint4*>(x + (int64_t)t * M) : nullptr;
     uint4 first[kUnroll];
-    if (src) {
+    if (src) {                                 // x is an input: no need to wait for it
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u)
         if (lane + 32 * u < nv) first[u] = ld_nc_v4(src + lane + 32 * u);
+    }
+    if (!waited) {
+      pdl_wait();                              // routing tables and offsets complete
+      waited = true;
     }
     int e = 0, s = -1;
     if (lane < k) {
@@ -120,6 +126,8 @@ __global__ void __launch_bounds__(kThreads, KM >= 8 ? 3 : 4) combine_kernel(cons
   const int warps = (gridDim.x * kThreads) >> 5;
   const int nv = (int)((int64_t)M * sizeof(T) / 16);
   constexpr int U = KM >= 4 ? 1 : 2;          // 16-byte vectors per lane per step
+  pdl_trigger();
+  pdl_wait();                                  // expert outputs complete
   for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < S; t += warps) {
     int e = 0, s = -1;
     float g = 0.f;
@@ -176,14 +184,15 @@ int grid_for(int S) {
 template <typename T, int KM>
 void dispatch_t(const void* x, int S, int M, int E, int k, int C, int64_t Cbuf, int nchunk,
                 const Routing& R, void* xbuf, int grid, cudaStream_t st) {
-  dispatch_kernel<T, KM><<<grid, kThreads, 0, st>>>((const T*)x, S, M, E, k, C, Cbuf, nchunk, R,
-                                                    (T*)xbuf);
+  launch_pdl(dispatch_kernel<T, KM>, dim3(grid), dim3(kThreads), 0, st, (const T*)x, S, M, E, k, C,
+             Cbuf, nchunk, R, (T*)xbuf);
 }
 
 template <typename T, int KM>
 void combine_t(const void* ybuf, int S, int M, int k, int64_t Cbuf, const Routing& R, void* y,
                int grid, cudaStream_t st) {
-  combine_kernel<T, KM><<<grid, kThreads, 0, st>>>((const T*)ybuf, S, M, k, Cbuf, R, (T*)y);
+  launch_pdl(combine_kernel<T, KM>, dim3(grid), dim3(kThreads), 0, st, (const T*)ybuf, S, M, k, Cbuf,
+             R, (T*)y);
 }
 
 template <typename T>

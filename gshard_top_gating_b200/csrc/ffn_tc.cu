@@ -39,8 +39,10 @@ struct Cfg {
   static constexpr uint32_t B_BYTES = BK * BN * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
-  // 1 KB alignment slack + stages + 512 B of barriers + misc words and the tile tables
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 512 + 16 + 4 * (3 * kMaxExperts + 1);
+  static constexpr uint32_t STAGING = 4 * 4096;   // one 32 x 64 bf16 store tile per epilogue warp
+  // 1 KB alignment slack + stages + staging + 512 B of barriers + misc words and the tile tables
+  static constexpr size_t SMEM =
+      1024 + (size_t)STAGES * STAGE_BYTES + STAGING + 512 + 16 + 4 * (3 * kMaxExperts + 1);
 };
 
 // Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: version 1 at bit 46,
@@ -74,24 +76,69 @@ struct TileIter {
   }
 };
 
+// Epilogue of one warp's 32 accumulator rows x BN columns: TMEM -> bf16 (+ReLU) ->
+// a 4 KB staging tile in shared memory laid out as the store tensor map's 128-byte
+// swizzle (row r, 16-byte chunk c at r*128 + ((c ^ (r % 8)) * 16)) -> one TMA store per
+// 64 columns.  Rows past n_e land in the expert's own padding rows (rows per expert
+// are a multiple of 128), which nothing reads.  The TMA engine writes whole 128-byte
+// rows, instead of each thread storing 16 bytes to 32 different rows per instruction.
+template <int BN, bool RELU>
+__device__ __forceinline__ void store_rows(const CUtensorMap* tmD, uint32_t tmem_rows,
+                                           uint32_t stage, int row0, int col0, int lane) {
+#pragma unroll 1
+  for (int b = 0; b < BN / 64; ++b) {
+    if (lane == 0) bulk_wait_read0();          // the previous store has read the staging tile
+    __syncwarp();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(tmem_rows + b * 64 + h * 32, r);
+      tmem_ld_wait();
+      uint32_t pk[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        float a = __uint_as_float(r[2 * j]), c = __uint_as_float(r[2 * j + 1]);
+        if (RELU) {
+          a = fmaxf(a, 0.f);
+          c = fmaxf(c, 0.f);
+        }
+        pk[j] = pack_bf16x2(a, c);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t cc = h * 4 + j;
+        st_shared_v4(stage + lane * 128 + ((cc ^ (lane & 7)) << 4), pk[4 * j], pk[4 * j + 1],
+                     pk[4 * j + 2], pk[4 * j + 3]);
+      }
+    }
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmD, stage, col0 + b * 64, row0);
+      bulk_commit();
+    }
+  }
+}
+
 template <int BN, bool RELU>
 __global__ void __launch_bounds__(kThreads, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                  __nv_bfloat16* __restrict__ D, const int32_t* __restrict__ nexp, int E,
+                  const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
                   int64_t Cbuf, int K, int N, unsigned* err, uint64_t limit_ns) {
   using C = Cfg<BN>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t base = (raw_base + 1023u) & ~1023u;                 // 1024-aligned for swizzle
   unsigned char* gbase = smem_raw + (base - raw_base);
-  const uint32_t bar0 = base + C::STAGES * C::STAGE_BYTES;
+  const uint32_t staging0 = base + C::STAGES * C::STAGE_BYTES;        // 4 x 4 KB store tiles
+  const uint32_t bar0 = staging0 + C::STAGING;
   // barriers: full[S], empty[S], tfull[2], tempty[2], done
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
   auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 2 + a); };
   const uint32_t done_bar = bar0 + 8u * (2 * C::STAGES + 4);
-  unsigned char* misc = gbase + C::STAGES * C::STAGE_BYTES + 512;
+  unsigned char* misc = gbase + C::STAGES * C::STAGE_BYTES + C::STAGING + 512;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   int* tile_pre = reinterpret_cast<int*>(misc + 16);                 // [E+1]
@@ -121,6 +168,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32((const void*)tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_trigger();
+  pdl_wait();                          // the producing kernel's rows and counts are complete
   if (warp == 2) {
     // tile prefix over experts (warp-parallel scan, ceil(E/32) experts per lane)
     const int per = (E + 31) / 32;
@@ -239,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;                     // TMEM lane quarter this warp may access
-    const int row = q * 32 + lane;
+    const uint32_t stage = staging0 + (warp - 2) * 4096u;
     TileIter it{tile_pre, mtiles, E, NT, 0};
     int e, mt, nt, i = 0;
     for (int tile = blockIdx.x; it.decode(tile, e, mt, nt); tile += gridDim.x, ++i) {
@@ -250,33 +299,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int grow = mt * BM + row;
-      const bool valid = grow < nrows[e];
-      __nv_bfloat16* dst = D + ((int64_t)e * Cbuf + grow) * N + (int64_t)nt * BN;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c * 32, r);
-        tmem_ld_wait();
-        if (valid) {
-          uint32_t p[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float a = __uint_as_float(r[2 * j]), b = __uint_as_float(r[2 * j + 1]);
-            if (RELU) {
-              a = fmaxf(a, 0.f);
-              b = fmaxf(b, 0.f);
-            }
-            p[j] = pack_bf16x2(a, b);
-          }
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) d4[j] = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
-        }
-      }
+      const int row0 = (int)(e * Cbuf + mt * BM + q * 32);
+      store_rows<BN, RELU>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
+                           nt * BN, lane);
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
     }
+    if (lane == 0) bulk_wait0();                // stores complete before the CTA exits
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -284,6 +314,226 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- CTA-pair variant
+//
+// Two CTAs of a cluster compute one 256 x 256 tile with cta_group::2 MMAs: CTA r
+// holds rows [128r, 128r+128) of the A tile and columns [128r, 128r+128) of the
+// B tile, so each SM loads 32 KB per k-block for the same MMA work that takes
+// 48 KB in the one-CTA kernel (the loads, not the tensor cores, bound that one).
+// The leader (rank 0) issues the MMAs; its full barrier counts the TMA bytes of
+// both CTAs; its commits arrive on both CTAs' barriers; both CTAs' epilogues
+// release an accumulator by arriving on the leader's barrier.
+namespace pairk {
+constexpr int BN = 256;                                   // pair tile columns
+constexpr int PM = 256;                                   // pair tile rows
+constexpr uint32_t B_HALF_BYTES = BK * (BN / 2) * 2;      // 16 KB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_HALF_BYTES;  // 32 KB per CTA
+constexpr int STAGES = 6;
+constexpr uint32_t TMEM_COLS = 2 * BN;                    // double-buffered accumulator
+constexpr uint32_t STAGING = 4 * 4096;                   // one 32 x 64 bf16 store tile per epilogue warp
+constexpr size_t SMEM =
+    1024 + (size_t)STAGES * STAGE_BYTES + STAGING + 512 + 16 + 4 * (3 * kMaxExperts + 1);
+constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;            // shared::cluster address -> rank 0
+}  // namespace pairk
+
+template <bool RELU>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    ffn_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
+                   int64_t Cbuf, int K, int N, unsigned* err, uint64_t limit_ns) {
+  using namespace pairk;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;   // same offset in both CTAs
+  unsigned char* gbase = smem_raw + (base - raw_base);
+  const uint32_t staging0 = base + STAGES * STAGE_BYTES;             // 4 x 4 KB store tiles
+  const uint32_t bar0 = staging0 + STAGING;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
+  unsigned char* misc = gbase + STAGES * STAGE_BYTES + STAGING + 512;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  int* tile_pre = reinterpret_cast<int*>(misc + 16);
+  int* mtiles = tile_pre + (kMaxExperts + 1);
+  int* nrows = mtiles + kMaxExperts;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int NT = N / BN;
+  const int KB = K / BK;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 2 * 128);     // epilogue threads of both CTAs
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32((const void*)tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  pdl_trigger();
+  pdl_wait();                          // the producing kernel's rows and counts are complete
+  if (warp == 2) {
+    const int per = (E + 31) / 32;
+    const int e0 = lane * per;
+    int sum = 0;
+    for (int e = e0; e < min(E, e0 + per); ++e) {
+      const int n = nexp[e];
+      const int m = (n + PM - 1) / PM;
+      nrows[e] = n;
+      mtiles[e] = m;
+      sum += m * NT;
+    }
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    int run = inc - sum;
+    for (int e = e0; e < min(E, e0 + per); ++e) {
+      tile_pre[e] = run;
+      run += mtiles[e] * NT;
+    }
+    if (lane == 31) tile_pre[E] = inc;
+  }
+  tc_fence_before();
+  cluster_sync_all();          // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      TileIter it{tile_pre, mtiles, E, NT, 0};
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int e, mt, nt;
+      for (int tile = pair; ok && it.decode(tile, e, mt, nt); tile += npairs) {
+        const int rowA = (int)(e * Cbuf + mt * PM + rank * (PM / 2));
+        const int rowB = e * K;
+        const int colB = nt * BN + rank * (BN / 2);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (*abort_flag || !mbar_wait(empty_bar(s), ph ^ 1u, err, limit_ns)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const uint32_t sa = base + s * STAGE_BYTES;
+          const uint32_t fb = full_bar(s) & kPeerBitMask;     // the leader's full barrier
+          if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * STAGE_BYTES);
+          tma_load_2d_pair(sa, &tmA, fb, kb * BK, rowA);
+#pragma unroll
+          for (int j = 0; j < BN / 128; ++j)
+            tma_load_2d_pair(sa + A_BYTES + j * 8192u, &tmB, fb, colB + j * 64, rowB + kb * BK);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && leader) {
+      TileIter it{tile_pre, mtiles, E, NT, 0};
+      // kind::f16, D fp32, A bf16 K-major, B bf16 MN-major, M=256, N=256
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                             ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(PM >> 4) << 24);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int e, mt, nt, i = 0;
+      for (int tile = pair; ok && it.decode(tile, e, mt, nt); tile += npairs, ++i) {
+        const int acc = i & 1;
+        const uint32_t aph = (i >> 1) & 1;
+        if (*abort_flag || !mbar_wait(tempty_bar(acc), aph ^ 1u, err, limit_ns)) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (*abort_flag || !mbar_wait(full_bar(s), ph, err, limit_ns)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base + s * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = desc_sw128(sa + kk * 32u, 16u, 1024u);
+            const uint64_t bd = desc_sw128(sb + kk * 2048u, 8192u, 1024u);
+            tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          }
+          tc_commit_pair(empty_bar(s), 0x3);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (ok) tc_commit_pair(tfull_bar(acc), 0x3);
+      }
+      if (!ok) {
+        tc_commit_pair(done_bar, 0x1);
+        mbar_wait(done_bar, 0, err, limit_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5, both CTAs)
+    const int q = warp & 3;
+    const uint32_t stage = staging0 + (warp - 2) * 4096u;
+    TileIter it{tile_pre, mtiles, E, NT, 0};
+    int e, mt, nt, i = 0;
+    for (int tile = pair; it.decode(tile, e, mt, nt); tile += npairs, ++i) {
+      const int acc = i & 1;
+      const uint32_t aph = (i >> 1) & 1;
+      if (*abort_flag || !mbar_wait(tfull_bar(acc), aph, err, limit_ns)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int row0 = (int)(e * Cbuf + mt * PM + (int)rank * (PM / 2) + q * 32);
+      store_rows<BN, RELU>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
+                           nt * BN, lane);
+      tc_fence_before();
+      if (leader) mbar_arrive(tempty_bar(acc));
+      else mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+    }
+    if (lane == 0) bulk_wait0();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();          // no CTA leaves while its pair may still use its smem or TMEM
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -314,6 +564,17 @@ bool encode_2d(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer,
   return r == CUDA_SUCCESS;
 }
 
+template <bool RELU>
+cudaError_t launch_pair(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint64_t limit_ns,
+                        int num_sms, cudaStream_t st) {
+  auto kern = ffn_tc2_kernel<RELU>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)pairk::SMEM);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(num_sms & ~1), dim3(kThreads), pairk::SMEM, st, p.tmA, p.tmB, p.tmD,
+                    nexp, p.E, p.Cbuf, p.K, p.N, err, limit_ns);
+}
+
 template <int BN, bool RELU>
 cudaError_t launch_t(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint64_t limit_ns,
                      int num_sms, cudaStream_t st) {
@@ -321,9 +582,8 @@ cudaError_t launch_t(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint
   const size_t smem = Cfg<BN>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<num_sms, kThreads, smem, st>>>(p.tmA, p.tmB, (__nv_bfloat16*)p.D, nexp, p.E, p.Cbuf, p.K,
-                                        p.N, err, limit_ns);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(num_sms), dim3(kThreads), smem, st, p.tmA, p.tmB, p.tmD, nexp, p.E,
+                    p.Cbuf, p.K, p.N, err, limit_ns);
 }
 
 }  // namespace
@@ -337,14 +597,19 @@ bool make_gemm_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, i
   p.D = D;
   p.relu = relu;
   p.BN = (N % 256 == 0) ? 256 : (N % 128 == 0 ? 128 : 64);
+  p.pair = (N % pairk::BN) == 0;      // CTA-pair kernel whenever the 256-wide tile divides N
   if (K % BK || N % 64) return false;
   if (!encode_2d(&p.tmA, A, (uint64_t)K, (uint64_t)E * Cbuf, BK, BM)) return false;
   if (!encode_2d(&p.tmB, B, (uint64_t)N, (uint64_t)E * K, 64, BK)) return false;
+  if (!encode_2d(&p.tmD, D, (uint64_t)N, (uint64_t)E * Cbuf, 64, 32)) return false;
   return true;
 }
 
 cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* err,
-                            uint64_t wait_limit_ns, int num_sms, cudaStream_t st) {
+                            uint64_t wait_limit_ns, int num_sms, bool want_pair, cudaStream_t st) {
+  if (p.pair && want_pair && (p.Cbuf % pairk::PM) == 0)
+    return p.relu ? launch_pair<true>(p, nexp, err, wait_limit_ns, num_sms, st)
+                  : launch_pair<false>(p, nexp, err, wait_limit_ns, num_sms, st);
   switch (p.BN) {
     case 256:
       return p.relu ? launch_t<256, true>(p, nexp, err, wait_limit_ns, num_sms, st)

@@ -5,11 +5,31 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace moe {
 
 constexpr int kMaxExperts = 256;
 constexpr int kMaxK = 8;
 constexpr int kChunk = 64;          // tokens per router CTA (= scan chunk)
+
+// Launch with programmatic stream serialization: the kernel may begin while the
+// previous kernel on the stream finishes, and orders itself with pdl_wait().
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Device tables of one forward (all owned by the handle's workspace).
 struct Routing {
@@ -54,15 +74,17 @@ cudaError_t launch_ffn_f32(const float* A, const float* B, float* D, const int32
 struct GemmPlan {
   CUtensorMap tmA;   // [E*Cbuf, K] bf16, box {64, 128}, 128B swizzle
   CUtensorMap tmB;   // [E*K, N]    bf16, box {64, 64},  128B swizzle
+  CUtensorMap tmD;   // [E*Cbuf, N] bf16, box {64, 32},  128B swizzle (epilogue stores)
   void* D;           // [E*Cbuf, N] bf16
   int E, K, N, BN;
   int64_t Cbuf;
   bool relu;
+  bool pair;         // the CTA-pair (cta_group::2, 256 x 256 tile) kernel can run (N % 256 == 0)
 };
 bool make_gemm_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, int64_t Cbuf, int K,
                     int N, bool relu);
 cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* err,
-                            uint64_t wait_limit_ns, int num_sms, cudaStream_t st);
+                            uint64_t wait_limit_ns, int num_sms, bool want_pair, cudaStream_t st);
 // selftest.cu
 cudaError_t launch_wait_selftest(unsigned* flag, unsigned* err, uint64_t limit_ns, cudaStream_t st);
 

@@ -183,7 +183,11 @@ moe_status moe_create(moe_handle* out, int64_t S_max, int64_t M, int64_t H, int3
   h->W1 = W1;
   h->W2 = W2;
   const int64_t C = capacity_of(capacity_factor, k, S_max, E);
-  h->Cbuf = C < S_max ? C : S_max;
+  // rows per expert: at most min(C, S_max) are kept; rounded up to 256 so every GEMM
+  // tile (128 rows, or 256 for a CTA pair) and its whole-tile stores stay inside the
+  // expert's own rows
+  const int64_t rows = C < S_max ? C : S_max;
+  h->Cbuf = (rows + 255) / 256 * 256;
   h->wait_limit_ns = 2000000000ull;   // 2 s per wait: far above any legitimate wait
   cudaError_t ce = cudaGetDevice(&h->device);
   if (ce == cudaSuccess)
@@ -279,9 +283,13 @@ moe_status moe_forward(moe_handle h, int64_t S, const void* x, void* y, void* st
   MOE_TRY(launch_dispatch(x, bf16, iS, iM, h->E, h->k, C, h->Cbuf, R, h->xbuf, st));
   MOE_TRY(mark(3));
   if (bf16) {
-    MOE_TRY(launch_ffn_bf16(h->plan1, R.nexp, R.err, h->wait_limit_ns, h->num_sms, st));
+    // CTA-pair GEMMs (256-row tiles) when the experts run at capacity, so the
+    // rows per expert are close to C and the 256-row padding stays small;
+    // otherwise 128-row tiles waste less on partly filled last tiles.
+    const bool saturated = (double)S * h->k / h->E >= (double)C;
+    MOE_TRY(launch_ffn_bf16(h->plan1, R.nexp, R.err, h->wait_limit_ns, h->num_sms, saturated, st));
     MOE_TRY(mark(4));
-    MOE_TRY(launch_ffn_bf16(h->plan2, R.nexp, R.err, h->wait_limit_ns, h->num_sms, st));
+    MOE_TRY(launch_ffn_bf16(h->plan2, R.nexp, R.err, h->wait_limit_ns, h->num_sms, saturated, st));
   } else {
     MOE_TRY(launch_ffn_f32((const float*)h->xbuf, (const float*)h->W1, (float*)h->hbuf, R.nexp,
                            h->E, h->Cbuf, iM, iH, true, st));

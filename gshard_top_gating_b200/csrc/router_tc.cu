@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x, tok0 = tile * C::TT;
+  pdl_trigger();                       // the scan may launch and wait while this grid runs
   const int KB = M / BK;
 
   if (warp == 0 && lane == 0) {

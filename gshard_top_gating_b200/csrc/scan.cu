@@ -65,6 +65,8 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(int S, int E, int k, int
   __shared__ int warp_sums[kThreads / 32];
   __shared__ double dsum[kThreads / 32];
   const int tid = threadIdx.x;
+  pdl_trigger();
+  pdl_wait();                                  // router tables complete
   if (blockIdx.x < (unsigned)E) {
     const int e = blockIdx.x;
     const int L = k * nchunk;                 // entries (r, chunk), r-major
@@ -127,8 +129,7 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(int S, int E, int k, int
 cudaError_t launch_scan(int S, int E, int k, int C, int64_t Cbuf, const Routing& R, cudaStream_t st) {
   const int nchunk = (S + kChunk - 1) / kChunk;
   const int cb = Cbuf < 0x7fffffff ? (int)Cbuf : 0x7fffffff;
-  scan_kernel<<<E + 1, kThreads, 0, st>>>(S, E, k, C, cb, nchunk, R);
-  return cudaGetLastError();
+  return launch_pdl(scan_kernel, dim3(E + 1), dim3(kThreads), 0, st, S, E, k, C, cb, nchunk, R);
 }
 
 }  // namespace moe

@@ -42,6 +42,8 @@ BF16_SHAPES = [
     (300, 128, 128, 200, 8, 1.25),    # router: E padded to 256, top-8
     (200, 192, 128, 100, 3, 1.0),     # router: E padded to 128
     (333, 64, 64, 33, 2, 1.0),        # router: E padded to 64
+    (600, 256, 512, 4, 2, 0.5),       # experts at capacity: CTA-pair GEMMs (256-row tiles)
+    (1000, 256, 256, 8, 1, 1.0),      # CTA pair, k=1, exactly at capacity
 ]
 
 
