@@ -1,0 +1,77 @@
+"""More CUDA-path vs oracle cases (GPU): handle reuse, host buffers, router tails.
+
+* one handle, several forwards with different token counts (capacity, tensor
+  maps and tables must follow S, nothing stale may leak between calls);
+* the host-buffer forward with S < S_max;
+* the tensor-core router's token tiles (64 or 128 tokens) with ragged tails,
+  several K-segments (M = 576 and 1536: 9 and 24 k-blocks of 64), a gate bias
+  with E padded to 256 and top-8.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from gshard_top_gating_b200.inputs import Workload, gate_bias, make_inputs
+from gshard_top_gating_b200.layer import MoeLayer
+from tests import gpu_helpers as G
+
+pytestmark = pytest.mark.gpu
+
+
+def test_one_handle_many_token_counts():
+    w = Workload("reuse", 1000, 256, 512, 16, 2, 0.75, "bf16", seed=21)
+    run = G.build(w)
+    for S in (1000, 37, 640, 1, 1000, 129):
+        G.full_check(run, S)
+    run.layer.close()
+
+
+def test_host_buffers_smaller_batch():
+    w = Workload("host", 700, 128, 256, 8, 2, 1.25, "bf16", seed=22)
+    run = G.build(w)
+    S = 333
+    xh = run.x[:S].cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    run.layer.forward_host(xh, yh)
+    torch.cuda.synchronize()
+    y_dev = run.layer(run.x[:S].contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(yh, y_dev.cpu())
+    G.full_check(run, S)
+    run.layer.close()
+
+
+ROUTER_SHAPES = [
+    # (S, M, H, E, k, cf)
+    (333, 256, 256, 100, 3, 1.0),     # EP = 128 -> 128-token CTAs, ragged tail of 77
+    (97, 128, 128, 40, 2, 1.0),       # EP = 64  -> 64-token CTAs, ragged tail of 33
+    (300, 576, 256, 24, 2, 1.25),     # 9 k-blocks: two K-segments, the last partial
+    (200, 1536, 256, 8, 2, 1.25),     # 24 k-blocks: three K-segments
+    (64, 256, 256, 256, 8, 1.25),     # E = 256, top-8, one CTA
+]
+
+
+@pytest.mark.parametrize("shape", ROUTER_SHAPES, ids=[str(s) for s in ROUTER_SHAPES])
+def test_router_tiles_and_segments(shape):
+    S, M, H, E, k, cf = shape
+    run = G.build(Workload("rt", S, M, H, E, k, cf, "bf16", seed=23))
+    G.full_check(run)
+    run.layer.close()
+
+
+def test_gate_bias_with_256_experts_top8():
+    w = Workload("bias256", 256, 128, 128, 200, 8, 1.0, "bf16", skew_bias=True, seed=24)
+    run = G.build(w)
+    out, rt = G.full_check(run)
+    assert (rt.slot < 0).any()                 # the bias makes low-index experts overflow
+    run.layer.close()
+
+
+def test_dropless_capacity_factor_keeps_everything():
+    # cf = E / k gives C = S: no assignment can be dropped (the "dropless" special case)
+    w = Workload("dropless", 500, 128, 256, 16, 2, 8.0, "bf16", seed=25)
+    run = G.build(w)
+    out, rt = G.full_check(run)
+    assert rt.C == 500 and np.all(rt.slot >= 0)
+    run.layer.close()
