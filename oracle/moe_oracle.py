@@ -1,4 +1,4 @@
-"""CPU oracle for the GShard top-2 (top-k) MoE layer forward.  TEST INFRASTRUCTURE.
+"""CPU oracle for the GShard top-2 (top-k) MoE layer, forward and backward.  TEST INFRASTRUCTURE.
 
 This file exists to check the CUDA path, never to serve it.  Only `tests/`,
 `__graft_entry__.smoke()` and `bench.py`'s CPU-baseline / reference arm may
@@ -39,9 +39,13 @@ Readings where the pages are silent (each one is listed in the design notes):
  * Top-k selects on the fp32 logits, ties to the lower expert index.
  * The expert FFN is relu(x W1[e]) W2[e] with no biases.
  * An empty batch (S = 0) has l_aux = z = 0.
+ * Backward: the routing (choices, slots, drops) and the first-choice fractions
+   f_j carry no gradient; every other step is differentiated exactly.
 
-Pins: every function here is checked in tests/test_oracle_pins.py against hand
-examples, closed forms, library routines, brute force and invariants.
+Pins: every forward function here is checked in tests/test_oracle_pins.py
+against hand examples, closed forms, library routines, brute force and
+invariants; the backward in tests/test_oracle_backward_pins.py against central
+finite differences of the forward and the textbook dense-FFN backward.
 """
 from __future__ import annotations
 
@@ -53,7 +57,8 @@ import numpy as np
 __all__ = [
     "capacity", "gate_logits", "softmax_stats", "top_k", "normalized_gates",
     "assign_slots", "expert_ffn", "dispatch", "combine", "aux_losses",
-    "route", "forward", "outputs_for_tokens",
+    "route", "forward", "expert_ffn_backward", "gates_backward", "aux_loss_backward",
+    "z_loss_backward", "backward", "outputs_for_tokens",
 ]
 
 
@@ -75,13 +80,18 @@ def capacity(S: int, E: int, k: int, cf: float) -> int:
     return int(math.ceil(cf * k * S / E))
 
 
-def gate_logits(x, Wg, bias=None) -> np.ndarray:
+def gate_logits(x, Wg, bias=None, round_fp32: bool = True) -> np.ndarray:
     """Gating logits l = x . W_g (+ b), returned as float32 [S, E].
 
     [blog] "Mixture-of-Experts Implementation", G(x) = Softmax(x . W_g): the
     product is taken in float64 and rounded once to float32; a per-expert bias,
-    when given, is added in float32 after that rounding.
+    when given, is added in float32 after that rounding.  With
+    round_fp32=False everything stays float64 (for finite-difference checks of
+    the backward pass, which fp32 rounding would drown).
     """
+    if not round_fp32:
+        l = _f64(x) @ _f64(Wg)
+        return l if bias is None else l + _f64(bias)
     l = (_f64(x) @ _f64(Wg)).astype(np.float32)
     if bias is not None:
         l = (l + np.asarray(_f64(bias), dtype=np.float32)).astype(np.float32)
@@ -109,9 +119,11 @@ def top_k(logits, k: int) -> np.ndarray:
 
     [note] "top-2"; [blog] "top-k experts (typically k=2)".  Selection is on
     the logits (order-equivalent to the probabilities); ties go to the lower
-    expert index (np.argmax returns the first maximum).
+    expert index (np.argmax returns the first maximum).  float64 logits are
+    compared as given.
     """
-    l = np.array(logits, dtype=np.float32, copy=True)
+    l = np.array(logits, dtype=np.float64 if np.asarray(logits).dtype == np.float64 else np.float32,
+                 copy=True)
     assert np.all(np.isfinite(l)), "logits must be finite"
     S = l.shape[0]
     ids = np.zeros((S, k), dtype=np.int32)
@@ -217,8 +229,11 @@ def route(logits, k: int, cf: float):
     """Routing of given fp32 logits: everything between the gate GEMM and dispatch.
 
     Returns a namespace with p, lse, ids, gates, C, slot, cnt, n, l_aux, z.
+    float64 logits (finite-difference checks) are routed without rounding.
     """
-    logits = np.asarray(logits, dtype=np.float32)
+    logits = np.asarray(logits)
+    if logits.dtype != np.float64:
+        logits = logits.astype(np.float32)
     S, E = logits.shape
     C = capacity(S, E, k, cf)
     p, lse = softmax_stats(logits)
@@ -230,12 +245,13 @@ def route(logits, k: int, cf: float):
                            n=np.minimum(cnt, C), l_aux=l_aux, z=z, f=f, P=P)
 
 
-def forward(x, Wg, bias, W1, W2, k: int, cf: float):
+def forward(x, Wg, bias, W1, W2, k: int, cf: float, round_fp32: bool = True):
     """The whole layer forward on the CPU (small cases).
 
-    Returns the `route` namespace plus logits and the output y[S, M] (float64).
+    Returns the `route` namespace plus logits, the per-expert buffers (xbuf,
+    pre-activation hpre, ybuf) and the output y[S, M] (float64).
     """
-    logits = gate_logits(x, Wg, bias)
+    logits = gate_logits(x, Wg, bias, round_fp32)
     rt = route(logits, k, cf)
     S, E = logits.shape
     C = rt.C
@@ -243,13 +259,109 @@ def forward(x, Wg, bias, W1, W2, k: int, cf: float):
     W2 = _f64(W2)
     xbuf = dispatch(x, rt.ids, rt.slot, E, C)
     ybuf = np.zeros_like(xbuf)
+    hpre = np.zeros((E, C, W1.shape[2]))
     for e in range(E):
         n = int(rt.n[e])
         if n:
             ybuf[e, :n] = expert_ffn(xbuf[e, :n], W1[e], W2[e])
+            hpre[e, :n] = xbuf[e, :n] @ W1[e]
     rt.logits = logits
+    rt.xbuf, rt.hpre, rt.ybuf = xbuf, hpre, ybuf
     rt.y = combine(ybuf, rt.ids, rt.gates, rt.slot)
     return rt
+
+
+def expert_ffn_backward(rows, hpre, dY, W1e, W2e):
+    """Backward of one expert's ReLU FFN y = relu(rows W1e) W2e ([blog] Expert Networks).
+
+    Given the upstream gradient dY of the expert's outputs: dW2 = relu(pre)^T dY,
+    dpre = (dY W2^T) * [pre > 0], dW1 = rows^T dpre, drows = dpre W1^T.
+    Returns (drows, dW1e, dW2e).
+    """
+    h = np.maximum(hpre, 0.0)
+    dW2e = h.T @ dY
+    dpre = (dY @ W2e.T) * (hpre > 0)
+    return dpre @ W1e.T, rows.T @ dpre, dW2e
+
+
+def gates_backward(gates, ids, dgate, E: int):
+    """Logit gradient through the normalised gates g_r = softmax over the k chosen logits.
+
+    [note] "softmax-normalised top-2 weights": dl[t, e_r] += g_r (dgate_r -
+    sum_r' g_r' dgate_r').  Returns dl[S, E].
+    """
+    S, k = gates.shape
+    dl = np.zeros((S, E))
+    inner = np.sum(gates * dgate, axis=1, keepdims=True)
+    np.add.at(dl, (np.arange(S)[:, None].repeat(k, 1), ids), gates * (dgate - inner))
+    return dl
+
+
+def aux_loss_backward(p, f, E: int):
+    """d l_aux / d logits with f_j held fixed (a count of argmax choices carries no gradient).
+
+    l_aux = E sum_j f_j P_j, P_j = mean_t p[t, j]; through the softmax:
+    dl[t] = E/S * p_t * (f - <p_t, f>).  Returns dl[S, E].
+    """
+    S = p.shape[0]
+    return E / S * p * (f[None, :] - (p @ f)[:, None])
+
+
+def z_loss_backward(p, lse):
+    """d z / d logits for z = mean_t lse_t^2: dl[t] = 2/S * lse_t * p_t.  Returns dl[S, E]."""
+    S = p.shape[0]
+    return 2.0 / S * lse[:, None] * p
+
+
+def backward(x, Wg, bias, W1, W2, k: int, cf: float, dy, a_aux: float = 0.0, a_z: float = 0.0,
+             round_fp32: bool = True):
+    """Gradients of  L = <dy, y> + a_aux * l_aux + a_z * z  with respect to x, W_g, b, W1, W2.
+
+    The routing (expert choice, slots, drops) is piecewise constant and carries
+    no gradient; everything else is differentiated exactly, in the forward's
+    order reversed:
+      combine: dY_e[slot_r] = g_r dy[t] and dgate_r = <dy[t], y_e[slot_r]>
+        (both 0 for a dropped assignment);
+      expert FFN: `expert_ffn_backward` per expert, dx[t] += sum of the kept
+        choices' row gradients;
+      gates, l_aux, z: `gates_backward`, `aux_loss_backward`, `z_loss_backward`
+        give the logit gradient dl;
+      gate GEMM ([blog] G(x) = Softmax(x . W_g)): dx += dl W_g^T, dW_g = x^T dl, db = sum_t dl.
+    Returns a namespace with dx, dWg, dbias, dW1, dW2 (float64), the
+    intermediates dl, dgate and the forward namespace fwd.
+    """
+    rt = forward(x, Wg, bias, W1, W2, k, cf, round_fp32)
+    xf, Wgf, W1f, W2f, dyf = _f64(x), _f64(Wg), _f64(W1), _f64(W2), _f64(dy)
+    S, E = rt.logits.shape
+    dgate = np.zeros((S, k))
+    dybuf = np.zeros_like(rt.ybuf)
+    for r in range(k):
+        keep = rt.slot[:, r] >= 0
+        t = np.nonzero(keep)[0]
+        e, sl = rt.ids[keep, r], rt.slot[keep, r]
+        dgate[t, r] = np.sum(dyf[t] * rt.ybuf[e, sl], axis=1)
+        dybuf[e, sl] = rt.gates[t, r][:, None] * dyf[t]
+    dW1 = np.zeros_like(W1f)
+    dW2 = np.zeros_like(W2f)
+    dxbuf = np.zeros_like(rt.xbuf)
+    for e in range(E):
+        n = int(rt.n[e])
+        if n:
+            dxbuf[e, :n], dW1[e], dW2[e] = expert_ffn_backward(
+                rt.xbuf[e, :n], rt.hpre[e, :n], dybuf[e, :n], W1f[e], W2f[e])
+    dx = np.zeros_like(xf)
+    for r in range(k):
+        keep = rt.slot[:, r] >= 0
+        dx[keep] += dxbuf[rt.ids[keep, r], rt.slot[keep, r]]
+    dl = np.zeros((S, E))
+    if S:
+        dl += gates_backward(rt.gates, rt.ids, dgate, E)
+        dl += a_aux * aux_loss_backward(rt.p, rt.f, E)
+        dl += a_z * z_loss_backward(rt.p, rt.lse)
+    dx += dl @ Wgf.T
+    dWg = xf.T @ dl
+    dbias = dl.sum(axis=0)
+    return SimpleNamespace(dx=dx, dWg=dWg, dbias=dbias, dW1=dW1, dW2=dW2, dl=dl, dgate=dgate, fwd=rt)
 
 
 def outputs_for_tokens(tokens, x_rows, ids, gates, slot, expert_weights):
