@@ -188,6 +188,103 @@ def algorithmic(w, A, n_active):
     }
 
 
+def algorithmic_bwd(w, A, pad_rows, nsplit):
+    """Algorithmic bytes / flops per launch of each backward stage (A kept assignments)."""
+    s = 2 if w.act == "bf16" else 4
+    S, M, H, E, k = w.S, w.M, w.H, w.E, w.k
+    return {
+        "gate_bwd": ("hbm", S * M * s + 2 * A * M * s + 2 * S * E * 4 + S * k * 16 + E * 4),
+        "pad_zero": ("hbm", pad_rows * (2 * M + H) * s),
+        "dW2": ("tensor", 2.0 * A * M * H),
+        "dP": ("tensor", 2.0 * A * M * H),
+        "dW1": ("tensor", 2.0 * A * M * H),
+        "dX_e": ("tensor", 2.0 * A * M * H),
+        "dx": ("hbm", (A + S) * M * s + S * E * 4 + M * E * 4 + S * k * 8),
+        "dWg": ("hbm", S * M * s + S * E * 4 + 2 * nsplit * (M + 1) * E * 4),
+    }
+
+
+def measure_backward(args, w, layer, x, y, flush, stream, pk, A, n_e):
+    """One training step = moe_forward + moe_backward of the same tokens, device-timed."""
+    from gshard_top_gating_b200 import _lib as L
+    from gshard_top_gating_b200.inputs import upstream_grad
+    dev = x.device
+    dy = upstream_grad(w, device=dev)
+    L.moe_enable_backward(layer.h)
+    dx = torch.empty_like(x)
+    dWg = torch.empty(w.M, w.E, dtype=torch.float32, device=dev)
+    dbias = torch.empty(w.E, dtype=torch.float32, device=dev) if w.skew_bias else None
+    dW1 = torch.empty(w.E, w.M, w.H, dtype=x.dtype, device=dev)
+    dW2 = torch.empty(w.E, w.H, w.M, dtype=x.dtype, device=dev)
+    a_aux, a_z = 0.01, 0.001
+
+    def bwd():
+        L.moe_backward(layer.h, w.S, x, dy, a_aux, a_z, dx, dWg, dbias, dW1, dW2)
+
+    for _ in range(3):
+        layer(x, out=y)
+        bwd()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 50))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    for i in range(n):
+        flush.zero_()
+        ev[i][0].record(stream)
+        layer(x, out=y)
+        ev[i][1].record(stream)
+        bwd()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    bwd_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    L.moe_set_profiling(layer.h, True)
+    per = [[] for _ in L.BWD_STAGES]
+    for _ in range(min(n, 20)):
+        flush.zero_()
+        layer(x, out=y)
+        bwd()
+        for j, t in enumerate(L.moe_get_backward_stage_times(layer.h)):
+            per[j].append(t)
+    L.moe_set_profiling(layer.h, False)
+    torch.cuda.synchronize()
+    stage_ms = {nm: statistics.mean(v) for nm, v in zip(L.BWD_STAGES, per)}
+    pad_rows = int(sum(((int(v) + 63) // 64) * 64 - int(v) for v in n_e.tolist()))
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    tiles = ((w.M + 64) // 64) * ((w.E + 63) // 64)
+    nsplit = max(1, min((2 * sms + tiles - 1) // tiles, (w.S + 255) // 256))
+    algo = algorithmic_bwd(w, A, pad_rows, nsplit)
+    stages = {}
+    for nm in L.BWD_STAGES:
+        b_, wk = algo[nm]
+        tt = stage_ms[nm] / 1e3
+        if tt <= 0:
+            continue
+        if b_ == "tensor":
+            stages[nm] = {"ms": round(stage_ms[nm], 4), "TFLOP/s": round(wk / tt / 1e12, 1),
+                          "frac_of_peak": round(wk / tt / 1e12 / pk["bf16_tflops"], 4)}
+        else:
+            stages[nm] = {"ms": round(stage_ms[nm], 4), "GB/s": round(wk / tt / 1e9, 1),
+                          "frac_of_peak": round(wk / tt / 1e9 / pk["hbm_gbs"], 4)}
+    dom = max(stage_ms, key=lambda k_: stage_ms[k_])
+    b_, wk = algo[dom]
+    tt = stage_ms[dom] / 1e3
+    if b_ == "tensor":
+        ach, peak, unit = wk / tt / 1e12, pk["bf16_tflops"], "TFLOP/s"
+    else:
+        ach, peak, unit = wk / tt / 1e9, pk["hbm_gbs"], "GB/s"
+    ffn = sum(stage_ms[k_] for k_ in ("dW2", "dP", "dW1", "dX_e"))
+    return {
+        "what": "moe_forward + moe_backward of the same tokens (dL/dy given; a_aux=0.01, a_z=0.001)",
+        "tokens_per_s": round(w.S / ((fwd_ms + bwd_ms) / 1e3), 1),
+        "ms_fwd": round(fwd_ms, 4), "ms_bwd": round(bwd_ms, 4), "steps": n,
+        "expert_gemm_TFLOP/s": round(4 * 2.0 * A * w.M * w.H / (ffn / 1e3) / 1e12, 1) if ffn > 0 else None,
+        "roofline": {"bound": b_, "kernel": dom, "achieved": round(ach, 2), "peak": peak, "unit": unit,
+                     "frac": round(ach / peak, 4)},
+        "stages": stages,
+        "gpu_launches": n * (L.moe_kernels_per_forward(layer.h, w.S) + L.moe_kernels_per_backward(layer.h, w.S)),
+    }
+
+
 def run_ours(args, rank, world, local):
     w = WORKLOADS[args.workload]
     from gshard_top_gating_b200 import _lib as L
@@ -326,6 +423,8 @@ def run_ours(args, rank, world, local):
             stages[n] = {"ms": round(stage_ms[n], 4), "GB/s": round(wk / tt / 1e9, 1),
                          "frac_of_peak": round(wk / tt / 1e9 / pk["hbm_gbs"], 4)}
 
+    train = None if args.no_backward else measure_backward(args, w, layer, x, y, flush, stream, pk, A, n_e)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_budget, x, Wg, b, W1, W2)
@@ -347,6 +446,7 @@ def run_ours(args, rank, world, local):
         "gpu_launches": args.steps * L.moe_kernels_per_forward(layer.h, w.S),
         "clocks": clocks,
         "cpu_baseline": cpu,
+        "train_step": train,
     }
     layer.close()
     return line
@@ -436,6 +536,8 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=120.0,
                     help="seconds of oracle work for the whole --impl reference run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the training-step (forward + backward) measurement")
     ap.add_argument("--eager", action="store_true",
                     help="time eager moe_forward calls instead of a CUDA-graph replay")
     args = ap.parse_args()

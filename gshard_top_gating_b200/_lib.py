@@ -20,6 +20,8 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_OOM, MOE
 MOE_F32, MOE_BF16 = 0, 1
 MOE_NUM_STAGES = 6
 STAGES = ("router", "scan", "dispatch", "ffn1", "ffn2", "combine")
+MOE_NUM_BWD_STAGES = 8
+BWD_STAGES = ("gate_bwd", "pad_zero", "dW2", "dP", "dW1", "dX_e", "dx", "dWg")
 
 
 class MoeError(RuntimeError):
@@ -50,6 +52,9 @@ def _load() -> ctypes.CDLL:
         "moe_get_stage_times": [P, ctypes.POINTER(ctypes.c_float), I32],
         "moe_selftest_wait_timeout": [I32, P],
         "moe_assign_slots_noalloc": [I64, I32, I32, I64, P, P, P, P],
+        "moe_enable_backward": [P],
+        "moe_get_backward_stage_times": [P, ctypes.POINTER(ctypes.c_float), I32],
+        "moe_backward": [P, I64, P, P, ctypes.c_float, ctypes.c_float, P, P, P, P, P, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -57,10 +62,14 @@ def _load() -> ctypes.CDLL:
         f.restype = ctypes.c_int
     lib.moe_kernels_per_forward.argtypes = [P, I64]
     lib.moe_kernels_per_forward.restype = I32
+    lib.moe_kernels_per_backward.argtypes = [P, I64]
+    lib.moe_kernels_per_backward.restype = I32
     lib.moe_status_string.argtypes = [ctypes.c_int]
     lib.moe_status_string.restype = ctypes.c_char_p
     lib.moe_stage_name.argtypes = [I32]
     lib.moe_stage_name.restype = ctypes.c_char_p
+    lib.moe_backward_stage_name.argtypes = [I32]
+    lib.moe_backward_stage_name.restype = ctypes.c_char_p
     return lib
 
 
@@ -168,3 +177,27 @@ def moe_assign_slots_noalloc(S, E, k, C, eidx, slot, cnt, stream=None) -> None:
     """Capacity slots from expert ids with no device allocation (see include/moe.h)."""
     _check("moe_assign_slots_noalloc",
            lib.moe_assign_slots_noalloc(S, E, k, C, _ptr(eidx), _ptr(slot), _ptr(cnt), _stream(stream)))
+
+
+def moe_enable_backward(h) -> None:
+    _check("moe_enable_backward", lib.moe_enable_backward(h))
+
+
+def moe_backward(h, S, x, dy, a_aux, a_z, dx, dWg, dbias, dW1, dW2, stream=None) -> None:
+    _check("moe_backward", lib.moe_backward(h, S, _ptr(x), _ptr(dy), float(a_aux), float(a_z), _ptr(dx),
+                                            _ptr(dWg), _ptr(dbias), _ptr(dW1), _ptr(dW2),
+                                            _stream(stream)))
+
+
+def moe_kernels_per_backward(h, S) -> int:
+    return int(lib.moe_kernels_per_backward(h, S))
+
+
+def moe_get_backward_stage_times(h):
+    buf = (ctypes.c_float * MOE_NUM_BWD_STAGES)()
+    _check("moe_get_backward_stage_times", lib.moe_get_backward_stage_times(h, buf, MOE_NUM_BWD_STAGES))
+    return list(buf)
+
+
+def moe_backward_stage_name(stage: int) -> str:
+    return lib.moe_backward_stage_name(stage).decode()

@@ -78,7 +78,8 @@ def build(verbose: bool = False, ptxas_info: bool = False) -> str:
     with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         list(ex.map(run, jobs))
     if jobs or _stale(LIB, objs):
-        cmd = [cc, *ARCH, "-shared", "-cudart", "static", "-o", LIB, *objs, "-ldl", "-lpthread", "-lrt"]
+        cmd = [cc, *ARCH, "-shared", "-cudart", "static", "-o", LIB, *objs, "-ldl", "-lpthread", "-lrt",
+               "-Xlinker", "--no-undefined"]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)

@@ -52,11 +52,12 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uin
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Instruction descriptor, kind::f16: D fp32, A bf16 (K-major), B bf16 (MN-major), M=128, N=BN.
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, M=128, N=BN; a_mn / b_mn
+// select the MN-major (transposed) operand layout (bits 15 / 16), else K-major.
 template <int BN>
-__device__ __forceinline__ uint32_t idesc_bf16() {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(BN >> 3) << 17) |
-         ((uint32_t)(BM >> 4) << 24);
+__device__ __forceinline__ uint32_t idesc_bf16(bool a_mn, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
 // Walks this CTA's tiles in the global order (expert, n-tile, m-tile).
@@ -76,31 +77,71 @@ struct TileIter {
   }
 };
 
-// Epilogue of one warp's 32 accumulator rows x BN columns: TMEM -> bf16 (+ReLU) ->
-// a 4 KB staging tile in shared memory laid out as the store tensor map's 128-byte
-// swizzle (row r, 16-byte chunk c at r*128 + ((c ^ (r % 8)) * 16)) -> one TMA store per
-// 64 columns.  Rows past n_e land in the expert's own padding rows (rows per expert
-// are a multiple of 128), which nothing reads.  The TMA engine writes whole 128-byte
-// rows, instead of each thread storing 16 bytes to 32 different rows per instruction.
-template <int BN, bool RELU>
+// Epilogue modes: plain store, ReLU, or the backward's ReLU mask (keep the
+// accumulator where the first layer's saved output h is > 0, else 0).
+enum { kEpiNone = 0, kEpiRelu = 1, kEpiMask = 2 };
+
+// 32 mask bits for 32 consecutive bf16 values of h: bit j set iff h[j] > 0
+// (bit patterns 0x0001 .. 0x7f80: positive finite or +inf).
+__device__ __forceinline__ uint32_t positive_bits(const uint4 (&v)[4]) {
+  uint32_t bits = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t lo = w[j] & 0xFFFFu, hi = w[j] >> 16;
+      bits |= (uint32_t)(lo - 1u < 0x7F80u) << (8 * q + 2 * j);
+      bits |= (uint32_t)(hi - 1u < 0x7F80u) << (8 * q + 2 * j + 1);
+    }
+  }
+  return bits;
+}
+
+// Epilogue of one warp's 32 accumulator rows x BN columns: TMEM -> bf16 (+ReLU or
+// mask) -> a 4 KB staging tile in shared memory laid out as the store tensor map's
+// 128-byte swizzle (row r, 16-byte chunk c at r*128 + ((c ^ (r % 8)) * 16)) -> one TMA
+// store per 64 columns.  Rows past n_e land in the expert's own padding rows (rows
+// per expert are a multiple of 128), which nothing reads as data.  The TMA engine
+// writes whole 128-byte rows, instead of each thread storing 16 bytes to 32
+// different rows per instruction.  `mrow` (kEpiMask) points at this lane's row of h
+// at the tile's first column; `zero` stores zeros without reading TMEM.
+template <int BN, int EPI>
 __device__ __forceinline__ void store_rows(const CUtensorMap* tmD, uint32_t tmem_rows,
-                                           uint32_t stage, int row0, int col0, int lane) {
+                                           uint32_t stage, int row0, int col0, int lane,
+                                           const uint16_t* mrow = nullptr, bool zero = false) {
 #pragma unroll 1
   for (int b = 0; b < BN / 64; ++b) {
     if (lane == 0) bulk_wait_read0();          // the previous store has read the staging tile
     __syncwarp();
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
+      uint32_t keep = 0xFFFFFFFFu;
+      if (EPI == kEpiMask) {
+        uint4 mv[4];
+        const uint4* mp = reinterpret_cast<const uint4*>(mrow + b * 64 + h * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mv[j] = ld_nc_v4(mp + j);
+        keep = positive_bits(mv);
+      }
       uint32_t r[32];
-      tmem_ld_32x32b_x32(tmem_rows + b * 64 + h * 32, r);
-      tmem_ld_wait();
+      if (zero) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = 0u;
+      } else {
+        tmem_ld_32x32b_x32(tmem_rows + b * 64 + h * 32, r);
+        tmem_ld_wait();
+      }
       uint32_t pk[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         float a = __uint_as_float(r[2 * j]), c = __uint_as_float(r[2 * j + 1]);
-        if (RELU) {
+        if (EPI == kEpiRelu) {
           a = fmaxf(a, 0.f);
           c = fmaxf(c, 0.f);
+        } else if (EPI == kEpiMask) {
+          a = ((keep >> (2 * j)) & 1u) ? a : 0.f;
+          c = ((keep >> (2 * j + 1)) & 1u) ? c : 0.f;
         }
         pk[j] = pack_bf16x2(a, c);
       }
@@ -120,11 +161,15 @@ __device__ __forceinline__ void store_rows(const CUtensorMap* tmD, uint32_t tmem
   }
 }
 
-template <int BN, bool RELU>
+// BKM = false: B[e] is [K, N] (N contiguous, the forward's weights).  BKM = true:
+// B[e] is [N, K] (K contiguous): the backward's products with a transposed weight,
+// dY W2[e]^T and dP W1[e]^T, read the weights in their stored layout.
+template <int BN, int EPI, bool BKM>
 __global__ void __launch_bounds__(kThreads, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
-                  int64_t Cbuf, int K, int N, unsigned* err, uint64_t limit_ns) {
+                  int64_t Cbuf, int K, int N, const uint16_t* __restrict__ mask, unsigned* err,
+                  uint64_t limit_ns) {
   using C = Cfg<BN>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -220,9 +265,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sa = base + s * C::STAGE_BYTES;
           mbar_arrive_expect_tx(full_bar(s), C::STAGE_BYTES);
           tma_load_2d(sa, &tmA, full_bar(s), kb * BK, rowA);
+          if (BKM) {
+            tma_load_2d(sa + A_BYTES, &tmB, full_bar(s), kb * BK, e * N + nt * BN);
+          } else {
 #pragma unroll
-          for (int j = 0; j < BN / 64; ++j)
-            tma_load_2d(sa + A_BYTES + j * 8192u, &tmB, full_bar(s), nt * BN + j * 64, rowB + kb * BK);
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(sa + A_BYTES + j * 8192u, &tmB, full_bar(s), nt * BN + j * 64,
+                          rowB + kb * BK);
+          }
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
           if (++s == C::STAGES) {
@@ -241,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       TileIter it{tile_pre, mtiles, E, NT, 0};
-      const uint32_t idesc = idesc_bf16<BN>();
+      const uint32_t idesc = idesc_bf16<BN>(false, !BKM);
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -268,7 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = desc_sw128(sa + kk * 32u, 16u, 1024u);
-            const uint64_t bd = desc_sw128(sb + kk * 2048u, 8192u, 1024u);
+            const uint64_t bd = BKM ? desc_sw128(sb + kk * 32u, 16u, 1024u)
+                                    : desc_sw128(sb + kk * 2048u, 8192u, 1024u);
             tc_mma_f16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
           }
           tc_commit(empty_bar(s));
@@ -300,12 +351,210 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int row0 = (int)(e * Cbuf + mt * BM + q * 32);
-      store_rows<BN, RELU>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
-                           nt * BN, lane);
+      const uint16_t* mrow = EPI == kEpiMask ? mask + (int64_t)(row0 + lane) * N + nt * BN : nullptr;
+      store_rows<BN, EPI>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
+                          nt * BN, lane, mrow);
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
     }
     if (lane == 0) bulk_wait0();                // stores complete before the CTA exits
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- weight gradients
+//
+//   D[e] = A[e, :n_e, :]^T . B[e, :n_e, :]        A [E*Cbuf, P], B [E*Cbuf, Q], D [E*P, Q]
+//
+// the backward's dW2[e] = h_e^T dY_e (P = H, Q = M) and dW1[e] = X_e^T dP_e (P = M,
+// Q = H).  The reduction runs over the expert's kept slots, so both operands are
+// read "MN-major" (slot rows, P or Q contiguous) in 64 x 64 TMA boxes and the MMA
+// takes them transposed.  The k-loop covers ceil(n_e / 64) blocks; rows n_e ..
+// ceil64(n_e) - 1 of both operands must hold zeros (the caller clears them).  An
+// expert with no kept slot gets D[e] = 0 (its tiles store zeros without an MMA).
+// Tiles are (expert, p-tile, q-tile), q fastest; roles as in ffn_tc_kernel.
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    wgrad_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp,
+                    int E, int64_t Cbuf, int P, int Q, unsigned* err, uint64_t limit_ns) {
+  using C = Cfg<BN>;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;
+  unsigned char* gbase = smem_raw + (base - raw_base);
+  const uint32_t staging0 = base + C::STAGES * C::STAGE_BYTES;
+  const uint32_t bar0 = staging0 + C::STAGING;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 2 + a); };
+  const uint32_t done_bar = bar0 + 8u * (2 * C::STAGES + 4);
+  unsigned char* misc = gbase + C::STAGES * C::STAGE_BYTES + C::STAGING + 512;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  int* kblocks = reinterpret_cast<int*>(misc + 16);                  // [E]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int PT = (P + BM - 1) / BM, QT = Q / BN;
+  const int per_e = PT * QT, total = E * per_e;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 128);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  pdl_trigger();
+  pdl_wait();                          // operands and counts complete
+  if (warp == 2)
+    for (int e = lane; e < E; e += 32) kblocks[e] = (min(nexp[e], (int)Cbuf) + BK - 1) / BK;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, issued = 0, issued_par = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const int e = tile / per_e, r = tile - e * per_e;
+        const int pt = r / QT, qt = r - pt * QT;
+        const int KB = kblocks[e];
+        for (int kb = 0; kb < KB; ++kb) {
+          if (*abort_flag || !mbar_wait(empty_bar(s), ph ^ 1u, err, limit_ns)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const uint32_t sa = base + s * C::STAGE_BYTES;
+          const int row = (int)(e * Cbuf + kb * BK);
+          mbar_arrive_expect_tx(full_bar(s), C::STAGE_BYTES);
+          // columns of A past P (a half-filled last p-tile) read as zeros
+#pragma unroll
+          for (int j = 0; j < BM / 64; ++j) tma_load_2d(sa + j * 8192u, &tmA, full_bar(s), pt * BM + j * 64, row);
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j)
+            tma_load_2d(sa + A_BYTES + j * 8192u, &tmB, full_bar(s), qt * BN + j * 64, row);
+          issued |= 1u << s;
+          issued_par = (issued_par & ~(1u << s)) | (ph << s);
+          if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        for (int q = 0; q < C::STAGES; ++q)
+          if ((issued >> q) & 1u) mbar_wait(full_bar(q), (issued_par >> q) & 1u, err, limit_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16<BN>(true, true);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int i = 0;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const int e = tile / per_e;
+        const int KB = kblocks[e];
+        if (KB == 0) continue;                  // zero tile: the epilogue stores zeros
+        const int acc = i & 1;
+        const uint32_t aph = (i >> 1) & 1;
+        ++i;
+        if (*abort_flag || !mbar_wait(tempty_bar(acc), aph ^ 1u, err, limit_ns)) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (*abort_flag || !mbar_wait(full_bar(s), ph, err, limit_ns)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base + s * C::STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = desc_sw128(sa + kk * 2048u, 8192u, 1024u);
+            const uint64_t bd = desc_sw128(sb + kk * 2048u, 8192u, 1024u);
+            tc_mma_f16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          }
+          tc_commit(empty_bar(s));
+          if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (ok) tc_commit(tfull_bar(acc));
+      }
+      if (!ok) {
+        tc_commit(done_bar);
+        mbar_wait(done_bar, 0, err, limit_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;
+    const uint32_t stage = staging0 + (warp - 2) * 4096u;
+    int i = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const int e = tile / per_e, r = tile - e * per_e;
+      const int pt = r / QT, qt = r - pt * QT;
+      const bool zero = kblocks[e] == 0;
+      const int prow = pt * BM + q * 32;        // P is a multiple of 64: warps hold 32 rows or none
+      const int row0 = e * P + prow;
+      int acc = 0;
+      if (!zero) {
+        acc = i & 1;
+        const uint32_t aph = (i >> 1) & 1;
+        ++i;
+        if (*abort_flag || !mbar_wait(tfull_bar(acc), aph, err, limit_ns)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+      }
+      if (prow < P)
+        store_rows<BN, kEpiNone>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage,
+                                 row0, qt * BN, lane, nullptr, zero);
+      if (!zero) {
+        tc_fence_before();
+        mbar_arrive(tempty_bar(acc));
+      }
+    }
+    if (lane == 0) bulk_wait0();
     __syncwarp();
   }
 
@@ -518,8 +767,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int row0 = (int)(e * Cbuf + mt * PM + (int)rank * (PM / 2) + q * 32);
-      store_rows<BN, RELU>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
-                           nt * BN, lane);
+      store_rows<BN, RELU ? kEpiRelu : kEpiNone>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN,
+                                                 stage, row0, nt * BN, lane);
       tc_fence_before();
       if (leader) mbar_arrive(tempty_bar(acc));
       else mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
@@ -575,10 +824,21 @@ cudaError_t launch_pair(const GemmPlan& p, const int32_t* nexp, unsigned* err, u
                     nexp, p.E, p.Cbuf, p.K, p.N, err, limit_ns);
 }
 
-template <int BN, bool RELU>
+template <int BN, int EPI, bool BKM>
 cudaError_t launch_t(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint64_t limit_ns,
                      int num_sms, cudaStream_t st) {
-  auto kern = ffn_tc_kernel<BN, RELU>;
+  auto kern = ffn_tc_kernel<BN, EPI, BKM>;
+  const size_t smem = Cfg<BN>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(num_sms), dim3(kThreads), smem, st, p.tmA, p.tmB, p.tmD, nexp, p.E,
+                    p.Cbuf, p.K, p.N, static_cast<const uint16_t*>(p.mask), err, limit_ns);
+}
+
+template <int BN>
+cudaError_t launch_w(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint64_t limit_ns,
+                     int num_sms, cudaStream_t st) {
+  auto kern = wgrad_tc_kernel<BN>;
   const size_t smem = Cfg<BN>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -586,17 +846,21 @@ cudaError_t launch_t(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint
                     p.Cbuf, p.K, p.N, err, limit_ns);
 }
 
+int pick_bn(int N) { return (N % 256 == 0) ? 256 : (N % 128 == 0 ? 128 : 64); }
+
 }  // namespace
 
 bool make_gemm_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, int64_t Cbuf, int K,
                     int N, bool relu) {
+  p = GemmPlan{};
+  p.kind = kGemmFwd;
   p.E = E;
   p.Cbuf = Cbuf;
   p.K = K;
   p.N = N;
   p.D = D;
   p.relu = relu;
-  p.BN = (N % 256 == 0) ? 256 : (N % 128 == 0 ? 128 : 64);
+  p.BN = pick_bn(N);
   p.pair = (N % pairk::BN) == 0;      // CTA-pair kernel whenever the 256-wide tile divides N
   if (K % BK || N % 64) return false;
   if (!encode_2d(&p.tmA, A, (uint64_t)K, (uint64_t)E * Cbuf, BK, BM)) return false;
@@ -605,21 +869,77 @@ bool make_gemm_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, i
   return true;
 }
 
+bool make_dgrad_plan(GemmPlan& p, const void* A, const void* Bt, void* D, const void* mask, int E,
+                     int64_t Cbuf, int K, int N) {
+  p = GemmPlan{};
+  p.kind = kGemmDgrad;
+  p.E = E;
+  p.Cbuf = Cbuf;
+  p.K = K;
+  p.N = N;
+  p.D = D;
+  p.mask = mask;
+  p.BN = pick_bn(N);
+  if (K % BK || N % 64) return false;
+  if (!encode_2d(&p.tmA, A, (uint64_t)K, (uint64_t)E * Cbuf, BK, BM)) return false;
+  if (!encode_2d(&p.tmB, Bt, (uint64_t)K, (uint64_t)E * N, BK, (uint32_t)p.BN)) return false;
+  if (!encode_2d(&p.tmD, D, (uint64_t)N, (uint64_t)E * Cbuf, 64, 32)) return false;
+  return true;
+}
+
+bool make_wgrad_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, int64_t Cbuf, int P,
+                     int Q) {
+  p = GemmPlan{};
+  p.kind = kGemmWgrad;
+  p.E = E;
+  p.Cbuf = Cbuf;
+  p.K = P;                             // rows of each expert's result
+  p.N = Q;
+  p.D = D;
+  p.BN = pick_bn(Q);
+  if (P % 64 || Q % 64 || Cbuf % BK) return false;
+  if (!encode_2d(&p.tmA, A, (uint64_t)P, (uint64_t)E * Cbuf, 64, BK)) return false;
+  if (!encode_2d(&p.tmB, B, (uint64_t)Q, (uint64_t)E * Cbuf, 64, BK)) return false;
+  if (!encode_2d(&p.tmD, D, (uint64_t)Q, (uint64_t)E * P, 64, 32)) return false;
+  return true;
+}
+
 cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* err,
                             uint64_t wait_limit_ns, int num_sms, bool want_pair, cudaStream_t st) {
+  if (p.kind == kGemmWgrad) {
+    switch (p.BN) {
+      case 256: return launch_w<256>(p, nexp, err, wait_limit_ns, num_sms, st);
+      case 128: return launch_w<128>(p, nexp, err, wait_limit_ns, num_sms, st);
+      default: return launch_w<64>(p, nexp, err, wait_limit_ns, num_sms, st);
+    }
+  }
+  if (p.kind == kGemmDgrad) {
+    const bool m = p.mask != nullptr;
+    switch (p.BN) {
+      case 256:
+        return m ? launch_t<256, kEpiMask, true>(p, nexp, err, wait_limit_ns, num_sms, st)
+                 : launch_t<256, kEpiNone, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+      case 128:
+        return m ? launch_t<128, kEpiMask, true>(p, nexp, err, wait_limit_ns, num_sms, st)
+                 : launch_t<128, kEpiNone, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+      default:
+        return m ? launch_t<64, kEpiMask, true>(p, nexp, err, wait_limit_ns, num_sms, st)
+                 : launch_t<64, kEpiNone, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+    }
+  }
   if (p.pair && want_pair && (p.Cbuf % pairk::PM) == 0)
     return p.relu ? launch_pair<true>(p, nexp, err, wait_limit_ns, num_sms, st)
                   : launch_pair<false>(p, nexp, err, wait_limit_ns, num_sms, st);
   switch (p.BN) {
     case 256:
-      return p.relu ? launch_t<256, true>(p, nexp, err, wait_limit_ns, num_sms, st)
-                    : launch_t<256, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      return p.relu ? launch_t<256, kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st)
+                    : launch_t<256, kEpiNone, false>(p, nexp, err, wait_limit_ns, num_sms, st);
     case 128:
-      return p.relu ? launch_t<128, true>(p, nexp, err, wait_limit_ns, num_sms, st)
-                    : launch_t<128, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      return p.relu ? launch_t<128, kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st)
+                    : launch_t<128, kEpiNone, false>(p, nexp, err, wait_limit_ns, num_sms, st);
     default:
-      return p.relu ? launch_t<64, true>(p, nexp, err, wait_limit_ns, num_sms, st)
-                    : launch_t<64, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      return p.relu ? launch_t<64, kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st)
+                    : launch_t<64, kEpiNone, false>(p, nexp, err, wait_limit_ns, num_sms, st);
   }
 }
 

@@ -42,6 +42,7 @@ struct Routing {
   int32_t* off;      // [k, nchunk, E] exclusive rank-major prefix of hist per expert
   int32_t* cnt;      // [E] demand per expert (before capacity)
   int32_t* nexp;     // [E] kept rows per expert = min(cnt, C)
+  int32_t* first;    // [E] tokens whose first choice is the expert (f_j * S)
   float* psum;       // [nchunk, E] per-chunk sum of softmax probabilities
   float* lse2;       // [nchunk]    per-chunk sum of lse^2
   float* losses;     // [2]  l_aux, z
@@ -71,11 +72,17 @@ cudaError_t launch_combine(const void* ybuf, bool bf16, int S, int M, int k, int
 cudaError_t launch_ffn_f32(const float* A, const float* B, float* D, const int32_t* nexp, int E,
                            int64_t Cbuf, int K, int N, bool relu, cudaStream_t st);
 // ffn_tc.cu  (bf16 activations, tcgen05)
+enum { kGemmFwd = 0, kGemmDgrad = 1, kGemmWgrad = 2 };
 struct GemmPlan {
-  CUtensorMap tmA;   // [E*Cbuf, K] bf16, box {64, 128}, 128B swizzle
-  CUtensorMap tmB;   // [E*K, N]    bf16, box {64, 64},  128B swizzle
-  CUtensorMap tmD;   // [E*Cbuf, N] bf16, box {64, 32},  128B swizzle (epilogue stores)
-  void* D;           // [E*Cbuf, N] bf16
+  // kGemmFwd   D[e,:n_e] = act(A[e,:n_e] . B[e])     A [E*Cbuf, K], B [E*K, N]
+  // kGemmDgrad D[e,:n_e] = (A[e,:n_e] . Bt[e]^T) (* [mask > 0])   Bt [E*N, K]
+  // kGemmWgrad D[e] = A[e,:n_e]^T . B[e,:n_e]        A [E*Cbuf, K=P], B [E*Cbuf, N=Q], D [E*P, Q]
+  CUtensorMap tmA;
+  CUtensorMap tmB;
+  CUtensorMap tmD;   // box {64, 32}, 128B swizzle (epilogue stores)
+  void* D;
+  const void* mask;  // kGemmDgrad: [E*Cbuf, N] bf16 values whose sign masks the result, or null
+  int kind;
   int E, K, N, BN;
   int64_t Cbuf;
   bool relu;
@@ -83,8 +90,42 @@ struct GemmPlan {
 };
 bool make_gemm_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, int64_t Cbuf, int K,
                     int N, bool relu);
+bool make_dgrad_plan(GemmPlan& p, const void* A, const void* Bt, void* D, const void* mask, int E,
+                     int64_t Cbuf, int K, int N);
+bool make_wgrad_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, int64_t Cbuf, int P,
+                     int Q);
 cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* err,
                             uint64_t wait_limit_ns, int num_sms, bool want_pair, cudaStream_t st);
+// backward.cu
+struct BwdArgs {
+  int S, M, H, E, k;
+  int64_t Cbuf;
+  bool bf16;
+  float a_aux, a_z;
+  const void* x;       // [S, M] act
+  const void* dy;      // [S, M] act
+  const float* Wg;     // [M, E]
+  const void* ybuf;    // [E*Cbuf, M] act (forward's expert outputs)
+  void* dybuf;         // [E*Cbuf, M] act (dY, later dX_e)
+  float* dl;           // [S, E]
+  float* dgate;        // [S, k]
+  float* part;         // split-K partials of dWg and dbias
+  size_t part_floats;
+  void* dx;            // [S, M] act
+  float* dWg;          // [M, E]
+  float* dbias;        // [E] or null
+};
+cudaError_t launch_gate_backward(const BwdArgs& a, const Routing& R, cudaStream_t st);
+cudaError_t launch_pad_zero(void* const* bufs, const int* widths, int nbuf, bool bf16, int E,
+                            int64_t Cbuf, const Routing& R, cudaStream_t st);
+cudaError_t launch_dx(const BwdArgs& a, const Routing& R, cudaStream_t st);
+cudaError_t launch_dwg(const BwdArgs& a, int num_sms, cudaStream_t st);
+size_t dwg_partial_floats(int S, int M, int E, int num_sms);
+// fp32 activations: the expert FFN's backward GEMMs on CUDA cores
+cudaError_t launch_ffn_bwd_f32(const float* xbuf, const float* hbuf, float* dybuf, float* dpre,
+                               const float* W1, const float* W2, float* dW1, float* dW2,
+                               const int32_t* nexp, int E, int64_t Cbuf, int M, int H,
+                               cudaStream_t st);
 // selftest.cu
 cudaError_t launch_wait_selftest(unsigned* flag, unsigned* err, uint64_t limit_ns, cudaStream_t st);
 

@@ -47,9 +47,24 @@ struct moe_layer {
   int64_t xmap_S;
   int64_t last_S;
   bool have_forward;
+  bool fwd_data;         // the expert buffers hold the last forward's (not a route-only call's)
   bool profiling;
+  // backward (moe_enable_backward)
+  void* bws;             // the backward's one device allocation
+  void* dybuf;           // [E, Cbuf, M] act: dY, then dX_e
+  void* dpre;            // [E, Cbuf, H] act: dP
+  float* dl;             // [S_max, E]
+  float* dgate;          // [S_max, k]
+  float* part;           // dW_g / dbias split-K partials
+  size_t part_floats;
+  GemmPlan plan_dp, plan_dx;        // dP = (dY W2^T)*[h>0],  dX = dP W1^T
+  GemmPlan plan_dw2, plan_dw1;      // dW2 = h^T dY,  dW1 = X^T dP (output pointers cached)
+  const void* dw2_ptr;
+  const void* dw1_ptr;
   cudaEvent_t ev[MOE_NUM_STAGES + 1];
+  cudaEvent_t evb[MOE_NUM_BWD_STAGES + 1];
   bool have_events;
+  bool have_backward_times;
   uint64_t wait_limit_ns;
 };
 
@@ -100,6 +115,7 @@ size_t carve(moe_layer* h, char* base) {
   R.off = c.take<int32_t>(k * nchunk * E);
   R.cnt = c.take<int32_t>(E);
   R.nexp = c.take<int32_t>(E);
+  R.first = c.take<int32_t>(E);
   R.psum = c.take<float>(nchunk * E);
   R.lse2 = c.take<float>(nchunk);
   R.losses = c.take<float>(2);
@@ -147,6 +163,12 @@ const char* moe_status_string(moe_status s) {
     case MOE_ERR_TIMEOUT: return "device wait timed out";
   }
   return "unknown status";
+}
+
+const char* moe_backward_stage_name(int32_t s) {
+  static const char* names[MOE_NUM_BWD_STAGES] = {"gate_bwd", "pad_zero", "dW2", "dP",
+                                                  "dW1",      "dX_e",     "dx",  "dWg"};
+  return (s >= 0 && s < MOE_NUM_BWD_STAGES) ? names[s] : "?";
 }
 
 const char* moe_stage_name(int32_t s) {
@@ -230,8 +252,10 @@ moe_status moe_create(moe_handle* out, int64_t S_max, int64_t M, int64_t H, int3
 moe_status moe_destroy(moe_handle h) {
   if (!h) return MOE_OK;
   cudaError_t ce = cudaDeviceSynchronize();
-  if (h->have_events)
+  if (h->have_events) {
     for (auto& e : h->ev) cudaEventDestroy(e);
+    for (auto& e : h->evb) cudaEventDestroy(e);
+  }
   cudaError_t fe = cudaFree(h->ws);
   delete h;
   if (ce != cudaSuccess) return from_cuda(ce);
@@ -255,6 +279,7 @@ moe_status moe_forward(moe_handle h, int64_t S, const void* x, void* y, void* st
   if (S > 0 && (!x || !y || !aligned(x, 16) || !aligned(y, 16))) return MOE_ERR_INVALID_ARG;
   h->last_S = S;
   h->have_forward = true;
+  h->fwd_data = true;
   if (S == 0) {
     MOE_TRY(cudaMemsetAsync(h->R.losses, 0, 2 * sizeof(float), st));
     return MOE_OK;
@@ -368,6 +393,7 @@ moe_status moe_route_from_logits(moe_handle h, int64_t S, const float* logits, v
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_S = S;
   h->have_forward = true;
+  h->fwd_data = false;
   if (S == 0) {
     MOE_TRY(cudaMemsetAsync(h->R.losses, 0, 2 * sizeof(float), st));
     return MOE_OK;
@@ -385,6 +411,7 @@ moe_status moe_set_profiling(moe_handle h, int32_t enable) {
   if (!h) return MOE_ERR_INVALID_ARG;
   if (enable && !h->have_events) {
     for (auto& e : h->ev) MOE_TRY(cudaEventCreate(&e));
+    for (auto& e : h->evb) MOE_TRY(cudaEventCreate(&e));
     h->have_events = true;
   }
   h->profiling = enable != 0;
@@ -396,6 +423,148 @@ moe_status moe_get_stage_times(moe_handle h, float* ms, int32_t n) {
   if (!h->profiling || !h->have_events || !h->have_forward || h->last_S == 0) return MOE_ERR_STATE;
   MOE_TRY(cudaEventSynchronize(h->ev[MOE_NUM_STAGES]));
   for (int i = 0; i < MOE_NUM_STAGES; ++i) MOE_TRY(cudaEventElapsedTime(&ms[i], h->ev[i], h->ev[i + 1]));
+  return MOE_OK;
+}
+
+moe_status moe_enable_backward(moe_handle h) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (h->bws) return MOE_OK;
+  const size_t as = act_bytes(h->act);
+  const int64_t rowsE = (int64_t)h->E * h->Cbuf;
+  h->part_floats = dwg_partial_floats((int)h->S_max, (int)h->M, h->E, h->num_sms);
+  Carver c{nullptr};
+  for (int pass = 0; pass < 2; ++pass) {
+    c.off = 0;
+    h->dybuf = c.take<char>((size_t)rowsE * h->M * as);
+    h->dpre = c.take<char>((size_t)rowsE * h->H * as);
+    h->dl = c.take<float>((size_t)h->S_max * h->E);
+    h->dgate = c.take<float>((size_t)h->S_max * h->k);
+    h->part = c.take<float>(h->part_floats);
+    if (pass == 0) {
+      const size_t bytes = c.off + 256;
+      cudaError_t ce = cudaMalloc(&h->bws, bytes);
+      if (ce != cudaSuccess) {
+        cudaGetLastError();
+        h->bws = nullptr;
+        return from_cuda(ce);
+      }
+      c.base = static_cast<char*>(h->bws);
+    }
+  }
+  if (h->act == MOE_BF16) {
+    const int M = (int)h->M, H = (int)h->H;
+    const bool ok = make_dgrad_plan(h->plan_dp, h->dybuf, h->W2, h->dpre, h->hbuf, h->E, h->Cbuf, M, H) &&
+                    make_dgrad_plan(h->plan_dx, h->dpre, h->W1, h->dybuf, nullptr, h->E, h->Cbuf, H, M);
+    if (!ok) {
+      cudaFree(h->bws);
+      h->bws = nullptr;
+      return MOE_ERR_CUDA;
+    }
+  }
+  h->dw1_ptr = h->dw2_ptr = nullptr;
+  return MOE_OK;
+}
+
+int32_t moe_kernels_per_backward(moe_handle h, int64_t S) {
+  if (!h || S <= 0) return 0;
+  return h->act == MOE_BF16 ? 9 : 8;
+}
+
+moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, float a_aux, float a_z,
+                        void* dx, float* dWg, float* dbias, void* dW1, void* dW2, void* stream) {
+  if (!h || S < 0 || S > h->S_max) return MOE_ERR_INVALID_ARG;
+  if (!h->bws || !h->have_forward || !h->fwd_data || S != h->last_S) return MOE_ERR_STATE;
+  if (!dWg || !dW1 || !dW2 || !aligned(dWg, 16) || !aligned(dW1, 16) || !aligned(dW2, 16) ||
+      (dbias && !aligned(dbias, 4)))
+    return MOE_ERR_INVALID_ARG;
+  if (S > 0 && (!x || !dy || !dx || !aligned(x, 16) || !aligned(dy, 16) || !aligned(dx, 16)))
+    return MOE_ERR_INVALID_ARG;
+  if (!isfinite(a_aux) || !isfinite(a_z)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t as = act_bytes(h->act);
+  const int E = h->E, M = (int)h->M, H = (int)h->H;
+  if (S == 0) {   // no tokens: every gradient is zero
+    MOE_TRY(cudaMemsetAsync(dWg, 0, (size_t)M * E * 4, st));
+    if (dbias) MOE_TRY(cudaMemsetAsync(dbias, 0, (size_t)E * 4, st));
+    MOE_TRY(cudaMemsetAsync(dW1, 0, (size_t)E * M * H * as, st));
+    MOE_TRY(cudaMemsetAsync(dW2, 0, (size_t)E * H * M * as, st));
+    return MOE_OK;
+  }
+  const bool bf16 = h->act == MOE_BF16;
+  BwdArgs a{};
+  a.S = (int)S;
+  a.M = M;
+  a.H = H;
+  a.E = E;
+  a.k = h->k;
+  a.Cbuf = h->Cbuf;
+  a.bf16 = bf16;
+  a.a_aux = a_aux;
+  a.a_z = a_z;
+  a.x = x;
+  a.dy = dy;
+  a.Wg = h->Wg;
+  a.ybuf = h->ybuf;
+  a.dybuf = h->dybuf;
+  a.dl = h->dl;
+  a.dgate = h->dgate;
+  a.part = h->part;
+  a.part_floats = h->part_floats;
+  a.dx = dx;
+  a.dWg = dWg;
+  a.dbias = dbias;
+  const Routing& R = h->R;
+  const bool prof = h->profiling && h->have_events;
+  auto mark = [&](int i) -> cudaError_t { return prof ? cudaEventRecord(h->evb[i], st) : cudaSuccess; };
+  h->have_backward_times = false;
+  MOE_TRY(mark(0));
+  MOE_TRY(launch_gate_backward(a, R, st));
+  MOE_TRY(mark(1));
+  if (bf16) {
+    if (h->dw2_ptr != dW2) {
+      if (!make_wgrad_plan(h->plan_dw2, h->hbuf, h->dybuf, dW2, E, h->Cbuf, H, M)) return MOE_ERR_CUDA;
+      h->dw2_ptr = dW2;
+    }
+    if (h->dw1_ptr != dW1) {
+      if (!make_wgrad_plan(h->plan_dw1, h->xbuf, h->dpre, dW1, E, h->Cbuf, M, H)) return MOE_ERR_CUDA;
+      h->dw1_ptr = dW1;
+    }
+    // the weight-gradient GEMMs reduce over whole 64-slot blocks: clear the rows
+    // between the kept count and the next multiple of 64
+    void* bufs[3] = {h->xbuf, h->hbuf, h->dybuf};
+    const int widths[3] = {M, H, M};
+    MOE_TRY(launch_pad_zero(bufs, widths, 3, true, E, h->Cbuf, R, st));
+    MOE_TRY(mark(2));
+    const uint64_t lim = h->wait_limit_ns;
+    MOE_TRY(launch_ffn_bf16(h->plan_dw2, R.nexp, R.err, lim, h->num_sms, false, st));
+    MOE_TRY(mark(3));
+    MOE_TRY(launch_ffn_bf16(h->plan_dp, R.nexp, R.err, lim, h->num_sms, false, st));
+    MOE_TRY(mark(4));
+    MOE_TRY(launch_ffn_bf16(h->plan_dw1, R.nexp, R.err, lim, h->num_sms, false, st));
+    MOE_TRY(mark(5));
+    MOE_TRY(launch_ffn_bf16(h->plan_dx, R.nexp, R.err, lim, h->num_sms, false, st));
+  } else {
+    MOE_TRY(mark(2));
+    MOE_TRY(launch_ffn_bwd_f32((const float*)h->xbuf, (const float*)h->hbuf, (float*)h->dybuf,
+                               (float*)h->dpre, (const float*)h->W1, (const float*)h->W2, (float*)dW1,
+                               (float*)dW2, R.nexp, E, h->Cbuf, M, H, st));
+    for (int i = 3; i <= 5; ++i) MOE_TRY(mark(i));   // the fp32 GEMMs are timed as one stage
+  }
+  MOE_TRY(mark(6));
+  MOE_TRY(launch_dx(a, R, st));
+  MOE_TRY(mark(7));
+  MOE_TRY(launch_dwg(a, h->num_sms, st));
+  MOE_TRY(mark(8));
+  h->have_backward_times = prof;
+  return MOE_OK;
+}
+
+moe_status moe_get_backward_stage_times(moe_handle h, float* ms, int32_t n) {
+  if (!h || !ms || n < MOE_NUM_BWD_STAGES) return MOE_ERR_INVALID_ARG;
+  if (!h->have_backward_times) return MOE_ERR_STATE;
+  MOE_TRY(cudaEventSynchronize(h->evb[MOE_NUM_BWD_STAGES]));
+  for (int i = 0; i < MOE_NUM_BWD_STAGES; ++i)
+    MOE_TRY(cudaEventElapsedTime(&ms[i], h->evb[i], h->evb[i + 1]));
   return MOE_OK;
 }
 

@@ -112,6 +112,7 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(int S, int E, int k, int
       f += part_f[g * E + j];
     }
     term += (double)f * P;
+    R.first[j] = (int32_t)f;                   // kept for the backward's d l_aux / d logits
   }
   const double fp = block_sum_f64(term, dsum);
   double zl = 0.0;

@@ -74,6 +74,7 @@ WORKLOADS = {
 
 # tensor ids of the counter-based stream
 TID_X, TID_WG, TID_W1, TID_W2 = 1, 2, 3, 4
+TID_DY = 5        # upstream gradient dL/dy of the backward
 
 _MASK64 = (1 << 64) - 1
 _GOLDEN = 0x9E3779B97F4A7C15
@@ -173,6 +174,12 @@ def make_inputs(w: Workload, device="cpu", S: int | None = None, weights: bool =
         W1 = normal((w.E, w.M, w.H), 1.0 / math.sqrt(w.M), w.seed, TID_W1, act, device)
         W2 = normal((w.E, w.H, w.M), 1.0 / math.sqrt(w.H), w.seed, TID_W2, act, device)
     return x, Wg, b, W1, W2
+
+
+def upstream_grad(w: Workload, device="cpu", S: int | None = None) -> torch.Tensor:
+    """dL/dy for the backward: [S, M] N(0, 1) entries in the activation dtype."""
+    S = w.S if S is None else S
+    return normal((S, w.M), 1.0, w.seed, TID_DY, w.torch_act, device)
 
 
 def expert_weights(w: Workload, e: int, device="cpu"):

@@ -3,6 +3,7 @@
     layer = MoeLayer(S_max, M, H, E, k, cf, Wg, bias, W1, W2)   # device tensors
     y = layer(x)                                                 # moe_forward
     l_aux, z = layer.aux_loss()                                  # moe_aux_loss
+    g = layer.backward(x, dy, a_aux, a_z)                        # moe_backward
 
 The tensors passed in are borrowed by the C library; this object keeps Python
 references to them so they outlive the handle.
@@ -43,6 +44,29 @@ class MoeLayer:
 
     def aux_loss(self, stream=None):
         return L.moe_aux_loss(self.h, stream)
+
+    def backward(self, x: torch.Tensor, dy: torch.Tensor, a_aux: float = 0.0, a_z: float = 0.0,
+                 stream=None) -> dict:
+        """Gradients of <dy, y> + a_aux*l_aux + a_z*z for the last forward (which took x).
+
+        Returns dx, dWg, dbias (None without a gate bias), dW1, dW2 as new tensors.
+        The backward workspace is allocated on the first call.
+        """
+        if not getattr(self, "_bwd", False):
+            L.moe_enable_backward(self.h)
+            self._bwd = True
+        for t in (x, dy):
+            if t.dtype != self.act or not t.is_contiguous() or t.dim() != 2 or t.shape[1] != self.M:
+                raise ValueError("x and dy must be contiguous [S, M] tensors of the activation dtype")
+        S = x.shape[0]
+        dev = x.device
+        dx = torch.empty_like(x)
+        dWg = torch.empty(self.M, self.E, dtype=torch.float32, device=dev)
+        dbias = torch.empty(self.E, dtype=torch.float32, device=dev) if self._keep[1] is not None else None
+        dW1 = torch.empty(self.E, self.M, self.H, dtype=self.act, device=dev)
+        dW2 = torch.empty(self.E, self.H, self.M, dtype=self.act, device=dev)
+        L.moe_backward(self.h, S, x, dy, a_aux, a_z, dx, dWg, dbias, dW1, dW2, stream)
+        return {"dx": dx, "dWg": dWg, "dbias": dbias, "dW1": dW1, "dW2": dW2}
 
     def capacity(self, S: int) -> int:
         return L.moe_get_capacity(self.h, S)

@@ -1,5 +1,5 @@
 /*
- * moe.h -- C ABI of a single-GPU GShard Mixture-of-Experts layer forward (B200, sm_100a).
+ * moe.h -- C ABI of a single-GPU GShard Mixture-of-Experts layer, forward and backward (B200, sm_100a).
  *
  * The layer (sources: "GShard: Scaling Giant Neural Networks with Conditional
  * Computation", section "Mixture-of-Experts Implementation" and its "Expert
@@ -83,7 +83,8 @@ enum { MOE_STAGE_ROUTER = 0, MOE_STAGE_SCAN = 1, MOE_STAGE_DISPATCH = 2, MOE_STA
  * Ownership: the weights and bias are BORROWED -- the caller keeps them alive
  * and unchanged until moe_destroy.  The handle owns its workspace (per-expert
  * buffers [E, min(C(S_max), S_max), M|H], routing tables and loss partials),
- * allocated here with one cudaMalloc; no later call allocates device memory.
+ * allocated here with one cudaMalloc; no later call allocates device memory
+ * except moe_enable_backward.
  * Must be called with the target device current.  On error *out is NULL.
  */
 MOE_API moe_status moe_create(moe_handle* out, int64_t S_max, int64_t M, int64_t H, int32_t E, int32_t k,
@@ -201,6 +202,80 @@ MOE_API moe_status moe_selftest_wait_timeout(int32_t limit_us, void* stream);
 MOE_API moe_status moe_assign_slots_noalloc(int64_t S, int32_t E, int32_t k, int64_t C,
                                             const int32_t* eidx_dev, int32_t* slot_dev,
                                             int32_t* cnt_dev, void* stream);
+
+/* ---- backward (training) ---------------------------------------------------- */
+
+/*
+ * moe_enable_backward -- allocate the workspace moe_backward needs (once per
+ * handle; a second call does nothing).  Inference-only handles never pay for
+ * these buffers:
+ *   dY  [E, Cbuf, M] act  (gradient of the expert outputs; reused for dX_e)
+ *   dP  [E, Cbuf, H] act  (gradient of the first layer's pre-activation)
+ *   dl  [S_max, E] fp32 (logit gradient), dgate [S_max, k] fp32, and the
+ *   split-K partials of the gate-weight gradient.
+ * Synchronous (cudaMalloc); call it outside stream capture.
+ */
+MOE_API moe_status moe_enable_backward(moe_handle h);
+
+/*
+ * moe_backward -- gradients of
+ *     L = <dy, y> + a_aux * l_aux + a_z * z
+ * ("GShard: Scaling Giant Neural Networks with Conditional Computation",
+ * "Training Methodology": the auxiliary loss joins the task loss with a small
+ * weight, here a_aux, and only experts that received tokens get a gradient)
+ * for the last moe_forward of this handle (same S, same x; the forward's saved
+ * routing and expert buffers are read, not changed, so moe_backward may run
+ * more than once per forward).  Enqueued on `stream`, no host synchronisation.
+ *
+ * The routing -- expert choices, slots, drops -- and the first-choice
+ * fractions f_j are piecewise constant and carry no gradient; every other step
+ * is differentiated exactly:
+ *   combine      dY_e[slot_r] = g_r dy[t],  dgate_r = <dy[t], y_e[slot_r]>
+ *                (both zero for a dropped assignment)
+ *   expert FFN   dW2[e] = relu(P_e)^T dY_e,  dP_e = (dY_e W2[e]^T) * [h_e > 0],
+ *                dW1[e] = X_e^T dP_e,  dx[t] += sum_{r kept} (dP_e W1[e]^T)[slot_r]
+ *   gates        dl[t, e_r] += g_r (dgate_r - sum_r' g_r' dgate_r')
+ *   l_aux        dl[t] += a_aux E/S p_t (f - <p_t, f>)
+ *   z-loss       dl[t] += a_z 2/S lse_t p_t
+ *   gate GEMM    dx += dl W_g^T,  dW_g = x^T dl,  dbias = sum_t dl
+ *
+ * x_dev     [S, M] act: the forward's input (unchanged since).
+ * dy_dev    [S, M] act: dL/dy.
+ * dx_dev    [S, M] act, overwritten.
+ * dWg_dev   [M, E] fp32, overwritten.      dbias_dev [E] fp32 overwritten, or NULL.
+ * dW1_dev   [E, M, H] act, overwritten.    dW2_dev   [E, H, M] act, overwritten
+ *           (experts that kept no token get zeros).
+ * Returns MOE_ERR_STATE unless moe_enable_backward succeeded and the last call
+ * that routed on this handle was a moe_forward of S tokens.  Every output
+ * pointer must be 16-byte aligned and must not alias the inputs.
+ */
+MOE_API moe_status moe_backward(moe_handle h, int64_t S, const void* x_dev, const void* dy_dev,
+                                float a_aux, float a_z, void* dx_dev, float* dWg_dev,
+                                float* dbias_dev, void* dW1_dev, void* dW2_dev, void* stream);
+
+/* Number of kernels one moe_backward of S tokens launches. */
+MOE_API int32_t moe_kernels_per_backward(moe_handle h, int64_t S);
+
+/* Stage indices of moe_get_backward_stage_times. */
+enum { MOE_BSTAGE_GATE = 0,     /* combine + gate backward: dY, dgate, dl */
+       MOE_BSTAGE_PAD = 1,      /* clearing the 64-row padding of the reduced buffers */
+       MOE_BSTAGE_DW2 = 2,      /* dW2 = h^T dY */
+       MOE_BSTAGE_DP = 3,       /* dP = (dY W2^T) * [h > 0] */
+       MOE_BSTAGE_DW1 = 4,      /* dW1 = X^T dP */
+       MOE_BSTAGE_DXE = 5,      /* dX_e = dP W1^T */
+       MOE_BSTAGE_DX = 6,       /* dx = gathered dX_e + dl W_g^T */
+       MOE_BSTAGE_DWG = 7,      /* dW_g = x^T dl, dbias (split-K + ordered sum) */
+       MOE_NUM_BWD_STAGES = 8 };
+
+/*
+ * With profiling on (moe_set_profiling), moe_backward records CUDA events on its
+ * stream between its stages; this synchronises and writes the last backward's
+ * per-stage milliseconds (MOE_NUM_BWD_STAGES values) to ms_host.
+ */
+MOE_API moe_status moe_get_backward_stage_times(moe_handle h, float* ms_host, int32_t n);
+
+/* Name of a MOE_BSTAGE_* index ("gate_bwd", "dW2", ...), or "?" */
+MOE_API const char* moe_backward_stage_name(int32_t stage);
 
 /* Static description of a status code (never NULL). */
 MOE_API const char* moe_status_string(moe_status s);

@@ -245,13 +245,16 @@ def route(logits, k: int, cf: float):
                            n=np.minimum(cnt, C), l_aux=l_aux, z=z, f=f, P=P)
 
 
-def forward(x, Wg, bias, W1, W2, k: int, cf: float, round_fp32: bool = True):
+def forward(x, Wg, bias, W1, W2, k: int, cf: float, round_fp32: bool = True, logits=None):
     """The whole layer forward on the CPU (small cases).
 
     Returns the `route` namespace plus logits, the per-expert buffers (xbuf,
-    pre-activation hpre, ybuf) and the output y[S, M] (float64).
+    pre-activation hpre, ybuf) and the output y[S, M] (float64).  Given
+    `logits` (fp32 [S, E], bias included) the routing uses them instead of
+    x . W_g + b, so that a check can hold the discrete routing decisions fixed.
     """
-    logits = gate_logits(x, Wg, bias, round_fp32)
+    if logits is None:
+        logits = gate_logits(x, Wg, bias, round_fp32)
     rt = route(logits, k, cf)
     S, E = logits.shape
     C = rt.C
@@ -297,24 +300,25 @@ def gates_backward(gates, ids, dgate, E: int):
     return dl
 
 
-def aux_loss_backward(p, f, E: int):
+def aux_loss_backward(p, f, E: int, S: int | None = None):
     """d l_aux / d logits with f_j held fixed (a count of argmax choices carries no gradient).
 
     l_aux = E sum_j f_j P_j, P_j = mean_t p[t, j]; through the softmax:
-    dl[t] = E/S * p_t * (f - <p_t, f>).  Returns dl[S, E].
+    dl[t] = E/S * p_t * (f - <p_t, f>).  Returns dl for the rows of p; S is the
+    batch's token count (default: the rows given).
     """
-    S = p.shape[0]
+    S = p.shape[0] if S is None else S
     return E / S * p * (f[None, :] - (p @ f)[:, None])
 
 
-def z_loss_backward(p, lse):
-    """d z / d logits for z = mean_t lse_t^2: dl[t] = 2/S * lse_t * p_t.  Returns dl[S, E]."""
-    S = p.shape[0]
+def z_loss_backward(p, lse, S: int | None = None):
+    """d z / d logits for z = mean_t lse_t^2: dl[t] = 2/S * lse_t * p_t (S as above)."""
+    S = p.shape[0] if S is None else S
     return 2.0 / S * lse[:, None] * p
 
 
 def backward(x, Wg, bias, W1, W2, k: int, cf: float, dy, a_aux: float = 0.0, a_z: float = 0.0,
-             round_fp32: bool = True):
+             round_fp32: bool = True, logits=None):
     """Gradients of  L = <dy, y> + a_aux * l_aux + a_z * z  with respect to x, W_g, b, W1, W2.
 
     The routing (expert choice, slots, drops) is piecewise constant and carries
@@ -328,9 +332,10 @@ def backward(x, Wg, bias, W1, W2, k: int, cf: float, dy, a_aux: float = 0.0, a_z
         give the logit gradient dl;
       gate GEMM ([blog] G(x) = Softmax(x . W_g)): dx += dl W_g^T, dW_g = x^T dl, db = sum_t dl.
     Returns a namespace with dx, dWg, dbias, dW1, dW2 (float64), the
-    intermediates dl, dgate and the forward namespace fwd.
+    intermediates dl, dgate, dybuf (the expert outputs' gradient) and the
+    forward namespace fwd.  `logits` as in `forward`.
     """
-    rt = forward(x, Wg, bias, W1, W2, k, cf, round_fp32)
+    rt = forward(x, Wg, bias, W1, W2, k, cf, round_fp32, logits)
     xf, Wgf, W1f, W2f, dyf = _f64(x), _f64(Wg), _f64(W1), _f64(W2), _f64(dy)
     S, E = rt.logits.shape
     dgate = np.zeros((S, k))
@@ -361,7 +366,8 @@ def backward(x, Wg, bias, W1, W2, k: int, cf: float, dy, a_aux: float = 0.0, a_z
     dx += dl @ Wgf.T
     dWg = xf.T @ dl
     dbias = dl.sum(axis=0)
-    return SimpleNamespace(dx=dx, dWg=dWg, dbias=dbias, dW1=dW1, dW2=dW2, dl=dl, dgate=dgate, fwd=rt)
+    return SimpleNamespace(dx=dx, dWg=dWg, dbias=dbias, dW1=dW1, dW2=dW2, dl=dl, dgate=dgate,
+                           dybuf=dybuf, fwd=rt)
 
 
 def outputs_for_tokens(tokens, x_rows, ids, gates, slot, expert_weights):

@@ -1,0 +1,258 @@
+"""Backward pass, CUDA path vs the oracle (GPU).
+
+The oracle routes the logits the GPU produced (the discrete routing decisions
+are held fixed, as in the forward checks) and differentiates in float64.
+
+Comparison: max|got - ref| / max|ref| per gradient, at most 1e-4 for fp32
+activations and 2e-2 for bf16 (the forward's output bar), after one allowance:
+the ReLU mask [h > 0] is a discontinuous decision taken on a pre-activation
+the GPU accumulates in fp32.  Where |pre| is within the fp32 accumulation
+bound K * 2^-23 * sum_i |x_i w_i| of zero, either decision is valid, and the
+two differ by |x| |dQ| in dW1 and |dQ| |W1| in dx (dQ = dY W2^T, the gradient
+before the mask).  The oracle-side slack for those ambiguous elements is
+subtracted before the comparison.  dW2, dWg and dbias are continuous in h and
+get no allowance.
+
+That bound is loose (it assumes every addition loses a full unit), so each
+gradient is also held to a global bar with no allowance at all: the Frobenius
+relative error ||got - ref|| / ||ref|| at most 1e-2 (bf16) / 1e-3 (fp32).  A
+rounding-decided mask flip moves one rank-one term of one expert, a small part
+of the whole norm, while a wrong term anywhere moves it by order one.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from gshard_top_gating_b200 import _lib as L
+from gshard_top_gating_b200.inputs import WORKLOADS, Workload, expert_weights, upstream_grad
+from tests import gpu_helpers as G
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+TOL_FRO = {"f32": 1e-3, "bf16": 1e-2}
+
+
+def _np(t) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def _excess_err(got, ref, slack=None) -> float:
+    d = np.abs(np.asarray(got, np.float64) - ref)
+    if slack is not None:
+        d = np.maximum(d - slack, 0.0)
+    den = np.abs(ref).max() if ref.size else 0.0
+    return float(d.max() / den) if den > 0 else float(d.max() if d.size else 0.0)
+
+
+def _fro_err(got, ref) -> float:
+    den = np.linalg.norm(ref)
+    num = np.linalg.norm(np.asarray(got, np.float64) - ref)
+    return float(num / den) if den > 0 else float(num)
+
+
+def _check_all(errs, act):
+    for name, e in errs.items():
+        bar = TOL_FRO[act] if name.startswith("fro ") else TOL[act]
+        assert e <= bar, (name, e)
+
+
+def _mask_slack(ref, W1, W2, K):
+    """Oracle-side bound on what an ambiguous ReLU decision can change."""
+    fwd = ref.fwd
+    E = W1.shape[0]
+    S, M = ref.dx.shape
+    s_dW1 = np.zeros_like(ref.dW1)
+    s_dxe = np.zeros_like(fwd.xbuf)
+    for e in range(E):
+        n = int(fwd.n[e])
+        if not n:
+            continue
+        xr = fwd.xbuf[e, :n]
+        bound = K * 2.0 ** -23 * (np.abs(xr) @ np.abs(W1[e]))
+        amb = np.abs(fwd.hpre[e, :n]) <= bound
+        if not amb.any():
+            continue
+        dq = np.abs(ref.dybuf[e, :n] @ W2[e].T) * amb
+        s_dW1[e] = np.abs(xr).T @ dq
+        s_dxe[e, :n] = dq @ np.abs(W1[e]).T
+    s_dx = np.zeros((S, M))
+    for r in range(fwd.slot.shape[1]):
+        keep = fwd.slot[:, r] >= 0
+        s_dx[keep] += s_dxe[fwd.ids[keep, r], fwd.slot[keep, r]]
+    return s_dW1, s_dx
+
+
+def backward_check(w, a_aux=0.7, a_z=0.3, S=None):
+    run = G.build(w, S=S)
+    out = G.forward(run)
+    G.check_routing(run, out)
+    dy = upstream_grad(w, device="cuda", S=run.S)
+    g = run.layer.backward(out.x, dy, a_aux, a_z)
+    torch.cuda.synchronize()
+    L.moe_check(run.layer.h)
+    W1, W2 = _np(run.W1), _np(run.W2)
+    ref = O.backward(_np(out.x), _np(run.Wg), None if run.b is None else _np(run.b), W1, W2, w.k,
+                     w.cf, _np(dy), a_aux, a_z, logits=out.logits)
+    s_dW1, s_dx = _mask_slack(ref, W1, W2, w.M)
+    errs = {
+        "dx": _excess_err(_np(g["dx"]), ref.dx, s_dx),
+        "dW1": _excess_err(_np(g["dW1"]), ref.dW1, s_dW1),
+        "dW2": _excess_err(_np(g["dW2"]), ref.dW2),
+        "dWg": _excess_err(_np(g["dWg"]), ref.dWg),
+    }
+    for name, r in (("dx", ref.dx), ("dW1", ref.dW1), ("dW2", ref.dW2), ("dWg", ref.dWg)):
+        errs["fro " + name] = _fro_err(_np(g[name]), r)
+    if run.b is not None:
+        errs["dbias"] = _excess_err(_np(g["dbias"]), ref.dbias)
+    else:
+        assert g["dbias"] is None
+    # experts that kept nothing get exactly zero weight gradients
+    empty = np.nonzero(ref.fwd.n == 0)[0]
+    for e in empty:
+        assert not g["dW1"][e].any() and not g["dW2"][e].any()
+    return run, out, g, ref, errs
+
+
+def test_f32_tiny_backward():
+    w = WORKLOADS["tiny"]
+    run, out, g, ref, errs = backward_check(w)
+    print(f"\ntiny f32 backward errors: {errs}")
+    _check_all(errs, "f32")
+    run.layer.close()
+
+
+def test_f32_backward_without_loss_terms():
+    w = WORKLOADS["tiny"].with_(S=200, cf=0.75)
+    run, out, g, ref, errs = backward_check(w, a_aux=0.0, a_z=0.0)
+    assert (out.slot < 0).any()
+    _check_all(errs, "f32")
+    run.layer.close()
+
+
+BF16_SHAPES = [
+    # (S, M, H, E, k, cf, skew_bias)
+    (600, 256, 512, 4, 2, 0.5, False),      # a third of the assignments dropped; 256-wide tiles
+    (1000, 256, 256, 8, 1, 1.0, False),     # top-1
+    (333, 128, 256, 16, 3, 1.0, False),     # ragged kept counts, k = 3
+    (257, 192, 320, 6, 2, 1.25, False),     # M, H = 64 mod 128: half-filled last weight-grad tiles
+    (512, 128, 128, 64, 2, 1.0, True),      # gate bias: many experts keep nothing (zero tiles)
+    (256, 256, 256, 32, 8, 1.25, False),    # top-8
+]
+
+
+@pytest.mark.parametrize("shape", BF16_SHAPES, ids=[str(s) for s in BF16_SHAPES])
+def test_bf16_backward(shape):
+    S, M, H, E, k, cf, skew = shape
+    w = Workload("bwd", S, M, H, E, k, cf, "bf16", skew_bias=skew, seed=31)
+    run, out, g, ref, errs = backward_check(w)
+    print(f"\n{shape}: {errs}")
+    _check_all(errs, "bf16")
+    run.layer.close()
+
+
+def test_backward_is_deterministic_and_repeatable():
+    w = Workload("det", 700, 256, 256, 8, 2, 1.0, "bf16", skew_bias=True, seed=32)
+    run = G.build(w)
+    x = run.x
+    y = run.layer(x)
+    dy = upstream_grad(w, device="cuda")
+    g1 = run.layer.backward(x, dy, 0.5, 0.1)
+    g2 = run.layer.backward(x, dy, 0.5, 0.1)      # a second backward of the same forward
+    torch.cuda.synchronize()
+    for key in g1:
+        assert torch.equal(g1[key], g2[key]), key
+    run.layer(x)                                   # a fresh forward, then again
+    g3 = run.layer.backward(x, dy, 0.5, 0.1)
+    torch.cuda.synchronize()
+    for key in g1:
+        assert torch.equal(g1[key], g3[key]), key
+    run.layer.close()
+
+
+def test_backward_call_order_is_checked():
+    w = Workload("order", 128, 128, 128, 4, 2, 1.0, "bf16", seed=33)
+    run = G.build(w)
+    dy = upstream_grad(w, device="cuda")
+    with pytest.raises(L.MoeError) as ei:             # no forward yet
+        run.layer.backward(run.x, dy)
+    assert ei.value.status == L.MOE_ERR_STATE
+    run.layer(run.x)
+    with pytest.raises(L.MoeError) as ei:             # a different token count
+        run.layer.backward(run.x[:64].contiguous(), dy[:64].contiguous())
+    assert ei.value.status == L.MOE_ERR_STATE
+    run.layer.route_from_logits(run.layer.logits(128))
+    with pytest.raises(L.MoeError) as ei:             # the buffers no longer hold a forward
+        run.layer.backward(run.x, dy)
+    assert ei.value.status == L.MOE_ERR_STATE
+    run.layer.close()
+
+
+def test_backward_mid_full_size():
+    """The mid workload at full size: every token's logit gradient (so dWg and
+    dbias in full), the weight gradients of four experts and dx of sampled
+    tokens, each from the oracle's step functions one expert or token at a time."""
+    w = WORKLOADS["mid"]
+    run = G.build(w)
+    out = G.forward(run)
+    rt = G.check_routing(run, out)
+    dy = upstream_grad(w, device="cuda")
+    a_aux, a_z = 0.01, 0.001
+    g = run.layer.backward(out.x, dy, a_aux, a_z)
+    torch.cuda.synchronize()
+    x = _np(out.x)
+    dyn = _np(dy)
+    Wg = _np(run.Wg)
+    S, E, k = w.S, w.E, w.k
+    dgate = np.zeros((S, k))
+    rng = np.random.default_rng(7)
+    sample_e = set(rng.choice(E, 4, replace=False).tolist())
+    tokens = np.unique(np.concatenate([[0, S - 1], rng.choice(S, 256, replace=False)]))
+    dxe_rows = {}
+    errs = {}
+    for e in range(E):
+        sel = [(t, r) for r in range(k) for t in np.nonzero((rt.ids[:, r] == e) & (rt.slot[:, r] >= 0))[0]]
+        if not sel:
+            continue
+        sel.sort(key=lambda tr: rt.slot[tr[0], tr[1]])
+        ts = np.array([t for t, _ in sel])
+        rs = np.array([r for _, r in sel])
+        W1e, W2e = (_np(t) for t in expert_weights(w, e))
+        xr = x[ts]
+        hpre = xr @ W1e
+        ye = O.expert_ffn(xr, W1e, W2e)
+        dgate[ts, rs] = np.sum(dyn[ts] * ye, axis=1)
+        dY = rt.gates[ts, rs][:, None] * dyn[ts]
+        want = np.isin(ts, tokens)
+        if e in sample_e or want.any():
+            dxe, dW1e, dW2e = O.expert_ffn_backward(xr, hpre, dY, W1e, W2e)
+            amb = np.abs(hpre) <= w.M * 2.0 ** -23 * (np.abs(xr) @ np.abs(W1e))
+            dq = np.abs(dY @ W2e.T) * amb
+            for i in np.nonzero(want)[0]:
+                dxe_rows[(ts[i], rs[i])] = (dxe[i], dq[i] @ np.abs(W1e).T)
+            if e in sample_e:
+                errs[f"dW1[{e}]"] = _excess_err(_np(g["dW1"][e]), dW1e, np.abs(xr).T @ dq)
+                errs[f"dW2[{e}]"] = _excess_err(_np(g["dW2"][e]), dW2e)
+                errs[f"fro dW1[{e}]"] = _fro_err(_np(g["dW1"][e]), dW1e)
+                errs[f"fro dW2[{e}]"] = _fro_err(_np(g["dW2"][e]), dW2e)
+    dl = O.gates_backward(rt.gates, rt.ids, dgate, E)
+    dl += a_aux * O.aux_loss_backward(rt.p, rt.f, E)
+    dl += a_z * O.z_loss_backward(rt.p, rt.lse)
+    errs["dWg"] = _excess_err(_np(g["dWg"]), x.T @ dl)
+    errs["fro dWg"] = _fro_err(_np(g["dWg"]), x.T @ dl)
+    errs["dbias"] = _excess_err(_np(g["dbias"]), dl.sum(axis=0)) if g["dbias"] is not None else 0.0
+    ref_dx = dl[tokens] @ Wg.T
+    slack = np.zeros_like(ref_dx)
+    for i, t in enumerate(tokens):
+        for r in range(k):
+            if (t, r) in dxe_rows:
+                ref_dx[i] += dxe_rows[(t, r)][0]
+                slack[i] += dxe_rows[(t, r)][1]
+    errs["dx"] = _excess_err(_np(g["dx"])[tokens], ref_dx, slack)
+    errs["fro dx"] = _fro_err(_np(g["dx"])[tokens], ref_dx)
+    print(f"\nmid backward errors: {errs}")
+    _check_all(errs, "bf16")
+    run.layer.close()
