@@ -279,7 +279,9 @@ def measure_backward(args, w, layer, x, y, flush, stream, pk, A, n_e):
         "ms_fwd": round(fwd_ms, 4), "ms_bwd": round(bwd_ms, 4), "steps": n,
         "expert_gemm_TFLOP/s": round(4 * 2.0 * A * w.M * w.H / (ffn / 1e3) / 1e12, 1) if ffn > 0 else None,
         "roofline": {"bound": b_, "kernel": dom, "achieved": round(ach, 2), "peak": peak, "unit": unit,
-                     "frac": round(ach / peak, 4)},
+                     "frac": round(ach / peak, 4), "peak_source": "measured, burst",
+                     "frac_of_sustained": (round(ach / pk["bf16_tflops_sustained"], 4)
+                                           if b_ == "tensor" and pk.get("bf16_tflops_sustained") else None)},
         "stages": stages,
         "gpu_launches": n * (L.moe_kernels_per_forward(layer.h, w.S) + L.moe_kernels_per_backward(layer.h, w.S)),
     }

@@ -15,11 +15,16 @@
 //              softmax over the chosen logits, "softmax-normalised top-2 weights")
 //   pad_zero   rows n_e .. ceil64(n_e) - 1 of the per-expert buffers the
 //              weight-gradient GEMMs reduce over are cleared
-//   dx         dx[t] = sum_{r kept} dX_e[slot_r] + dl[t] W_g^T      (tiled FFMA)
+//   dx         dx[t] = sum_{r kept} dX_e[slot_r] + dl[t] W_g^T
 //   dwg        dW_g = x^T dl and dbias = sum_t dl: split-K partials in a fixed
 //              order, then a fixed-order sum (no atomics: bitwise reproducible)
-//   f32 FFN    for fp32 activations the four expert GEMMs of the backward run on
-//              the same tiled FFMA kernel (tensor cores would lose fp32 accuracy)
+// bf16 activations: dl also leaves gate_bwd as a two-term bf16 split
+// (hi = bf16(dl), lo = bf16(dl - hi)), the operand of two tensor-core GEMMs in
+// ffn_tc.cu: dl_hi W_g,hi^T straight into dx (which dx_gather then adds the
+// expert rows to), and x^T [dl_hi | dl_lo] as fp32 split-K partials that
+// dwg_tc_reduce sums with the bias partials gate_bwd leaves per CTA.
+// fp32 activations: dx, dW_g and the four expert GEMMs of the backward run on
+// the tiled FFMA kernel below (tensor cores would lose fp32 accuracy).
 #include "common.cuh"
 #include "internal.h"
 
@@ -69,8 +74,16 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // ---------------------------------------------------------------- combine + gate backward
-template <typename T, int KM, int RE>
+template <typename T, int KM, int RE, bool TC>
 __global__ void __launch_bounds__(kThreads) gate_bwd_kernel(BwdArgs a, Routing R) {
+  __shared__ float bred[TC ? kThreads / 32 : 1][TC ? 32 * RE : 1];
+  float bacc[RE];
+#pragma unroll
+  for (int i = 0; i < RE; ++i) bacc[i] = 0.f;
+  if (TC && blockIdx.x == 0 && threadIdx.x == 0) {
+    a.cnt_rows[0] = a.S;                       // rows of the one-expert gate GEMMs
+    for (int z = 0; z < a.nsplit; ++z) a.cnt_rows[1 + z] = max(0, min(a.kchunk, a.S - z * a.kchunk));
+  }
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * kThreads) >> 5;
   const int nv = (int)((int64_t)a.M * sizeof(T) / 16);
@@ -167,27 +180,132 @@ __global__ void __launch_bounds__(kThreads) gate_bwd_kernel(BwdArgs a, Routing R
     }
     pf = warp_sum(pf);
     const float ca = a.a_aux * (float)E * invS, cz = a.a_z * 2.f * invS * lse;
-    float* drow = a.dl + (int64_t)t * E;
+    float dd[RE];
 #pragma unroll
     for (int i = 0; i < RE; ++i) {
       const int j = lane + 32 * i;
-      if (j >= E) continue;
       float d = ca * v[i] * (fj[i] - pf) + cz * v[i];
 #pragma unroll
       for (int r = 0; r < KM; ++r)
         if (r < k && er[r] == j) d += gr[r] * (dot[r] - inner);
-      drow[j] = d;
+      dd[i] = j < E ? d : 0.f;
+    }
+    if (TC) {
+      __nv_bfloat16* hrow = static_cast<__nv_bfloat16*>(a.dlb) + (int64_t)t * 2 * a.EPb;
+      const int nI = a.EPb / 32;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (i >= nI) break;
+        float d = 0.f;
+#pragma unroll
+        for (int q = 0; q < RE; ++q)
+          if (q == i) d = dd[q];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(d);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(d - __bfloat162float(hi));
+        hrow[lane + 32 * i] = hi;
+        hrow[a.EPb + lane + 32 * i] = lo;
+      }
+#pragma unroll
+      for (int i = 0; i < RE; ++i) bacc[i] += dd[i];
+    } else {
+      float* drow = a.dl + (int64_t)t * E;
+#pragma unroll
+      for (int i = 0; i < RE; ++i)
+        if (lane + 32 * i < E) drow[lane + 32 * i] = dd[i];
+    }
+  }
+  if (TC) {
+    // bias partial of this CTA: its warps' sums added in warp order
+    const int warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int i = 0; i < RE; ++i) bred[warp][lane + 32 * i] = bacc[i];
+    __syncthreads();
+    for (int j = threadIdx.x; j < E; j += kThreads) {
+      float sum = 0.f;
+      for (int w = 0; w < kThreads / 32; ++w) sum += bred[w][j];
+      a.bpart[(int64_t)blockIdx.x * E + j] = sum;
     }
   }
 }
 
 template <typename T, int KM>
 void gate_bwd_re(const BwdArgs& a, const Routing& R, int grid, cudaStream_t st) {
+  constexpr bool TC = sizeof(T) == 2;
   const int re = (a.E + 31) / 32;
-  if (re <= 1) gate_bwd_kernel<T, KM, 1><<<grid, kThreads, 0, st>>>(a, R);
-  else if (re <= 2) gate_bwd_kernel<T, KM, 2><<<grid, kThreads, 0, st>>>(a, R);
-  else if (re <= 4) gate_bwd_kernel<T, KM, 4><<<grid, kThreads, 0, st>>>(a, R);
-  else gate_bwd_kernel<T, KM, 8><<<grid, kThreads, 0, st>>>(a, R);
+  if (re <= 1) gate_bwd_kernel<T, KM, 1, TC><<<grid, kThreads, 0, st>>>(a, R);
+  else if (re <= 2) gate_bwd_kernel<T, KM, 2, TC><<<grid, kThreads, 0, st>>>(a, R);
+  else if (re <= 4) gate_bwd_kernel<T, KM, 4, TC><<<grid, kThreads, 0, st>>>(a, R);
+  else gate_bwd_kernel<T, KM, 8, TC><<<grid, kThreads, 0, st>>>(a, R);
+}
+
+// dx[t] += sum over kept choices of dX_e[slot] (r ascending, fp32), in place on
+// the bf16 dx that holds dl W_g^T; one warp per token, 16-byte vectors.
+template <int KM>
+__global__ void __launch_bounds__(kThreads) dx_gather_kernel(BwdArgs a, Routing R) {
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * kThreads) >> 5;
+  const int nv = a.M / 8;
+  const int k = a.k;
+  const __nv_bfloat16* dxe = static_cast<const __nv_bfloat16*>(a.dybuf);
+  for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < a.S; t += warps) {
+    int e = 0, s = -1;
+    if (lane < k) {
+      e = R.eidx[(int64_t)t * k + lane];
+      s = R.slot[(int64_t)t * k + lane];
+    }
+    const uint4* src[KM];
+#pragma unroll
+    for (int r = 0; r < KM; ++r) {
+      const int er = __shfl_sync(0xffffffffu, e, r);
+      const int sr = __shfl_sync(0xffffffffu, s, r);
+      src[r] = (r < k && sr >= 0) ? reinterpret_cast<const uint4*>(dxe + ((int64_t)er * a.Cbuf + sr) * a.M)
+                                  : nullptr;
+    }
+    uint4* row = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.dx) + (int64_t)t * a.M);
+    for (int v = lane; v < nv; v += 32) {
+      uint4 val[KM];
+#pragma unroll
+      for (int r = 0; r < KM; ++r)
+        if (src[r] != nullptr) val[r] = ld_nc_v4(src[r] + v);
+      float acc[8];
+      V16<__nv_bfloat16>::unpack(row[v], acc);
+#pragma unroll
+      for (int r = 0; r < KM; ++r) {
+        if (src[r] == nullptr) continue;
+        float f[8];
+        V16<__nv_bfloat16>::unpack(val[r], f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] += f[q];
+      }
+      row[v] = V16<__nv_bfloat16>::pack(acc);
+    }
+  }
+}
+
+// dW_g[m, e] = sum over splits z of (P[z][m][e] + P[z][m][EPb + e]) (hi and lo
+// halves of dl), dbias[e] = sum over gate_bwd's CTAs of their partials, both in order.
+__global__ void __launch_bounds__(kThreads) dwg_tc_reduce_kernel(const float* __restrict__ part,
+                                                                int nsplit, int M, int E, int EPb,
+                                                                const float* __restrict__ bpart,
+                                                                int nbpart, float* dWg, float* dbias) {
+  const int64_t n = (int64_t)M * E;
+  const int64_t zstride = (int64_t)M * 2 * EPb;
+  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n + E;
+       i += (int64_t)gridDim.x * kThreads) {
+    if (i < n) {
+      const int64_t m = i / E, e = i - m * E;
+      const float* p = part + m * 2 * EPb + e;
+      float s = 0.f;
+#pragma unroll 8
+      for (int z = 0; z < nsplit; ++z) s += __ldg(p + z * zstride) + __ldg(p + z * zstride + EPb);
+      dWg[i] = s;
+    } else if (dbias) {
+      const int64_t e = i - n;
+      float s = 0.f;
+      for (int b = 0; b < nbpart; ++b) s += bpart[(int64_t)b * E + e];
+      dbias[e] = s;
+    }
+  }
 }
 
 template <typename T>
@@ -387,12 +505,33 @@ int sms_of_device() {
 
 }  // namespace
 
+int gate_backward_grid(int S, int num_sms) {
+  const int want = (S + (kThreads / 32) - 1) / (kThreads / 32);
+  return want < num_sms * 4 ? want : num_sms * 4;
+}
+
 cudaError_t launch_gate_backward(const BwdArgs& a, const Routing& R, cudaStream_t st) {
-  const int sms = sms_of_device();
-  const int want = (a.S + (kThreads / 32) - 1) / (kThreads / 32);
-  const int grid = want < sms * 4 ? want : sms * 4;
+  const int grid = gate_backward_grid(a.S, sms_of_device());
   if (a.bf16) gate_bwd_k<__nv_bfloat16>(a, R, grid, st);
   else gate_bwd_k<float>(a, R, grid, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dx_gather(const BwdArgs& a, const Routing& R, cudaStream_t st) {
+  const int grid = gate_backward_grid(a.S, sms_of_device());
+  if (a.k <= 1) dx_gather_kernel<1><<<grid, kThreads, 0, st>>>(a, R);
+  else if (a.k <= 2) dx_gather_kernel<2><<<grid, kThreads, 0, st>>>(a, R);
+  else if (a.k <= 4) dx_gather_kernel<4><<<grid, kThreads, 0, st>>>(a, R);
+  else dx_gather_kernel<8><<<grid, kThreads, 0, st>>>(a, R);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dwg_tc_reduce(const BwdArgs& a, int nbpart, int num_sms, cudaStream_t st) {
+  const int64_t n = (int64_t)a.M * a.E + a.E;
+  int grid = (int)((n + kThreads - 1) / kThreads);
+  if (grid > 4 * num_sms) grid = 4 * num_sms;
+  dwg_tc_reduce_kernel<<<grid, kThreads, 0, st>>>(a.part, a.nsplit, a.M, a.E, a.EPb, a.bpart, nbpart,
+                                                  a.dWg, a.dbias);
   return cudaGetLastError();
 }
 
@@ -427,6 +566,24 @@ cudaError_t launch_dx(const BwdArgs& a, const Routing& R, cudaStream_t st) {
   g.k = a.k;
   if (a.bf16) return run_simt<float, float, __nv_bfloat16, kSgDx>(g, a.S, 1, R, st);
   return run_simt<float, float, float, kSgDx>(g, a.S, 1, R, st);
+}
+
+int dwg_tc_split_bound(int S, int M, int EPb, int num_sms) {
+  const int Q = 2 * EPb;
+  const int bn = Q % 256 == 0 ? 256 : (Q % 128 == 0 ? 128 : 64);
+  const int tiles = ((M + 127) / 128) * (Q / bn);
+  int ns = (num_sms + tiles - 1) / tiles;
+  const int maxs = (S + 63) / 64;
+  if (ns > maxs) ns = maxs;
+  return ns < 1 ? 1 : ns;
+}
+
+void dwg_tc_split(int S, int M, int EPb, int num_sms, int& nsplit, int& kchunk) {
+  const int ns = dwg_tc_split_bound(S, M, EPb, num_sms);
+  kchunk = ((S + ns - 1) / ns + 63) / 64 * 64;
+  if (kchunk < 64) kchunk = 64;
+  nsplit = (S + kchunk - 1) / kchunk;
+  if (nsplit < 1) nsplit = 1;
 }
 
 size_t dwg_partial_floats(int S, int M, int E, int num_sms) {

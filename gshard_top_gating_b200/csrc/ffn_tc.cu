@@ -79,7 +79,7 @@ struct TileIter {
 
 // Epilogue modes: plain store, ReLU, or the backward's ReLU mask (keep the
 // accumulator where the first layer's saved output h is > 0, else 0).
-enum { kEpiNone = 0, kEpiRelu = 1, kEpiMask = 2 };
+enum { kEpiNone = 0, kEpiRelu = 1, kEpiMask = 2, kEpiF32 = 3 };
 
 // 32 mask bits for 32 consecutive bf16 values of h: bit j set iff h[j] > 0
 // (bit patterns 0x0001 .. 0x7f80: positive finite or +inf).
@@ -110,18 +110,59 @@ template <int BN, int EPI>
 __device__ __forceinline__ void store_rows(const CUtensorMap* tmD, uint32_t tmem_rows,
                                            uint32_t stage, int row0, int col0, int lane,
                                            const uint16_t* mrow = nullptr, bool zero = false) {
+  if (EPI == kEpiF32) {
+    // fp32 result: 32 columns (128 bytes) per row per store, same swizzled staging
+#pragma unroll 1
+    for (int b = 0; b < BN / 32; ++b) {
+      if (lane == 0) bulk_wait_read0();
+      __syncwarp();
+      uint32_t r[32];
+      if (zero) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = 0u;
+      } else {
+        tmem_ld_32x32b_x32(tmem_rows + b * 32, r);
+        tmem_ld_wait();
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        st_shared_v4(stage + lane * 128 + ((j ^ (lane & 7)) << 4), r[4 * j], r[4 * j + 1], r[4 * j + 2],
+                     r[4 * j + 3]);
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmD, stage, col0 + b * 32, row0);
+        bulk_commit();
+      }
+    }
+    return;
+  }
+  // kEpiMask: the mask of 64-column chunk b + 1 is in flight while chunk b is stored
+  uint4 mnext[8];
+  if (EPI == kEpiMask) {
+    const uint4* mp = reinterpret_cast<const uint4*>(mrow);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mnext[j] = ld_nc_v4(mp + j);
+  }
 #pragma unroll 1
   for (int b = 0; b < BN / 64; ++b) {
+    uint4 mcur[8];
+    if (EPI == kEpiMask) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mcur[j] = mnext[j];
+      if (b + 1 < BN / 64) {
+        const uint4* mp = reinterpret_cast<const uint4*>(mrow + (b + 1) * 64);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mnext[j] = ld_nc_v4(mp + j);
+      }
+    }
     if (lane == 0) bulk_wait_read0();          // the previous store has read the staging tile
     __syncwarp();
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t keep = 0xFFFFFFFFu;
       if (EPI == kEpiMask) {
-        uint4 mv[4];
-        const uint4* mp = reinterpret_cast<const uint4*>(mrow + b * 64 + h * 32);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) mv[j] = ld_nc_v4(mp + j);
+        const uint4 mv[4] = {mcur[4 * h], mcur[4 * h + 1], mcur[4 * h + 2], mcur[4 * h + 3]};
         keep = positive_bits(mv);
       }
       uint32_t r[32];
@@ -168,8 +209,8 @@ template <int BN, int EPI, bool BKM>
 __global__ void __launch_bounds__(kThreads, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
-                  int64_t Cbuf, int K, int N, const uint16_t* __restrict__ mask, unsigned* err,
-                  uint64_t limit_ns) {
+                  int64_t Cbuf, int K, int N, const uint16_t* __restrict__ mask, int64_t row_limit,
+                  unsigned* err, uint64_t limit_ns) {
   using C = Cfg<BN>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -345,15 +386,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; it.decode(tile, e, mt, nt); tile += gridDim.x, ++i) {
       const int acc = i & 1;
       const uint32_t aph = (i >> 1) & 1;
+      const int row0 = (int)(e * Cbuf + mt * BM + q * 32);
+      const uint16_t* mrow = EPI == kEpiMask ? mask + (int64_t)(row0 + lane) * N + nt * BN : nullptr;
+      if (EPI == kEpiMask) {           // bring this row's mask into L2 while the MMAs run
+#pragma unroll
+        for (int c = 0; c < BN * 2 / 128; ++c) prefetch_l2(reinterpret_cast<const char*>(mrow) + c * 128);
+      }
       if (*abort_flag || !mbar_wait(tfull_bar(acc), aph, err, limit_ns)) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const int row0 = (int)(e * Cbuf + mt * BM + q * 32);
-      const uint16_t* mrow = EPI == kEpiMask ? mask + (int64_t)(row0 + lane) * N + nt * BN : nullptr;
-      store_rows<BN, EPI>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
-                          nt * BN, lane, mrow);
+      if (row0 < row_limit)           // a store box starts inside the tensor (TMA clips its tail)
+        store_rows<BN, EPI>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
+                            nt * BN, lane, mrow);
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
     }
@@ -377,10 +423,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Q = H).  The reduction runs over the expert's kept slots, so both operands are
 // read "MN-major" (slot rows, P or Q contiguous) in 64 x 64 TMA boxes and the MMA
 // takes them transposed.  The k-loop covers ceil(n_e / 64) blocks; rows n_e ..
-// ceil64(n_e) - 1 of both operands must hold zeros (the caller clears them).  An
-// expert with no kept slot gets D[e] = 0 (its tiles store zeros without an MMA).
+// ceil64(n_e) - 1 of both operands must hold zeros (the caller clears them), or lie
+// past the tensor maps' last row (TMA fills zeros).  An expert with no kept slot
+// gets D[e] = 0 (its tiles store zeros without an MMA).  EPI = kEpiF32 stores the
+// fp32 accumulator; the "experts" may also be consecutive row ranges of one
+// operand pair (a split of a long reduction, whose partial results the caller adds).
 // Tiles are (expert, p-tile, q-tile), q fastest; roles as in ffn_tc_kernel.
-template <int BN>
+template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     wgrad_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp,
@@ -547,8 +596,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
       }
       if (prow < P)
-        store_rows<BN, kEpiNone>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage,
-                                 row0, qt * BN, lane, nullptr, zero);
+        store_rows<BN, EPI>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
+                            qt * BN, lane, nullptr, zero);
       if (!zero) {
         tc_fence_before();
         mbar_arrive(tempty_bar(acc));
@@ -799,17 +848,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// 2-D row-major tensor of `outer` rows x `inner` elements (row pitch `pitch` bytes,
+// 0 = dense), 128-byte swizzle.
 bool encode_2d(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_in,
-               uint32_t box_out) {
+               uint32_t box_out, bool f32 = false, uint64_t pitch = 0) {
   auto fn = encode_fn();
   if (!fn) return false;
+  const uint64_t es = f32 ? 4 : 2;
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
+  cuuint64_t strides[1] = {pitch ? pitch : inner * es};
   cuuint32_t box[2] = {box_in, box_out};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(tm, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -831,14 +884,15 @@ cudaError_t launch_t(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint
   const size_t smem = Cfg<BN>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  const int64_t row_limit = p.row_limit > 0 ? p.row_limit : (int64_t)p.E * p.Cbuf;
   return launch_pdl(kern, dim3(num_sms), dim3(kThreads), smem, st, p.tmA, p.tmB, p.tmD, nexp, p.E,
-                    p.Cbuf, p.K, p.N, static_cast<const uint16_t*>(p.mask), err, limit_ns);
+                    p.Cbuf, p.K, p.N, static_cast<const uint16_t*>(p.mask), row_limit, err, limit_ns);
 }
 
-template <int BN>
+template <int BN, int EPI>
 cudaError_t launch_w(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint64_t limit_ns,
                      int num_sms, cudaStream_t st) {
-  auto kern = wgrad_tc_kernel<BN>;
+  auto kern = wgrad_tc_kernel<BN, EPI>;
   const size_t smem = Cfg<BN>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -888,7 +942,7 @@ bool make_dgrad_plan(GemmPlan& p, const void* A, const void* Bt, void* D, const 
 }
 
 bool make_wgrad_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, int64_t Cbuf, int P,
-                     int Q) {
+                     int Q, bool f32out, int64_t rows_ab) {
   p = GemmPlan{};
   p.kind = kGemmWgrad;
   p.E = E;
@@ -896,21 +950,51 @@ bool make_wgrad_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, 
   p.K = P;                             // rows of each expert's result
   p.N = Q;
   p.D = D;
+  p.f32out = f32out;
   p.BN = pick_bn(Q);
   if (P % 64 || Q % 64 || Cbuf % BK) return false;
-  if (!encode_2d(&p.tmA, A, (uint64_t)P, (uint64_t)E * Cbuf, 64, BK)) return false;
-  if (!encode_2d(&p.tmB, B, (uint64_t)Q, (uint64_t)E * Cbuf, 64, BK)) return false;
-  if (!encode_2d(&p.tmD, D, (uint64_t)Q, (uint64_t)E * P, 64, 32)) return false;
+  const uint64_t rows = rows_ab > 0 ? (uint64_t)rows_ab : (uint64_t)E * Cbuf;
+  if (!encode_2d(&p.tmA, A, (uint64_t)P, rows, 64, BK)) return false;
+  if (!encode_2d(&p.tmB, B, (uint64_t)Q, rows, 64, BK)) return false;
+  if (!encode_2d(&p.tmD, D, (uint64_t)Q, (uint64_t)E * P, f32out ? 32 : 64, 32, f32out)) return false;
+  return true;
+}
+
+bool make_gate_dx_plan(GemmPlan& p, const void* dlb, int64_t S, int EPb, const void* wsplit,
+                       int EPr, void* dx, int M) {
+  p = GemmPlan{};
+  p.kind = kGemmFwd;
+  p.E = 1;
+  p.Cbuf = S;
+  p.K = EPb;
+  p.N = M;
+  p.D = dx;
+  p.BN = pick_bn(M);
+  if (EPb % BK || M % 64 || 3 * EPr < EPb) return false;
+  // A: the hi half of dl's bf16 split, rows of 2*EPb elements
+  if (!encode_2d(&p.tmA, dlb, (uint64_t)EPb, (uint64_t)S, BK, BM, false, (uint64_t)EPb * 4)) return false;
+  // B: W_g's hi part [EPr, M] (E contiguous rows past E are zero; rows EPr.. of the
+  // next part only meet zero columns of A)
+  if (!encode_2d(&p.tmB, wsplit, (uint64_t)M, (uint64_t)3 * EPr, 64, BK)) return false;
+  if (!encode_2d(&p.tmD, dx, (uint64_t)M, (uint64_t)S, 64, 32)) return false;
+  p.row_limit = S;
   return true;
 }
 
 cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* err,
                             uint64_t wait_limit_ns, int num_sms, bool want_pair, cudaStream_t st) {
   if (p.kind == kGemmWgrad) {
+    if (p.f32out) {
+      switch (p.BN) {
+        case 256: return launch_w<256, kEpiF32>(p, nexp, err, wait_limit_ns, num_sms, st);
+        case 128: return launch_w<128, kEpiF32>(p, nexp, err, wait_limit_ns, num_sms, st);
+        default: return launch_w<64, kEpiF32>(p, nexp, err, wait_limit_ns, num_sms, st);
+      }
+    }
     switch (p.BN) {
-      case 256: return launch_w<256>(p, nexp, err, wait_limit_ns, num_sms, st);
-      case 128: return launch_w<128>(p, nexp, err, wait_limit_ns, num_sms, st);
-      default: return launch_w<64>(p, nexp, err, wait_limit_ns, num_sms, st);
+      case 256: return launch_w<256, kEpiNone>(p, nexp, err, wait_limit_ns, num_sms, st);
+      case 128: return launch_w<128, kEpiNone>(p, nexp, err, wait_limit_ns, num_sms, st);
+      default: return launch_w<64, kEpiNone>(p, nexp, err, wait_limit_ns, num_sms, st);
     }
   }
   if (p.kind == kGemmDgrad) {

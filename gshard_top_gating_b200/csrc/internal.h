@@ -87,13 +87,20 @@ struct GemmPlan {
   int64_t Cbuf;
   bool relu;
   bool pair;         // the CTA-pair (cta_group::2, 256 x 256 tile) kernel can run (N % 256 == 0)
+  bool f32out;       // kGemmWgrad: D is fp32
+  int64_t row_limit; // rows of D (0 = E*Cbuf): stores of 32-row groups starting past it are skipped
 };
 bool make_gemm_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, int64_t Cbuf, int K,
                     int N, bool relu);
 bool make_dgrad_plan(GemmPlan& p, const void* A, const void* Bt, void* D, const void* mask, int E,
                      int64_t Cbuf, int K, int N);
+// rows_ab: rows of the A / B tensor maps (0 = E*Cbuf); rows past it read as zeros
 bool make_wgrad_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, int64_t Cbuf, int P,
-                     int Q);
+                     int Q, bool f32out = false, int64_t rows_ab = 0);
+// dx = dl_hi . W_g,hi^T as a one-expert forward GEMM: A = dlb [S, 2*EPb] (hi half),
+// B = the router's W_g split [3*EPr, M], D = dx [S, M]
+bool make_gate_dx_plan(GemmPlan& p, const void* dlb, int64_t S, int EPb, const void* wsplit,
+                       int EPr, void* dx, int M);
 cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* err,
                             uint64_t wait_limit_ns, int num_sms, bool want_pair, cudaStream_t st);
 // backward.cu
@@ -114,13 +121,26 @@ struct BwdArgs {
   void* dx;            // [S, M] act
   float* dWg;          // [M, E]
   float* dbias;        // [E] or null
+  // bf16 activations (tensor-core gate gradients)
+  void* dlb;           // [S, 2*EPb] bf16: dl hi in columns [0, EPb), lo in [EPb, 2*EPb)
+  int EPb;             // E rounded up to 64
+  float* bpart;        // [gate_bwd CTAs, E] bias partials
+  int32_t* cnt_rows;   // [1 + nsplit]: S, then the rows of each dW_g split
+  int nsplit, kchunk;  // dW_g split-K: nsplit splits of kchunk tokens
 };
 cudaError_t launch_gate_backward(const BwdArgs& a, const Routing& R, cudaStream_t st);
 cudaError_t launch_pad_zero(void* const* bufs, const int* widths, int nbuf, bool bf16, int E,
                             int64_t Cbuf, const Routing& R, cudaStream_t st);
 cudaError_t launch_dx(const BwdArgs& a, const Routing& R, cudaStream_t st);
+int gate_backward_grid(int S, int num_sms);
+cudaError_t launch_dx_gather(const BwdArgs& a, const Routing& R, cudaStream_t st);
+cudaError_t launch_dwg_tc_reduce(const BwdArgs& a, int nbpart, int num_sms, cudaStream_t st);
 cudaError_t launch_dwg(const BwdArgs& a, int num_sms, cudaStream_t st);
 size_t dwg_partial_floats(int S, int M, int E, int num_sms);
+// bf16 dW_g: split-K over tokens, about one tile per SM; splits of kchunk (a multiple
+// of 64) tokens.  nsplit(S) <= dwg_tc_split_bound(S_max) for every S <= S_max.
+void dwg_tc_split(int S, int M, int EPb, int num_sms, int& nsplit, int& kchunk);
+int dwg_tc_split_bound(int S, int M, int EPb, int num_sms);
 // fp32 activations: the expert FFN's backward GEMMs on CUDA cores
 cudaError_t launch_ffn_bwd_f32(const float* xbuf, const float* hbuf, float* dybuf, float* dpre,
                                const float* W1, const float* W2, float* dW1, float* dW2,

@@ -61,6 +61,15 @@ struct moe_layer {
   GemmPlan plan_dw2, plan_dw1;      // dW2 = h^T dY,  dW1 = X^T dP (output pointers cached)
   const void* dw2_ptr;
   const void* dw1_ptr;
+  // bf16: tensor-core gate gradients
+  int EPb;                          // E rounded up to 64
+  void* dlb;                        // [S_max, 2*EPb] bf16 split of dl
+  float* bpart;                     // [4*num_sms, E] bias partials
+  int32_t* cnt_rows;                // [1 + max splits]
+  GemmPlan plan_gdx, plan_dwg;      // dx = dl W_g^T;  dW_g partials = x^T [dl_hi | dl_lo]
+  const void* gdx_ptr;
+  const void* dwg_ptr;
+  int64_t gdx_S, dwg_S;
   cudaEvent_t ev[MOE_NUM_STAGES + 1];
   cudaEvent_t evb[MOE_NUM_BWD_STAGES + 1];
   bool have_events;
@@ -431,15 +440,22 @@ moe_status moe_enable_backward(moe_handle h) {
   if (h->bws) return MOE_OK;
   const size_t as = act_bytes(h->act);
   const int64_t rowsE = (int64_t)h->E * h->Cbuf;
-  h->part_floats = dwg_partial_floats((int)h->S_max, (int)h->M, h->E, h->num_sms);
+  const bool bf16 = h->act == MOE_BF16;
+  h->EPb = (h->E + 63) / 64 * 64;
+  const int ns_max = dwg_tc_split_bound((int)h->S_max, (int)h->M, h->EPb, h->num_sms);
+  h->part_floats = bf16 ? (size_t)ns_max * h->M * 2 * h->EPb
+                        : dwg_partial_floats((int)h->S_max, (int)h->M, h->E, h->num_sms);
   Carver c{nullptr};
   for (int pass = 0; pass < 2; ++pass) {
     c.off = 0;
     h->dybuf = c.take<char>((size_t)rowsE * h->M * as);
     h->dpre = c.take<char>((size_t)rowsE * h->H * as);
-    h->dl = c.take<float>((size_t)h->S_max * h->E);
+    h->dl = bf16 ? nullptr : c.take<float>((size_t)h->S_max * h->E);
     h->dgate = c.take<float>((size_t)h->S_max * h->k);
     h->part = c.take<float>(h->part_floats);
+    h->dlb = bf16 ? c.take<char>((size_t)h->S_max * 2 * h->EPb * 2) : nullptr;
+    h->bpart = bf16 ? c.take<float>((size_t)4 * h->num_sms * h->E) : nullptr;
+    h->cnt_rows = bf16 ? c.take<int32_t>((size_t)1 + ns_max) : nullptr;
     if (pass == 0) {
       const size_t bytes = c.off + 256;
       cudaError_t ce = cudaMalloc(&h->bws, bytes);
@@ -462,12 +478,14 @@ moe_status moe_enable_backward(moe_handle h) {
     }
   }
   h->dw1_ptr = h->dw2_ptr = nullptr;
+  h->gdx_ptr = h->dwg_ptr = nullptr;
+  h->gdx_S = h->dwg_S = -1;
   return MOE_OK;
 }
 
 int32_t moe_kernels_per_backward(moe_handle h, int64_t S) {
   if (!h || S <= 0) return 0;
-  return h->act == MOE_BF16 ? 9 : 8;
+  return h->act == MOE_BF16 ? 10 : 8;
 }
 
 moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, float a_aux, float a_z,
@@ -513,6 +531,26 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
   a.dx = dx;
   a.dWg = dWg;
   a.dbias = dbias;
+  if (bf16) {
+    a.dlb = h->dlb;
+    a.EPb = h->EPb;
+    a.bpart = h->bpart;
+    a.cnt_rows = h->cnt_rows;
+    dwg_tc_split((int)S, M, h->EPb, h->num_sms, a.nsplit, a.kchunk);
+    if ((size_t)a.nsplit * M * 2 * h->EPb > h->part_floats) return MOE_ERR_STATE;
+    if (h->gdx_ptr != dx || h->gdx_S != S) {
+      if (!make_gate_dx_plan(h->plan_gdx, h->dlb, S, h->EPb, h->wsplit, router_tc_pad(E), dx, M))
+        return MOE_ERR_CUDA;
+      h->gdx_ptr = dx;
+      h->gdx_S = S;
+    }
+    if (h->dwg_ptr != x || h->dwg_S != S) {
+      if (!make_wgrad_plan(h->plan_dwg, x, h->dlb, h->part, a.nsplit, a.kchunk, M, 2 * h->EPb, true, S))
+        return MOE_ERR_CUDA;
+      h->dwg_ptr = x;
+      h->dwg_S = S;
+    }
+  }
   const Routing& R = h->R;
   const bool prof = h->profiling && h->have_events;
   auto mark = [&](int i) -> cudaError_t { return prof ? cudaEventRecord(h->evb[i], st) : cudaSuccess; };
@@ -551,9 +589,18 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
     for (int i = 3; i <= 5; ++i) MOE_TRY(mark(i));   // the fp32 GEMMs are timed as one stage
   }
   MOE_TRY(mark(6));
-  MOE_TRY(launch_dx(a, R, st));
-  MOE_TRY(mark(7));
-  MOE_TRY(launch_dwg(a, h->num_sms, st));
+  if (bf16) {
+    const uint64_t lim = h->wait_limit_ns;
+    MOE_TRY(launch_ffn_bf16(h->plan_gdx, h->cnt_rows, R.err, lim, h->num_sms, false, st));
+    MOE_TRY(launch_dx_gather(a, R, st));
+    MOE_TRY(mark(7));
+    MOE_TRY(launch_ffn_bf16(h->plan_dwg, h->cnt_rows + 1, R.err, lim, h->num_sms, false, st));
+    MOE_TRY(launch_dwg_tc_reduce(a, gate_backward_grid((int)S, h->num_sms), h->num_sms, st));
+  } else {
+    MOE_TRY(launch_dx(a, R, st));
+    MOE_TRY(mark(7));
+    MOE_TRY(launch_dwg(a, h->num_sms, st));
+  }
   MOE_TRY(mark(8));
   h->have_backward_times = prof;
   return MOE_OK;
