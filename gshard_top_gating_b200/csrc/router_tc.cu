@@ -18,11 +18,12 @@
 // it into a second TMEM region with ordinary round-to-nearest fp32 adds.  The
 // logits so carry fp32-level error at tensor-core speed.
 //
-// One CTA = 128 tokens x EP experts (E padded to 32/64/128/256), 256 threads:
-// warp 0 TMA producer (x tile 128x64 + three W_g parts EPx64 per stage, K-major,
+// One CTA = 128 tokens (64 for small batches with E <= 64) x EP experts (E padded
+// to 32/64/128/256), 512 threads:
+// warp 0 TMA producer (x tile TTx64 + three W_g parts EPx64 per stage, K-major,
 // 128B swizzle), warp 1 TMEM owner and single-thread MMA issuer, warps 2-5 fold
 // the K-segments (one token row per thread, as TMEM lanes dictate) and leave the
-// final logits tile in shared memory.  Then all eight warps route warp-per-token
+// final logits tile in shared memory.  Then all sixteen warps route warp-per-token
 // (lanes over experts, shuffle max / sum / argmax, ties to the lower index) and
 // write the same per-64-token chunk tables (probability sums, lse^2 sums,
 // rank-r histograms, local ranks) as the CUDA-core router.
@@ -35,25 +36,31 @@
 
 namespace moe {
 
+int router_tokens_per_cta(int E, int S);
+
 namespace {
 
 constexpr int BM = 128, BK = 64;
 constexpr int kThreads = 512;   // 16 warps: all route; warps 0/1/2-5 also load / issue / fold
 constexpr uint32_t A_BYTES = BM * BK * 2;
-constexpr int kPrefetchX = 12;     // L2 prefetch distance of the token tiles, k-blocks
 constexpr int kSegBlocks = 8;      // k-blocks (of 64) accumulated before each fp32 round-to-nearest add
 
-template <int EP>
+template <int EP, int TT_>
 struct RCfg {
-  // tokens per CTA: 64 for small E (twice the CTAs stream x; the MMA keeps M=128
-  // and its upper 64 accumulator rows are ignored), 128 otherwise
-  static constexpr int TT = EP <= 64 ? 64 : 128;
+  // tokens per CTA: 128, or 64 when 128-token CTAs would not fill the SMs (twice
+  // the CTAs stream x; the MMA keeps M=128 and its upper 64 accumulator rows are
+  // ignored)
+  static constexpr int TT = TT_;
   static constexpr int NCH = TT / kChunk;                       // 64-token chunks per CTA
   static constexpr uint32_t X_BYTES = TT * BK * 2;              // bytes TMA writes into the A tile
   static constexpr uint32_t PART_BYTES = EP * BK * 2;           // one W_g part, EP x 64 bf16
   static constexpr uint32_t STAGE_BYTES = A_BYTES + 3 * PART_BYTES;
   static constexpr uint32_t TX_BYTES = X_BYTES + 3 * PART_BYTES;
   static constexpr int STAGES = (EP == 256) ? 2 : (EP == 128 ? 3 : (EP == 64 ? 5 : 7));
+  // L2 prefetch distance of the token tiles, in k-blocks.  With 3 or more stages in
+  // flight the prefetches only queue ahead of the loads in the TMA unit (measured:
+  // slower); with 2 stages (E > 128) they hide the DRAM latency of x.
+  static constexpr int PREFETCH_X = STAGES <= 2 ? 12 : 0;
   static constexpr uint32_t TMEM_COLS = 2 * EP;        // accumulator + running sum
   // epilogue scratch reuses the stage buffers: logits L [TT][EP+1] f32 (padded row),
   // per-warp probability sums red [16][EP] f32, per-warp lse^2 [16], sel [TT][8] i32,
@@ -80,12 +87,12 @@ __device__ __forceinline__ uint32_t idesc_router() {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(EP >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
-template <int EP>
+template <int EP, int TT>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const float* __restrict__ bias, int S, int M, int E, int k, int nchunk,
                      Routing R, uint64_t limit_ns) {
-  using C = RCfg<EP>;
+  using C = RCfg<EP, TT>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -131,10 +138,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_par = 0;
       bool ok = true;
-      // x streams from DRAM once: prefetch it into L2 kPrefetchX k-blocks ahead
-      for (int kb = 0; kb < KB && kb < kPrefetchX; ++kb) tma_prefetch_l2_2d(&tmX, kb * BK, tok0);
+      // x streams from DRAM once: with few stages, prefetch it into L2 ahead of the loads
+      constexpr int PF = C::PREFETCH_X;
+      for (int kb = 0; kb < KB && kb < PF; ++kb) tma_prefetch_l2_2d(&tmX, kb * BK, tok0);
       for (int kb = 0; kb < KB; ++kb) {
-        if (kb + kPrefetchX < KB) tma_prefetch_l2_2d(&tmX, (kb + kPrefetchX) * BK, tok0);
+        if (PF > 0 && kb + PF < KB) tma_prefetch_l2_2d(&tmX, (kb + PF) * BK, tok0);
         if (*abort_flag || !mbar_wait(empty_bar(s), ph ^ 1u, R.err, limit_ns)) {
           *abort_flag = 1;
           ok = false;
@@ -248,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < EP; ++c) Ls[row * C::LD + c] = 0.f;
   }
 
-  // ------------------------------------------------------------ route, all 8 warps
+  // ------------------------------------------------------------ route, all 16 warps
   __syncthreads();
   {
     float* Ls = reinterpret_cast<float*>(gbase + C::L_OFF);
@@ -385,22 +393,50 @@ bool encode_kmajor(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t ou
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int EP, int TT>
+cudaError_t launch_tt(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias, int S, int M,
+                      int E, int k, const Routing& R, uint64_t limit_ns, cudaStream_t st) {
+  auto kern = router_tc_kernel<EP, TT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)RCfg<EP, TT>::SMEM);
+  if (e != cudaSuccess) return e;
+  const int nchunk = (S + kChunk - 1) / kChunk;
+  kern<<<(S + TT - 1) / TT, kThreads, RCfg<EP, TT>::SMEM, st>>>(tmX, tmW, bias, S, M, E, k, nchunk, R,
+                                                                limit_ns);
+  return cudaGetLastError();
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!cached[dev]) {
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = sms;
+  }
+  return cached[dev];
+}
+
 template <int EP>
 cudaError_t launch_t(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias, int S, int M,
                      int E, int k, const Routing& R, uint64_t limit_ns, cudaStream_t st) {
-  auto kern = router_tc_kernel<EP>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)RCfg<EP>::SMEM);
-  if (e != cudaSuccess) return e;
-  const int nchunk = (S + kChunk - 1) / kChunk;
-  kern<<<(S + RCfg<EP>::TT - 1) / RCfg<EP>::TT, kThreads, RCfg<EP>::SMEM, st>>>(
-      tmX, tmW, bias, S, M, E, k, nchunk, R, limit_ns);
-  return cudaGetLastError();
+  if (router_tokens_per_cta(E, S) == 128)
+    return launch_tt<EP, 128>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);
+  return launch_tt<EP, 64>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);
 }
 
 }  // namespace
 
 int router_tc_pad(int E) { return E <= 32 ? 32 : (E <= 64 ? 64 : (E <= 128 ? 128 : 256)); }
+
+// 128 tokens per CTA halves the W_g bytes each token costs; 64 only for E <= 64 and
+// batches too small for 128-token CTAs to fill every SM once.
+int router_tokens_per_cta(int E, int S) {
+  if (router_tc_pad(E) > 64) return 128;
+  return (S + 127) / 128 >= sm_count() ? 128 : 64;
+}
 
 cudaError_t split_gate_weights(const float* Wg, int M, int E, void* out3, cudaStream_t st) {
   const int EP = router_tc_pad(E);
@@ -416,8 +452,7 @@ bool make_router_wmap(CUtensorMap* tm, const void* wsplit, int M, int E) {
 }
 
 bool make_router_xmap(CUtensorMap* tm, const void* x, int S, int M, int E) {
-  const int TT = router_tc_pad(E) <= 64 ? 64 : 128;      // = RCfg<EP>::TT
-  return encode_kmajor(tm, x, (uint64_t)M, (uint64_t)S, (uint32_t)TT);
+  return encode_kmajor(tm, x, (uint64_t)M, (uint64_t)S, (uint32_t)router_tokens_per_cta(E, S));
 }
 
 cudaError_t launch_router_tc(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias, int S,
