@@ -637,11 +637,14 @@ constexpr size_t SMEM =
 constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;            // shared::cluster address -> rank 0
 }  // namespace pairk
 
-template <bool RELU>
+// EPI and BKM as in ffn_tc_kernel; with BKM each CTA's B box is its 128 rows of
+// the [N, K] weight (box {64, 128}).
+template <int EPI, bool BKM>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ffn_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
-                   int64_t Cbuf, int K, int N, unsigned* err, uint64_t limit_ns) {
+                   int64_t Cbuf, int K, int N, const uint16_t* __restrict__ mask, unsigned* err,
+                   uint64_t limit_ns) {
   using namespace pairk;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -740,9 +743,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t fb = full_bar(s) & kPeerBitMask;     // the leader's full barrier
           if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * STAGE_BYTES);
           tma_load_2d_pair(sa, &tmA, fb, kb * BK, rowA);
+          if (BKM) {
+            tma_load_2d_pair(sa + A_BYTES, &tmB, fb, kb * BK, e * N + colB);
+          } else {
 #pragma unroll
-          for (int j = 0; j < BN / 128; ++j)
-            tma_load_2d_pair(sa + A_BYTES + j * 8192u, &tmB, fb, colB + j * 64, rowB + kb * BK);
+            for (int j = 0; j < BN / 128; ++j)
+              tma_load_2d_pair(sa + A_BYTES + j * 8192u, &tmB, fb, colB + j * 64, rowB + kb * BK);
+          }
           if (++s == STAGES) {
             s = 0;
             ph ^= 1u;
@@ -755,8 +762,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (lane == 0 && leader) {
       TileIter it{tile_pre, mtiles, E, NT, 0};
-      // kind::f16, D fp32, A bf16 K-major, B bf16 MN-major, M=256, N=256
-      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+      // kind::f16, D fp32, A bf16 K-major, B bf16 MN-major (K-major with BKM), M=256, N=256
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(!BKM) << 16) |
                              ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(PM >> 4) << 24);
       int s = 0;
       uint32_t ph = 0;
@@ -784,7 +791,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = desc_sw128(sa + kk * 32u, 16u, 1024u);
-            const uint64_t bd = desc_sw128(sb + kk * 2048u, 8192u, 1024u);
+            const uint64_t bd = BKM ? desc_sw128(sb + kk * 32u, 16u, 1024u)
+                                    : desc_sw128(sb + kk * 2048u, 8192u, 1024u);
             tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
           }
           tc_commit_pair(empty_bar(s), 0x3);
@@ -816,11 +824,204 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int row0 = (int)(e * Cbuf + mt * PM + (int)rank * (PM / 2) + q * 32);
-      store_rows<BN, RELU ? kEpiRelu : kEpiNone>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN,
-                                                 stage, row0, nt * BN, lane);
+      const uint16_t* mrow = EPI == kEpiMask ? mask + (int64_t)(row0 + lane) * N + nt * BN : nullptr;
+      store_rows<BN, EPI>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
+                          nt * BN, lane, mrow);
       tc_fence_before();
       if (leader) mbar_arrive(tempty_bar(acc));
       else mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+    }
+    if (lane == 0) bulk_wait0();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();          // no CTA leaves while its pair may still use its smem or TMEM
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+// Weight gradients on CTA pairs: D[e] tile of 256 (P) x 256 (Q) per pair, CTA r holding
+// rows [128r, 128r+128) of the tile (its A columns) and columns [128r, 128r+128) of
+// B.  Both operands MN-major as in wgrad_tc_kernel; the k-loop covers the expert's
+// kept slots in 64-slot blocks (the caller clears the rows up to the next multiple
+// of 64).  An expert with no kept slot gets zero tiles, stored by both CTAs without
+// an MMA.  Same barrier and TMEM handshake as ffn_tc2_kernel.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    wgrad_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
+                     int64_t Cbuf, int P, int Q, unsigned* err, uint64_t limit_ns) {
+  using namespace pairk;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;   // same offset in both CTAs
+  unsigned char* gbase = smem_raw + (base - raw_base);
+  const uint32_t staging0 = base + STAGES * STAGE_BYTES;
+  const uint32_t bar0 = staging0 + STAGING;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
+  unsigned char* misc = gbase + STAGES * STAGE_BYTES + STAGING + 512;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  int* kblocks = reinterpret_cast<int*>(misc + 16);                  // [E]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int PT = (P + PM - 1) / PM, QT = Q / BN;
+  const int per_e = PT * QT, total = E * per_e;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 2 * 128);     // epilogue threads of both CTAs
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32((const void*)tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  pdl_trigger();
+  pdl_wait();                          // operands and counts complete
+  if (warp == 2)
+    for (int e = lane; e < E; e += 32) kblocks[e] = (min(nexp[e], (int)Cbuf) + BK - 1) / BK;
+  tc_fence_before();
+  cluster_sync_all();          // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total; tile += npairs) {
+        const int e = tile / per_e, r = tile - e * per_e;
+        const int pt = r / QT, qt = r - pt * QT;
+        const int KB = kblocks[e];
+        const int colA = pt * PM + (int)rank * (PM / 2), colB = qt * BN + (int)rank * (BN / 2);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (*abort_flag || !mbar_wait(empty_bar(s), ph ^ 1u, err, limit_ns)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const uint32_t sa = base + s * STAGE_BYTES;
+          const uint32_t fb = full_bar(s) & kPeerBitMask;     // the leader's full barrier
+          if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * STAGE_BYTES);
+          const int row = (int)(e * Cbuf + kb * BK);
+          // columns of A past P (the second CTA of a half-filled last p-tile) read as zeros
+#pragma unroll
+          for (int j = 0; j < 2; ++j) tma_load_2d_pair(sa + j * 8192u, &tmA, fb, colA + j * 64, row);
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            tma_load_2d_pair(sa + A_BYTES + j * 8192u, &tmB, fb, colB + j * 64, row);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && leader) {
+      // kind::f16, D fp32, A and B bf16 MN-major, M=256, N=256
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                             ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(PM >> 4) << 24);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int i = 0;
+      for (int tile = pair; ok && tile < total; tile += npairs) {
+        const int KB = kblocks[tile / per_e];
+        if (KB == 0) continue;                  // zero tile: the epilogues store zeros
+        const int acc = i & 1;
+        const uint32_t aph = (i >> 1) & 1;
+        ++i;
+        if (*abort_flag || !mbar_wait(tempty_bar(acc), aph ^ 1u, err, limit_ns)) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (*abort_flag || !mbar_wait(full_bar(s), ph, err, limit_ns)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base + s * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = desc_sw128(sa + kk * 2048u, 8192u, 1024u);
+            const uint64_t bd = desc_sw128(sb + kk * 2048u, 8192u, 1024u);
+            tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          }
+          tc_commit_pair(empty_bar(s), 0x3);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (ok) tc_commit_pair(tfull_bar(acc), 0x3);
+      }
+      if (!ok) {
+        tc_commit_pair(done_bar, 0x1);
+        mbar_wait(done_bar, 0, err, limit_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5, both CTAs)
+    const int q = warp & 3;
+    const uint32_t stage = staging0 + (warp - 2) * 4096u;
+    int i = 0;
+    for (int tile = pair; tile < total; tile += npairs) {
+      const int e = tile / per_e, r = tile - e * per_e;
+      const int pt = r / QT, qt = r - pt * QT;
+      const bool zero = kblocks[e] == 0;
+      const int prow = pt * PM + (int)rank * (PM / 2) + q * 32;   // P is a multiple of 64
+      int acc = 0;
+      if (!zero) {
+        acc = i & 1;
+        const uint32_t aph = (i >> 1) & 1;
+        ++i;
+        if (*abort_flag || !mbar_wait(tfull_bar(acc), aph, err, limit_ns)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+      }
+      if (prow < P)
+        store_rows<BN, kEpiNone>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage,
+                                 e * P + prow, qt * BN, lane, nullptr, zero);
+      if (!zero) {
+        tc_fence_before();
+        if (leader) mbar_arrive(tempty_bar(acc));
+        else mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+      }
     }
     if (lane == 0) bulk_wait0();
     __syncwarp();
@@ -866,15 +1067,16 @@ bool encode_2d(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer,
   return r == CUDA_SUCCESS;
 }
 
-template <bool RELU>
+template <int EPI, bool BKM>
 cudaError_t launch_pair(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint64_t limit_ns,
                         int num_sms, cudaStream_t st) {
-  auto kern = ffn_tc2_kernel<RELU>;
+  auto kern = ffn_tc2_kernel<EPI, BKM>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)pairk::SMEM);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(num_sms & ~1), dim3(kThreads), pairk::SMEM, st, p.tmA, p.tmB, p.tmD,
-                    nexp, p.E, p.Cbuf, p.K, p.N, err, limit_ns);
+  return launch_pdl(kern, dim3(num_sms & ~1), dim3(kThreads), pairk::SMEM, st, p.tmA,
+                    BKM ? p.tmB2 : p.tmB, p.tmD, nexp, p.E, p.Cbuf, p.K, p.N,
+                    static_cast<const uint16_t*>(p.mask), err, limit_ns);
 }
 
 template <int BN, int EPI, bool BKM>
@@ -898,6 +1100,16 @@ cudaError_t launch_w(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(num_sms), dim3(kThreads), smem, st, p.tmA, p.tmB, p.tmD, nexp, p.E,
                     p.Cbuf, p.K, p.N, err, limit_ns);
+}
+
+cudaError_t launch_w2(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint64_t limit_ns,
+                      int num_sms, cudaStream_t st) {
+  auto kern = wgrad_tc2_kernel;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)pairk::SMEM);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(num_sms & ~1), dim3(kThreads), pairk::SMEM, st, p.tmA, p.tmB, p.tmD,
+                    nexp, p.E, p.Cbuf, p.K, p.N, err, limit_ns);
 }
 
 int pick_bn(int N) { return (N % 256 == 0) ? 256 : (N % 128 == 0 ? 128 : 64); }
@@ -934,9 +1146,11 @@ bool make_dgrad_plan(GemmPlan& p, const void* A, const void* Bt, void* D, const 
   p.D = D;
   p.mask = mask;
   p.BN = pick_bn(N);
+  p.pair = (N % pairk::BN) == 0;
   if (K % BK || N % 64) return false;
   if (!encode_2d(&p.tmA, A, (uint64_t)K, (uint64_t)E * Cbuf, BK, BM)) return false;
   if (!encode_2d(&p.tmB, Bt, (uint64_t)K, (uint64_t)E * N, BK, (uint32_t)p.BN)) return false;
+  if (p.pair && !encode_2d(&p.tmB2, Bt, (uint64_t)K, (uint64_t)E * N, BK, pairk::BN / 2)) return false;
   if (!encode_2d(&p.tmD, D, (uint64_t)N, (uint64_t)E * Cbuf, 64, 32)) return false;
   return true;
 }
@@ -952,6 +1166,7 @@ bool make_wgrad_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, 
   p.D = D;
   p.f32out = f32out;
   p.BN = pick_bn(Q);
+  p.pair = !f32out && (Q % pairk::BN) == 0;   // wgrad_tc2_kernel: 256 x 256 tiles on CTA pairs
   if (P % 64 || Q % 64 || Cbuf % BK) return false;
   const uint64_t rows = rows_ab > 0 ? (uint64_t)rows_ab : (uint64_t)E * Cbuf;
   if (!encode_2d(&p.tmA, A, (uint64_t)P, rows, 64, BK)) return false;
@@ -984,6 +1199,7 @@ bool make_gate_dx_plan(GemmPlan& p, const void* dlb, int64_t S, int EPb, const v
 cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* err,
                             uint64_t wait_limit_ns, int num_sms, bool want_pair, cudaStream_t st) {
   if (p.kind == kGemmWgrad) {
+    if (!p.f32out && p.pair && want_pair) return launch_w2(p, nexp, err, wait_limit_ns, num_sms, st);
     if (p.f32out) {
       switch (p.BN) {
         case 256: return launch_w<256, kEpiF32>(p, nexp, err, wait_limit_ns, num_sms, st);
@@ -999,6 +1215,9 @@ cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* er
   }
   if (p.kind == kGemmDgrad) {
     const bool m = p.mask != nullptr;
+    if (p.pair && want_pair && (p.Cbuf % pairk::PM) == 0)
+      return m ? launch_pair<kEpiMask, true>(p, nexp, err, wait_limit_ns, num_sms, st)
+               : launch_pair<kEpiNone, true>(p, nexp, err, wait_limit_ns, num_sms, st);
     switch (p.BN) {
       case 256:
         return m ? launch_t<256, kEpiMask, true>(p, nexp, err, wait_limit_ns, num_sms, st)
@@ -1012,8 +1231,8 @@ cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* er
     }
   }
   if (p.pair && want_pair && (p.Cbuf % pairk::PM) == 0)
-    return p.relu ? launch_pair<true>(p, nexp, err, wait_limit_ns, num_sms, st)
-                  : launch_pair<false>(p, nexp, err, wait_limit_ns, num_sms, st);
+    return p.relu ? launch_pair<kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st)
+                  : launch_pair<kEpiNone, false>(p, nexp, err, wait_limit_ns, num_sms, st);
   switch (p.BN) {
     case 256:
       return p.relu ? launch_t<256, kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st)

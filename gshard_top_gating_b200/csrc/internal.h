@@ -80,6 +80,7 @@ struct GemmPlan {
   CUtensorMap tmA;
   CUtensorMap tmB;
   CUtensorMap tmD;   // box {64, 32}, 128B swizzle (epilogue stores)
+  CUtensorMap tmB2;  // kGemmDgrad CTA pairs: B box {64, 128} (each CTA's half of the N rows)
   void* D;
   const void* mask;  // kGemmDgrad: [E*Cbuf, N] bf16 values whose sign masks the result, or null
   int kind;

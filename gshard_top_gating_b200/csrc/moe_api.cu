@@ -574,13 +574,16 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
     MOE_TRY(launch_pad_zero(bufs, widths, 3, true, E, h->Cbuf, R, st));
     MOE_TRY(mark(2));
     const uint64_t lim = h->wait_limit_ns;
-    MOE_TRY(launch_ffn_bf16(h->plan_dw2, R.nexp, R.err, lim, h->num_sms, false, st));
+    // CTA pairs (256-row / 256-column tiles) under the forward's rule: experts at capacity
+    const int C = (int)capacity_of(h->cf, h->k, S, E);
+    const bool pair = (double)S * h->k / E >= (double)C;
+    MOE_TRY(launch_ffn_bf16(h->plan_dw2, R.nexp, R.err, lim, h->num_sms, pair, st));
     MOE_TRY(mark(3));
-    MOE_TRY(launch_ffn_bf16(h->plan_dp, R.nexp, R.err, lim, h->num_sms, false, st));
+    MOE_TRY(launch_ffn_bf16(h->plan_dp, R.nexp, R.err, lim, h->num_sms, pair, st));
     MOE_TRY(mark(4));
-    MOE_TRY(launch_ffn_bf16(h->plan_dw1, R.nexp, R.err, lim, h->num_sms, false, st));
+    MOE_TRY(launch_ffn_bf16(h->plan_dw1, R.nexp, R.err, lim, h->num_sms, pair, st));
     MOE_TRY(mark(5));
-    MOE_TRY(launch_ffn_bf16(h->plan_dx, R.nexp, R.err, lim, h->num_sms, false, st));
+    MOE_TRY(launch_ffn_bf16(h->plan_dx, R.nexp, R.err, lim, h->num_sms, pair, st));
   } else {
     MOE_TRY(mark(2));
     MOE_TRY(launch_ffn_bwd_f32((const float*)h->xbuf, (const float*)h->hbuf, (float*)h->dybuf,

@@ -141,6 +141,10 @@ BF16_SHAPES = [
     (257, 192, 320, 6, 2, 1.25, False),     # M, H = 64 mod 128: half-filled last weight-grad tiles
     (512, 128, 128, 64, 2, 1.0, True),      # gate bias: many experts keep nothing (zero tiles)
     (256, 256, 256, 32, 8, 1.25, False),    # top-8
+    # experts at capacity (S k / E >= C): the CTA-pair kernels run where 256 divides N or Q
+    (768, 384, 256, 4, 2, 1.0, False),      # pair dP and dW1 (P = 384: half-filled last pair tile)
+    (1024, 256, 256, 16, 2, 1.0, True),     # pair kernels with experts that keep nothing
+    (4096, 512, 1024, 8, 2, 1.0, False),    # several 256-row pair tiles per expert
 ]
 
 
