@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libgshard_moe.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_OOM, MOE_ERR_STATE, \
     MOE_ERR_TIMEOUT = range(7)
 MOE_F32, MOE_BF16 = 0, 1
+MOE_BWD_SKIP_EMPTY_EXPERTS = 1
 MOE_NUM_STAGES = 6
 STAGES = ("router", "scan", "dispatch", "ffn1", "ffn2", "combine")
 MOE_NUM_BWD_STAGES = 8
@@ -53,6 +54,7 @@ def _load() -> ctypes.CDLL:
         "moe_selftest_wait_timeout": [I32, P],
         "moe_assign_slots_noalloc": [I64, I32, I32, I64, P, P, P, P],
         "moe_enable_backward": [P],
+        "moe_set_backward_flags": [P, ctypes.c_uint32],
         "moe_get_backward_stage_times": [P, ctypes.POINTER(ctypes.c_float), I32],
         "moe_backward": [P, I64, P, P, ctypes.c_float, ctypes.c_float, P, P, P, P, P, P],
     }
@@ -201,3 +203,7 @@ def moe_get_backward_stage_times(h):
 
 def moe_backward_stage_name(stage: int) -> str:
     return lib.moe_backward_stage_name(stage).decode()
+
+
+def moe_set_backward_flags(h, flags: int) -> None:
+    _check("moe_set_backward_flags", lib.moe_set_backward_flags(h, int(flags)))

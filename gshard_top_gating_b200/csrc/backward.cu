@@ -355,6 +355,7 @@ struct SimtGemm {
   int64_t a_z, a_i, a_k, b_z, b_k, b_j;
   int rows, cols, K;
   bool rows_from_n, k_from_n;   // rows / K = the expert's kept count
+  bool skip_empty;              // k_from_n: an expert with no kept row leaves D untouched
   int ones_row;                 // A(i, kk) = 1 for i == ones_row (bias gradient), else -1
   int kchunk;                   // split-K: z covers [z*kchunk, (z+1)*kchunk)
   void* D;
@@ -388,6 +389,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemm g, Routing R) {
   }
   const int i0 = blockIdx.y * TM, j0 = blockIdx.x * TN;
   if (i0 >= rows) return;
+  if (g.skip_empty && g.k_from_n && k1 <= 0) return;
   const TA* A = static_cast<const TA*>(g.A) + (g.kchunk > 0 ? 0 : z * g.a_z);
   const TB* B = static_cast<const TB*>(g.B) + (g.kchunk > 0 ? 0 : z * g.b_z);
   __shared__ float As[TK][TM + 4];
@@ -622,7 +624,7 @@ cudaError_t launch_dwg(const BwdArgs& a, int num_sms, cudaStream_t st) {
 cudaError_t launch_ffn_bwd_f32(const float* xbuf, const float* hbuf, float* dybuf, float* dpre,
                                const float* W1, const float* W2, float* dW1, float* dW2,
                                const int32_t* nexp, int E, int64_t Cbuf, int M, int H,
-                               cudaStream_t st) {
+                               bool skip_empty, cudaStream_t st) {
   Routing none{};
   const int rows_cap = (int)Cbuf;
   cudaError_t e;
@@ -632,6 +634,7 @@ cudaError_t launch_ffn_bwd_f32(const float* xbuf, const float* hbuf, float* dybu
     g.A = hbuf; g.a_z = Cbuf * H; g.a_i = 1; g.a_k = H;
     g.B = dybuf; g.b_z = Cbuf * M; g.b_k = M; g.b_j = 1;
     g.rows = H; g.cols = M; g.k_from_n = true; g.nexp = nexp; g.Cbuf = Cbuf; g.ones_row = -1;
+    g.skip_empty = skip_empty;
     g.D = dW2; g.d_z = (int64_t)H * M; g.d_i = M;
     if ((e = run_simt<float, float, float, kSgStore>(g, H, E, none, st)) != cudaSuccess) return e;
   }
@@ -650,6 +653,7 @@ cudaError_t launch_ffn_bwd_f32(const float* xbuf, const float* hbuf, float* dybu
     g.A = xbuf; g.a_z = Cbuf * M; g.a_i = 1; g.a_k = M;
     g.B = dpre; g.b_z = Cbuf * H; g.b_k = H; g.b_j = 1;
     g.rows = M; g.cols = H; g.k_from_n = true; g.nexp = nexp; g.Cbuf = Cbuf; g.ones_row = -1;
+    g.skip_empty = skip_empty;
     g.D = dW1; g.d_z = (int64_t)M * H; g.d_i = H;
     if ((e = run_simt<float, float, float, kSgStore>(g, M, E, none, st)) != cudaSuccess) return e;
   }

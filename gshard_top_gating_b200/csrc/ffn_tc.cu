@@ -425,7 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // takes them transposed.  The k-loop covers ceil(n_e / 64) blocks; rows n_e ..
 // ceil64(n_e) - 1 of both operands must hold zeros (the caller clears them), or lie
 // past the tensor maps' last row (TMA fills zeros).  An expert with no kept slot
-// gets D[e] = 0 (its tiles store zeros without an MMA).  EPI = kEpiF32 stores the
+// gets D[e] = 0 (its tiles store zeros without an MMA), or keeps D[e] untouched when
+// store_zero is 0.  EPI = kEpiF32 stores the
 // fp32 accumulator; the "experts" may also be consecutive row ranges of one
 // operand pair (a split of a long reduction, whose partial results the caller adds).
 // Tiles are (expert, p-tile, q-tile), q fastest; roles as in ffn_tc_kernel.
@@ -433,7 +434,8 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     wgrad_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp,
-                    int E, int64_t Cbuf, int P, int Q, unsigned* err, uint64_t limit_ns) {
+                    int E, int64_t Cbuf, int P, int Q, int store_zero, unsigned* err,
+                    uint64_t limit_ns) {
   using C = Cfg<BN>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -595,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
       }
-      if (prow < P)
+      if (prow < P && (!zero || store_zero))
         store_rows<BN, EPI>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
                             qt * BN, lane, nullptr, zero);
       if (!zero) {
@@ -853,7 +855,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     wgrad_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
-                     int64_t Cbuf, int P, int Q, unsigned* err, uint64_t limit_ns) {
+                     int64_t Cbuf, int P, int Q, int store_zero, unsigned* err, uint64_t limit_ns) {
   using namespace pairk;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -1014,7 +1016,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
       }
-      if (prow < P)
+      if (prow < P && (!zero || store_zero))
         store_rows<BN, kEpiNone>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage,
                                  e * P + prow, qt * BN, lane, nullptr, zero);
       if (!zero) {
@@ -1099,7 +1101,7 @@ cudaError_t launch_w(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(num_sms), dim3(kThreads), smem, st, p.tmA, p.tmB, p.tmD, nexp, p.E,
-                    p.Cbuf, p.K, p.N, err, limit_ns);
+                    p.Cbuf, p.K, p.N, p.skip_zero ? 0 : 1, err, limit_ns);
 }
 
 cudaError_t launch_w2(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint64_t limit_ns,
@@ -1109,7 +1111,7 @@ cudaError_t launch_w2(const GemmPlan& p, const int32_t* nexp, unsigned* err, uin
                                        (int)pairk::SMEM);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(num_sms & ~1), dim3(kThreads), pairk::SMEM, st, p.tmA, p.tmB, p.tmD,
-                    nexp, p.E, p.Cbuf, p.K, p.N, err, limit_ns);
+                    nexp, p.E, p.Cbuf, p.K, p.N, p.skip_zero ? 0 : 1, err, limit_ns);
 }
 
 int pick_bn(int N) { return (N % 256 == 0) ? 256 : (N % 128 == 0 ? 128 : 64); }

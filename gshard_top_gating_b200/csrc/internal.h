@@ -89,6 +89,7 @@ struct GemmPlan {
   bool relu;
   bool pair;         // the CTA-pair (cta_group::2, 256 x 256 tile) kernel can run (N % 256 == 0)
   bool f32out;       // kGemmWgrad: D is fp32
+  bool skip_zero;    // kGemmWgrad: experts with no kept row leave D[e] untouched (else zeros)
   int64_t row_limit; // rows of D (0 = E*Cbuf): stores of 32-row groups starting past it are skipped
 };
 bool make_gemm_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, int64_t Cbuf, int K,
@@ -146,7 +147,7 @@ int dwg_tc_split_bound(int S, int M, int EPb, int num_sms);
 cudaError_t launch_ffn_bwd_f32(const float* xbuf, const float* hbuf, float* dybuf, float* dpre,
                                const float* W1, const float* W2, float* dW1, float* dW2,
                                const int32_t* nexp, int E, int64_t Cbuf, int M, int H,
-                               cudaStream_t st);
+                               bool skip_empty, cudaStream_t st);
 // selftest.cu
 cudaError_t launch_wait_selftest(unsigned* flag, unsigned* err, uint64_t limit_ns, cudaStream_t st);
 

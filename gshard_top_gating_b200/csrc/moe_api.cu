@@ -61,6 +61,7 @@ struct moe_layer {
   GemmPlan plan_dw2, plan_dw1;      // dW2 = h^T dY,  dW1 = X^T dP (output pointers cached)
   const void* dw2_ptr;
   const void* dw1_ptr;
+  uint32_t bwd_flags;               // MOE_BWD_* flags
   // bf16: tensor-core gate gradients
   int EPb;                          // E rounded up to 64
   void* dlb;                        // [S_max, 2*EPb] bf16 split of dl
@@ -483,6 +484,12 @@ moe_status moe_enable_backward(moe_handle h) {
   return MOE_OK;
 }
 
+moe_status moe_set_backward_flags(moe_handle h, uint32_t flags) {
+  if (!h || (flags & ~(uint32_t)MOE_BWD_SKIP_EMPTY_EXPERTS)) return MOE_ERR_INVALID_ARG;
+  h->bwd_flags = flags;
+  return MOE_OK;
+}
+
 int32_t moe_kernels_per_backward(moe_handle h, int64_t S) {
   if (!h || S <= 0) return 0;
   return h->act == MOE_BF16 ? 10 : 8;
@@ -504,8 +511,10 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
   if (S == 0) {   // no tokens: every gradient is zero
     MOE_TRY(cudaMemsetAsync(dWg, 0, (size_t)M * E * 4, st));
     if (dbias) MOE_TRY(cudaMemsetAsync(dbias, 0, (size_t)E * 4, st));
-    MOE_TRY(cudaMemsetAsync(dW1, 0, (size_t)E * M * H * as, st));
-    MOE_TRY(cudaMemsetAsync(dW2, 0, (size_t)E * H * M * as, st));
+    if (!(h->bwd_flags & MOE_BWD_SKIP_EMPTY_EXPERTS)) {   // every expert is empty
+      MOE_TRY(cudaMemsetAsync(dW1, 0, (size_t)E * M * H * as, st));
+      MOE_TRY(cudaMemsetAsync(dW2, 0, (size_t)E * H * M * as, st));
+    }
     return MOE_OK;
   }
   const bool bf16 = h->act == MOE_BF16;
@@ -567,6 +576,9 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
       if (!make_wgrad_plan(h->plan_dw1, h->xbuf, h->dpre, dW1, E, h->Cbuf, M, H)) return MOE_ERR_CUDA;
       h->dw1_ptr = dW1;
     }
+    const bool skip = (h->bwd_flags & MOE_BWD_SKIP_EMPTY_EXPERTS) != 0;
+    h->plan_dw2.skip_zero = skip;
+    h->plan_dw1.skip_zero = skip;
     // the weight-gradient GEMMs reduce over whole 64-slot blocks: clear the rows
     // between the kept count and the next multiple of 64
     void* bufs[3] = {h->xbuf, h->hbuf, h->dybuf};
@@ -588,7 +600,8 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
     MOE_TRY(mark(2));
     MOE_TRY(launch_ffn_bwd_f32((const float*)h->xbuf, (const float*)h->hbuf, (float*)h->dybuf,
                                (float*)h->dpre, (const float*)h->W1, (const float*)h->W2, (float*)dW1,
-                               (float*)dW2, R.nexp, E, h->Cbuf, M, H, st));
+                               (float*)dW2, R.nexp, E, h->Cbuf, M, H,
+                               (h->bwd_flags & MOE_BWD_SKIP_EMPTY_EXPERTS) != 0, st));
     for (int i = 3; i <= 5; ++i) MOE_TRY(mark(i));   // the fp32 GEMMs are timed as one stage
   }
   MOE_TRY(mark(6));

@@ -46,11 +46,14 @@ class MoeLayer:
         return L.moe_aux_loss(self.h, stream)
 
     def backward(self, x: torch.Tensor, dy: torch.Tensor, a_aux: float = 0.0, a_z: float = 0.0,
-                 stream=None) -> dict:
+                 stream=None, out: dict | None = None, skip_empty_experts: bool = False) -> dict:
         """Gradients of <dy, y> + a_aux*l_aux + a_z*z for the last forward (which took x).
 
-        Returns dx, dWg, dbias (None without a gate bias), dW1, dW2 as new tensors.
-        The backward workspace is allocated on the first call.
+        Returns dx, dWg, dbias (None without a gate bias), dW1, dW2: new tensors,
+        or the tensors of `out` (same keys) written in place.  With
+        skip_empty_experts, dW1[e] and dW2[e] of experts that kept no token are
+        left as they were (MOE_BWD_SKIP_EMPTY_EXPERTS).  The backward workspace is
+        allocated on the first call.
         """
         if not getattr(self, "_bwd", False):
             L.moe_enable_backward(self.h)
@@ -60,11 +63,22 @@ class MoeLayer:
                 raise ValueError("x and dy must be contiguous [S, M] tensors of the activation dtype")
         S = x.shape[0]
         dev = x.device
-        dx = torch.empty_like(x)
-        dWg = torch.empty(self.M, self.E, dtype=torch.float32, device=dev)
-        dbias = torch.empty(self.E, dtype=torch.float32, device=dev) if self._keep[1] is not None else None
-        dW1 = torch.empty(self.E, self.M, self.H, dtype=self.act, device=dev)
-        dW2 = torch.empty(self.E, self.H, self.M, dtype=self.act, device=dev)
+        out = dict(out or {})
+        dx = out.get("dx") if out.get("dx") is not None else torch.empty_like(x)
+        dWg = out.get("dWg") if out.get("dWg") is not None else \
+            torch.empty(self.M, self.E, dtype=torch.float32, device=dev)
+        dbias = None
+        if self._keep[1] is not None:
+            dbias = out.get("dbias") if out.get("dbias") is not None else \
+                torch.empty(self.E, dtype=torch.float32, device=dev)
+        dW1 = out.get("dW1") if out.get("dW1") is not None else \
+            torch.empty(self.E, self.M, self.H, dtype=self.act, device=dev)
+        dW2 = out.get("dW2") if out.get("dW2") is not None else \
+            torch.empty(self.E, self.H, self.M, dtype=self.act, device=dev)
+        for t in (dx, dWg, dW1, dW2) + ((dbias,) if dbias is not None else ()):
+            if not (t.is_cuda and t.is_contiguous()):
+                raise ValueError("gradient buffers must be contiguous CUDA tensors")
+        L.moe_set_backward_flags(self.h, L.MOE_BWD_SKIP_EMPTY_EXPERTS if skip_empty_experts else 0)
         L.moe_backward(self.h, S, x, dy, a_aux, a_z, dx, dWg, dbias, dW1, dW2, stream)
         return {"dx": dx, "dWg": dWg, "dbias": dbias, "dW1": dW1, "dW2": dW2}
 

@@ -244,7 +244,8 @@ MOE_API moe_status moe_enable_backward(moe_handle h);
  * dx_dev    [S, M] act, overwritten.
  * dWg_dev   [M, E] fp32, overwritten.      dbias_dev [E] fp32 overwritten, or NULL.
  * dW1_dev   [E, M, H] act, overwritten.    dW2_dev   [E, H, M] act, overwritten
- *           (experts that kept no token get zeros).
+ *           (experts that kept no token get zeros, or are skipped: see
+ *           moe_set_backward_flags).
  * Returns MOE_ERR_STATE unless moe_enable_backward succeeded and the last call
  * that routed on this handle was a moe_forward of S tokens.  Every output
  * pointer must be 16-byte aligned and must not alias the inputs.
@@ -255,6 +256,21 @@ MOE_API moe_status moe_backward(moe_handle h, int64_t S, const void* x_dev, cons
 
 /* Number of kernels one moe_backward of S tokens launches. */
 MOE_API int32_t moe_kernels_per_backward(moe_handle h, int64_t S);
+
+/* Flags of moe_set_backward_flags. */
+enum { MOE_BWD_SKIP_EMPTY_EXPERTS = 1 };
+
+/*
+ * moe_set_backward_flags -- options of the following moe_backward calls (default 0).
+ * MOE_BWD_SKIP_EMPTY_EXPERTS: dW1[e] and dW2[e] of an expert that kept no token in
+ * the forward are not written (the caller's buffer keeps what it held), instead of
+ * being set to zero.  Only the experts a batch activated get a gradient ("GShard:
+ * Scaling Giant Neural Networks with Conditional Computation", "Training
+ * Methodology", "Gradient Synchronization"); a caller that applies sparse updates
+ * reads which experts those were from moe_get_routing's cnt (cnt[e] > 0).
+ * Returns MOE_ERR_INVALID_ARG for unknown bits.
+ */
+MOE_API moe_status moe_set_backward_flags(moe_handle h, uint32_t flags);
 
 /* Stage indices of moe_get_backward_stage_times. */
 enum { MOE_BSTAGE_GATE = 0,     /* combine + gate backward: dY, dgate, dl */

@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
     for want in ("moe_create", "moe_forward", "moe_aux_loss", "moe_destroy", "moe_get_logits",
                  "moe_get_routing", "moe_route_from_logits", "moe_status_string",
                  "moe_forward_host", "moe_enable_backward", "moe_backward",
-                 "moe_kernels_per_backward"):
+                 "moe_kernels_per_backward", "moe_set_backward_flags",
+                 "moe_get_backward_stage_times"):
         assert want in names
 
 
@@ -88,3 +89,4 @@ def test_null_handle_calls_are_rejected(L):
     assert L.lib.moe_enable_backward(None) == 1
     assert L.lib.moe_backward(None, 1, FAKE, FAKE, 0.0, 0.0, FAKE, FAKE, None, FAKE, FAKE, None) == 1
     assert L.lib.moe_kernels_per_backward(None, 10) == 0
+    assert L.lib.moe_set_backward_flags(None, 0) == 1

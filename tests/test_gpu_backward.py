@@ -260,3 +260,34 @@ def test_backward_mid_full_size():
     print(f"\nmid backward errors: {errs}")
     _check_all(errs, "bf16")
     run.layer.close()
+
+
+@pytest.mark.parametrize("act,shape", [
+    ("bf16", (512, 128, 256, 64, 2, 1.25)),         # one-CTA weight-gradient kernels
+    ("bf16", (1024, 256, 256, 16, 2, 1.0)),         # CTA-pair weight-gradient kernels
+    ("f32", (256, 64, 128, 32, 2, 1.0)),            # FFMA weight gradients
+])
+def test_skip_empty_experts_leaves_their_gradients(act, shape):
+    """MOE_BWD_SKIP_EMPTY_EXPERTS: experts that kept no token keep the caller's
+    bytes; every other gradient equals the dense backward bit for bit."""
+    S, M, H, E, k, cf = shape
+    w = Workload("skip", S, M, H, E, k, cf, act, skew_bias=True, seed=34)
+    run = G.build(w)
+    x = run.x
+    run.layer(x)
+    dy = upstream_grad(w, device="cuda")
+    dense = run.layer.backward(x, dy, 0.5, 0.1)
+    sentinel = {"dW1": torch.full_like(dense["dW1"], 7.0), "dW2": torch.full_like(dense["dW2"], -3.0)}
+    sparse = run.layer.backward(x, dy, 0.5, 0.1, out=sentinel, skip_empty_experts=True)
+    torch.cuda.synchronize()
+    _, _, _, cnt = run.layer.routing(S)
+    empty = (cnt == 0).cpu()
+    assert empty.any() and not empty.all()
+    for key, fill in (("dW1", 7.0), ("dW2", -3.0)):
+        got, ref = sparse[key].cpu(), dense[key].cpu()
+        assert torch.all(got[empty] == fill), key
+        assert torch.equal(got[~empty], ref[~empty]), key
+    for key in ("dx", "dWg", "dbias"):
+        if dense[key] is not None:
+            assert torch.equal(sparse[key], dense[key]), key
+    run.layer.close()
