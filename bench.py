@@ -413,7 +413,9 @@ def run_ours(args, rank, world, local):
         achieved, peak, unit = work / t / 1e9, pk["hbm_gbs"], "GB/s"
     roof = {"bound": bound, "kernel": dom, "achieved": round(achieved, 2), "peak": peak,
             "unit": unit, "frac": round(achieved / peak, 4), "traffic": ncu_traffic(dom, w.name),
-            "peak_source": pk_kind}
+            "peak_source": f"{pk_kind}, burst" if bound == "tensor" else pk_kind,
+            "frac_of_sustained": (round(achieved / pk["bf16_tflops_sustained"], 4)
+                                  if bound == "tensor" and pk.get("bf16_tflops_sustained") else None)}
     stages = {}
     for n in STAGES:
         b_, wk = algo[n]
