@@ -38,8 +38,14 @@ struct moe_layer {
   void* xbuf;
   void* hbuf;
   void* ybuf;
-  void* xstage;          // moe_forward_host staging
-  void* ystage;
+  void* xstage[2];       // moe_forward_host staging, two slots so calls overlap
+  void* ystage[2];
+  // moe_forward_host pipeline: copy-in, compute and copy-out streams (created on first use)
+  bool host_ready;
+  cudaStream_t hs_in, hs_comp, hs_out;
+  cudaEvent_t ev_xready[2], ev_fwd[2], ev_yfree[2], ev_entry;
+  int host_slot;
+  bool last_was_host;    // the handle's last device work was a moe_forward_host
   GemmPlan plan1, plan2;
   void* wsplit;          // bf16 tokens: W_g split into three bf16 parts [3][EP][M]
   CUtensorMap wmap, xmap;
@@ -133,8 +139,10 @@ size_t carve(moe_layer* h, char* base) {
   h->xbuf = c.take<char>((size_t)E * h->Cbuf * h->M * as);
   h->hbuf = c.take<char>((size_t)E * h->Cbuf * h->H * as);
   h->ybuf = c.take<char>((size_t)E * h->Cbuf * h->M * as);
-  h->xstage = c.take<char>((size_t)S * h->M * as);
-  h->ystage = c.take<char>((size_t)S * h->M * as);
+  for (int b = 0; b < 2; ++b) {
+    h->xstage[b] = c.take<char>((size_t)S * h->M * as);
+    h->ystage[b] = c.take<char>((size_t)S * h->M * as);
+  }
   h->wsplit = h->act == MOE_BF16 ? c.take<char>((size_t)3 * router_tc_pad(h->E) * h->M * 2) : nullptr;
   return c.off + 256;
 }
@@ -266,6 +274,15 @@ moe_status moe_destroy(moe_handle h) {
     for (auto& e : h->ev) cudaEventDestroy(e);
     for (auto& e : h->evb) cudaEventDestroy(e);
   }
+  if (h->host_ready) {
+    for (cudaStream_t s_ : {h->hs_in, h->hs_comp, h->hs_out}) cudaStreamDestroy(s_);
+    for (int b = 0; b < 2; ++b) {
+      cudaEventDestroy(h->ev_xready[b]);
+      cudaEventDestroy(h->ev_fwd[b]);
+      cudaEventDestroy(h->ev_yfree[b]);
+    }
+    cudaEventDestroy(h->ev_entry);
+  }
   cudaError_t fe = cudaFree(h->ws);
   delete h;
   if (ce != cudaSuccess) return from_cuda(ce);
@@ -283,9 +300,12 @@ int32_t moe_kernels_per_forward(moe_handle h, int64_t S) {
   return 6;
 }
 
-moe_status moe_forward(moe_handle h, int64_t S, const void* x, void* y, void* stream) {
+}  // extern "C"
+
+namespace {
+
+moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStream_t st) {
   if (!h || S < 0 || S > h->S_max) return MOE_ERR_INVALID_ARG;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (S > 0 && (!x || !y || !aligned(x, 16) || !aligned(y, 16))) return MOE_ERR_INVALID_ARG;
   h->last_S = S;
   h->have_forward = true;
@@ -338,20 +358,80 @@ moe_status moe_forward(moe_handle h, int64_t S, const void* x, void* y, void* st
   return MOE_OK;
 }
 
+cudaError_t host_pipeline_init(moe_handle h) {
+  if (h->host_ready) return cudaSuccess;
+  cudaError_t e = cudaSuccess;
+  for (cudaStream_t* s_ : {&h->hs_in, &h->hs_comp, &h->hs_out})
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(s_, cudaStreamNonBlocking);
+  for (int b = 0; b < 2 && e == cudaSuccess; ++b) {
+    e = cudaEventCreateWithFlags(&h->ev_xready[b], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fwd[b], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_yfree[b], cudaEventDisableTiming);
+  }
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_entry, cudaEventDisableTiming);
+  if (e == cudaSuccess) h->host_ready = true;    // (a failure leaks the few objects made)
+  return e;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_forward(moe_handle h, int64_t S, const void* x, void* y, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  h->last_was_host = false;
+  return forward_impl(h, S, x, y, static_cast<cudaStream_t>(stream));
+}
+
+// Three stages on the handle's own streams, so that consecutive calls overlap: the
+// copy of call i+1's x runs during call i's compute, and call i's y travels back
+// during call i+1's compute.  Staging slot b = call parity; events hand a slot
+// from one stage to the next and back.  Ordering with the caller:
+//  - `stream` waits for this call's copy back of y, so work later on `stream`
+//    (or a synchronisation of it) sees the result;
+//  - a call whose predecessor on this handle was not a host call first waits for
+//    the work enqueued on `stream` so far (the handle's workspace may still be
+//    read there); between host calls that wait is skipped, which is what lets
+//    the copies overlap.
 moe_status moe_forward_host(moe_handle h, int64_t S, const void* x_host, void* y_host, void* stream) {
   if (!h || S < 0 || S > h->S_max) return MOE_ERR_INVALID_ARG;
   if (S > 0 && (!x_host || !y_host)) return MOE_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (S == 0) {
+    h->last_was_host = false;
+    return forward_impl(h, 0, nullptr, nullptr, st);
+  }
+  MOE_TRY(host_pipeline_init(h));
   const size_t bytes = (size_t)S * h->M * act_bytes(h->act);
-  if (S > 0) MOE_TRY(cudaMemcpyAsync(h->xstage, x_host, bytes, cudaMemcpyHostToDevice, st));
-  moe_status s = moe_forward(h, S, h->xstage, h->ystage, stream);
+  const int b = h->host_slot;
+  if (!h->last_was_host) {
+    MOE_TRY(cudaEventRecord(h->ev_entry, st));
+    MOE_TRY(cudaStreamWaitEvent(h->hs_in, h->ev_entry, 0));
+    MOE_TRY(cudaStreamWaitEvent(h->hs_comp, h->ev_entry, 0));
+  }
+  // copy in: slot b's x was last read by the compute of call i-2
+  MOE_TRY(cudaStreamWaitEvent(h->hs_in, h->ev_fwd[b], 0));
+  MOE_TRY(cudaMemcpyAsync(h->xstage[b], x_host, bytes, cudaMemcpyHostToDevice, h->hs_in));
+  MOE_TRY(cudaEventRecord(h->ev_xready[b], h->hs_in));
+  // compute: needs this x, and slot b's y copied out by call i-2
+  MOE_TRY(cudaStreamWaitEvent(h->hs_comp, h->ev_xready[b], 0));
+  MOE_TRY(cudaStreamWaitEvent(h->hs_comp, h->ev_yfree[b], 0));
+  moe_status s = forward_impl(h, S, h->xstage[b], h->ystage[b], h->hs_comp);
   if (s != MOE_OK) return s;
-  if (S > 0) MOE_TRY(cudaMemcpyAsync(y_host, h->ystage, bytes, cudaMemcpyDeviceToHost, st));
+  MOE_TRY(cudaEventRecord(h->ev_fwd[b], h->hs_comp));
+  // copy out, then make the caller's stream wait for it
+  MOE_TRY(cudaStreamWaitEvent(h->hs_out, h->ev_fwd[b], 0));
+  MOE_TRY(cudaMemcpyAsync(y_host, h->ystage[b], bytes, cudaMemcpyDeviceToHost, h->hs_out));
+  MOE_TRY(cudaEventRecord(h->ev_yfree[b], h->hs_out));
+  MOE_TRY(cudaStreamWaitEvent(st, h->ev_yfree[b], 0));
+  h->host_slot = b ^ 1;
+  h->last_was_host = true;
   return MOE_OK;
 }
 
 moe_status moe_aux_loss(moe_handle h, float* l_aux, float* z_loss, void* stream) {
   if (!h || !l_aux || !z_loss) return MOE_ERR_INVALID_ARG;
+  h->last_was_host = false;
   if (!h->have_forward) return MOE_ERR_STATE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float v[2] = {0.f, 0.f};
@@ -370,6 +450,7 @@ moe_status moe_check(moe_handle h, void* stream) {
 
 moe_status moe_get_logits(moe_handle h, float* logits, void* stream) {
   if (!h || !logits) return MOE_ERR_INVALID_ARG;
+  h->last_was_host = false;
   if (!h->have_forward) return MOE_ERR_STATE;
   if (h->last_S == 0) return MOE_OK;
   MOE_TRY(cudaMemcpyAsync(logits, h->R.logits, (size_t)h->last_S * h->E * sizeof(float),
@@ -380,6 +461,7 @@ moe_status moe_get_logits(moe_handle h, float* logits, void* stream) {
 moe_status moe_get_routing(moe_handle h, int32_t* eidx, float* gate, int32_t* slot, int32_t* cnt,
                            void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
+  h->last_was_host = false;
   if (!h->have_forward) return MOE_ERR_STATE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t n = (size_t)h->last_S * h->k;
@@ -399,6 +481,7 @@ moe_status moe_get_routing(moe_handle h, int32_t* eidx, float* gate, int32_t* sl
 
 moe_status moe_route_from_logits(moe_handle h, int64_t S, const float* logits, void* stream) {
   if (!h || S < 0 || S > h->S_max) return MOE_ERR_INVALID_ARG;
+  h->last_was_host = false;
   if (S > 0 && (!logits || !aligned(logits, 4))) return MOE_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_S = S;
@@ -498,6 +581,7 @@ int32_t moe_kernels_per_backward(moe_handle h, int64_t S) {
 moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, float a_aux, float a_z,
                         void* dx, float* dWg, float* dbias, void* dW1, void* dW2, void* stream) {
   if (!h || S < 0 || S > h->S_max) return MOE_ERR_INVALID_ARG;
+  h->last_was_host = false;
   if (!h->bws || !h->have_forward || !h->fwd_data || S != h->last_S) return MOE_ERR_STATE;
   if (!dWg || !dW1 || !dW2 || !aligned(dWg, 16) || !aligned(dW1, 16) || !aligned(dW2, 16) ||
       (dbias && !aligned(dbias, 4)))

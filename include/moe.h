@@ -102,10 +102,19 @@ MOE_API moe_status moe_forward(moe_handle h, int64_t S, const void* x_dev, void*
 
 /*
  * moe_forward_host -- the same forward from and to HOST memory: copies x_host
- * ([S, M] act) into the handle's device staging buffer, runs moe_forward and
- * copies y back into y_host ([S, M] act), all enqueued on `stream`.  The host
- * buffers must stay valid until the stream reaches this point; page-locked
- * (pinned) buffers make the copies asynchronous.
+ * ([S, M] act) into a device staging buffer of the handle, runs the forward and
+ * copies y back into y_host ([S, M] act).
+ *
+ * The three steps run on the handle's own copy-in, compute and copy-out streams
+ * with two staging slots, so back-to-back calls overlap: call i+1's input copy
+ * runs during call i's compute, and call i's output copy during call i+1's.
+ * Ordering: `stream` is made to wait for this call's copy back of y (synchronise
+ * `stream` before reading y_host).  A call that follows another kind of call on
+ * the handle first waits for the work already enqueued on `stream`; a call that
+ * follows a moe_forward_host does not, so it must not depend on device work the
+ * caller enqueued on `stream` in between (its input is host memory).  x_host and
+ * y_host must stay valid, and x_host unchanged, until `stream` passes this call.
+ * Page-locked (pinned) buffers make the copies asynchronous.
  */
 MOE_API moe_status moe_forward_host(moe_handle h, int64_t S, const void* x_host, void* y_host, void* stream);
 

@@ -75,3 +75,27 @@ def test_dropless_capacity_factor_keeps_everything():
     out, rt = G.full_check(run)
     assert rt.C == 500 and np.all(rt.slot >= 0)
     run.layer.close()
+
+
+def test_host_pipeline_back_to_back_calls():
+    """moe_forward_host calls issued back to back (their copies overlap the previous
+    call's compute) each return exactly what a device forward of the same batch does,
+    also with a device forward and different token counts in between."""
+    w = Workload("pipe", 700, 128, 256, 8, 2, 1.25, "bf16", seed=26)
+    run = G.build(w)
+    batches = []
+    for i, S in enumerate((700, 333, 700, 1, 512, 700)):
+        xd = torch.roll(run.x, shifts=37 * i, dims=0)[:S].contiguous()
+        batches.append((xd, xd.cpu().pin_memory(), torch.empty(S, w.M, dtype=xd.dtype).pin_memory()))
+    y_mid = None
+    for i, (xd, xh, yh) in enumerate(batches):
+        run.layer.forward_host(xh, yh)
+        if i == 2:
+            y_mid = run.layer(batches[1][0])        # a device forward between host calls
+    torch.cuda.synchronize()
+    for xd, xh, yh in batches:
+        ref = run.layer(xd)
+        torch.cuda.synchronize()
+        assert torch.equal(yh, ref.cpu())
+    assert torch.equal(y_mid, run.layer(batches[1][0]))
+    run.layer.close()
