@@ -291,3 +291,83 @@ def test_skip_empty_experts_leaves_their_gradients(act, shape):
         if dense[key] is not None:
             assert torch.equal(sparse[key], dense[key]), key
     run.layer.close()
+
+
+def test_backward_large_sampled():
+    """The large workload at full size (experts at capacity: the CTA-pair backward
+    kernels over many tiles and waves): 16 rows of dW2[e] and 16 columns of dW1[e]
+    for four experts, and dx of tokens whose kept choices all lie in those experts,
+    each from the oracle's step functions (no gate-weight gradient here: it needs
+    every kept row's FFN output; the mid test checks it in full)."""
+    w = WORKLOADS["large"]
+    run = G.build(w)
+    out = G.forward(run)
+    rt = G.check_routing(run, out)
+    dy = upstream_grad(w, device="cuda")
+    a_aux, a_z = 0.01, 0.001
+    g = run.layer.backward(out.x, dy, a_aux, a_z)
+    torch.cuda.synchronize()
+    S, E, k, M, H = w.S, w.E, w.k, w.M, w.H
+    rng = np.random.default_rng(11)
+    sample_e = sorted(rng.choice(E, 4, replace=False).tolist())
+    errs = {}
+    W = {}
+    for e in sample_e:
+        W[e] = (_np(run.W1[e]), _np(run.W2[e]))
+        sel = [(t, r) for r in range(k) for t in np.nonzero((rt.ids[:, r] == e) & (rt.slot[:, r] >= 0))[0]]
+        sel.sort(key=lambda tr: rt.slot[tr[0], tr[1]])
+        ts = np.array([t for t, _ in sel])
+        rs = np.array([r for _, r in sel])
+        W1e, W2e = W[e]
+        xr = _np(out.x[torch.as_tensor(ts, device="cuda")])
+        dY = rt.gates[ts, rs][:, None] * _np(dy[torch.as_tensor(ts, device="cuda")])
+        cols = rng.choice(H, 16, replace=False)
+        # dW2[e][cols, :] = relu(pre[:, cols])^T dY
+        pre_c = xr @ W1e[:, cols]
+        ref2 = np.maximum(pre_c, 0.0).T @ dY
+        got2 = _np(g["dW2"][e])[cols]
+        errs[f"dW2[{e}] rows"] = _excess_err(got2, ref2)
+        errs[f"fro dW2[{e}] rows"] = _fro_err(got2, ref2)
+        # dW1[e][:, cols] = X^T ((dY W2[e][cols]^T) * [pre[:, cols] > 0])
+        dq = dY @ W2e[cols].T
+        amb = np.abs(pre_c) <= M * 2.0 ** -23 * (np.abs(xr) @ np.abs(W1e[:, cols]))
+        ref1 = xr.T @ (dq * (pre_c > 0))
+        slack1 = np.abs(xr).T @ (np.abs(dq) * amb)
+        got1 = _np(g["dW1"][e])[:, cols]
+        errs[f"dW1[{e}] cols"] = _excess_err(got1, ref1, slack1)
+        errs[f"fro dW1[{e}] cols"] = _fro_err(got1, ref1)
+    # dx of tokens whose kept choices all lie in the sampled experts
+    kept = rt.slot >= 0
+    inset = np.isin(rt.ids, sample_e) | ~kept
+    toks = np.nonzero(inset.all(axis=1) & kept.any(axis=1))[0][:48]
+    assert len(toks) >= 8
+    xs = _np(out.x[torch.as_tensor(toks, device="cuda")])
+    dys = _np(dy[torch.as_tensor(toks, device="cuda")])
+    Wg = _np(run.Wg)
+    dgate = np.zeros((len(toks), k))
+    dxe = np.zeros((len(toks), M))
+    slack = np.zeros((len(toks), M))
+    for i, t in enumerate(toks):
+        for r in range(k):
+            if rt.slot[t, r] < 0:
+                continue
+            W1e, W2e = W[int(rt.ids[t, r])]
+            pre = xs[i] @ W1e
+            yrow = np.maximum(pre, 0.0) @ W2e
+            dgate[i, r] = dys[i] @ yrow
+            dq = (rt.gates[t, r] * dys[i]) @ W2e.T
+            amb = np.abs(pre) <= M * 2.0 ** -23 * (np.abs(xs[i]) @ np.abs(W1e))
+            dxe[i] += (dq * (pre > 0)) @ W1e.T
+            slack[i] += (np.abs(dq) * amb) @ np.abs(W1e).T
+    dl = O.gates_backward(rt.gates[toks], rt.ids[toks], dgate, E)
+    dl += a_aux * O.aux_loss_backward(rt.p[toks], rt.f, E, S=S)
+    dl += a_z * O.z_loss_backward(rt.p[toks], rt.lse[toks], S=S)
+    ref_dx = dxe + dl @ Wg.T
+    got_dx = _np(g["dx"][torch.as_tensor(toks, device="cuda")])
+    errs["dx"] = _excess_err(got_dx, ref_dx, slack)
+    errs["fro dx"] = _fro_err(got_dx, ref_dx)
+    print(f"\nlarge backward errors ({len(toks)} tokens): {errs}")
+    _check_all(errs, "bf16")
+    run.layer.close()
+    del run
+    torch.cuda.empty_cache()
