@@ -105,12 +105,12 @@ def _gates_uncentred(gates, ids, dgate, E):
     return dl
 
 
-def _aux_uncentred(p, f, E):
-    return E / p.shape[0] * p * f[None, :]
+def _aux_uncentred(p, f, E, S=None):
+    return E / (p.shape[0] if S is None else S) * p * f[None, :]
 
 
-def _z_wrong_sign(p, lse):
-    return -2.0 / p.shape[0] * lse[:, None] * p
+def _z_wrong_sign(p, lse, S=None):
+    return -2.0 / (p.shape[0] if S is None else S) * lse[:, None] * p
 
 
 PLANTS = {
