@@ -371,3 +371,20 @@ def test_backward_large_sampled():
     run.layer.close()
     del run
     torch.cuda.empty_cache()
+
+
+def test_backward_stage_times():
+    """With profiling on, the backward records its eight stages."""
+    w = Workload("prof", 512, 256, 256, 8, 2, 1.25, "bf16", seed=35)
+    run = G.build(w)
+    run.layer(run.x)
+    dy = upstream_grad(w, device="cuda")
+    run.layer.backward(run.x, dy)                # allocates the backward workspace
+    L.moe_set_profiling(run.layer.h, True)
+    run.layer(run.x)
+    run.layer.backward(run.x, dy)
+    ms = L.moe_get_backward_stage_times(run.layer.h)
+    L.moe_set_profiling(run.layer.h, False)
+    assert len(ms) == L.MOE_NUM_BWD_STAGES and all(t >= 0.0 for t in ms) and sum(ms) > 0.0
+    assert [L.moe_backward_stage_name(i) for i in range(len(ms))] == list(L.BWD_STAGES)
+    run.layer.close()

@@ -99,3 +99,29 @@ def test_host_pipeline_back_to_back_calls():
         assert torch.equal(yh, ref.cpu())
     assert torch.equal(y_mid, run.layer(batches[1][0]))
     run.layer.close()
+
+
+def test_cuda_graph_replay_matches_eager():
+    """moe_forward captured in a CUDA graph (as the bench times it) and replayed on
+    new contents of the same input buffer gives what an eager call gives."""
+    w = Workload("graph", 512, 256, 512, 8, 2, 1.25, "bf16", seed=27)
+    run = G.build(w)
+    x = run.x.clone()
+    y = torch.empty_like(x)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run.layer(x, out=y)                      # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run.layer(x, out=y)
+    for shift in (0, 101, 7):
+        x.copy_(torch.roll(run.x, shifts=shift, dims=0))
+        graph.replay()
+        torch.cuda.synchronize()
+        ref = run.layer(x.clone())
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref), shift
+    del graph
+    run.layer.close()
