@@ -388,3 +388,26 @@ def test_backward_stage_times():
     assert len(ms) == L.MOE_NUM_BWD_STAGES and all(t >= 0.0 for t in ms) and sum(ms) > 0.0
     assert [L.moe_backward_stage_name(i) for i in range(len(ms))] == list(L.BWD_STAGES)
     run.layer.close()
+
+
+EDGE = [
+    # (S, M, H, E, k, cf, act, skew_bias)
+    (1, 128, 128, 4, 2, 1.0, "bf16", False),      # one token
+    (300, 128, 256, 1, 1, 1.0, "bf16", False),    # one expert: a dense FFN, no gate gradient
+    (200, 128, 128, 4, 4, 1.0, "bf16", False),    # k = E
+    (97, 64, 128, 6, 2, 0.75, "f32", True),       # fp32 with a gate bias and drops
+    (65, 64, 64, 3, 3, 2.0, "f32", False),        # fp32, k = E, no drops
+]
+
+
+@pytest.mark.parametrize("shape", EDGE, ids=[str(s) for s in EDGE])
+def test_backward_edge_shapes(shape):
+    S, M, H, E, k, cf, act, skew = shape
+    w = Workload("edge", S, M, H, E, k, cf, act, skew_bias=skew, seed=36)
+    # one expert: the gate and l_aux gradients vanish (g = p = 1); with a_z = 0 so does dW_g
+    run, out, g, ref, errs = backward_check(w, a_z=0.0 if E == 1 else 0.3)
+    print(f"\n{shape}: {errs}")
+    _check_all(errs, act)
+    if E == 1:
+        assert np.abs(_np(g["dWg"])).max() <= 1e-6 * np.abs(_np(g["dx"])).max()
+    run.layer.close()
