@@ -79,7 +79,12 @@ struct TileIter {
 
 // Epilogue modes: plain store, ReLU, or the backward's ReLU mask (keep the
 // accumulator where the first layer's saved output h is > 0, else 0).
-enum { kEpiNone = 0, kEpiRelu = 1, kEpiMask = 2, kEpiF32 = 3 };
+enum { kEpiNone = 0, kEpiRelu = 1, kEpiMask = 2, kEpiF32 = 3, kEpiReluBits = 4, kEpiMaskBits = 5 };
+// kEpiReluBits: ReLU, and one bit per stored element, set when the stored bf16 value
+// is > 0 (the backward's mask, 1/16 of the bytes of h).  kEpiMaskBits: keep the
+// accumulator where that bit is set.  Bit j of word w of a row covers column 32w + j;
+// the words are stored word-major, bits[w][row] (rows = E * Cbuf), so a warp's 32
+// consecutive rows write and read one 128-byte line per word.
 
 // 32 mask bits for 32 consecutive bf16 values of h: bit j set iff h[j] > 0
 // (bit patterns 0x0001 .. 0x7f80: positive finite or +inf).
@@ -109,7 +114,9 @@ __device__ __forceinline__ uint32_t positive_bits(const uint4 (&v)[4]) {
 template <int BN, int EPI>
 __device__ __forceinline__ void store_rows(const CUtensorMap* tmD, uint32_t tmem_rows,
                                            uint32_t stage, int row0, int col0, int lane,
-                                           const uint16_t* mrow = nullptr, bool zero = false) {
+                                           const uint16_t* mrow = nullptr, bool zero = false,
+                                           uint32_t* brow = nullptr, const uint32_t* bw = nullptr,
+                                           int64_t bstride = 0) {
   if (EPI == kEpiF32) {
     // fp32 result: 32 columns (128 bytes) per row per store, same swizzled staging
 #pragma unroll 1
@@ -164,6 +171,8 @@ __device__ __forceinline__ void store_rows(const CUtensorMap* tmD, uint32_t tmem
       if (EPI == kEpiMask) {
         const uint4 mv[4] = {mcur[4 * h], mcur[4 * h + 1], mcur[4 * h + 2], mcur[4 * h + 3]};
         keep = positive_bits(mv);
+      } else if (EPI == kEpiMaskBits) {
+        keep = bw[2 * b + h];
       }
       uint32_t r[32];
       if (zero) {
@@ -177,14 +186,23 @@ __device__ __forceinline__ void store_rows(const CUtensorMap* tmD, uint32_t tmem
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         float a = __uint_as_float(r[2 * j]), c = __uint_as_float(r[2 * j + 1]);
-        if (EPI == kEpiRelu) {
+        if (EPI == kEpiRelu || EPI == kEpiReluBits) {
           a = fmaxf(a, 0.f);
           c = fmaxf(c, 0.f);
-        } else if (EPI == kEpiMask) {
+        } else if (EPI == kEpiMask || EPI == kEpiMaskBits) {
           a = ((keep >> (2 * j)) & 1u) ? a : 0.f;
           c = ((keep >> (2 * j + 1)) & 1u) ? c : 0.f;
         }
         pk[j] = pack_bf16x2(a, c);
+      }
+      if (EPI == kEpiReluBits) {    // positive stored values: bit patterns 0x0001 .. 0x7f80
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          word |= (uint32_t)((pk[j] & 0xFFFFu) - 1u < 0x7F80u) << (2 * j);
+          word |= (uint32_t)((pk[j] >> 16) - 1u < 0x7F80u) << (2 * j + 1);
+        }
+        brow[(int64_t)(2 * b + h) * bstride] = word;
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -210,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
                   int64_t Cbuf, int K, int N, const uint16_t* __restrict__ mask, int64_t row_limit,
-                  unsigned* err, uint64_t limit_ns) {
+                  uint32_t* __restrict__ bits, unsigned* err, uint64_t limit_ns) {
   using C = Cfg<BN>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -392,6 +410,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < BN * 2 / 128; ++c) prefetch_l2(reinterpret_cast<const char*>(mrow) + c * 128);
       }
+      const int64_t bstride = (int64_t)E * Cbuf;
+      uint32_t* brow = (EPI == kEpiReluBits || EPI == kEpiMaskBits)
+                           ? bits + (int64_t)nt * (BN / 32) * bstride + row0 + lane : nullptr;
+      uint32_t bw[BN / 32];
+      if (EPI == kEpiMaskBits) {       // this row's mask words, loaded while the MMAs run
+#pragma unroll
+        for (int w = 0; w < BN / 32; ++w) bw[w] = __ldg(brow + w * bstride);
+      }
       if (*abort_flag || !mbar_wait(tfull_bar(acc), aph, err, limit_ns)) {
         *abort_flag = 1;
         break;
@@ -399,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (row0 < row_limit)           // a store box starts inside the tensor (TMA clips its tail)
         store_rows<BN, EPI>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
-                            nt * BN, lane, mrow);
+                            nt * BN, lane, mrow, false, brow, bw, bstride);
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
     }
@@ -645,8 +671,8 @@ template <int EPI, bool BKM>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ffn_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
-                   int64_t Cbuf, int K, int N, const uint16_t* __restrict__ mask, unsigned* err,
-                   uint64_t limit_ns) {
+                   int64_t Cbuf, int K, int N, const uint16_t* __restrict__ mask,
+                   uint32_t* __restrict__ bits, unsigned* err, uint64_t limit_ns) {
   using namespace pairk;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -820,15 +846,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int tile = pair; it.decode(tile, e, mt, nt); tile += npairs, ++i) {
       const int acc = i & 1;
       const uint32_t aph = (i >> 1) & 1;
+      const int row0 = (int)(e * Cbuf + mt * PM + (int)rank * (PM / 2) + q * 32);
+      const uint16_t* mrow = EPI == kEpiMask ? mask + (int64_t)(row0 + lane) * N + nt * BN : nullptr;
+      const int64_t bstride = (int64_t)E * Cbuf;
+      uint32_t* brow = (EPI == kEpiReluBits || EPI == kEpiMaskBits)
+                           ? bits + (int64_t)nt * (BN / 32) * bstride + row0 + lane : nullptr;
+      uint32_t bw[BN / 32];
+      if (EPI == kEpiMaskBits) {       // this row's mask words, loaded while the MMAs run
+#pragma unroll
+        for (int w = 0; w < BN / 32; ++w) bw[w] = __ldg(brow + w * bstride);
+      }
       if (*abort_flag || !mbar_wait(tfull_bar(acc), aph, err, limit_ns)) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const int row0 = (int)(e * Cbuf + mt * PM + (int)rank * (PM / 2) + q * 32);
-      const uint16_t* mrow = EPI == kEpiMask ? mask + (int64_t)(row0 + lane) * N + nt * BN : nullptr;
       store_rows<BN, EPI>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
-                          nt * BN, lane, mrow);
+                          nt * BN, lane, mrow, false, brow, bw, bstride);
       tc_fence_before();
       if (leader) mbar_arrive(tempty_bar(acc));
       else mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
@@ -1078,7 +1112,7 @@ cudaError_t launch_pair(const GemmPlan& p, const int32_t* nexp, unsigned* err, u
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(num_sms & ~1), dim3(kThreads), pairk::SMEM, st, p.tmA,
                     BKM ? p.tmB2 : p.tmB, p.tmD, nexp, p.E, p.Cbuf, p.K, p.N,
-                    static_cast<const uint16_t*>(p.mask), err, limit_ns);
+                    static_cast<const uint16_t*>(p.mask), p.bits, err, limit_ns);
 }
 
 template <int BN, int EPI, bool BKM>
@@ -1090,7 +1124,8 @@ cudaError_t launch_t(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint
   if (e != cudaSuccess) return e;
   const int64_t row_limit = p.row_limit > 0 ? p.row_limit : (int64_t)p.E * p.Cbuf;
   return launch_pdl(kern, dim3(num_sms), dim3(kThreads), smem, st, p.tmA, p.tmB, p.tmD, nexp, p.E,
-                    p.Cbuf, p.K, p.N, static_cast<const uint16_t*>(p.mask), row_limit, err, limit_ns);
+                    p.Cbuf, p.K, p.N, static_cast<const uint16_t*>(p.mask), row_limit, p.bits, err,
+                    limit_ns);
 }
 
 template <int BN, int EPI>
@@ -1216,35 +1251,47 @@ cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* er
     }
   }
   if (p.kind == kGemmDgrad) {
-    const bool m = p.mask != nullptr;
-    if (p.pair && want_pair && (p.Cbuf % pairk::PM) == 0)
-      return m ? launch_pair<kEpiMask, true>(p, nexp, err, wait_limit_ns, num_sms, st)
-               : launch_pair<kEpiNone, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+    const int epi = (p.bits && p.use_bits) ? kEpiMaskBits : (p.mask ? kEpiMask : kEpiNone);
+    if (p.pair && want_pair && (p.Cbuf % pairk::PM) == 0) {
+      if (epi == kEpiMaskBits) return launch_pair<kEpiMaskBits, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+      if (epi == kEpiMask) return launch_pair<kEpiMask, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+      return launch_pair<kEpiNone, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+    }
     switch (p.BN) {
       case 256:
-        return m ? launch_t<256, kEpiMask, true>(p, nexp, err, wait_limit_ns, num_sms, st)
-                 : launch_t<256, kEpiNone, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+        if (epi == kEpiMaskBits) return launch_t<256, kEpiMaskBits, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+        if (epi == kEpiMask) return launch_t<256, kEpiMask, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+        return launch_t<256, kEpiNone, true>(p, nexp, err, wait_limit_ns, num_sms, st);
       case 128:
-        return m ? launch_t<128, kEpiMask, true>(p, nexp, err, wait_limit_ns, num_sms, st)
-                 : launch_t<128, kEpiNone, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+        if (epi == kEpiMaskBits) return launch_t<128, kEpiMaskBits, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+        if (epi == kEpiMask) return launch_t<128, kEpiMask, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+        return launch_t<128, kEpiNone, true>(p, nexp, err, wait_limit_ns, num_sms, st);
       default:
-        return m ? launch_t<64, kEpiMask, true>(p, nexp, err, wait_limit_ns, num_sms, st)
-                 : launch_t<64, kEpiNone, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+        if (epi == kEpiMaskBits) return launch_t<64, kEpiMaskBits, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+        if (epi == kEpiMask) return launch_t<64, kEpiMask, true>(p, nexp, err, wait_limit_ns, num_sms, st);
+        return launch_t<64, kEpiNone, true>(p, nexp, err, wait_limit_ns, num_sms, st);
     }
   }
-  if (p.pair && want_pair && (p.Cbuf % pairk::PM) == 0)
-    return p.relu ? launch_pair<kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st)
-                  : launch_pair<kEpiNone, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+  // forward: ReLU (and the backward's mask bits when a bit buffer is set) or none
+  const int epi = p.relu ? (p.bits ? kEpiReluBits : kEpiRelu) : kEpiNone;
+  if (p.pair && want_pair && (p.Cbuf % pairk::PM) == 0) {
+    if (epi == kEpiReluBits) return launch_pair<kEpiReluBits, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+    if (epi == kEpiRelu) return launch_pair<kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+    return launch_pair<kEpiNone, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+  }
   switch (p.BN) {
     case 256:
-      return p.relu ? launch_t<256, kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st)
-                    : launch_t<256, kEpiNone, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      if (epi == kEpiReluBits) return launch_t<256, kEpiReluBits, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      if (epi == kEpiRelu) return launch_t<256, kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      return launch_t<256, kEpiNone, false>(p, nexp, err, wait_limit_ns, num_sms, st);
     case 128:
-      return p.relu ? launch_t<128, kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st)
-                    : launch_t<128, kEpiNone, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      if (epi == kEpiReluBits) return launch_t<128, kEpiReluBits, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      if (epi == kEpiRelu) return launch_t<128, kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      return launch_t<128, kEpiNone, false>(p, nexp, err, wait_limit_ns, num_sms, st);
     default:
-      return p.relu ? launch_t<64, kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st)
-                    : launch_t<64, kEpiNone, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      if (epi == kEpiReluBits) return launch_t<64, kEpiReluBits, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      if (epi == kEpiRelu) return launch_t<64, kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      return launch_t<64, kEpiNone, false>(p, nexp, err, wait_limit_ns, num_sms, st);
   }
 }
 

@@ -83,6 +83,9 @@ struct GemmPlan {
   CUtensorMap tmB2;  // kGemmDgrad CTA pairs: B box {64, 128} (each CTA's half of the N rows)
   void* D;
   const void* mask;  // kGemmDgrad: [E*Cbuf, N] bf16 values whose sign masks the result, or null
+  uint32_t* bits;    // [N/32, E*Cbuf] mask bits, word-major: kGemmFwd with ReLU writes them (h > 0);
+                     // kGemmDgrad reads them instead of `mask` when use_bits is set
+  bool use_bits;
   int kind;
   int E, K, N, BN;
   int64_t Cbuf;

@@ -68,6 +68,8 @@ struct moe_layer {
   const void* dw2_ptr;
   const void* dw1_ptr;
   uint32_t bwd_flags;               // MOE_BWD_* flags
+  uint32_t* hbits;                  // [H/32, E*Cbuf] bits of h > 0, written by FFN1 once enabled
+  bool bits_valid;                  // the last forward wrote hbits
   // bf16: tensor-core gate gradients
   int EPb;                          // E rounded up to 64
   void* dlb;                        // [S_max, 2*EPb] bf16 split of dl
@@ -310,6 +312,7 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
   h->last_S = S;
   h->have_forward = true;
   h->fwd_data = true;
+  h->bits_valid = false;
   if (S == 0) {
     MOE_TRY(cudaMemsetAsync(h->R.losses, 0, 2 * sizeof(float), st));
     return MOE_OK;
@@ -343,6 +346,7 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
     // otherwise 128-row tiles waste less on partly filled last tiles.
     const bool saturated = (double)S * h->k / h->E >= (double)C;
     MOE_TRY(launch_ffn_bf16(h->plan1, R.nexp, R.err, h->wait_limit_ns, h->num_sms, saturated, st));
+    h->bits_valid = h->plan1.bits != nullptr;
     MOE_TRY(mark(4));
     MOE_TRY(launch_ffn_bf16(h->plan2, R.nexp, R.err, h->wait_limit_ns, h->num_sms, saturated, st));
   } else {
@@ -487,6 +491,7 @@ moe_status moe_route_from_logits(moe_handle h, int64_t S, const float* logits, v
   h->last_S = S;
   h->have_forward = true;
   h->fwd_data = false;
+  h->bits_valid = false;
   if (S == 0) {
     MOE_TRY(cudaMemsetAsync(h->R.losses, 0, 2 * sizeof(float), st));
     return MOE_OK;
@@ -540,6 +545,7 @@ moe_status moe_enable_backward(moe_handle h) {
     h->dlb = bf16 ? c.take<char>((size_t)h->S_max * 2 * h->EPb * 2) : nullptr;
     h->bpart = bf16 ? c.take<float>((size_t)4 * h->num_sms * h->E) : nullptr;
     h->cnt_rows = bf16 ? c.take<int32_t>((size_t)1 + ns_max) : nullptr;
+    h->hbits = bf16 ? c.take<uint32_t>((size_t)rowsE * (h->H / 32)) : nullptr;
     if (pass == 0) {
       const size_t bytes = c.off + 256;
       cudaError_t ce = cudaMalloc(&h->bws, bytes);
@@ -560,6 +566,10 @@ moe_status moe_enable_backward(moe_handle h) {
       h->bws = nullptr;
       return MOE_ERR_CUDA;
     }
+    // from now on FFN1 also writes the bits of h > 0, which dP reads instead of h
+    h->plan1.bits = h->hbits;
+    h->plan_dp.bits = h->hbits;
+    h->bits_valid = false;
   }
   h->dw1_ptr = h->dw2_ptr = nullptr;
   h->gdx_ptr = h->dwg_ptr = nullptr;
@@ -663,6 +673,7 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
     const bool skip = (h->bwd_flags & MOE_BWD_SKIP_EMPTY_EXPERTS) != 0;
     h->plan_dw2.skip_zero = skip;
     h->plan_dw1.skip_zero = skip;
+    h->plan_dp.use_bits = h->bits_valid;   // else the mask is read from h itself
     // the weight-gradient GEMMs reduce over whole 64-slot blocks: clear the rows
     // between the kept count and the next multiple of 64
     void* bufs[3] = {h->xbuf, h->hbuf, h->dybuf};
