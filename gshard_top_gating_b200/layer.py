@@ -45,6 +45,14 @@ class MoeLayer:
     def aux_loss(self, stream=None):
         return L.moe_aux_loss(self.h, stream)
 
+    def enable_backward(self) -> None:
+        """Allocate the backward workspace now (moe_enable_backward).  Forwards
+        that run after it also store the ReLU mask bits the backward reads; a
+        backward of a forward that ran before it re-reads h instead."""
+        if not getattr(self, "_bwd", False):
+            L.moe_enable_backward(self.h)
+            self._bwd = True
+
     def backward(self, x: torch.Tensor, dy: torch.Tensor, a_aux: float = 0.0, a_z: float = 0.0,
                  stream=None, out: dict | None = None, skip_empty_experts: bool = False) -> dict:
         """Gradients of <dy, y> + a_aux*l_aux + a_z*z for the last forward (which took x).
@@ -55,9 +63,7 @@ class MoeLayer:
         left as they were (MOE_BWD_SKIP_EMPTY_EXPERTS).  The backward workspace is
         allocated on the first call.
         """
-        if not getattr(self, "_bwd", False):
-            L.moe_enable_backward(self.h)
-            self._bwd = True
+        self.enable_backward()
         for t in (x, dy):
             if t.dtype != self.act or not t.is_contiguous() or t.dim() != 2 or t.shape[1] != self.M:
                 raise ValueError("x and dy must be contiguous [S, M] tensors of the activation dtype")

@@ -86,8 +86,12 @@ def _mask_slack(ref, W1, W2, K):
     return s_dW1, s_dx
 
 
-def backward_check(w, a_aux=0.7, a_z=0.3, S=None):
+def backward_check(w, a_aux=0.7, a_z=0.3, S=None, train=True):
+    """train: the backward is enabled before the forward, so FFN1 stores the
+    ReLU mask bits that dP reads; otherwise dP re-reads h."""
     run = G.build(w, S=S)
+    if train:
+        run.layer.enable_backward()
     out = G.forward(run)
     G.check_routing(run, out)
     dy = upstream_grad(w, device="cuda", S=run.S)
@@ -158,6 +162,26 @@ def test_bf16_backward(shape):
     run.layer.close()
 
 
+@pytest.mark.parametrize("shape", [(700, 256, 256, 8, 2, 1.0), (4096, 512, 1024, 8, 2, 1.0)],
+                         ids=["one-cta", "cta-pair"])
+def test_mask_bits_equal_mask_from_h(shape):
+    """dP's ReLU mask from the bits FFN1 stores in training mode and from
+    re-reading h select the same elements: all gradients are bitwise equal.
+    The second shape puts every expert at capacity (CTA-pair kernels)."""
+    S, M, H, E, k, cf = shape
+    w = Workload("bits", S, M, H, E, k, cf, "bf16", seed=34)
+    run = G.build(w)
+    dy = upstream_grad(w, device="cuda")
+    run.layer(run.x)                               # forward before the backward is enabled
+    g_h = run.layer.backward(run.x, dy, 0.5, 0.1)  # dP re-reads h
+    run.layer(run.x)                               # forward in training mode: mask bits
+    g_bits = run.layer.backward(run.x, dy, 0.5, 0.1)
+    torch.cuda.synchronize()
+    for key in g_h:
+        assert torch.equal(g_h[key], g_bits[key]), key
+    run.layer.close()
+
+
 def test_backward_is_deterministic_and_repeatable():
     w = Workload("det", 700, 256, 256, 8, 2, 1.0, "bf16", skew_bias=True, seed=32)
     run = G.build(w)
@@ -201,6 +225,7 @@ def test_backward_mid_full_size():
     tokens, each from the oracle's step functions one expert or token at a time."""
     w = WORKLOADS["mid"]
     run = G.build(w)
+    run.layer.enable_backward()                    # training mode: FFN1 stores the mask bits
     out = G.forward(run)
     rt = G.check_routing(run, out)
     dy = upstream_grad(w, device="cuda")
@@ -301,6 +326,7 @@ def test_backward_large_sampled():
     every kept row's FFN output; the mid test checks it in full)."""
     w = WORKLOADS["large"]
     run = G.build(w)
+    run.layer.enable_backward()                    # training mode: FFN1 stores the mask bits
     out = G.forward(run)
     rt = G.check_routing(run, out)
     dy = upstream_grad(w, device="cuda")
