@@ -11,12 +11,16 @@
 // W_g = hi + mid + lo (about 24 significant bits, the bf16x3 scheme of Henry,
 // Tang and Heinecke, "Leveraging the bfloat16 artificial intelligence datatype
 // for higher-precision computations", ARITH 2019).  The three products
-// x.hi + x.mid + x.lo accumulate in an fp32 TMEM accumulator.  The tensor
-// core's fp32 accumulation does not round to nearest, and over a long K its
-// rounding error builds up coherently, so K is cut into segments of
-// kSegBlocks*64: each segment accumulates from zero and the epilogue warps add
-// it into a second TMEM region with ordinary round-to-nearest fp32 adds.  The
-// logits so carry fp32-level error at tensor-core speed.
+// x.hi, x.mid, x.lo accumulate in fp32 TMEM columns: for EP <= 64 each part has
+// its own column group and one MMA of N = 3*EP covers all three, so a 16-deep K
+// step is one instruction instead of three and reads the token tile from shared
+// memory once; for EP >= 128 (MMAs of N >= 128, long enough on their own) the
+// three parts add into one accumulator.  The tensor core's fp32 accumulation does not round to
+// nearest, and over a long K its rounding error builds up coherently, so K is
+// cut into segments of kSegBlocks*64: each segment accumulates from zero and the
+// epilogue warps add it (lo + mid, then + hi) into a running sum with ordinary
+// round-to-nearest fp32 adds.  The logits so carry fp32-level error at
+// tensor-core speed.
 //
 // One CTA = 128 tokens (64 for small batches with E <= 64) x EP experts (E padded
 // to 32/64/128/256), 512 threads:
@@ -61,17 +65,24 @@ struct RCfg {
   // flight the prefetches only queue ahead of the loads in the TMA unit (measured:
   // slower); with 2 stages (E > 128) they hide the DRAM latency of x.
   static constexpr int PREFETCH_X = STAGES <= 2 ? 12 : 0;
-  static constexpr uint32_t TMEM_COLS = 2 * EP;        // accumulator + running sum
+  // column groups of the accumulator: hi | mid | lo for EP <= 64, one shared group above
+  static constexpr int NG = EP <= 64 ? 3 : 1;
+  static constexpr uint32_t ACC_COLS = NG * EP;        // the running sum follows
+  static constexpr uint32_t TMEM_COLS =
+      ACC_COLS + EP <= 128 ? 128 : (ACC_COLS + EP <= 256 ? 256 : 512);
   // epilogue scratch reuses the stage buffers: logits L [TT][EP+1] f32 (padded row),
   // per-warp probability sums red [16][EP] f32, per-warp lse^2 [16], sel [TT][8] i32,
-  // hist [NCH][8][EP] i32
+  // running counts / hist [NCH][8][EP] i32
   static constexpr uint32_t LD = EP + 1;
   static constexpr uint32_t L_OFF = 0;
   static constexpr uint32_t RED_OFF = L_OFF + TT * LD * 4;
   static constexpr uint32_t LSE_OFF = RED_OFF + 16 * EP * 4;
   static constexpr uint32_t SEL_OFF = LSE_OFF + 16 * 4;
   static constexpr uint32_t H_OFF = SEL_OFF + TT * kMaxK * 4;
-  static constexpr uint32_t EPI_END = H_OFF + NCH * kMaxK * EP * 4;
+  // E <= 64 (thread-per-token routing): probabilities P [TT][EP+1] f32, lse^2 per token [TT]
+  static constexpr uint32_t P_OFF = H_OFF + NCH * kMaxK * EP * 4;
+  static constexpr uint32_t LSET_OFF = P_OFF + (EP <= 64 ? TT * LD * 4 : 0);
+  static constexpr uint32_t EPI_END = LSET_OFF + (EP <= 64 ? TT * 4 : 0);
   static_assert(EPI_END <= STAGES * STAGE_BYTES, "epilogue scratch must fit in the stage buffers");
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + 16;
 };
@@ -81,10 +92,11 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
          (1ull << 46) | (2ull << 61);
 }
 
-// kind::f16, D fp32, A bf16 K-major, B bf16 K-major, M=128, N=EP
-template <int EP>
+// kind::f16, D fp32, A bf16 K-major, B bf16 K-major, M=128, N (a multiple of 16, <= 256)
+template <int N>
 __device__ __forceinline__ uint32_t idesc_router() {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(EP >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N out of range");
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
 template <int EP, int TT>
@@ -168,7 +180,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_router<EP>();
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -191,13 +202,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t sa = base + s * C::STAGE_BYTES;
+        if constexpr (C::NG == 3) {
+          // the three parts sit back to back (1024-byte aligned), one K-major operand of 3*EP rows
+          const uint32_t sb = sa + A_BYTES;
 #pragma unroll
-        for (int part = 2; part >= 0; --part) {       // smallest part first
-          const uint32_t sb = sa + A_BYTES + part * C::PART_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
+          for (int kk = 0; kk < BK / 16; ++kk) {
             tc_mma_f16(tmem_base, desc_kmajor_sw128(sa + kk * 32u), desc_kmajor_sw128(sb + kk * 32u),
-                       idesc, !(seg_first && kk == 0 && part == 2));
+                       idesc_router<3 * EP>(), !(seg_first && kk == 0));
+          }
+        } else {
+#pragma unroll
+          for (int part = 2; part >= 0; --part) {       // smallest part first
+            const uint32_t sb = sa + A_BYTES + part * C::PART_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              tc_mma_f16(tmem_base, desc_kmajor_sw128(sa + kk * 32u), desc_kmajor_sw128(sb + kk * 32u),
+                         idesc_router<EP>(), !(seg_first && kk == 0 && part == 2));
+          }
         }
         tc_commit(empty_bar(s));
         if (seg_last) tc_commit(tfull_bar);
@@ -231,8 +252,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < EP / 32; ++c) {
         uint32_t a[32], b[32];
-        tmem_ld_32x32b_x32(tlane + c * 32, a);
-        if (seg > 0) tmem_ld_32x32b_x32(tlane + EP + c * 32, b);
+        if constexpr (C::NG == 3) {    // this segment's x.lo + x.mid, then + x.hi
+          tmem_ld_32x32b_x32(tlane + 2 * EP + c * 32, a);
+          tmem_ld_32x32b_x32(tlane + EP + c * 32, b);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) + __uint_as_float(b[i]));
+          tmem_ld_32x32b_x32(tlane + c * 32, b);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) + __uint_as_float(b[i]));
+        } else {
+          tmem_ld_32x32b_x32(tlane + c * 32, a);
+        }
+        if (seg > 0) tmem_ld_32x32b_x32(tlane + C::ACC_COLS + c * 32, b);
         tmem_ld_wait();
         if (seg > 0) {
 #pragma unroll
@@ -245,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             Ls[row * C::LD + j] = __uint_as_float(a[i]) + ((bias && j < E) ? __ldg(bias + j) : 0.f);
           }
         } else {
-          tmem_st_32x32b_x32(tlane + EP + c * 32, a);
+          tmem_st_32x32b_x32(tlane + C::ACC_COLS + c * 32, a);
         }
       }
       if (!last) tmem_st_wait();
@@ -265,70 +298,185 @@ __global__ void __launch_bounds__(kThreads, 1)
     int32_t* sel = reinterpret_cast<int32_t*>(gbase + C::SEL_OFF);
     int32_t* Hs = reinterpret_cast<int32_t*>(gbase + C::H_OFF);
     constexpr int RE = EP / 32;
-    constexpr int TPW = C::TT / 16;                         // tokens per warp (4 or 8)
-    constexpr int WPC = 16 / C::NCH;                        // warps per 64-token chunk
     const int tid = threadIdx.x;
     const bool good = !*abort_flag;
-    float psum[RE];
-#pragma unroll
-    for (int i = 0; i < RE; ++i) psum[i] = 0.f;
-    float lse2 = 0.f;
     const int ntile = good ? min(C::TT, S - tok0) : 0;
-    for (int t = warp * TPW; t < warp * TPW + TPW && t < ntile; t += 2) {   // two tokens in flight
-      if (t + 1 < ntile) {
-        float v[2][RE];
+    const int chunk0 = tile * C::NCH;
+    for (int i = tid; i < C::NCH * kMaxK * EP; i += kThreads) Hs[i] = 0;
+    if constexpr (EP <= 64) {
+      // One thread per token: the whole logit row is read from shared memory (row
+      // stride EP + 1 words, so the 32 tokens of a warp hit 32 banks).  The warps
+      // without tokens copy the logits tile out, coalesced.
+      float* Ps = reinterpret_cast<float*>(gbase + C::P_OFF);
+      float* lse_t = reinterpret_cast<float*>(gbase + C::LSET_OFF);
+      if (warp < C::TT / 32) {
+        const int t = warp * 32 + lane;
+        if (t < ntile) {
+          const float* Lr = Ls + t * C::LD;
+          float* Pr = Ps + t * C::LD;
+          float mx = -INFINITY;
+#pragma unroll 8
+          for (int j = 0; j < E; ++j) mx = fmaxf(mx, Lr[j]);
+          float sum = 0.f;
+#pragma unroll 8
+          for (int j = 0; j < E; ++j) {
+            const float ex = expf(Lr[j] - mx);
+            Pr[j] = ex;
+            sum += ex;
+          }
+          const float inv = 1.f / sum;
+#pragma unroll 8
+          for (int j = 0; j < E; ++j) Pr[j] *= inv;
+          const float lse = mx + logf(sum);
+          lse_t[t] = lse * lse;
+          // top-k on the logits, ties to the lower expert index (an ascending scan
+          // replaces the incumbent only on a strictly larger logit)
+          uint64_t taken = 0;
+          int er[kMaxK];
+          float lr[kMaxK];
 #pragma unroll
-        for (int n = 0; n < 2; ++n)
+          for (int r = 0; r < kMaxK; ++r) {
+            er[r] = 0;
+            lr[r] = 0.f;
+            if (r < k) {
+              float bv = -INFINITY;
+              int bj = -1;
+#pragma unroll 8
+              for (int j = 0; j < E; ++j) {
+                const float v = Lr[j];
+                if (!((taken >> j) & 1ull) && (v > bv || bj < 0)) {
+                  bv = v;
+                  bj = j;
+                }
+              }
+              if (bj < 0) {                 // k > E: rejected by the host, never reached
+                atomicOr(R.err, DEVERR_BOUNDS);
+                bj = 0;
+              }
+              taken |= 1ull << bj;
+              er[r] = bj;
+              lr[r] = bv;
+            }
+          }
+          float gs = 0.f, gr[kMaxK];
+#pragma unroll
+          for (int r = 0; r < kMaxK; ++r) {
+            gr[r] = (r < k) ? expf(lr[r] - lr[0]) : 0.f;
+            gs += gr[r];
+          }
+          const float ginv = 1.f / gs;
+          const int64_t tok = tok0 + t;
+#pragma unroll
+          for (int r = 0; r < kMaxK; ++r) {
+            if (r < k) {
+              R.eidx[tok * k + r] = er[r];
+              R.gate[tok * k + r] = gr[r] * ginv;
+              sel[t * kMaxK + r] = er[r];
+            }
+          }
+        }
+      } else {
+        const int nthr = kThreads - C::TT;
+        for (int idx = tid - C::TT; idx < ntile * E; idx += nthr) {
+          const int t = idx / E, j = idx - t * E;
+          R.logits[(int64_t)tok0 * E + idx] = Ls[t * C::LD + j];
+        }
+      }
+      __syncthreads();
+      // per-chunk probability sums (tokens in order, four interleaved partial sums)
+      // and lse^2 sums (one warp per chunk, fixed shuffle tree)
+      for (int idx = tid; idx < C::NCH * E; idx += kThreads) {
+        const int cc = idx / E, j = idx - cc * E;
+        const int chunk = chunk0 + cc;
+        if (chunk >= nchunk) continue;
+        const int t0 = cc * kChunk, t1 = min(t0 + kChunk, ntile);
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        int t = t0;
+        for (; t + 4 <= t1; t += 4) {
+          a0 += Ps[t * C::LD + j];
+          a1 += Ps[(t + 1) * C::LD + j];
+          a2 += Ps[(t + 2) * C::LD + j];
+          a3 += Ps[(t + 3) * C::LD + j];
+        }
+        for (; t < t1; ++t) a0 += Ps[t * C::LD + j];
+        R.psum[(int64_t)chunk * E + j] = (a0 + a1) + (a2 + a3);
+      }
+      if (warp < C::NCH && chunk0 + warp < nchunk) {
+        const int t = warp * kChunk + lane;
+        float a = (t < ntile ? lse_t[t] : 0.f) + (t + 32 < ntile ? lse_t[t + 32] : 0.f);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) R.lse2[chunk0 + warp] = a;
+      }
+    } else {
+      // E > 64: one warp per token, lanes over experts
+      constexpr int TPW = C::TT / 16;                         // tokens per warp (4 or 8)
+      constexpr int WPC = 16 / C::NCH;                        // warps per 64-token chunk
+      float psum[RE];
+#pragma unroll
+      for (int i = 0; i < RE; ++i) psum[i] = 0.f;
+      float lse2 = 0.f;
+      for (int t = warp * TPW; t < warp * TPW + TPW && t < ntile; t += 2) {   // two tokens in flight
+        if (t + 1 < ntile) {
+          float v[2][RE];
+#pragma unroll
+          for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int i = 0; i < RE; ++i) {
+              const int j = lane + 32 * i;
+              v[n][i] = j < E ? Ls[(t + n) * C::LD + j] : -INFINITY;
+            }
+          const int64_t tk[2] = {tok0 + t, tok0 + t + 1};
+          int32_t* const rows[2] = {sel + t * kMaxK, sel + (t + 1) * kMaxK};
+          route_tokens<RE, 2>(v, tk, E, k, true, R, psum, lse2, rows);
+        } else {
+          float v[RE];
 #pragma unroll
           for (int i = 0; i < RE; ++i) {
             const int j = lane + 32 * i;
-            v[n][i] = j < E ? Ls[(t + n) * C::LD + j] : -INFINITY;
+            v[i] = j < E ? Ls[t * C::LD + j] : -INFINITY;
           }
-        const int64_t tk[2] = {tok0 + t, tok0 + t + 1};
-        int32_t* const rows[2] = {sel + t * kMaxK, sel + (t + 1) * kMaxK};
-        route_tokens<RE, 2>(v, tk, E, k, true, R, psum, lse2, rows);
-      } else {
-        float v[RE];
-#pragma unroll
-        for (int i = 0; i < RE; ++i) {
-          const int j = lane + 32 * i;
-          v[i] = j < E ? Ls[t * C::LD + j] : -INFINITY;
+          route_token<RE>(v, tok0 + t, E, k, true, R, psum, lse2, sel + t * kMaxK);
         }
-        route_token<RE>(v, tok0 + t, E, k, true, R, psum, lse2, sel + t * kMaxK);
+      }
+#pragma unroll
+      for (int i = 0; i < RE; ++i) red[warp * EP + lane + 32 * i] = psum[i];
+      if (lane == 0) lse_w[warp] = lse2;
+      __syncthreads();
+      // per-chunk probability and lse^2 sums, warps of a chunk added in order
+      for (int cc = 0; cc < C::NCH; ++cc) {
+        const int chunk = chunk0 + cc;
+        if (chunk >= nchunk) break;
+        for (int j = tid; j < E; j += kThreads) {
+          float acc = 0.f;
+#pragma unroll
+          for (int w = 0; w < WPC; ++w) acc += red[(cc * WPC + w) * EP + j];
+          R.psum[(int64_t)chunk * E + j] = acc;
+        }
+        if (tid == 0) {
+          float acc = 0.f;
+#pragma unroll
+          for (int w = 0; w < WPC; ++w) acc += lse_w[cc * WPC + w];
+          R.lse2[chunk] = acc;
+        }
       }
     }
-#pragma unroll
-    for (int i = 0; i < RE; ++i) red[warp * EP + lane + 32 * i] = psum[i];
-    if (lane == 0) lse_w[warp] = lse2;
-    for (int i = tid; i < C::NCH * kMaxK * EP; i += kThreads) Hs[i] = 0;
-    __syncthreads();
-    // per-chunk probability and lse^2 sums, warps of a chunk added in order
-    const int chunk0 = tile * C::NCH;
-    for (int cc = 0; cc < C::NCH; ++cc) {
-      const int chunk = chunk0 + cc;
-      if (chunk >= nchunk) break;
-      for (int j = tid; j < E; j += kThreads) {
-        float acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < WPC; ++w) acc += red[(cc * WPC + w) * EP + j];
-        R.psum[(int64_t)chunk * E + j] = acc;
+    // local ranks within each 64-token chunk and rank-r histograms: one warp per
+    // (chunk, rank), 32 tokens at a time; tokens choosing the same expert find one
+    // another with a match, and a running count per expert carries over
+    for (int pi = warp; pi < C::NCH * k; pi += kThreads / 32) {
+      const int cc = pi / k, r = pi - cc * k;
+      int32_t* cnt = Hs + (cc * kMaxK + r) * EP;
+      for (int h = 0; h < kChunk / 32; ++h) {
+        const int t = cc * kChunk + h * 32 + lane;
+        const bool valid = t < ntile;
+        const int e = valid ? sel[t * kMaxK + r] : EP + lane;       // unmatched when invalid
+        const unsigned m = __match_any_sync(0xffffffffu, e);
+        if (valid) R.lrank[(int64_t)(tok0 + t) * k + r] = cnt[e] + __popc(m & ((1u << lane) - 1u));
+        __syncwarp();
+        if (valid && lane == __ffs(m) - 1) cnt[e] += __popc(m);
+        __syncwarp();
       }
-      if (tid == 0) {
-        float acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < WPC; ++w) acc += lse_w[cc * WPC + w];
-        R.lse2[chunk] = acc;
-      }
-    }
-    // local ranks within each 64-token chunk and rank-r histograms
-    for (int idx = tid; idx < ntile * k; idx += kThreads) {
-      const int t = idx / k, r = idx - t * k;
-      const int e = sel[t * kMaxK + r];
-      const int cbeg = (t >> 6) << 6;
-      int c = 0;
-      for (int u = cbeg; u < t; ++u) c += (sel[u * kMaxK + r] == e);
-      R.lrank[(int64_t)(tok0 + t) * k + r] = c;
-      atomicAdd(&Hs[((t >> 6) * kMaxK + r) * EP + e], 1);
     }
     __syncthreads();
     for (int cc = 0; cc < C::NCH; ++cc) {
