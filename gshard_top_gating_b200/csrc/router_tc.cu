@@ -23,14 +23,17 @@
 // tensor-core speed.
 //
 // One CTA = 128 tokens (64 for small batches with E <= 64) x EP experts (E padded
-// to 32/64/128/256), 512 threads:
+// to 32/64/128/256), 16 warps; or, for 128-token CTAs with E <= 64, 8 warps and
+// fewer stages so that two CTAs share an SM and one's epilogue overlaps the
+// other's loads:
 // warp 0 TMA producer (x tile TTx64 + three W_g parts EPx64 per stage, K-major,
-// 128B swizzle), warp 1 TMEM owner and single-thread MMA issuer, warps 2-5 fold
+// 128B swizzle), warp 1 TMEM owner and single-thread MMA issuer, four warps fold
 // the K-segments (one token row per thread, as TMEM lanes dictate) and leave the
-// final logits tile in shared memory.  Then all sixteen warps route warp-per-token
-// (lanes over experts, shuffle max / sum / argmax, ties to the lower index) and
-// write the same per-64-token chunk tables (probability sums, lse^2 sums,
-// rank-r histograms, local ranks) as the CUDA-core router.
+// final logits tile in shared memory.  Then all warps route (E <= 64: a thread per
+// token; above: a warp per token, lanes over experts, shuffle max / sum / argmax;
+// ties to the lower index) and write the same per-64-token chunk tables
+// (probability sums, lse^2 sums, rank-r histograms, local ranks) as the CUDA-core
+// router.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -45,22 +48,28 @@ int router_tokens_per_cta(int E, int S);
 namespace {
 
 constexpr int BM = 128, BK = 64;
-constexpr int kThreads = 512;   // 16 warps: all route; warps 0/1/2-5 also load / issue / fold
 constexpr uint32_t A_BYTES = BM * BK * 2;
 constexpr int kSegBlocks = 8;      // k-blocks (of 64) accumulated before each fp32 round-to-nearest add
 
-template <int EP, int TT_>
+template <int EP, int TT_, int NW_>
 struct RCfg {
   // tokens per CTA: 128, or 64 when 128-token CTAs would not fill the SMs (twice
   // the CTAs stream x; the MMA keeps M=128 and its upper 64 accumulator rows are
   // ignored)
   static constexpr int TT = TT_;
+  // warps: 16 (one CTA per SM), or 8 (two per SM: 128 tokens and E <= 64 only)
+  static constexpr int NW = NW_;
+  static constexpr int NT = NW * 32;
+  static constexpr int FOLD0 = NW == 8 ? 4 : 2;       // first of the four fold warps
+  static_assert(NW == 16 || (NW == 8 && TT == 128 && EP <= 64), "8-warp CTAs: 128 tokens, E <= 64");
   static constexpr int NCH = TT / kChunk;                       // 64-token chunks per CTA
   static constexpr uint32_t X_BYTES = TT * BK * 2;              // bytes TMA writes into the A tile
   static constexpr uint32_t PART_BYTES = EP * BK * 2;           // one W_g part, EP x 64 bf16
   static constexpr uint32_t STAGE_BYTES = A_BYTES + 3 * PART_BYTES;
   static constexpr uint32_t TX_BYTES = X_BYTES + 3 * PART_BYTES;
-  static constexpr int STAGES = (EP == 256) ? 2 : (EP == 128 ? 3 : (EP == 64 ? 5 : 7));
+  // two 8-warp CTAs per SM must each fit in half the shared memory
+  static constexpr int STAGES = NW == 8 ? (EP == 64 ? 2 : 3)
+                                        : ((EP == 256) ? 2 : (EP == 128 ? 3 : (EP == 64 ? 5 : 7)));
   // L2 prefetch distance of the token tiles, in k-blocks.  With 3 or more stages in
   // flight the prefetches only queue ahead of the loads in the TMA unit (measured:
   // slower); with 2 stages (E > 128) they hide the DRAM latency of x.
@@ -99,12 +108,13 @@ __device__ __forceinline__ uint32_t idesc_router() {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
-template <int EP, int TT>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int EP, int TT, int NW>
+__global__ void __launch_bounds__(NW * 32, (NW == 8) ? 2 : 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const float* __restrict__ bias, int S, int M, int E, int k, int nchunk,
                      Routing R, uint64_t limit_ns) {
-  using C = RCfg<EP, TT>;
+  using C = RCfg<EP, TT, NW>;
+  constexpr int kThreads = C::NT;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -120,7 +130,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x, tok0 = tile * C::TT;
-  pdl_trigger();                       // the scan may launch and wait while this grid runs
   const int KB = M / BK;
 
   if (warp == 0 && lane == 0) {
@@ -144,6 +153,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The scan may launch and wait while this grid runs.  Triggered after the TMEM
+  // allocation, so no dependent grid is resident before every CTA of this one holds
+  // its columns.
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -233,8 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp < 6 && (warp & 3) < C::TT / 32) {
-    // ------------------------------------------------------------ fold K-segments (warps 2-5)
+  } else if (warp >= C::FOLD0 && warp < C::FOLD0 + 4 && (warp & 3) < C::TT / 32) {
+    // ------------------------------------------------------------ fold K-segments (four warps)
     const int q = warp & 3;
     const int row = q * 32 + lane;              // token row within the tile (= TMEM lane)
     const uint32_t tlane = tmem_base + ((uint32_t)(q * 32) << 16);
@@ -289,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < EP; ++c) Ls[row * C::LD + c] = 0.f;
   }
 
-  // ------------------------------------------------------------ route, all 16 warps
+  // ------------------------------------------------------------ route, all warps
   __syncthreads();
   {
     float* Ls = reinterpret_cast<float*>(gbase + C::L_OFF);
@@ -410,6 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else {
       // E > 64: one warp per token, lanes over experts
+      static_assert(C::NW == 16, "warp-per-token routing assumes 16 warps");
       constexpr int TPW = C::TT / 16;                         // tokens per warp (4 or 8)
       constexpr int WPC = 16 / C::NCH;                        // warps per 64-token chunk
       float psum[RE];
@@ -464,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // local ranks within each 64-token chunk and rank-r histograms: one warp per
     // (chunk, rank), 32 tokens at a time; tokens choosing the same expert find one
     // another with a match, and a running count per expert carries over
-    for (int pi = warp; pi < C::NCH * k; pi += kThreads / 32) {
+    for (int pi = warp; pi < C::NCH * k; pi += C::NW) {
       const int cc = pi / k, r = pi - cc * k;
       int32_t* cnt = Hs + (cc * kMaxK + r) * EP;
       for (int h = 0; h < kChunk / 32; ++h) {
@@ -541,16 +555,15 @@ bool encode_kmajor(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t ou
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EP, int TT>
+template <int EP, int TT, int NW>
 cudaError_t launch_tt(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias, int S, int M,
                       int E, int k, const Routing& R, uint64_t limit_ns, cudaStream_t st) {
-  auto kern = router_tc_kernel<EP, TT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)RCfg<EP, TT>::SMEM);
+  using C = RCfg<EP, TT, NW>;
+  auto kern = router_tc_kernel<EP, TT, NW>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int nchunk = (S + kChunk - 1) / kChunk;
-  kern<<<(S + TT - 1) / TT, kThreads, RCfg<EP, TT>::SMEM, st>>>(tmX, tmW, bias, S, M, E, k, nchunk, R,
-                                                                limit_ns);
+  kern<<<(S + TT - 1) / TT, C::NT, C::SMEM, st>>>(tmX, tmW, bias, S, M, E, k, nchunk, R, limit_ns);
   return cudaGetLastError();
 }
 
@@ -571,8 +584,8 @@ template <int EP>
 cudaError_t launch_t(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias, int S, int M,
                      int E, int k, const Routing& R, uint64_t limit_ns, cudaStream_t st) {
   if (router_tokens_per_cta(E, S) == 128)
-    return launch_tt<EP, 128>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);
-  return launch_tt<EP, 64>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);
+    return launch_tt<EP, 128, (EP <= 64 ? 8 : 16)>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);
+  return launch_tt<EP, 64, 16>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);
 }
 
 }  // namespace

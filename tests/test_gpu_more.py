@@ -49,6 +49,11 @@ ROUTER_SHAPES = [
     (300, 576, 256, 24, 2, 1.25),     # 9 k-blocks: two K-segments, the last partial
     (200, 1536, 256, 8, 2, 1.25),     # 24 k-blocks: three K-segments
     (64, 256, 256, 256, 8, 1.25),     # E = 256, top-8, one CTA
+    # enough tokens for 128-token CTAs with E <= 64 on 148 SMs: the 8-warp, two-per-SM
+    # router; ragged last tiles whose second 64-token chunk is empty or partial
+    (19001, 576, 256, 40, 2, 1.0),    # EP = 64, two K-segments, last tile 57 tokens
+    (20000, 128, 128, 24, 3, 1.25),   # EP = 32, top-3, last tile 32 tokens
+    (19050, 192, 128, 64, 1, 1.0),    # EP = 64, top-1, last tile 106 tokens
 ]
 
 
