@@ -204,6 +204,44 @@ def algorithmic_bwd(w, A, pad_rows, nsplit):
     }
 
 
+def measure_copies(args, x, xh, yh, stream):
+    """The e2e step's copies without the layer: its input host -> device, its output
+    device -> host, each direction alone and both at once on two streams (pinned host
+    buffers, the same bytes per step).  The slower of "both" and the device step bounds
+    what the overlapped host-buffer pipeline can reach."""
+    xd = torch.empty_like(x)
+    yd = torch.empty_like(x)
+    other = torch.cuda.Stream()
+    reps = max(3, min(args.steps, 50))
+
+    def run(h2d, d2h):
+        for _ in range(2):                          # warm-up
+            if h2d:
+                xd.copy_(xh, non_blocking=True)
+            if d2h:
+                yh.copy_(yd, non_blocking=True)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        other.wait_stream(stream)
+        for _ in range(reps):
+            if h2d:
+                xd.copy_(xh, non_blocking=True)
+            if d2h:
+                with torch.cuda.stream(other):
+                    yh.copy_(yd, non_blocking=True)
+        stream.wait_stream(other)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    nbytes = x.numel() * x.element_size()
+    h2d, d2h, both = run(True, False), run(False, True), run(True, True)
+    return {"h2d_ms": round(h2d, 4), "d2h_ms": round(d2h, 4), "both_ms": round(both, 4),
+            "h2d_GBps": round(nbytes / h2d / 1e6, 1), "d2h_GBps": round(nbytes / d2h / 1e6, 1)}
+
+
 def measure_backward(args, w, layer, x, y, flush, stream, pk, A, n_e):
     """One training step = moe_forward + moe_backward of the same tokens, device-timed."""
     from gshard_top_gating_b200 import _lib as L
@@ -386,6 +424,7 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), world)
     nbytes = x.numel() * x.element_size()
+    copies = measure_copies(args, x, xh, yh, stream)
 
     # clocks: the timed region itself when it held enough samples, else a soak of
     # the same forward right after it (the timed region was too short to sample)
@@ -446,7 +485,9 @@ def run_ours(args, rank, world, local):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roof, "stages": stages,
         "e2e": {"value": round(job_throughput(w.S, args.steps, e2e_ms, world), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes},
+                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+                "ms_per_step": round(e2e_ms / args.steps, 4),
+                "copies_alone": copies},
         "gpu_launches": args.steps * L.moe_kernels_per_forward(layer.h, w.S),
         "clocks": clocks,
         "cpu_baseline": cpu,
