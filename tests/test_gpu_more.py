@@ -7,6 +7,8 @@
   several K-segments (M = 576 and 1536: 9 and 24 k-blocks of 64), a gate bias
   with E padded to 256 and top-8.
 """
+from types import SimpleNamespace
+
 import numpy as np
 import pytest
 import torch
@@ -54,6 +56,7 @@ ROUTER_SHAPES = [
     (19001, 576, 256, 40, 2, 1.0),    # EP = 64, two K-segments, last tile 57 tokens
     (20000, 128, 128, 24, 3, 1.25),   # EP = 32, top-3, last tile 32 tokens
     (19050, 192, 128, 64, 1, 1.0),    # EP = 64, top-1, last tile 106 tokens
+    (257, 128, 128, 12, 8, 1.0),      # EP = 32, top-8 of 12 (thread-per-token), one-token last tile
 ]
 
 
@@ -63,6 +66,39 @@ def test_router_tiles_and_segments(shape):
     run = G.build(Workload("rt", S, M, H, E, k, cf, "bf16", seed=23))
     G.full_check(run)
     run.layer.close()
+
+
+TIE_SHAPES = [
+    # (S, M, H, E, k, cf)
+    (300, 128, 128, 16, 4, 1.25),     # EP = 32: a thread per token, 64-token CTAs
+    (19001, 128, 128, 40, 3, 1.0),    # EP = 64: 8-warp CTAs, two per SM
+    (300, 128, 128, 100, 4, 1.0),     # EP = 128: a warp per token
+]
+
+
+@pytest.mark.parametrize("shape", TIE_SHAPES, ids=[str(s) for s in TIE_SHAPES])
+def test_tensor_core_router_exact_ties(shape):
+    """W_g whose odd columns repeat the even column before them: the tensor-core
+    router computes both columns from the same operand values, so every token's
+    logits tie in pairs, bitwise.  Top-k then has to take the lower index of a tied
+    pair first; routing against the oracle on those logits stays bit-exact."""
+    S, M, H, E, k, cf = shape
+    w = Workload("ties_tc", S, M, H, E, k, cf, "bf16", seed=37)
+    x, Wg, b, W1, W2 = make_inputs(w, device="cuda")
+    Wg[:, 1::2] = Wg[:, 0::2]
+    layer = MoeLayer(S, M, H, E, k, cf, Wg, b, W1, W2)
+    run = SimpleNamespace(w=w, S=S, x=x, Wg=Wg, b=b, W1=W1, W2=W2, layer=layer)
+    out = G.forward(run)
+    assert np.array_equal(out.logits[:, 1::2], out.logits[:, 0::2])
+    rt = G.check_routing(run, out)
+    # an odd expert is chosen only after the even expert it ties with (lower index first)
+    ids = out.eidx
+    for r in range(k):
+        e = ids[:, r]
+        before = (ids[:, :r] == (e - 1)[:, None]).any(axis=1)
+        assert np.all((e % 2 == 0) | before), r
+    G.check_outputs(run, out, rt, np.arange(min(S, 2048)))
+    layer.close()
 
 
 def test_gate_bias_with_256_experts_top8():
