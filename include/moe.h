@@ -221,7 +221,13 @@ MOE_API moe_status moe_assign_slots_noalloc(int64_t S, int32_t E, int32_t k, int
  *   dY  [E, Cbuf, M] act  (gradient of the expert outputs; reused for dX_e)
  *   dP  [E, Cbuf, H] act  (gradient of the first layer's pre-activation)
  *   dl  [S_max, E] fp32 (logit gradient), dgate [S_max, k] fp32, and the
- *   split-K partials of the gate-weight gradient.
+ *   split-K partials of the gate-weight gradient;
+ *   bf16 only: the ReLU mask bits [H/32, E*Cbuf] uint32, one bit per element
+ *   of the first layer's output (set when the stored bf16 value is > 0).
+ * Training mode: every bf16 forward after this call also stores those bits
+ * (1/16 of the bytes of h), and moe_backward's dP step reads them instead of
+ * re-reading h.  A backward of a forward that ran before this call re-reads h;
+ * both give bitwise-equal gradients.
  * Synchronous (cudaMalloc); call it outside stream capture.
  */
 MOE_API moe_status moe_enable_backward(moe_handle h);
