@@ -242,13 +242,18 @@ def measure_copies(args, x, xh, yh, stream):
             "h2d_GBps": round(nbytes / h2d / 1e6, 1), "d2h_GBps": round(nbytes / d2h / 1e6, 1)}
 
 
-def measure_backward(args, w, layer, x, y, flush, stream, pk, A, n_e):
-    """One training step = moe_forward + moe_backward of the same tokens, device-timed."""
+def measure_backward(args, w, weights, x, y, flush, stream, pk, A, n_e):
+    """One training step = moe_forward + moe_backward of the same tokens, device-timed.
+
+    On a handle of its own, in training mode from its first forward (the backward
+    enabled first), as a training loop would use the layer."""
     from gshard_top_gating_b200 import _lib as L
     from gshard_top_gating_b200.inputs import upstream_grad
+    from gshard_top_gating_b200.layer import MoeLayer
     dev = x.device
     dy = upstream_grad(w, device=dev)
-    L.moe_enable_backward(layer.h)
+    layer = MoeLayer(w.S, w.M, w.H, w.E, w.k, w.cf, *weights)
+    layer.enable_backward()
     dx = torch.empty_like(x)
     dWg = torch.empty(w.M, w.E, dtype=torch.float32, device=dev)
     dbias = torch.empty(w.E, dtype=torch.float32, device=dev) if w.skew_bias else None
@@ -311,6 +316,8 @@ def measure_backward(args, w, layer, x, y, flush, stream, pk, A, n_e):
     else:
         ach, peak, unit = wk / tt / 1e9, pk["hbm_gbs"], "GB/s"
     ffn = sum(stage_ms[k_] for k_ in ("dW2", "dP", "dW1", "dX_e"))
+    launches = n * (L.moe_kernels_per_forward(layer.h, w.S) + L.moe_kernels_per_backward(layer.h, w.S))
+    layer.close()
     return {
         "what": "moe_forward + moe_backward of the same tokens (dL/dy given; a_aux=0.01, a_z=0.001)",
         "tokens_per_s": round(w.S / ((fwd_ms + bwd_ms) / 1e3), 1),
@@ -321,7 +328,7 @@ def measure_backward(args, w, layer, x, y, flush, stream, pk, A, n_e):
                      "frac_of_sustained": (round(ach / pk["bf16_tflops_sustained"], 4)
                                            if b_ == "tensor" and pk.get("bf16_tflops_sustained") else None)},
         "stages": stages,
-        "gpu_launches": n * (L.moe_kernels_per_forward(layer.h, w.S) + L.moe_kernels_per_backward(layer.h, w.S)),
+        "gpu_launches": launches,
     }
 
 
@@ -466,7 +473,8 @@ def run_ours(args, rank, world, local):
             stages[n] = {"ms": round(stage_ms[n], 4), "GB/s": round(wk / tt / 1e9, 1),
                          "frac_of_peak": round(wk / tt / 1e9 / pk["hbm_gbs"], 4)}
 
-    train = None if args.no_backward else measure_backward(args, w, layer, x, y, flush, stream, pk, A, n_e)
+    train = (None if args.no_backward
+             else measure_backward(args, w, (Wg, b, W1, W2), x, y, flush, stream, pk, A, n_e))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -70,6 +70,10 @@ struct moe_layer {
   uint32_t bwd_flags;               // MOE_BWD_* flags
   uint32_t* hbits;                  // [H/32, E*Cbuf] bits of h > 0, written by FFN1 once enabled
   bool bits_valid;                  // the last forward wrote hbits
+  // A forward was captured into a CUDA graph without the bits epilogue: a replay of
+  // that graph rewrites h but not hbits, and the host cannot see replays, so from
+  // then on the backward reads its ReLU mask from h.
+  bool graph_without_bits;
   // bf16: tensor-core gate gradients
   int EPb;                          // E rounded up to 64
   void* dlb;                        // [S_max, 2*EPb] bf16 split of dl
@@ -313,6 +317,12 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
   h->have_forward = true;
   h->fwd_data = true;
   h->bits_valid = false;
+  if (h->act == MOE_BF16 && !h->plan1.bits) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    // an error (a capture elsewhere in global mode) counts as capturing
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+      h->graph_without_bits = true;
+  }
   if (S == 0) {
     MOE_TRY(cudaMemsetAsync(h->R.losses, 0, 2 * sizeof(float), st));
     return MOE_OK;
@@ -673,7 +683,8 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
     const bool skip = (h->bwd_flags & MOE_BWD_SKIP_EMPTY_EXPERTS) != 0;
     h->plan_dw2.skip_zero = skip;
     h->plan_dw1.skip_zero = skip;
-    h->plan_dp.use_bits = h->bits_valid;   // else the mask is read from h itself
+    // else the mask is read from h itself
+    h->plan_dp.use_bits = h->bits_valid && !h->graph_without_bits;
     // the weight-gradient GEMMs reduce over whole 64-slot blocks: clear the rows
     // between the kept count and the next multiple of 64
     void* bufs[3] = {h->xbuf, h->hbuf, h->dybuf};

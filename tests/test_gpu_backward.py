@@ -185,6 +185,43 @@ def test_mask_bits_equal_mask_from_h(shape):
     run.layer.close()
 
 
+def test_graph_captured_before_training_mode_never_uses_stale_mask_bits():
+    """A forward captured in a CUDA graph before the backward is enabled stores no
+    mask bits, and the host cannot see its replays.  After a training-mode forward of
+    other tokens (which stores bits), a replay of that graph followed by a backward
+    must give the replayed forward's gradients: the same as an eager forward and
+    backward of the replayed tokens."""
+    w = Workload("gbits", 512, 256, 512, 8, 2, 1.25, "bf16", seed=38)
+    run = G.build(w)
+    dy = upstream_grad(w, device="cuda")
+    x = run.x.clone()
+    y = torch.empty_like(x)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run.layer(x, out=y)                        # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run.layer(x, out=y)                        # inference epilogue: no mask bits
+    run.layer.enable_backward()
+    run.layer(torch.roll(run.x, shifts=77, dims=0).contiguous())   # stores bits of other tokens
+    x.copy_(torch.flip(run.x, dims=[0]))
+    graph.replay()
+    g_replay = run.layer.backward(x, dy, 0.5, 0.1)
+    torch.cuda.synchronize()
+    x_eager = x.clone()
+    run.layer(x_eager)
+    g_eager = run.layer.backward(x_eager, dy, 0.5, 0.1)
+    torch.cuda.synchronize()
+    for key in g_eager:
+        if g_eager[key] is None:
+            continue
+        assert torch.equal(g_replay[key], g_eager[key]), key
+    del graph
+    run.layer.close()
+
+
 def test_backward_is_deterministic_and_repeatable():
     w = Workload("det", 700, 256, 256, 8, 2, 1.0, "bf16", skew_bias=True, seed=32)
     run = G.build(w)
