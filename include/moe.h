@@ -227,7 +227,10 @@ MOE_API moe_status moe_assign_slots_noalloc(int64_t S, int32_t E, int32_t k, int
  * Training mode: every bf16 forward after this call also stores those bits
  * (1/16 of the bytes of h), and moe_backward's dP step reads them instead of
  * re-reading h.  A backward of a forward that ran before this call re-reads h;
- * both give bitwise-equal gradients.
+ * both give bitwise-equal gradients.  Once any forward of the handle has been
+ * captured into a CUDA graph without the bits (captured before this call), the
+ * backward always re-reads h, since replays of that graph are invisible to the
+ * host: capture training graphs after this call to keep the faster path.
  * Synchronous (cudaMalloc); call it outside stream capture.
  */
 MOE_API moe_status moe_enable_backward(moe_handle h);
