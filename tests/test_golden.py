@@ -1,0 +1,75 @@
+"""The oracle against the hand-worked examples in tests/golden/ (CPU only).
+
+The source pages print no worked example.  Each fixture works a small case out by
+hand from the definitions (its `cite` and `reading` fields name the passage and
+the reading used) and states the expected values exactly: integers, fractions, or
+closed forms in exp and log.  Nothing in a fixture comes from the oracle or the
+CUDA path, so a wrong index, sign, normalisation or slot order in the oracle
+fails here.
+"""
+import json
+import math
+import pathlib
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+GOLDEN = pathlib.Path(__file__).parent / "golden"
+
+
+def value(expr) -> float:
+    """A fixture number: an int, a float, or a string in +-*/, **, exp and log."""
+    if isinstance(expr, (int, float)):
+        return float(expr)
+    if "/" in expr and not any(c.isalpha() for c in expr):
+        return float(Fraction(expr))
+    return float(eval(expr, {"__builtins__": {}}, {"exp": math.exp, "log": math.log}))
+
+
+def values(a) -> np.ndarray:
+    return np.array([[value(v) for v in row] for row in a]) if isinstance(a[0], list) else \
+        np.array([value(v) for v in a])
+
+
+def load(name):
+    with open(GOLDEN / name) as fh:
+        return json.load(fh)
+
+
+def check_route(rt, exp, E):
+    assert rt.C == exp["C"]
+    assert np.array_equal(rt.ids, np.array(exp["ids"]))
+    assert np.array_equal(rt.slot, np.array(exp["slot"]))
+    assert np.array_equal(rt.cnt, np.array(exp["cnt"]))
+    if "n" in exp:
+        assert np.array_equal(rt.n, np.array(exp["n"]))
+    np.testing.assert_allclose(rt.gates, values(exp["gates"]), rtol=1e-12, atol=1e-15)
+    if "f" in exp:
+        np.testing.assert_allclose(rt.f, values(exp["f"]), rtol=1e-12, atol=1e-15)
+    if "P" in exp:
+        np.testing.assert_allclose(rt.P, values(exp["P"]), rtol=1e-12)
+    if "l_aux" in exp:
+        assert math.isclose(rt.l_aux, value(exp["l_aux"]), rel_tol=1e-12)
+    if "z" in exp:
+        assert math.isclose(rt.z, value(exp["z"]), rel_tol=1e-12)
+
+
+def test_route_rank_major_fixture():
+    g = load("route_rank_major.json")
+    assert g["cite"] and g["reading"]
+    logits = np.array(g["logits"], dtype=np.float64)
+    rt = O.route(logits, g["k"], g["cf"])
+    check_route(rt, g["expect"], g["E"])
+
+
+@pytest.mark.parametrize("i", range(3))
+def test_losses_and_gates_fixture(i):
+    g = load("losses_and_gates.json")
+    assert g["cite"] and g["reading"]
+    case = g["cases"][i]
+    logits = values(g["logits"])
+    rt = O.route(logits, case["k"], case["cf"])
+    check_route(rt, case["expect"], g["E"])
