@@ -73,3 +73,22 @@ def test_losses_and_gates_fixture(i):
     logits = values(g["logits"])
     rt = O.route(logits, case["k"], case["cf"])
     check_route(rt, case["expect"], g["E"])
+
+
+def test_backward_closed_form_fixture():
+    g = load("backward_closed_form.json")
+    assert g["cite"] and g["reading"]
+    a = g["aux_and_z"]
+    p, f, lse = values(a["p"]), values(a["f"]), values(a["lse"])
+    np.testing.assert_allclose(O.aux_loss_backward(p, f, a["E"], a["S"]), values(a["expect_aux"]),
+                               rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(O.z_loss_backward(p, lse, a["S"]), values(a["expect_z"]), rtol=1e-12)
+    gt = g["gates"]
+    dl = O.gates_backward(values(gt["gates"]), np.array(gt["ids"]), values(gt["dgate"]), gt["E"])
+    np.testing.assert_allclose(dl, values(gt["expect"]), rtol=1e-12, atol=1e-15)
+    fx = g["expert_ffn"]
+    rows, W1, W2, dY = (values(fx[n]) for n in ("rows", "W1", "W2", "dY"))
+    drows, dW1, dW2 = O.expert_ffn_backward(rows, rows @ W1, dY, W1, W2)
+    np.testing.assert_allclose(drows, values(fx["expect_drows"]), rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(dW1, values(fx["expect_dW1"]), rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(dW2, values(fx["expect_dW2"]), rtol=1e-12, atol=1e-15)
