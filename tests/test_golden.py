@@ -92,3 +92,47 @@ def test_backward_closed_form_fixture():
     np.testing.assert_allclose(drows, values(fx["expect_drows"]), rtol=1e-12, atol=1e-15)
     np.testing.assert_allclose(dW1, values(fx["expect_dW1"]), rtol=1e-12, atol=1e-15)
     np.testing.assert_allclose(dW2, values(fx["expect_dW2"]), rtol=1e-12, atol=1e-15)
+
+
+# ---------------------------------------------------------------- the fixtures catch plants
+# The planted mistakes of the other pin files, restricted to those a routing, loss or
+# step-gradient fixture can see (the fixtures have no ties, compute no logits and run no
+# forward FFN, dispatch or combine): each must make at least one fixture test fail.
+def _golden_pins():
+    return [test_route_rank_major_fixture] + \
+        [lambda i=i: test_losses_and_gates_fixture(i) for i in range(3)] + \
+        [test_backward_closed_form_fixture]
+
+
+def _planted():
+    import tests.test_oracle_backward_pins as B
+    import tests.test_oracle_mutations as MU
+    fwd = [("normalized_gates", MU._mut_gates_unnormalised),
+           ("assign_slots", MU._mut_slots_token_major),
+           ("assign_slots", MU._mut_slots_second_choice_uses_raw_count),
+           ("capacity", MU._mut_capacity_floor_plus_one),
+           ("aux_losses", MU._mut_aux_all_choices),
+           ("aux_losses", MU._mut_aux_z_not_squared),
+           ("aux_losses", MU._mut_aux_no_E),
+           ("softmax_stats", MU._mut_softmax_wrong_sign)]
+    bwd = [(n, f) for n, fs in B.PLANTS.items() for f in fs]
+    return fwd + bwd
+
+
+PLANTED = _planted()
+
+
+@pytest.mark.parametrize("fn,mutant", PLANTED, ids=[m.__name__ for _, m in PLANTED])
+def test_fixtures_catch_planted_mistake(fn, mutant, monkeypatch):
+    import oracle.moe_oracle as M
+    monkeypatch.setitem(M.__dict__, "_orig_aux", M.aux_losses)
+    monkeypatch.setitem(M.__dict__, "_orig_softmax", M.softmax_stats)
+    monkeypatch.setattr(M, fn, mutant)
+    monkeypatch.setattr(O, fn, mutant, raising=False)
+    failed = []
+    for pin in _golden_pins():
+        try:
+            pin()
+        except Exception:
+            failed.append(pin)
+    assert failed, f"no fixture caught the planted mistake {mutant.__name__} in {fn}"
