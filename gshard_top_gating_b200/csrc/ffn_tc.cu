@@ -43,6 +43,13 @@ struct Cfg {
   // 1 KB alignment slack + stages + staging + 512 B of barriers + misc words and the tile tables
   static constexpr size_t SMEM =
       1024 + (size_t)STAGES * STAGE_BYTES + STAGING + 512 + 16 + 4 * (3 * kMaxExperts + 1);
+  // A GEMM CTA owns its SM: beside its shared memory no other TMEM-using CTA of the
+  // library fits (the smallest, an 8-warp router CTA, takes over 80 KB of the SM's
+  // 228 KB), so a TMEM allocation (up to 512 columns) never waits on a co-resident CTA
+  // that may itself be waiting on this kernel.
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  static_assert(SMEM + 1024 + 80 * 1024 > 228 * 1024, "a GEMM CTA must own its SM");
+  static_assert(TMEM_COLS <= 512, "TMEM columns");
 };
 
 // Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: version 1 at bit 46,
@@ -663,6 +670,9 @@ constexpr uint32_t STAGING = 4 * 4096;                   // one 32 x 64 bf16 sto
 constexpr size_t SMEM =
     1024 + (size_t)STAGES * STAGE_BYTES + STAGING + 512 + 16 + 4 * (3 * kMaxExperts + 1);
 constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;            // shared::cluster address -> rank 0
+static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+static_assert(SMEM + 1024 + 80 * 1024 > 228 * 1024, "a GEMM CTA must own its SM (as Cfg)");
+static_assert(TMEM_COLS <= 512, "TMEM columns");
 }  // namespace pairk
 
 // EPI and BKM as in ffn_tc_kernel; with BKM each CTA's B box is its 128 rows of

@@ -94,6 +94,13 @@ struct RCfg {
   static constexpr uint32_t EPI_END = LSET_OFF + (EP <= 64 ? TT * 4 : 0);
   static_assert(EPI_END <= STAGES * STAGE_BYTES, "epilogue scratch must fit in the stage buffers");
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + 16;
+  // residency: a 16-warp CTA owns its SM; two 8-warp CTAs share one SM's 228 KB of
+  // shared memory (1 KB reserved per CTA) and its 512 TMEM columns, so neither CTA's
+  // allocation can wait on the other
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  static_assert(NW == 16 || 2 * (SMEM + 1024) <= 228 * 1024, "two 8-warp CTAs per SM");
+  static_assert(SMEM > 80 * 1024, "the GEMM kernels' residency argument assumes more than 80 KB");
+  static_assert((NW == 8 ? 2 : 1) * TMEM_COLS <= 512, "TMEM columns of the CTAs on one SM");
 };
 
 __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
