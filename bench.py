@@ -175,33 +175,59 @@ def ncu_traffic(kernel: str, workload: str):
 
 
 def algorithmic(w, A, n_active):
-    """Algorithmic bytes / flops per launch of each stage (A kept assignments)."""
+    """Algorithmic work per launch of each stage (A kept assignments, n_active experts
+    with a kept row): ("hbm", bytes), or ("gemm", flops, bytes) for an expert GEMM,
+    whose bytes are its operands read once (the active experts' weights) and its
+    result written once."""
     s = 2 if w.act == "bf16" else 4
     S, M, H, E, k = w.S, w.M, w.H, w.E, w.k
+    wts = n_active * M * H * s
     return {
         "router": ("hbm", S * M * s + 4 * M * E + S * E * 4 + S * k * 12),
         "scan": ("hbm", 0),
         "dispatch": ("hbm", (S + A) * M * s),
-        "ffn1": ("tensor", 2.0 * A * M * H),
-        "ffn2": ("tensor", 2.0 * A * M * H),
+        "ffn1": ("gemm", 2.0 * A * M * H, A * M * s + wts + A * H * s),
+        "ffn2": ("gemm", 2.0 * A * M * H, A * H * s + wts + A * M * s),
         "combine": ("hbm", (A + S) * M * s + S * k * 12),
     }
 
 
-def algorithmic_bwd(w, A, pad_rows, nsplit):
-    """Algorithmic bytes / flops per launch of each backward stage (A kept assignments)."""
+def algorithmic_bwd(w, A, n_active, pad_rows, nsplit):
+    """Algorithmic work per launch of each backward stage, as algorithmic().  The
+    weight gradients are written for every expert (zeros for the empty ones: the
+    default, MOE_BWD_SKIP_EMPTY_EXPERTS off); dP reads one mask bit per element."""
     s = 2 if w.act == "bf16" else 4
     S, M, H, E, k = w.S, w.M, w.H, w.E, w.k
+    wts, grads = n_active * M * H * s, E * M * H * s
+    f = 2.0 * A * M * H
     return {
         "gate_bwd": ("hbm", S * M * s + 2 * A * M * s + 2 * S * E * 4 + S * k * 16 + E * 4),
         "pad_zero": ("hbm", pad_rows * (2 * M + H) * s),
-        "dW2": ("tensor", 2.0 * A * M * H),
-        "dP": ("tensor", 2.0 * A * M * H),
-        "dW1": ("tensor", 2.0 * A * M * H),
-        "dX_e": ("tensor", 2.0 * A * M * H),
+        "dW2": ("gemm", f, A * H * s + A * M * s + grads),
+        "dP": ("gemm", f, A * M * s + wts + A * H // 8 + A * H * s),
+        "dW1": ("gemm", f, A * M * s + A * H * s + grads),
+        "dX_e": ("gemm", f, A * H * s + wts + A * M * s),
         "dx": ("hbm", (A + S) * M * s + S * E * 4 + M * E * 4 + S * k * 8),
         "dWg": ("hbm", S * M * s + S * E * 4 + 2 * nsplit * (M + 1) * E * 4),
     }
+
+
+def stage_roof(entry, seconds, pk):
+    """(bound, achieved, peak, unit) of one stage.  An expert GEMM is bound by the slower
+    of its flops at the bf16 tensor peak and its bytes at the HBM peak (a GEMM over few
+    rows per expert streams weights faster than it can use the tensor cores)."""
+    if entry[0] == "gemm":
+        flops, nbytes = entry[1], entry[2]
+        if flops / (pk["bf16_tflops"] * 1e12) >= nbytes / (pk["hbm_gbs"] * 1e9):
+            return "tensor", flops / seconds / 1e12, pk["bf16_tflops"], "TFLOP/s"
+        return "hbm", nbytes / seconds / 1e9, pk["hbm_gbs"], "GB/s"
+    return "hbm", entry[1] / seconds / 1e9, pk["hbm_gbs"], "GB/s"
+
+
+def stage_entry(entry, ms, pk):
+    b_, ach, peak, unit = stage_roof(entry, ms / 1e3, pk)
+    return {"ms": round(ms, 4), unit: round(ach, 1), "frac_of_peak": round(ach / peak, 4),
+            "bound": b_}
 
 
 def measure_copies(args, x, xh, yh, stream):
@@ -295,26 +321,11 @@ def measure_backward(args, w, weights, x, y, flush, stream, pk, A, n_e):
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     tiles = ((w.M + 64) // 64) * ((w.E + 63) // 64)
     nsplit = max(1, min((2 * sms + tiles - 1) // tiles, (w.S + 255) // 256))
-    algo = algorithmic_bwd(w, A, pad_rows, nsplit)
-    stages = {}
-    for nm in L.BWD_STAGES:
-        b_, wk = algo[nm]
-        tt = stage_ms[nm] / 1e3
-        if tt <= 0:
-            continue
-        if b_ == "tensor":
-            stages[nm] = {"ms": round(stage_ms[nm], 4), "TFLOP/s": round(wk / tt / 1e12, 1),
-                          "frac_of_peak": round(wk / tt / 1e12 / pk["bf16_tflops"], 4)}
-        else:
-            stages[nm] = {"ms": round(stage_ms[nm], 4), "GB/s": round(wk / tt / 1e9, 1),
-                          "frac_of_peak": round(wk / tt / 1e9 / pk["hbm_gbs"], 4)}
+    n_active = int((n_e > 0).sum().item())
+    algo = algorithmic_bwd(w, A, n_active, pad_rows, nsplit)
+    stages = {nm: stage_entry(algo[nm], stage_ms[nm], pk) for nm in L.BWD_STAGES if stage_ms[nm] > 0}
     dom = max(stage_ms, key=lambda k_: stage_ms[k_])
-    b_, wk = algo[dom]
-    tt = stage_ms[dom] / 1e3
-    if b_ == "tensor":
-        ach, peak, unit = wk / tt / 1e12, pk["bf16_tflops"], "TFLOP/s"
-    else:
-        ach, peak, unit = wk / tt / 1e9, pk["hbm_gbs"], "GB/s"
+    b_, ach, peak, unit = stage_roof(algo[dom], stage_ms[dom] / 1e3, pk)
     ffn = sum(stage_ms[k_] for k_ in ("dW2", "dP", "dW1", "dX_e"))
     launches = n * (L.moe_kernels_per_forward(layer.h, w.S) + L.moe_kernels_per_backward(layer.h, w.S))
     layer.close()
@@ -324,7 +335,8 @@ def measure_backward(args, w, weights, x, y, flush, stream, pk, A, n_e):
         "ms_fwd": round(fwd_ms, 4), "ms_bwd": round(bwd_ms, 4), "steps": n,
         "expert_gemm_TFLOP/s": round(4 * 2.0 * A * w.M * w.H / (ffn / 1e3) / 1e12, 1) if ffn > 0 else None,
         "roofline": {"bound": b_, "kernel": dom, "achieved": round(ach, 2), "peak": peak, "unit": unit,
-                     "frac": round(ach / peak, 4), "peak_source": "measured, burst",
+                     "frac": round(ach / peak, 4),
+                     "peak_source": "measured, burst" if b_ == "tensor" else "measured",
                      "frac_of_sustained": (round(ach / pk["bf16_tflops_sustained"], 4)
                                            if b_ == "tensor" and pk.get("bf16_tflops_sustained") else None)},
         "stages": stages,
@@ -451,27 +463,13 @@ def run_ours(args, rank, world, local):
     pk, pk_kind = peaks()
     algo = algorithmic(w, A, n_active)
     dom = max(stage_ms, key=lambda n: stage_ms[n])
-    bound, work = algo[dom]
-    t = stage_ms[dom] / 1e3
-    if bound == "tensor":
-        achieved, peak, unit = work / t / 1e12, pk["bf16_tflops"], "TFLOP/s"
-    else:
-        achieved, peak, unit = work / t / 1e9, pk["hbm_gbs"], "GB/s"
+    bound, achieved, peak, unit = stage_roof(algo[dom], stage_ms[dom] / 1e3, pk)
     roof = {"bound": bound, "kernel": dom, "achieved": round(achieved, 2), "peak": peak,
             "unit": unit, "frac": round(achieved / peak, 4), "traffic": ncu_traffic(dom, w.name),
             "peak_source": f"{pk_kind}, burst" if bound == "tensor" else pk_kind,
             "frac_of_sustained": (round(achieved / pk["bf16_tflops_sustained"], 4)
                                   if bound == "tensor" and pk.get("bf16_tflops_sustained") else None)}
-    stages = {}
-    for n in STAGES:
-        b_, wk = algo[n]
-        tt = stage_ms[n] / 1e3
-        if b_ == "tensor":
-            stages[n] = {"ms": round(stage_ms[n], 4), "TFLOP/s": round(wk / tt / 1e12, 1),
-                         "frac_of_peak": round(wk / tt / 1e12 / pk["bf16_tflops"], 4)}
-        else:
-            stages[n] = {"ms": round(stage_ms[n], 4), "GB/s": round(wk / tt / 1e9, 1),
-                         "frac_of_peak": round(wk / tt / 1e9 / pk["hbm_gbs"], 4)}
+    stages = {n: stage_entry(algo[n], stage_ms[n], pk) for n in STAGES if stage_ms[n] > 0}
 
     train = (None if args.no_backward
              else measure_backward(args, w, (Wg, b, W1, W2), x, y, flush, stream, pk, A, n_e))
