@@ -533,9 +533,13 @@ def cpu_baseline(w, budget_s, x, Wg, b, W1, W2):
     probe = min(w.S, 256)
     c = _oracle_step(O, w, inp, probe) / probe                 # seconds per token
     ntok = int(max(64, min(w.S, budget_s / max(c, 1e-9))))
+    dt = _oracle_step(O, w, inp, ntok)
+    reps = 1
     # a whole workload shorter than the budget is run again until the budget is spent
-    reps = max(1, min(20, int(budget_s / max(c * ntok, 1e-9)))) if ntok == w.S else 1
-    dt = sum(_oracle_step(O, w, inp, ntok) for _ in range(reps))
+    if ntok == w.S:
+        more = max(0, min(19, int((budget_s - dt) / max(dt, 1e-9))))
+        dt += sum(_oracle_step(O, w, inp, ntok) for _ in range(more))
+        reps += more
     what = (f"first {ntok} of {w.S} tokens of the {w.name} workload (same M, H, E, k, cf; "
             f"C scaled to the sample)" if ntok < w.S else
             f"the whole {w.name} workload ({w.S} tokens), {reps} pass{'es' if reps > 1 else ''}")
