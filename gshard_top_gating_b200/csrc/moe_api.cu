@@ -10,6 +10,7 @@
 // The data-dependent per-expert counts stay on the device: the grouped GEMMs
 // read them there.
 #include <math.h>
+#include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -234,6 +235,11 @@ moe_status moe_create(moe_handle* out, int64_t S_max, int64_t M, int64_t H, int3
   // expert's own rows
   const int64_t rows = C < S_max ? C : S_max;
   h->Cbuf = (rows + 255) / 256 * 256;
+  // expert-buffer rows and token choices are 32-bit indices (TMA coordinates, tables)
+  if ((int64_t)E * h->Cbuf > INT32_MAX || S_max * k > INT32_MAX) {
+    delete h;
+    return MOE_ERR_UNSUPPORTED;
+  }
   h->wait_limit_ns = 2000000000ull;   // 2 s per wait: far above any legitimate wait
   cudaError_t ce = cudaGetDevice(&h->device);
   if (ce == cudaSuccess)

@@ -70,7 +70,10 @@ enum { MOE_STAGE_ROUTER = 0, MOE_STAGE_SCAN = 1, MOE_STAGE_DISPATCH = 2, MOE_STA
 /*
  * moe_create -- build a layer handle and allocate its device workspace.
  *
- * S_max            largest token count a forward will be given (>= 1).
+ * S_max            largest token count a forward will be given (1 .. 2^30).  The
+ *                  expert buffers' rows, E * round256(min(C(S_max), S_max)), and
+ *                  S_max * k must stay below 2^31 (32-bit row indices and TMA
+ *                  coordinates); larger sizes return MOE_ERR_UNSUPPORTED.
  * M, H             model and expert-hidden widths; multiples of 64.
  * E, k             number of experts and choices per token, 1 <= k <= E <= 256.
  * capacity_factor  > 0 and finite; C = ceil(capacity_factor * k * S / E) per forward.

@@ -65,6 +65,9 @@ FAKE = 1 << 20   # 16-byte aligned, never dereferenced: validation fails first
     ((64, 64, 100, 8, 2, 1.0), 1),         # H not a multiple of 64
     ((64, 64, 64, 300, 2, 1.0), 2),        # E > 256 unsupported
     ((64, 64, 64, 16, 9, 1.0), 2),         # k > 8 unsupported
+    ((1 << 30, 64, 64, 256, 8, 8.0), 2),   # E * expert rows >= 2^31: 32-bit row indices
+    ((1 << 30, 64, 64, 8, 4, 0.001), 2),   # S_max * k >= 2^31
+    ((1 << 31, 64, 64, 8, 2, 1.0), 2),     # S_max > 2^30
 ])
 def test_create_rejects_bad_arguments_before_device_work(L, args, status):
     h = ctypes.c_void_p(123)
