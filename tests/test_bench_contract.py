@@ -28,3 +28,38 @@ def test_reference_arm_prints_one_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert d["config"]["S"] == 256 and d["config"]["E"] == 8
+
+
+def _bench_module():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    argv, sys.argv = sys.argv, ["bench.py"]
+    try:
+        spec.loader.exec_module(mod)
+    finally:
+        sys.argv = argv
+    return mod
+
+
+def test_expert_gemm_stages_take_the_slower_bound():
+    """An expert GEMM is reported against the tensor peak when its flops take longer
+    than its bytes at HBM bandwidth, else against HBM (few rows per active expert)."""
+    b = _bench_module()
+    from gshard_top_gating_b200.inputs import WORKLOADS
+    pk = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}
+    mid, skewed = WORKLOADS["mid"], WORKLOADS["skewed"]
+    e = b.algorithmic(mid, 16384, 32)["ffn1"]
+    assert e[0] == "gemm" and e[1] == 2.0 * 16384 * 1024 * 4096
+    assert e[2] == 16384 * 1024 * 2 + 32 * 1024 * 4096 * 2 + 16384 * 4096 * 2
+    bound, ach, peak, unit = b.stage_roof(e, 1e-4, pk)
+    assert (bound, unit, peak) == ("tensor", "TFLOP/s", 1000.0) and abs(ach - e[1] / 1e-4 / 1e12) < 1e-9
+    e = b.algorithmic(skewed, 2300, 20)["ffn1"]
+    bound, ach, peak, unit = b.stage_roof(e, 1e-4, pk)
+    assert (bound, unit, peak) == ("hbm", "GB/s", 5000.0) and abs(ach - e[2] / 1e-4 / 1e9) < 1e-9
+    # the backward's weight gradients are written for every expert (zeros for empty ones)
+    d = b.algorithmic_bwd(skewed, 2300, 20, 0, 1)["dW2"]
+    assert d[2] >= skewed.E * skewed.M * skewed.H * 2
+    # 5 GB in 1 ms is 5000 GB/s, the whole of this HBM peak
+    assert b.stage_entry(("hbm", 5e9), 1.0, pk) == {"ms": 1.0, "GB/s": 5000.0, "frac_of_peak": 1.0,
+                                                     "bound": "hbm"}
