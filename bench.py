@@ -1,13 +1,15 @@
 """Benchmark of the GShard MoE layer forward on B200 (one JSON line on stdout).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload mid]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload large]
 
 A step is one whole layer forward (router, capacity scan, dispatch, two grouped
 expert GEMMs, combine, losses) over one batch of synthetic tokens already
-resident in HBM.  The default workload is the mid configuration (S=8192
-tokens, M=1024, H=4096, E=32, top-2, capacity factor 2.0, bf16).  L2 is flushed
-(a 256 MB write) before every timed step and each step is timed with CUDA
-events on the launching stream; the sum over the K steps is the timed region.
+resident in HBM.  The headline workload is the largest single-GPU
+configuration, "large" (S=65536 tokens, M=2048, H=8192, E=64, top-2, capacity
+factor 1.0, bf16).  L2 is flushed (a 256 MB write) before every timed step and
+each step is timed with CUDA events on the launching stream; the sum over the
+K steps is the timed region.  The other four workloads are timed the same way
+in the same run and reported under "per_workload" (--workload-only skips them).
 
 With N > 1 (launched by torch.distributed.run) every rank runs an independent
 replica of the layer on its own GPU and batch (the forward has no exchange on
@@ -176,20 +178,43 @@ def ncu_traffic(kernel: str, workload: str):
 
 def algorithmic(w, A, n_active):
     """Algorithmic work per launch of each stage (A kept assignments, n_active experts
-    with a kept row): ("hbm", bytes), or ("gemm", flops, bytes) for an expert GEMM,
-    whose bytes are its operands read once (the active experts' weights) and its
-    result written once."""
+    with a kept row): ("hbm", bytes), ("latency", bytes) for a stage whose bytes are
+    too few to be bound by HBM, or ("gemm", flops, bytes) for an expert GEMM, whose
+    bytes are its operands read once (the active experts' weights) and its result
+    written once."""
     s = 2 if w.act == "bf16" else 4
     S, M, H, E, k = w.S, w.M, w.H, w.E, w.k
     wts = n_active * M * H * s
+    nchunk = (S + 63) // 64
     return {
         "router": ("hbm", S * M * s + 4 * M * E + S * E * 4 + S * k * 12),
-        "scan": ("hbm", 0),
+        # chunk histograms read, their prefix offsets written, loss partials read
+        "scan": ("latency", 2 * k * nchunk * E * 4 + nchunk * (E + 1) * 4),
         "dispatch": ("hbm", (S + A) * M * s),
         "ffn1": ("gemm", 2.0 * A * M * H, A * M * s + wts + A * H * s),
         "ffn2": ("gemm", 2.0 * A * M * H, A * H * s + wts + A * M * s),
         "combine": ("hbm", (A + S) * M * s + S * k * 12),
     }
+
+
+def layer_roofline(w, A, algo, ms_per_step, pk):
+    """The layer's bound: its expert-FFN flops (4*A*M*H) at the bf16 tensor peak or
+    the total algorithmic bytes of all its stages at the HBM peak, whichever takes
+    longer; frac = that time over the measured step."""
+    flops = 4.0 * A * w.M * w.H
+    nbytes = sum(e[2] if e[0] == "gemm" else e[1] for e in algo.values())
+    t_tc = flops / (pk["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    t = max(t_tc, t_hbm)
+    out = {"bound": "tensor" if t_tc >= t_hbm else "hbm", "ffn_flops": flops, "total_bytes": nbytes,
+           "t_tensor_us": round(t_tc * 1e6, 2), "t_hbm_us": round(t_hbm * 1e6, 2),
+           "t_bound_us": round(t * 1e6, 2), "ms_per_step": round(ms_per_step, 5),
+           "frac": round(t / (ms_per_step / 1e3), 4),
+           "peaks": "bf16 burst and HBM copy"}
+    if pk.get("bf16_tflops_sustained"):
+        t_s = max(flops / (pk["bf16_tflops_sustained"] * 1e12), t_hbm)
+        out["frac_of_sustained"] = round(t_s / (ms_per_step / 1e3), 4)
+    return out
 
 
 def algorithmic_bwd(w, A, n_active, pad_rows, nsplit):
@@ -215,7 +240,10 @@ def algorithmic_bwd(w, A, n_active, pad_rows, nsplit):
 def stage_roof(entry, seconds, pk):
     """(bound, achieved, peak, unit) of one stage.  An expert GEMM is bound by the slower
     of its flops at the bf16 tensor peak and its bytes at the HBM peak (a GEMM over few
-    rows per expert streams weights faster than it can use the tensor cores)."""
+    rows per expert streams weights faster than it can use the tensor cores).  A
+    latency-bound stage reports its bytes per second with no peak."""
+    if entry[0] == "latency":
+        return "latency", entry[1] / seconds / 1e9, None, "GB/s"
     if entry[0] == "gemm":
         flops, nbytes = entry[1], entry[2]
         if flops / (pk["bf16_tflops"] * 1e12) >= nbytes / (pk["hbm_gbs"] * 1e9):
@@ -226,8 +254,8 @@ def stage_roof(entry, seconds, pk):
 
 def stage_entry(entry, ms, pk):
     b_, ach, peak, unit = stage_roof(entry, ms / 1e3, pk)
-    return {"ms": round(ms, 4), unit: round(ach, 1), "frac_of_peak": round(ach / peak, 4),
-            "bound": b_}
+    return {"ms": round(ms, 4), unit: round(ach, 1),
+            "frac_of_peak": round(ach / peak, 4) if peak else None, "bound": b_}
 
 
 def measure_copies(args, x, xh, yh, stream):
@@ -344,18 +372,78 @@ def measure_backward(args, w, weights, x, y, flush, stream, pk, A, n_e):
     }
 
 
-def run_ours(args, rank, world, local):
-    w = WORKLOADS[args.workload]
+def workload_config(w, world):
+    """The workload as both arms name it (same keys and values on the reference arm)."""
+    return {"workload": f"{w.name} (S={w.S}, M={w.M}, H={w.H}, E={w.E}, k={w.k}, cf={w.cf})",
+            "S": w.S, "M": w.M, "H": w.H, "E": w.E, "k": w.k, "capacity_factor": w.cf,
+            "C": math.ceil(w.cf * w.k * w.S / w.E),
+            "l2": "flushed before every timed step (256 MB write)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+def capture_step(layer, x, y, dev, eager):
+    """A CUDA graph of one moe_forward (its six kernels and their programmatic
+    dependencies), or None to time eager calls; with the launch note."""
+    if eager:
+        return None, "eager moe_forward"
+    try:
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            layer(x, out=y)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layer(x, out=y)
+        torch.cuda.synchronize()
+        return graph, "CUDA graph of moe_forward"
+    except Exception as exc:            # capture unsupported: time eager calls instead
+        torch.cuda.synchronize()
+        return None, f"eager moe_forward (graph capture failed: {type(exc).__name__})"
+
+
+def time_steps(step, flush, stream, steps, world):
+    """K steps, L2 flushed before each, device time per step; (total ms over ranks, t0, t1)."""
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.monotonic()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.monotonic()
+    barrier(world)
+    total = max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in zip(starts, ends)), world)
+    return total, t0, t1
+
+
+def stage_times(layer, x, y, flush, steps):
+    """Per-stage device times: events the library records on the stream between its kernels."""
+    from gshard_top_gating_b200 import _lib as L
+    L.moe_set_profiling(layer.h, True)
+    per = [[] for _ in STAGES]
+    for _ in range(steps):
+        flush.zero_()
+        layer(x, out=y)
+        for j, t in enumerate(L.moe_get_stage_times(layer.h)):
+            per[j].append(t)
+    L.moe_set_profiling(layer.h, False)
+    return {n: statistics.mean(v) for n, v in zip(STAGES, per)}
+
+
+def measure_workload(args, w, dev, world, flush, pk, pk_kind, headline):
+    """Time one workload's layer forward.  The headline workload also gets the clock
+    record, the end-to-end host-buffer number, the training step and the CPU baseline."""
     from gshard_top_gating_b200 import _lib as L
     from gshard_top_gating_b200.layer import MoeLayer
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
     x, Wg, b, W1, W2 = make_inputs(w, device=dev)
     layer = MoeLayer(w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b, W1, W2)
     y = torch.empty_like(x)
     stream = torch.cuda.current_stream()
-    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MB > L2
-
     for _ in range(args.warmup):
         layer(x, out=y)
     torch.cuda.synchronize()
@@ -364,27 +452,7 @@ def run_ours(args, rank, world, local):
     n_e = torch.clamp(cnt.long(), max=C)
     A = int(n_e.sum().item())
     n_active = int((n_e > 0).sum().item())
-
-    # ---- the step: one layer forward, replayed from a CUDA graph of moe_forward
-    # (its six kernels and their programmatic dependencies) unless --eager
-    graph = None
-    launch_note = "eager moe_forward"
-    if not args.eager:
-        try:
-            side = torch.cuda.Stream(device=dev)
-            side.wait_stream(torch.cuda.current_stream())
-            with torch.cuda.stream(side):
-                layer(x, out=y)
-            torch.cuda.current_stream().wait_stream(side)
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
-                layer(x, out=y)
-            torch.cuda.synchronize()
-            launch_note = "CUDA graph of moe_forward"
-        except Exception as exc:            # capture unsupported: time eager calls instead
-            graph = None
-            launch_note = f"eager moe_forward (graph capture failed: {type(exc).__name__})"
-            torch.cuda.synchronize()
+    graph, launch_note = capture_step(layer, x, y, dev, args.eager)
 
     def step():
         if graph is not None:
@@ -396,36 +464,34 @@ def run_ours(args, rank, world, local):
         step()
     torch.cuda.synchronize()
 
-    # ---- timed region: K forwards, L2 flushed before each, device time per step
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    clk = ClockSampler(local).__enter__()
-    barrier(world)
-    torch.cuda.synchronize()
-    t_begin = time.monotonic()
-    for i in range(args.steps):
-        flush.zero_()
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-    torch.cuda.synchronize()
-    t_end = time.monotonic()
-    barrier(world)
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = max_over_ranks(sum(step_ms), world)
+    clk = ClockSampler(dev.index or 0).__enter__() if headline else None
+    total_ms, t_begin, t_end = time_steps(step, flush, stream, args.steps, world)
     ms_per_step = total_ms / args.steps
     value = job_throughput(w.S, args.steps, total_ms, world)
+    stage_ms = stage_times(layer, x, y, flush, args.steps)
 
-    # ---- per-stage device times (events recorded by the library on the same stream)
-    L.moe_set_profiling(layer.h, True)
-    per_stage = [[] for _ in STAGES]
-    for i in range(args.steps):
-        flush.zero_()
-        layer(x, out=y)
-        for j, t in enumerate(L.moe_get_stage_times(layer.h)):
-            per_stage[j].append(t)
-    L.moe_set_profiling(layer.h, False)
-    stage_ms = {n: statistics.mean(v) for n, v in zip(STAGES, per_stage)}
+    algo = algorithmic(w, A, n_active)
+    stages = {n: stage_entry(algo[n], stage_ms[n], pk) for n in STAGES if stage_ms[n] > 0}
+    if w.act == "bf16":
+        dom = max(stage_ms, key=lambda n: stage_ms[n])
+        bound, achieved, peak, unit = stage_roof(algo[dom], stage_ms[dom] / 1e3, pk)
+        roof = {"bound": bound, "kernel": dom, "achieved": round(achieved, 2), "peak": peak,
+                "unit": unit, "frac": round(achieved / peak, 4), "traffic": ncu_traffic(dom, w.name),
+                "peak_source": f"{pk_kind}, burst" if bound == "tensor" else pk_kind,
+                "frac_of_sustained": (round(achieved / pk["bf16_tflops_sustained"], 4)
+                                      if bound == "tensor" and pk.get("bf16_tflops_sustained") else None),
+                "layer": layer_roofline(w, A, algo, ms_per_step, pk)}
+    else:
+        roof = {"bound": "latency", "note": "fp32 activations on FFMA kernels: a parity "
+                "configuration, bound by launch latency, with no roofline target"}
+    out = {"value": round(value, 1), "unit": "tokens/s", "ms_per_step": round(ms_per_step, 5),
+           "dtype": w.act, "config": workload_config(w, world),
+           "run": {"kept_assignments": A, "active_experts": n_active, "launch": launch_note},
+           "roofline": roof, "stages": stages,
+           "gpu_launches": args.steps * L.moe_kernels_per_forward(layer.h, w.S)}
+    if not headline:
+        layer.close()
+        return out
 
     # ---- end to end through the C ABI with host buffers (copies inside the timed region)
     xh = x.cpu().pin_memory()
@@ -444,6 +510,7 @@ def run_ours(args, rank, world, local):
     e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), world)
     nbytes = x.numel() * x.element_size()
     copies = measure_copies(args, x, xh, yh, stream)
+    del xh, yh
 
     # clocks: the timed region itself when it held enough samples, else a soak of
     # the same forward right after it (the timed region was too short to sample)
@@ -452,62 +519,60 @@ def run_ours(args, rank, world, local):
     else:
         s0 = time.monotonic()
         while time.monotonic() - s0 < 1.5:
-            for _ in range(20):
+            for _ in range(5):
                 flush.zero_()
                 step()
             torch.cuda.synchronize()
         clocks = clk.summary(s0, time.monotonic(),
                              "1.5 s soak of the same step right after the timed region")
     clk.__exit__()
+    del graph
 
+    out["e2e"] = {"value": round(job_throughput(w.S, args.steps, e2e_ms, world), 1), "unit": "tokens/s",
+                  "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+                  "ms_per_step": round(e2e_ms / args.steps, 4), "copies_alone": copies}
+    out["clocks"] = clocks
+    out["train_step"] = (None if args.no_backward
+                         else measure_backward(args, w, (Wg, b, W1, W2), x, y, flush, stream, pk, A, n_e))
+    layer.close()
+    out["_inputs"] = (x, Wg, b, W1, W2)
+    return out
+
+
+def run_ours(args, rank, world, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MB > L2
     pk, pk_kind = peaks()
-    algo = algorithmic(w, A, n_active)
-    dom = max(stage_ms, key=lambda n: stage_ms[n])
-    bound, achieved, peak, unit = stage_roof(algo[dom], stage_ms[dom] / 1e3, pk)
-    roof = {"bound": bound, "kernel": dom, "achieved": round(achieved, 2), "peak": peak,
-            "unit": unit, "frac": round(achieved / peak, 4), "traffic": ncu_traffic(dom, w.name),
-            "peak_source": f"{pk_kind}, burst" if bound == "tensor" else pk_kind,
-            "frac_of_sustained": (round(achieved / pk["bf16_tflops_sustained"], 4)
-                                  if bound == "tensor" and pk.get("bf16_tflops_sustained") else None)}
-    stages = {n: stage_entry(algo[n], stage_ms[n], pk) for n in STAGES if stage_ms[n] > 0}
-
-    train = (None if args.no_backward
-             else measure_backward(args, w, (Wg, b, W1, W2), x, y, flush, stream, pk, A, n_e))
-
+    w = WORKLOADS[args.workload]
+    head = measure_workload(args, w, dev, world, flush, pk, pk_kind, headline=True)
+    x, Wg, b, W1, W2 = head.pop("_inputs")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_budget, x, Wg, b, W1, W2)
+    del x, Wg, b, W1, W2
+    torch.cuda.empty_cache()
+
+    per = {}
+    if not args.workload_only:
+        for name, wl in WORKLOADS.items():
+            if name == w.name:
+                continue
+            per[name] = measure_workload(args, wl, dev, world, flush, pk, pk_kind, headline=False)
+            torch.cuda.empty_cache()
 
     line = {
         "metric": "MoE-layer tokens/sec on 1 B200; FFN % of bf16 TC peak; dispatch/combine HBM GB/s",
-        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.act, "data": "synthetic",
-        "config": {"workload": f"{w.name} (S={w.S}, M={w.M}, H={w.H}, E={w.E}, k={w.k}, cf={w.cf})",
-                   "S": w.S, "M": w.M, "H": w.H, "E": w.E, "k": w.k, "capacity_factor": w.cf,
-                   "C": C, "kept_assignments": A, "active_experts": n_active,
-                   "l2": "flushed before every timed step (256 MB write)",
-                   "launch": launch_note,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "roofline": roof, "stages": stages,
-        "e2e": {"value": round(job_throughput(w.S, args.steps, e2e_ms, world), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
-                "ms_per_step": round(e2e_ms / args.steps, 4),
-                "copies_alone": copies},
-        "gpu_launches": args.steps * L.moe_kernels_per_forward(layer.h, w.S),
-        "clocks": clocks,
-        "cpu_baseline": cpu,
-        "train_step": train,
+        "config": head["config"], "run": head["run"],
+        "roofline": head["roofline"], "stages": head["stages"], "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+        "cpu_baseline": cpu, "train_step": head["train_step"],
+        "per_workload": per,
     }
-    layer.close()
     return line
-
-
-def _oracle_inputs(w, x, Wg, b, W1, W2):
-    """Host float64 copies of the workload's inputs (the oracle's input form)."""
-    import numpy as np
-    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
-    return (f64(x), f64(Wg), None if b is None else f64(b), f64(W1), f64(W2))
 
 
 def _blas_threads() -> int:
@@ -519,52 +584,102 @@ def _blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def _oracle_step(O, w, inp, ntok):
-    xs, Wg, b, W1, W2 = inp
-    t0 = time.perf_counter()
-    O.forward(xs[:ntok], Wg, b, W1, W2, w.k, w.cf)
-    return time.perf_counter() - t0
+class OracleSample:
+    """The oracle's forward over the first ntok tokens of a workload, as a batch of
+    their own (C scaled to the sample): gate logits, routing, and every sampled
+    token's output through its kept experts (`outputs_for_tokens`).
+
+    The expert weights are handed to the oracle one expert at a time in float64;
+    fetching and converting them is timed apart and left out of the oracle's time.
+    """
+
+    def __init__(self, w, x, Wg, b, W1, W2):
+        import numpy as np
+        f64 = lambda t: None if t is None else t.detach().to("cpu", torch.float64).numpy()
+        self.w = w
+        self.x = x
+        self.Wg, self.b = f64(Wg), f64(b)
+        self.W1, self.W2 = W1, W2
+        self.np = np
+
+    def run(self, ntok):
+        import oracle as O
+        w = self.w
+        fetch = [0.0]
+
+        def expert_weights(e):
+            t0 = time.perf_counter()
+            pair = (self.W1[e].to(torch.float64).cpu().numpy(), self.W2[e].to(torch.float64).cpu().numpy())
+            fetch[0] += time.perf_counter() - t0
+            return pair
+
+        t0 = time.perf_counter()
+        xs = self.x[:ntok].to(torch.float64).cpu().numpy()
+        fetch[0] += time.perf_counter() - t0
+        t0 = time.perf_counter()
+        logits = O.gate_logits(xs, self.Wg, self.b)
+        rt = O.route(logits, w.k, w.cf)
+        O.outputs_for_tokens(self.np.arange(ntok), xs, rt.ids, rt.gates, rt.slot, expert_weights)
+        return time.perf_counter() - t0 - fetch[0]
+
+
+def _sized_runs(sample, budget_s, S, probe=64, max_passes=20):
+    """Oracle passes on a token sample sized to about budget_s seconds of oracle time:
+    a probe pass sizes the sample; a whole workload shorter than the budget is run
+    again (at most max_passes).  Returns (tokens per pass, passes, seconds)."""
+    probe = min(S, probe)
+    c = sample.run(probe) / probe
+    ntok = int(max(probe, min(S, budget_s / max(c, 1e-9))))
+    dt = sample.run(ntok)
+    reps = 1
+    if ntok == S:
+        more = max(0, min(max_passes - 1, int((budget_s - dt) / max(dt, 1e-9))))
+        dt += sum(sample.run(ntok) for _ in range(more))
+        reps += more
+    return ntok, reps, dt
 
 
 def cpu_baseline(w, budget_s, x, Wg, b, W1, W2):
-    """The oracle as it stands, timed on the host cores on a bounded token sample."""
-    import oracle as O
-    inp = _oracle_inputs(w, x, Wg, b, W1, W2)
-    probe = min(w.S, 256)
-    c = _oracle_step(O, w, inp, probe) / probe                 # seconds per token
-    ntok = int(max(64, min(w.S, budget_s / max(c, 1e-9))))
-    dt = _oracle_step(O, w, inp, ntok)
-    reps = 1
-    # a whole workload shorter than the budget is run again until the budget is spent
-    if ntok == w.S:
-        more = max(0, min(19, int((budget_s - dt) / max(dt, 1e-9))))
-        dt += sum(_oracle_step(O, w, inp, ntok) for _ in range(more))
-        reps += more
-    what = (f"first {ntok} of {w.S} tokens of the {w.name} workload (same M, H, E, k, cf; "
-            f"C scaled to the sample)" if ntok < w.S else
-            f"the whole {w.name} workload ({w.S} tokens), {reps} pass{'es' if reps > 1 else ''}")
-    return {"value": round(reps * ntok / dt, 2), "unit": "tokens/s", "cores": _blas_threads(),
-            "kind": "oracle",
-            "sample": f"{what}; float64 oracle forward, {dt:.1f} s; weights converted to float64 "
-                      f"once, outside the timing"}
+    """The oracle as it stands, timed on the host cores on a bounded token sample: with
+    every BLAS thread, and with one thread."""
+    sample = OracleSample(w, x, Wg, b, W1, W2)
+
+    def describe(ntok, reps, dt):
+        what = (f"first {ntok} of {w.S} tokens of the {w.name} workload as their own batch "
+                f"(same M, H, E, k, cf; C scaled to the sample)" if ntok < w.S else
+                f"the whole {w.name} workload ({w.S} tokens), {reps} pass{'es' if reps > 1 else ''}")
+        return (f"{what}; float64 oracle forward (gate logits, routing, outputs of every sampled "
+                f"token), {dt:.1f} s of oracle time; each expert's weights fetched and converted "
+                f"to float64 outside that time")
+
+    ntok, reps, dt = _sized_runs(sample, budget_s, w.S)
+    out = {"value": round(reps * ntok / dt, 2), "unit": "tokens/s", "cores": _blas_threads(),
+           "kind": "oracle", "sample": describe(ntok, reps, dt)}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            n1, r1, d1 = _sized_runs(sample, budget_s / 2, w.S, probe=16, max_passes=5)
+        out["single_thread"] = {"value": round(r1 * n1 / d1, 2), "unit": "tokens/s", "cores": 1,
+                                "sample": describe(n1, r1, d1)}
+    except ImportError:
+        out["single_thread"] = None
+    return out
 
 
 def run_reference(args, rank, world):
     w = WORKLOADS[args.workload]
     if rank != 0:
         return None
-    import oracle as O
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    inp = _oracle_inputs(w, *make_inputs(w, device=dev))
-    torch.cuda.empty_cache() if dev == "cuda" else None
-    probe = min(w.S, 256)
-    c = _oracle_step(O, w, inp, probe) / probe
+    sample = OracleSample(w, *make_inputs(w, device=dev))
+    probe = min(w.S, 64)
+    c = sample.run(probe) / probe
     # per-step sample sized so the whole run stays near args.ref_budget seconds
     per_step = args.ref_budget / max(1, args.steps + args.warmup)
-    ntok = int(max(64, min(w.S, per_step / max(c, 1e-9))))
+    ntok = int(max(min(w.S, 16), min(w.S, per_step / max(c, 1e-9))))
     for _ in range(args.warmup):
-        _oracle_step(O, w, inp, ntok)
-    times = [_oracle_step(O, w, inp, ntok) for _ in range(args.steps)]
+        sample.run(ntok)
+    times = [sample.run(ntok) for _ in range(args.steps)]
     tot = sum(times)
     v = round(ntok * args.steps / tot, 2)
     return {
@@ -574,11 +689,12 @@ def run_reference(args, rank, world):
         "warmup": args.warmup, "ms_per_step": round(1e3 * tot / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": f"{w.name} (S={w.S}, M={w.M}, H={w.H}, E={w.E}, k={w.k}, cf={w.cf})",
-                   "S": w.S, "M": w.M, "H": w.H, "E": w.E, "k": w.k, "capacity_factor": w.cf},
+        "config": workload_config(w, world),
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
-                         "sample": f"first {ntok} of {w.S} tokens per step (same M, H, E, k, cf; "
-                                   f"C scaled to the sample); float64 oracle forward"},
+                         "sample": f"first {ntok} of {w.S} tokens per step as their own batch "
+                                   f"(same M, H, E, k, cf; C scaled to the sample); float64 oracle "
+                                   f"forward; each expert's weights fetched and converted to "
+                                   f"float64 outside the timed oracle work"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -586,10 +702,13 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(WORKLOADS), default="mid")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="large",
+                    help="the headline workload (default: large, the largest single-GPU one)")
+    ap.add_argument("--workload-only", action="store_true",
+                    help="time the headline workload alone (no per_workload lines)")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the CPU baseline sample")
     ap.add_argument("--ref-budget", type=float, default=120.0,

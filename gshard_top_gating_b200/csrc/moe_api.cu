@@ -521,6 +521,24 @@ moe_status moe_route_from_logits(moe_handle h, int64_t S, const float* logits, v
   return MOE_OK;
 }
 
+moe_status moe_get_expert_rows(moe_handle h, int32_t which, int32_t e, int64_t nrows, void* dst,
+                               void* stream) {
+  if (!h || which < MOE_BUF_X || which > MOE_BUF_Y || e < 0 || e >= h->E || nrows < 0 ||
+      nrows > h->Cbuf || (nrows > 0 && !dst))
+    return MOE_ERR_INVALID_ARG;
+  h->last_was_host = false;
+  if (!h->have_forward || !h->fwd_data) return MOE_ERR_STATE;
+  if (nrows == 0) return MOE_OK;
+  const size_t as = act_bytes(h->act);
+  const int64_t width = which == MOE_BUF_H ? h->H : h->M;
+  const void* base = which == MOE_BUF_X ? h->xbuf : which == MOE_BUF_H ? h->hbuf : h->ybuf;
+  const size_t row_bytes = (size_t)width * as;
+  const char* src = static_cast<const char*>(base) + (size_t)e * h->Cbuf * row_bytes;
+  MOE_TRY(cudaMemcpyAsync(dst, src, (size_t)nrows * row_bytes, cudaMemcpyDeviceToDevice,
+                          static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
 moe_status moe_set_profiling(moe_handle h, int32_t enable) {
   if (!h) return MOE_ERR_INVALID_ARG;
   if (enable && !h->have_events) {

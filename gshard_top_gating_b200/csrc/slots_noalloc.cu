@@ -37,11 +37,16 @@ constexpr int kMaxDevices = 64;
 
 std::mutex g_scratch_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
+int g_num_sms[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device.  In host code the
-// array's name is only a host-side stand-in, so the real address is looked up
-// once per device (with that device current) and cached.
-cudaError_t scratch_address(void** out) {
+// Set-up, once per device: the device address of the scratch array and the
+// device's SM count.  In host code the array's name is only a host-side
+// stand-in, so the real address is looked up with that device current and
+// cached for later calls.  The cache belongs to the device's primary context:
+// after cudaDeviceReset the library's module is loaded afresh, the cached
+// address no longer names the array, and this entry point must not be called
+// again in that process.
+cudaError_t scratch_setup(void** out, int* num_sms) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -49,11 +54,15 @@ cudaError_t scratch_address(void** out) {
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
   if (!g_scratch_addr[dev]) {
     void* p = nullptr;
+    int sms = 0;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     g_scratch_addr[dev] = p;
+    g_num_sms[dev] = sms > 0 ? sms : 1;
   }
   *out = g_scratch_addr[dev];
+  *num_sms = g_num_sms[dev];
   return cudaSuccess;
 }
 
@@ -178,7 +187,8 @@ extern "C" MOE_API moe_status moe_assign_slots_noalloc(int64_t S, int32_t E, int
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   void* base = nullptr;
-  cudaError_t ce = scratch_address(&base);
+  int num_sms = 1;
+  cudaError_t ce = scratch_setup(&base, &num_sms);
   if (ce != cudaSuccess) return status_of(ce);
   if (S == 0) return status_of(cudaMemsetAsync(cnt_dev, 0, (size_t)E * 4, st));
 
@@ -188,8 +198,9 @@ extern "C" MOE_API moe_status moe_assign_slots_noalloc(int64_t S, int32_t E, int
   int32_t* off = reinterpret_cast<int32_t*>(p + lrank_bytes + table_bytes);
   na_chunk_kernel<<<nchunk, kThreads, 0, st>>>(eidx_dev, (int)S, E, k, nchunk, lrank, hist);
   na_scan_kernel<<<E, kThreads, 0, st>>>(E, k, nchunk, hist, off, cnt_dev);
-  const int64_t n = S * k;
-  const int grid = (int)((n + kThreads - 1) / kThreads < 148 * 8 ? (n + kThreads - 1) / kThreads : 148 * 8);
+  // grid-stride slot pass: at most 8 blocks of 256 threads per SM
+  const int64_t n = S * k, blocks = (n + kThreads - 1) / kThreads, cap = (int64_t)num_sms * 8;
+  const int grid = (int)(blocks < cap ? blocks : cap);
   na_slot_kernel<<<grid, kThreads, 0, st>>>(eidx_dev, (int)S, E, k, C, nchunk, off, lrank, slot_dev);
   return status_of(cudaGetLastError());
 }

@@ -104,6 +104,13 @@ class MoeLayer:
         L.moe_get_routing(self.h, eidx, gate, slot, cnt, stream)
         return eidx, gate, slot, cnt
 
+    def expert_rows(self, which: int, e: int, nrows: int, stream=None) -> torch.Tensor:
+        """Rows 0..nrows-1 of expert e in xbuf / hbuf / ybuf (L.MOE_BUF_X / _H / _Y)."""
+        width = self.H if which == L.MOE_BUF_H else self.M
+        out = torch.empty(nrows, width, dtype=self.act, device="cuda")
+        L.moe_get_expert_rows(self.h, which, e, nrows, out, stream)
+        return out
+
     def route_from_logits(self, logits: torch.Tensor, stream=None) -> None:
         L.moe_route_from_logits(self.h, logits.shape[0], logits, stream)
 

@@ -161,6 +161,23 @@ MOE_API moe_status moe_get_routing(moe_handle h, int32_t* eidx_dev, float* gate_
  */
 MOE_API moe_status moe_route_from_logits(moe_handle h, int64_t S, const float* logits_dev, void* stream);
 
+/* Buffers of moe_get_expert_rows. */
+enum { MOE_BUF_X = 0,   /* xbuf [E, Cbuf, M] act: the dispatched token rows */
+       MOE_BUF_H = 1,   /* hbuf [E, Cbuf, H] act: relu(xbuf W1[e]) */
+       MOE_BUF_Y = 2 }; /* ybuf [E, Cbuf, M] act: hbuf W2[e] */
+
+/*
+ * moe_get_expert_rows -- copy rows 0 .. nrows-1 of expert e's slots in one of the
+ * per-expert buffers of the last moe_forward (which = MOE_BUF_X, MOE_BUF_H or
+ * MOE_BUF_Y) to dst_dev, a device buffer of nrows rows of M (or H for MOE_BUF_H)
+ * act elements.  Row i is the assignment the capacity scan gave slot i of expert
+ * e; only rows below n_e = min(cnt[e], C) hold data.  0 <= nrows <= the handle's
+ * rows per expert (min(C(S_max), S_max) rounded up to 256).  Device-to-device copy
+ * on `stream`.  Returns MOE_ERR_STATE unless the last routing call was a moe_forward.
+ */
+MOE_API moe_status moe_get_expert_rows(moe_handle h, int32_t which, int32_t e, int64_t nrows,
+                                       void* dst_dev, void* stream);
+
 /* Capacity C this handle uses for S tokens (host arithmetic, no device work). */
 MOE_API moe_status moe_get_capacity(moe_handle h, int64_t S, int64_t* C_out);
 
@@ -205,9 +222,11 @@ MOE_API moe_status moe_selftest_wait_timeout(int32_t limit_us, void* stream);
  * every GPU that loads the library holds until the process exits.  The call
  * needs round256(4*S*k) + 2*round256(4*k*ceil(S/64)*E) bytes of it and
  * returns MOE_ERR_UNSUPPORTED, with no device work, when that exceeds 8 MiB.
- * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture.  Every call shares the array and leaves its contents behind, so
+ * The first call on a device looks up the array's device address and the
+ * device's SM count (with that device current) and caches them; make that
+ * first call before any stream capture.  The cache does not survive
+ * cudaDeviceReset: after a reset, do not call this entry point again in the
+ * same process.  Every call shares the array and leaves its contents behind, so
  * calls whose work overlaps on the GPU (other streams, other host threads)
  * race.  Enqueued on `stream`; no host synchronisation.
  */

@@ -63,3 +63,35 @@ def test_expert_gemm_stages_take_the_slower_bound():
     # 5 GB in 1 ms is 5000 GB/s, the whole of this HBM peak
     assert b.stage_entry(("hbm", 5e9), 1.0, pk) == {"ms": 1.0, "GB/s": 5000.0, "frac_of_peak": 1.0,
                                                      "bound": "hbm"}
+
+
+def test_reference_arm_names_the_same_workload_config():
+    """Both arms print the same config dict for a workload, so the driver can pair them."""
+    b = _bench_module()
+    from gshard_top_gating_b200.inputs import WORKLOADS
+    for name in ("tiny", "large"):
+        cfg = b.workload_config(WORKLOADS[name], 1)
+        assert cfg["S"] == WORKLOADS[name].S and "l2" in cfg and cfg["workload"].startswith(name)
+    assert b.workload_config(WORKLOADS["large"], 1)["C"] == 2048
+    assert b.workload_config(WORKLOADS["wide"], 1)["C"] == 640
+
+
+def test_layer_roofline_takes_the_slower_of_tensor_and_hbm():
+    """The layer's bound is max(4*A*M*H flops at the tensor peak, all stages' bytes at HBM)."""
+    b = _bench_module()
+    from gshard_top_gating_b200.inputs import WORKLOADS
+    pk = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}
+    w = WORKLOADS["large"]
+    A = 2 * w.S
+    algo = b.algorithmic(w, A, w.E)
+    r = b.layer_roofline(w, A, algo, 10.0, pk)
+    flops = 4.0 * A * w.M * w.H
+    nbytes = sum(e[2] if e[0] == "gemm" else e[1] for e in algo.values())
+    assert r["ffn_flops"] == flops and r["total_bytes"] == nbytes
+    assert r["bound"] == "tensor" and abs(r["t_tensor_us"] - flops / 1e15 * 1e6) < 0.01
+    assert abs(r["frac"] - flops / 1e15 / 10e-3) < 1e-4
+    # few kept rows over many experts' weights: bytes dominate
+    r = b.layer_roofline(WORKLOADS["skewed"], 2300, b.algorithmic(WORKLOADS["skewed"], 2300, 20), 1.0, pk)
+    assert r["bound"] == "hbm" and r["t_bound_us"] == r["t_hbm_us"]
+    # the capacity scan is reported as latency-bound, with no fraction of a peak
+    assert b.stage_entry(b.algorithmic(w, A, w.E)["scan"], 0.05, pk)["bound"] == "latency"

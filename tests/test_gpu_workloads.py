@@ -1,20 +1,50 @@
 """The five benchmark workloads at full size, in the launch configuration the bench times (GPU).
 
-Routing is compared in full (every token, bit-exact given the GPU's logits);
-logits and layer outputs on seeded token samples the oracle computes one by
-one (every output row depends only on its own token once the routing is
-fixed); losses against the oracle both on the GPU's logits and on its own.
+Routing is compared in full (every token, bit-exact given the GPU's logits).
+Logits and layer outputs are compared on seeded token samples the oracle
+computes one by one (every output row depends only on its own token once the
+routing is fixed): every token of the tiny workload, and at least 2048 tokens
+of each bf16 workload.  For three seeded experts of each bf16 workload (the
+most loaded one and two others with kept rows), every kept row of the
+expert's first-layer output h and second-layer output is read back from the
+per-expert buffers and compared with the oracle's expert FFN of the same
+dispatched token rows, so every GEMM tile of those experts is checked.  Losses
+are compared both on the GPU's logits and on the oracle's own.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle as O
+from gshard_top_gating_b200 import _lib as L
 from gshard_top_gating_b200.inputs import WORKLOADS
 from tests import gpu_helpers as G
 
 pytestmark = pytest.mark.gpu
 
-SAMPLES = {"tiny": None, "mid": 768, "skewed": 768, "large": 384, "wide": 48}
+SAMPLES = {"tiny": None, "mid": 2048, "skewed": 2048, "large": 2048, "wide": 2048}
+
+
+def _expert_rows_check(run, out, rt, e):
+    """Every kept row of expert e: x, h = relu(x W1[e]) and y = h W2[e] in the
+    expert buffers against the oracle's float64 expert FFN of the same tokens."""
+    n = int(min(rt.cnt[e], rt.C))
+    tok = np.full(n, -1, dtype=np.int64)
+    for r in range(run.w.k):
+        sel = np.nonzero((rt.ids[:, r] == e) & (rt.slot[:, r] >= 0))[0]
+        tok[rt.slot[sel, r]] = sel
+    assert np.all(tok >= 0), "every slot below n_e holds one assignment"
+    xs = run.x[torch.as_tensor(tok, device=run.x.device)]
+    got_x = run.layer.expert_rows(L.MOE_BUF_X, e, n)
+    assert torch.equal(got_x, xs), "dispatched rows"
+    W1e, W2e = run.W1[e].cpu(), run.W2[e].cpu()
+    h_ref = np.maximum(O._f64(xs.cpu()) @ O._f64(W1e), 0.0)
+    y_ref = O.expert_ffn(xs.cpu(), W1e, W2e)
+    e_h = G.rel_err(run.layer.expert_rows(L.MOE_BUF_H, e, n).float().cpu().numpy(), h_ref)
+    e_y = G.rel_err(run.layer.expert_rows(L.MOE_BUF_Y, e, n).float().cpu().numpy(), y_ref)
+    tol = G.TOL_Y[run.w.act]
+    assert e_h <= tol and e_y <= tol, (e, e_h, e_y)
+    return n, e_h, e_y
 
 
 @pytest.mark.parametrize("name", list(WORKLOADS))
@@ -24,19 +54,42 @@ def test_workload_full_size(name):
     out = G.forward(run)
     rt = G.check_routing(run, out)
     n = SAMPLES[name]
+    rng = np.random.default_rng(2024)
     if n is None:
         tokens = np.arange(w.S)
     else:
-        rng = np.random.default_rng(2024)
         tokens = np.unique(np.concatenate([[0, w.S - 1], rng.choice(w.S, n, replace=False)]))
     e_logits = G.check_logits(run, out, tokens)
     e_y = G.check_outputs(run, out, rt, tokens)
     G.check_losses_own_logits(run, out)
-    print(f"\n{name}: logits rel err {e_logits:.3e}, output rel err {e_y:.3e}, "
-          f"dropped {(out.slot < 0).mean():.4f}, l_aux {out.l_aux:.6f}, z {out.z:.6f}")
+    msg = (f"\n{name}: {len(tokens)} tokens: logits rel err {e_logits:.3e}, output rel err {e_y:.3e}, "
+           f"dropped {(out.slot < 0).mean():.4f}, l_aux {out.l_aux:.6f}, z {out.z:.6f}")
+    if w.act == "bf16":
+        n_e = np.minimum(rt.cnt, rt.C)
+        live = np.nonzero(n_e > 0)[0]
+        others = rng.choice(np.setdiff1d(live, [int(np.argmax(n_e))]), 2, replace=False)
+        for e in [int(np.argmax(n_e))] + [int(v) for v in others]:
+            rows, e_h, e_ye = _expert_rows_check(run, out, rt, e)
+            msg += f"\n  expert {e}: {rows} kept rows, h rel err {e_h:.3e}, expert output rel err {e_ye:.3e}"
+    print(msg)
     # capacity invariants at full size
     n_e = np.minimum(rt.cnt, rt.C)
     assert np.all(n_e <= rt.C) and (out.slot >= 0).sum() == n_e.sum()
     run.layer.close()
     del run
     torch.cuda.empty_cache()
+
+
+def test_expert_rows_getter_rejects_bad_arguments():
+    w = WORKLOADS["tiny"]
+    run = G.build(w, S=64)
+    buf = torch.empty(4, w.M, dtype=torch.float32, device="cuda")
+    with pytest.raises(L.MoeError) as ei:
+        run.layer.expert_rows(L.MOE_BUF_Y, 0, 4)         # before any forward
+    assert ei.value.status == L.MOE_ERR_STATE
+    G.forward(run)
+    for which, e, nrows in ((3, 0, 4), (L.MOE_BUF_X, w.E, 4), (L.MOE_BUF_X, 0, 10 ** 6)):
+        with pytest.raises(L.MoeError) as ei:
+            L.moe_get_expert_rows(run.layer.h, which, e, nrows, buf)
+        assert ei.value.status == L.MOE_ERR_INVALID_ARG
+    run.layer.close()
