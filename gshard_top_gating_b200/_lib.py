@@ -60,10 +60,27 @@ def _load() -> ctypes.CDLL:
         "moe_get_backward_stage_times": [P, ctypes.POINTER(ctypes.c_float), I32],
         "moe_backward": [P, I64, P, P, ctypes.c_float, ctypes.c_float, P, P, P, P, P, P],
     }
+    I64P = ctypes.POINTER(I64)
+    sig.update({
+        "moe_ep_plan": [I32, I32, I32, I32, D, P, P, I64P, P, P, P, P],
+        "moe_ep_create": [ctypes.POINTER(P), I32, I32, I64, I64, I64, I64, I32, I32, D, ctypes.c_int,
+                          P, P, P, P],
+        "moe_ep_destroy": [P],
+        "moe_ep_buffer_rows": [P, I64P, I64P],
+        "moe_ep_route": [P, I64, P, P, P],
+        "moe_ep_dispatch": [P, P, P, P, P, P, P],
+        "moe_ep_experts": [P, P, P],
+        "moe_ep_combine": [P, P, P, P],
+        "moe_ep_aux_loss": [P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)],
+        "moe_ep_get_routing": [P, P, P, P, P, P, P],
+        "moe_ep_check": [P, P],
+    })
     for name, args in sig.items():
         f = getattr(lib, name)
         f.argtypes = args
         f.restype = ctypes.c_int
+    lib.moe_ep_stats_len.argtypes = [I32, I32]
+    lib.moe_ep_stats_len.restype = I32
     lib.moe_kernels_per_forward.argtypes = [P, I64]
     lib.moe_kernels_per_forward.restype = I32
     lib.moe_kernels_per_backward.argtypes = [P, I64]
@@ -213,3 +230,86 @@ def moe_backward_stage_name(stage: int) -> str:
 
 def moe_set_backward_flags(h, flags: int) -> None:
     _check("moe_set_backward_flags", lib.moe_set_backward_flags(h, int(flags)))
+
+
+# ---- expert parallelism (include/moe.h): host buffers are numpy int64 / float64 arrays
+
+def _np_ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def moe_ep_stats_len(E, k) -> int:
+    return int(lib.moe_ep_stats_len(E, k))
+
+
+def moe_ep_plan(G, g, E, k, capacity_factor, counts, S):
+    """Host exchange plan of rank g: (C, send_rows[G], recv_rows[G], base[G,k,E], kept[G,k,E])."""
+    import numpy as np
+    cnt = np.ascontiguousarray(counts, dtype=np.int64)
+    Sv = np.ascontiguousarray(S, dtype=np.int64)
+    C = ctypes.c_int64()
+    send = np.zeros(G, dtype=np.int64)
+    recv = np.zeros(G, dtype=np.int64)
+    base = np.zeros((G, k, E), dtype=np.int64)
+    kept = np.zeros((G, k, E), dtype=np.int64)
+    _check("moe_ep_plan", lib.moe_ep_plan(G, g, E, k, float(capacity_factor), _np_ptr(cnt), _np_ptr(Sv),
+                                          ctypes.byref(C), _np_ptr(send), _np_ptr(recv), _np_ptr(base),
+                                          _np_ptr(kept)))
+    return C.value, send, recv, base, kept
+
+
+def moe_ep_create(G, g, S_max, S_total_max, M, H, E, k, capacity_factor, act, Wg, gate_bias, W1, W2) -> int:
+    h = ctypes.c_void_p()
+    dt = MOE_BF16 if act in ("bf16", torch.bfloat16, MOE_BF16) else MOE_F32
+    _check("moe_ep_create", lib.moe_ep_create(ctypes.byref(h), G, g, S_max, S_total_max, M, H, E, k,
+                                              float(capacity_factor), dt, _ptr(Wg), _ptr(gate_bias),
+                                              _ptr(W1), _ptr(W2)))
+    return h.value
+
+
+def moe_ep_destroy(h) -> None:
+    _check("moe_ep_destroy", lib.moe_ep_destroy(h))
+
+
+def moe_ep_buffer_rows(h):
+    a, b = ctypes.c_int64(), ctypes.c_int64()
+    _check("moe_ep_buffer_rows", lib.moe_ep_buffer_rows(h, ctypes.byref(a), ctypes.byref(b)))
+    return a.value, b.value
+
+
+def moe_ep_route(h, S, x, stats, stream=None) -> None:
+    _check("moe_ep_route", lib.moe_ep_route(h, S, _ptr(x), _ptr(stats), _stream(stream)))
+
+
+def moe_ep_dispatch(h, stats_all, x, sendbuf, G, stream=None):
+    """stats_all: numpy float64 [G, stats_len]; returns (send_rows[G], recv_rows[G]) int64."""
+    import numpy as np
+    st = np.ascontiguousarray(stats_all, dtype=np.float64)
+    send = np.zeros(G, dtype=np.int64)
+    recv = np.zeros(G, dtype=np.int64)
+    _check("moe_ep_dispatch", lib.moe_ep_dispatch(h, _np_ptr(st), _ptr(x), _ptr(sendbuf), _np_ptr(send),
+                                                  _np_ptr(recv), _stream(stream)))
+    return send, recv
+
+
+def moe_ep_experts(h, recvbuf, stream=None) -> None:
+    _check("moe_ep_experts", lib.moe_ep_experts(h, _ptr(recvbuf), _stream(stream)))
+
+
+def moe_ep_combine(h, sendbuf, y, stream=None) -> None:
+    _check("moe_ep_combine", lib.moe_ep_combine(h, _ptr(sendbuf), _ptr(y), _stream(stream)))
+
+
+def moe_ep_aux_loss(h):
+    a, z = ctypes.c_float(), ctypes.c_float()
+    _check("moe_ep_aux_loss", lib.moe_ep_aux_loss(h, ctypes.byref(a), ctypes.byref(z)))
+    return a.value, z.value
+
+
+def moe_ep_get_routing(h, eidx=None, gate=None, slot=None, spos=None, logits=None, stream=None) -> None:
+    _check("moe_ep_get_routing", lib.moe_ep_get_routing(h, _ptr(eidx), _ptr(gate), _ptr(slot), _ptr(spos),
+                                                        _ptr(logits), _stream(stream)))
+
+
+def moe_ep_check(h, stream=None) -> None:
+    _check("moe_ep_check", lib.moe_ep_check(h, _stream(stream)))

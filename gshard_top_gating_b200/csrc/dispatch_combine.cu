@@ -10,6 +10,8 @@
 // are dropped).  Both kernels are token-centric (one warp per token), read and
 // write whole rows in 16-byte vectors, and need no atomics, so the result does
 // not depend on scheduling.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -173,6 +175,119 @@ __global__ void __launch_bounds__(kThreads, KM >= 8 ? 3 : 4) combine_kernel(cons
   }
 }
 
+// Expert parallelism, sending side: the global rank-major slot of each of the rank's
+// choices is base[r][e] (all earlier ranks' and earlier choice ranks' demand of e, from
+// the exchanged counts) plus the rank-local position off[r][c][e] + lrank.  Kept rows go
+// to the send buffer, where each (expert, rank r) run of this rank's kept choices starts
+// at soff[r][e]; a run's kept choices are a prefix of it, so row = soff + local position.
+template <typename T, int KM>
+__global__ void __launch_bounds__(kThreads, 4) ep_dispatch_kernel(const T* __restrict__ x, int S, int M,
+                                                                  int E, int k, int C, int nchunk,
+                                                                  Routing R, const int32_t* __restrict__ base,
+                                                                  const int32_t* __restrict__ soff,
+                                                                  int32_t* __restrict__ spos,
+                                                                  T* __restrict__ sendbuf) {
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * kThreads) >> 5;
+  const int nv = (int)((int64_t)M * sizeof(T) / 16);
+  pdl_trigger();
+  pdl_wait();                                  // local offsets and the exchanged plan complete
+  for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < S; t += warps) {
+    int sp = -1;
+    if (lane < k) {
+      const int e = R.eidx[(int64_t)t * k + lane];
+      int s = -1;
+      if (e >= 0 && e < E) {
+        const int local = R.off[((int64_t)lane * nchunk + t / kChunk) * E + e] + R.lrank[(int64_t)t * k + lane];
+        const int g = base[lane * E + e] + local;
+        if (g < C) {
+          s = g;
+          sp = soff[lane * E + e] + local;
+        }
+      } else {
+        atomicOr(R.err, DEVERR_BOUNDS);
+      }
+      R.slot[(int64_t)t * k + lane] = s;
+      spos[(int64_t)t * k + lane] = sp;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)t * M);
+    uint4* dst[KM];
+    bool any = false;
+#pragma unroll
+    for (int r = 0; r < KM; ++r) {
+      const int pr = __shfl_sync(0xffffffffu, sp, r);
+      dst[r] = (r < k && pr >= 0) ? reinterpret_cast<uint4*>(sendbuf + (int64_t)pr * M) : nullptr;
+      any |= dst[r] != nullptr;
+    }
+    if (!any) continue;                        // every choice dropped: the row is not sent
+    for (int v0 = lane; v0 < nv; v0 += 32 * kUnroll) {
+      uint4 val[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (v0 + 32 * u < nv) val[u] = ld_nc_v4(src + v0 + 32 * u);
+#pragma unroll
+      for (int r = 0; r < KM; ++r) {
+        if (dst[r] == nullptr) continue;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+          if (v0 + 32 * u < nv) dst[r][v0 + 32 * u] = val[u];
+      }
+    }
+  }
+}
+
+// Expert parallelism, receiving side: one warp per received row.  The row's segment is
+// the last q with seg_start[q] <= j (empty segments share their start with the next
+// one, so the last such q is the non-empty segment holding j).
+__global__ void __launch_bounds__(kThreads) ep_unpack_kernel(const uint4* __restrict__ recv, int nrows,
+                                                             int nv, const int32_t* __restrict__ seg_start,
+                                                             const int32_t* __restrict__ seg_dst, int nseg,
+                                                             int32_t* __restrict__ rowmap,
+                                                             uint4* __restrict__ xbuf, unsigned* err,
+                                                             int64_t xrows) {
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * kThreads) >> 5;
+  pdl_trigger();
+  pdl_wait();
+  for (int j = (blockIdx.x * kThreads + threadIdx.x) >> 5; j < nrows; j += warps) {
+    int lo = 0, hi = nseg;                     // first q with seg_start[q] > j
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (seg_start[mid] <= j) lo = mid + 1;
+      else hi = mid;
+    }
+    const int q = lo - 1;
+    const int64_t row = q >= 0 ? (int64_t)seg_dst[q] + (j - seg_start[q]) : -1;
+    if (row < 0 || row >= xrows) {             // a plan inconsistent with the rows received
+      if (lane == 0) {
+        atomicOr(err, DEVERR_BOUNDS);
+        rowmap[j] = -1;
+      }
+      continue;
+    }
+    if (lane == 0) rowmap[j] = (int32_t)row;
+    const uint4* s = recv + (int64_t)j * nv;
+    uint4* d = xbuf + row * nv;
+    for (int v = lane; v < nv; v += 32) d[v] = ld_nc_v4(s + v);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) ep_repack_kernel(const uint4* __restrict__ ybuf, int nrows, int nv,
+                                                             const int32_t* __restrict__ rowmap,
+                                                             uint4* __restrict__ recv) {
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * kThreads) >> 5;
+  pdl_trigger();
+  pdl_wait();                                  // expert outputs complete
+  for (int j = (blockIdx.x * kThreads + threadIdx.x) >> 5; j < nrows; j += warps) {
+    const int row = rowmap[j];
+    if (row < 0) continue;
+    const uint4* s = ybuf + (int64_t)row * nv;
+    uint4* d = recv + (int64_t)j * nv;
+    for (int v = lane; v < nv; v += 32) d[v] = ld_nc_v4(s + v);
+  }
+}
+
 int grid_for(int S) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -224,6 +339,46 @@ cudaError_t launch_dispatch(const void* x, bool bf16, int S, int M, int E, int k
   else
     dispatch_k<float>(k, x, S, M, E, C, Cbuf, nchunk, R, xbuf, grid, st);
   return cudaGetLastError();
+}
+
+cudaError_t launch_ep_dispatch(const void* x, bool bf16, int S, int M, int E, int k, int C,
+                               const Routing& R, const int32_t* base, const int32_t* soff,
+                               int32_t* spos, void* sendbuf, cudaStream_t st) {
+  const int nchunk = (S + kChunk - 1) / kChunk;
+  const int grid = grid_for(S);
+  auto go = [&](auto tag, auto km) {
+    using T = decltype(tag);
+    constexpr int KM = decltype(km)::value;
+    return launch_pdl(ep_dispatch_kernel<T, KM>, dim3(grid), dim3(kThreads), 0, st, (const T*)x, S, M, E,
+                      k, C, nchunk, R, base, soff, spos, (T*)sendbuf);
+  };
+  using I1 = std::integral_constant<int, 1>;
+  using I2 = std::integral_constant<int, 2>;
+  using I4 = std::integral_constant<int, 4>;
+  using I8 = std::integral_constant<int, 8>;
+  if (bf16) {
+    const __nv_bfloat16 b{};
+    return k <= 1 ? go(b, I1{}) : k <= 2 ? go(b, I2{}) : k <= 4 ? go(b, I4{}) : go(b, I8{});
+  }
+  return k <= 1 ? go(0.f, I1{}) : k <= 2 ? go(0.f, I2{}) : k <= 4 ? go(0.f, I4{}) : go(0.f, I8{});
+}
+
+cudaError_t launch_ep_unpack(const void* recvbuf, bool bf16, int nrows, int M, const int32_t* seg_start,
+                             const int32_t* seg_dst, int nseg, int32_t* rowmap, void* xbuf,
+                             unsigned* err, int64_t xrows, cudaStream_t st) {
+  if (nrows <= 0) return cudaSuccess;
+  const int nv = (int)((int64_t)M * (bf16 ? 2 : 4) / 16);
+  return launch_pdl(ep_unpack_kernel, dim3(grid_for(nrows)), dim3(kThreads), 0, st,
+                    (const uint4*)recvbuf, nrows, nv, seg_start, seg_dst, nseg, rowmap, (uint4*)xbuf, err,
+                    xrows);
+}
+
+cudaError_t launch_ep_repack(const void* ybuf, bool bf16, int nrows, int M, const int32_t* rowmap,
+                             void* recvbuf, cudaStream_t st) {
+  if (nrows <= 0) return cudaSuccess;
+  const int nv = (int)((int64_t)M * (bf16 ? 2 : 4) / 16);
+  return launch_pdl(ep_repack_kernel, dim3(grid_for(nrows)), dim3(kThreads), 0, st, (const uint4*)ybuf,
+                    nrows, nv, rowmap, (uint4*)recvbuf);
 }
 
 cudaError_t launch_combine(const void* ybuf, bool bf16, int S, int M, int k, int64_t Cbuf,

@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 
 #include <utility>
@@ -12,6 +13,16 @@ namespace moe {
 constexpr int kMaxExperts = 256;
 constexpr int kMaxK = 8;
 constexpr int kChunk = 64;          // tokens per router CTA (= scan chunk)
+
+// Expert capacity C = ceil(capacity_factor * k * S / E), evaluated in double left to
+// right ("GShard: Scaling Giant Models with Conditional Computation and Automatic
+// Sharding", paper-note summary: tokens beyond an expert's capacity, set by the
+// capacity factor, are dropped); clamped to 2^31 - 1.
+inline int64_t capacity_of(double cf, int k, int64_t S, int E) {
+  const double c = ceil(cf * (double)k * (double)S / (double)E);
+  if (!(c < 2147483647.0)) return 2147483647;
+  return (int64_t)c;
+}
 
 // Launch with programmatic stream serialization: the kernel may begin while the
 // previous kernel on the stream finishes, and orders itself with pdl_wait().
@@ -63,6 +74,27 @@ cudaError_t launch_router_tc(const CUtensorMap& tmX, const CUtensorMap& tmW, con
                              int M, int E, int k, const Routing& R, uint64_t limit_ns, cudaStream_t st);
 // scan.cu
 cudaError_t launch_scan(int S, int E, int k, int C, int64_t Cbuf, const Routing& R, cudaStream_t st);
+// scan.cu, expert parallelism: per-rank scan of one rank's tokens.  off[r][c][e] gets the
+// exclusive prefix of hist[r][.][e] over chunks; stats (doubles, ep_stats_len(E, k)):
+// [r*E + e] rank-r demand of expert e, [k*E + j] sum over tokens of p_tj,
+// [k*E + E] sum of lse^2, [k*E + E + 1] the rank's token count S.
+inline int ep_stats_len(int E, int k) { return k * E + E + 2; }
+cudaError_t launch_ep_scan(int S, int E, int k, const Routing& R, double* stats, cudaStream_t st);
+// dispatch_combine.cu, expert parallelism (one rank's side of the two exchanges):
+//   ep_dispatch: slot[t][r] = base[r][e] + off[r][c][e] + lrank (global rank-major slot),
+//     kept iff < C; a kept row goes to sendbuf[soff[r][e] + off + lrank] (runs ordered by
+//     destination rank, expert, rank r), spos[t][r] = that row or -1
+//   ep_unpack: received row j of segment q (starts seg_start[q], sorted) goes to expert row
+//     seg_dst[q] + (j - seg_start[q]); rowmap[j] records it
+//   ep_repack: recvbuf[j] = ybuf[rowmap[j]] (the expert outputs go back in arrival order)
+cudaError_t launch_ep_dispatch(const void* x, bool bf16, int S, int M, int E, int k, int C,
+                               const Routing& R, const int32_t* base, const int32_t* soff,
+                               int32_t* spos, void* sendbuf, cudaStream_t st);
+cudaError_t launch_ep_unpack(const void* recvbuf, bool bf16, int nrows, int M, const int32_t* seg_start,
+                             const int32_t* seg_dst, int nseg, int32_t* rowmap, void* xbuf,
+                             unsigned* err, int64_t xrows, cudaStream_t st);
+cudaError_t launch_ep_repack(const void* ybuf, bool bf16, int nrows, int M, const int32_t* rowmap,
+                             void* recvbuf, cudaStream_t st);
 // dispatch_combine.cu
 cudaError_t launch_dispatch(const void* x, bool bf16, int S, int M, int E, int k, int C,
                             int64_t Cbuf, const Routing& R, void* xbuf, cudaStream_t st);

@@ -103,12 +103,6 @@ moe_status from_cuda(cudaError_t e) {
   return MOE_ERR_CUDA;
 }
 
-// C = ceil(capacity_factor * k * S / E), evaluated in double left to right.
-int64_t capacity_of(double cf, int k, int64_t S, int E) {
-  const double c = ceil(cf * (double)k * (double)S / (double)E);
-  if (!(c < 2147483647.0)) return 2147483647;
-  return (int64_t)c;
-}
 
 struct Carver {
   char* base;

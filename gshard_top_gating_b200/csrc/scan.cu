@@ -125,7 +125,66 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(int S, int E, int k, int
   }
 }
 
+// Expert parallelism: the scan of one rank's own tokens.  Block e (< E): for every
+// rank r, the exclusive prefix of hist[r][.][e] over the rank's chunks (the position of
+// each chunk's first rank-r choice of e among the rank's own rank-r choices of e) and
+// the total.  Block E: the loss partials of the rank's tokens, summed in double in a
+// fixed order (chunk groups as in scan_kernel), and the token count.
+__global__ void __launch_bounds__(kThreads) ep_scan_kernel(int S, int E, int k, int nchunk, Routing R,
+                                                           double* __restrict__ stats) {
+  __shared__ int warp_sums[kThreads / 32];
+  __shared__ double dsum[kThreads / 32];
+  const int tid = threadIdx.x;
+  pdl_trigger();
+  pdl_wait();                                  // router tables complete
+  if (blockIdx.x < (unsigned)E) {
+    const int e = blockIdx.x;
+    const int seg = (nchunk + kThreads - 1) / kThreads;
+    const int a = min(nchunk, tid * seg), b = min(nchunk, a + seg);
+    for (int r = 0; r < k; ++r) {
+      const int64_t q0 = (int64_t)r * nchunk;
+      int local = 0;
+      for (int c = a; c < b; ++c) local += R.hist[(q0 + c) * E + e];
+      int total;
+      int run = block_exclusive_scan(local, warp_sums, total);
+      for (int c = a; c < b; ++c) {
+        R.off[(q0 + c) * E + e] = run;
+        run += R.hist[(q0 + c) * E + e];
+      }
+      if (tid == 0) stats[(int64_t)r * E + e] = (double)total;
+      __syncthreads();                         // warp_sums is reused by the next rank
+    }
+    return;
+  }
+  __shared__ double part_P[kThreads];
+  const int G = E >= kThreads ? 1 : kThreads / E;
+  if (tid < E * G) {
+    const int j = tid % E, g = tid / E;
+    double P = 0.0;
+    for (int c = g; c < nchunk; c += G) P += (double)R.psum[(int64_t)c * E + j];
+    part_P[tid] = P;
+  }
+  __syncthreads();
+  for (int j = tid; j < E; j += kThreads) {
+    double P = 0.0;
+    for (int g = 0; g < G; ++g) P += part_P[g * E + j];
+    stats[(int64_t)k * E + j] = P;
+  }
+  double zl = 0.0;
+  for (int c = tid; c < nchunk; c += kThreads) zl += (double)R.lse2[c];
+  const double zs = block_sum_f64(zl, dsum);
+  if (tid == 0) {
+    stats[(int64_t)k * E + E] = zs;
+    stats[(int64_t)k * E + E + 1] = (double)S;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_ep_scan(int S, int E, int k, const Routing& R, double* stats, cudaStream_t st) {
+  const int nchunk = (S + kChunk - 1) / kChunk;
+  return launch_pdl(ep_scan_kernel, dim3(E + 1), dim3(kThreads), 0, st, S, E, k, nchunk, R, stats);
+}
 
 cudaError_t launch_scan(int S, int E, int k, int C, int64_t Cbuf, const Routing& R, cudaStream_t st) {
   const int nchunk = (S + kChunk - 1) / kChunk;

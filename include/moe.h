@@ -234,6 +234,106 @@ MOE_API moe_status moe_assign_slots_noalloc(int64_t S, int32_t E, int32_t k, int
                                             const int32_t* eidx_dev, int32_t* slot_dev,
                                             int32_t* cnt_dev, void* stream);
 
+/* ---- expert parallelism: one layer over G ranks, one GPU each ------------------ */
+
+/*
+ * The layer with its experts spread over G ranks ("GShard (Expert Parallelism)", "In
+ * plain words": each device hosts some experts; tokens go to them by an all-to-all and
+ * come back by a second one; the "WideEP" claim: 256 experts on 8 GPUs, 32 per GPU,
+ * results returned by a second all-to-all).  Rank g holds a contiguous block of the
+ * batch's tokens (ranks in order) and the experts [g*E/G, (g+1)*E/G) (E % G == 0);
+ * every rank holds the whole gate W_g.
+ *
+ * Capacity and slots keep their one-device meaning over the whole batch:
+ * C = ceil(capacity_factor * k * S_total / E), and slots are rank-major over the
+ * concatenated tokens.  The result -- expert ids, slots, drops, outputs, losses -- is
+ * the single-GPU layer's on the concatenated batch.
+ *
+ * The library computes; the caller moves bytes between ranks (NCCL, or any transport)
+ * at three points of one forward:
+ *   1. moe_ep_route(x) -> stats_dev       [ALL-GATHER the stats of every rank, to host]
+ *   2. moe_ep_dispatch(stats_all) -> sendbuf, send_rows[G], recv_rows[G]
+ *                                         [ALL-TO-ALL: sendbuf -> recvbuf, row counts given]
+ *   3. moe_ep_experts(recvbuf)            [ALL-TO-ALL back: recvbuf -> sendbuf, counts reversed]
+ *   4. moe_ep_combine(sendbuf) -> y;  moe_ep_aux_loss
+ * Rows are M act elements.  Rank g's send buffer holds, for each destination rank in
+ * order, the rows of its kept choices ordered by expert, then choice rank, then token;
+ * the receiver gets each source's rows in that order, source after source, and
+ * moe_ep_experts writes each expert output over the row it came from, so the second
+ * exchange is the first one reversed.
+ */
+typedef struct moe_ep_layer* moe_ep_handle;
+
+/* Doubles per rank in the stats vector: k*E counts (rank-r demand of expert e at
+ * [r*E + e]), E probability sums, the sum of lse^2, the rank's token count. */
+MOE_API int32_t moe_ep_stats_len(int32_t E, int32_t k);
+
+/*
+ * moe_ep_plan -- the exchange plan of rank g (host arithmetic, no device work; the
+ * entry points below use the same).  counts_host [G][k][E]: rank q's rank-r demand of
+ * expert e; S_host [G]: tokens per rank.  Outputs: C_out (capacity of the batch),
+ * send_rows_host [G] rows rank g sends to each rank, recv_rows_host [G] rows it
+ * receives from each, and (optional, may be NULL) base_host [G][k][E] -- the first
+ * global slot of each (rank q, choice rank r, expert e) run -- and kept_host [G][k][E],
+ * the kept rows of each run.  MOE_ERR_INVALID_ARG for negative or inconsistent counts
+ * (each rank's rank-r counts must sum to its token count).
+ */
+MOE_API moe_status moe_ep_plan(int32_t G, int32_t g, int32_t E, int32_t k, double capacity_factor,
+                               const int64_t* counts_host, const int64_t* S_host, int64_t* C_out,
+                               int64_t* send_rows_host, int64_t* recv_rows_host, int64_t* base_host,
+                               int64_t* kept_host);
+
+/*
+ * moe_ep_create -- rank g's handle.  S_max: most tokens this rank routes in a forward;
+ * S_total_max: most tokens of a batch over all ranks (sizes the expert buffers).
+ * Wg_dev [M, E] and gate_bias_dev [E] (or NULL) as in moe_create; W1_local_dev
+ * [E/G, M, H] and W2_local_dev [E/G, H, M]: this rank's experts.  Borrowed, as in
+ * moe_create.  One cudaMalloc here; the forward allocates nothing.
+ */
+MOE_API moe_status moe_ep_create(moe_ep_handle* out, int32_t G, int32_t g, int64_t S_max,
+                                 int64_t S_total_max, int64_t M, int64_t H, int32_t E, int32_t k,
+                                 double capacity_factor, moe_dtype act, const float* Wg_dev,
+                                 const float* gate_bias_dev, const void* W1_local_dev,
+                                 const void* W2_local_dev);
+MOE_API moe_status moe_ep_destroy(moe_ep_handle h);
+
+/* Rows the caller's buffers need: send buffer S_max*k, receive buffer E/G * min(C, S_total_max). */
+MOE_API moe_status moe_ep_buffer_rows(moe_ep_handle h, int64_t* send_rows_max, int64_t* recv_rows_max);
+
+/* Step 1: router and the rank's own scan on S tokens (x_dev [S, M] act); writes the
+ * rank's stats (moe_ep_stats_len doubles, 8-byte aligned device memory) on `stream`. */
+MOE_API moe_status moe_ep_route(moe_ep_handle h, int64_t S, const void* x_dev, double* stats_dev,
+                                void* stream);
+
+/* Step 2: stats_all_host [G][moe_ep_stats_len] (every rank's stats, rank order) ->
+ * plan, send_rows_host / recv_rows_host [G], and the kept rows of x_dev (the same x as
+ * step 1) packed into sendbuf_dev (>= sum(send_rows) rows).  Host arithmetic, then
+ * one table upload and one kernel on `stream`. */
+MOE_API moe_status moe_ep_dispatch(moe_ep_handle h, const double* stats_all_host, const void* x_dev,
+                                   void* sendbuf_dev, int64_t* send_rows_host, int64_t* recv_rows_host,
+                                   void* stream);
+
+/* Step 3: the received rows (recvbuf_dev, sum(recv_rows) rows) into the local experts'
+ * slots, both expert GEMMs, and each expert output written over its received row. */
+MOE_API moe_status moe_ep_experts(moe_ep_handle h, void* recvbuf_dev, void* stream);
+
+/* Step 4: y_dev [S, M] act from the returned rows in sendbuf_dev (fully overwritten;
+ * a token whose choices were all dropped gets 0). */
+MOE_API moe_status moe_ep_combine(moe_ep_handle h, const void* sendbuf_dev, void* y_dev, void* stream);
+
+/* l_aux and z of the whole batch, from the stats given to the last moe_ep_dispatch (host). */
+MOE_API moe_status moe_ep_aux_loss(moe_ep_handle h, float* l_aux_host, float* z_loss_host);
+
+/* This rank's routing of the last forward (device copies; any pointer may be NULL):
+ * eidx / gate [S, k], slot [S, k] global slot or -1, spos [S, k] send-buffer row or -1
+ * (slot and spos need step 2), logits [S, E]. */
+MOE_API moe_status moe_ep_get_routing(moe_ep_handle h, int32_t* eidx_dev, float* gate_dev,
+                                      int32_t* slot_dev, int32_t* spos_dev, float* logits_dev,
+                                      void* stream);
+
+/* Synchronise `stream` and report a pending device error of this handle (as moe_check). */
+MOE_API moe_status moe_ep_check(moe_ep_handle h, void* stream);
+
 /* ---- backward (training) ---------------------------------------------------- */
 
 /*
