@@ -38,6 +38,9 @@ Readings where the pages are silent (each one is listed in the design notes):
    contributes zero; the surviving weights are not renormalised.
  * Top-k selects on the fp32 logits, ties to the lower expert index.
  * The expert FFN is relu(x W1[e]) W2[e] with no biases.
+ * Rerouting (optional, off by default): a dropped assignment is offered once
+   to the token's next-ranked unchosen expert, in the capacity pass's order,
+   into the capacity left over; it keeps its gate weight (see `reroute`).
  * An empty batch (S = 0) has l_aux = z = 0.
  * Backward: the routing (choices, slots, drops) and the first-choice fractions
    f_j carry no gradient; every other step is differentiated exactly.
@@ -56,7 +59,7 @@ import numpy as np
 
 __all__ = [
     "capacity", "gate_logits", "softmax_stats", "top_k", "normalized_gates",
-    "assign_slots", "expert_ffn", "dispatch", "combine", "aux_losses",
+    "assign_slots", "reroute", "expert_ffn", "dispatch", "combine", "aux_losses",
     "route", "forward", "expert_ffn_backward", "gates_backward", "aux_loss_backward",
     "z_loss_backward", "backward", "outputs_for_tokens",
 ]
@@ -168,6 +171,46 @@ def assign_slots(ids, E: int, C: int):
     return slot, cnt
 
 
+def reroute(logits, ids, slot, cnt, C: int):
+    """Second chance for the assignments the capacity pass dropped.
+
+    [blog] "Expert Capacity": tokens over an expert's capacity are either dropped
+    or routed to alternative experts; the page gives no rule for the second
+    option.  Reading taken here: each dropped assignment (t, r) is offered to one
+    alternative expert, the best-ranked expert of token t (largest logit, ties to
+    the lower index) that t did not choose and that no earlier dropped
+    assignment of t was offered -- the token's j-th dropped assignment (in r
+    order) is offered its (k + j)-th ranked expert.  Offers are taken in the
+    capacity pass's order (r, then t); an expert accepts while it has free slots
+    (C minus the rows the capacity pass kept) and gives the next one.  A rerouted
+    assignment keeps its gate weight g_r; one not accepted stays dropped.
+
+    Returns dest[S, k] (the expert that serves each assignment: the chosen one
+    unless rerouted), slot[S, k] (-1 if dropped) and n[E] (kept rows per expert).
+    """
+    l = np.asarray(logits)
+    ids = np.asarray(ids)
+    S, k = ids.shape
+    E = l.shape[1]
+    ranking = top_k(l, E)                       # every expert, best first
+    n = np.minimum(np.asarray(cnt), C).astype(np.int64)
+    dest = ids.astype(np.int32).copy()
+    out = np.array(slot, dtype=np.int32, copy=True)
+    j = np.zeros((S, k), dtype=np.int64)        # earlier dropped assignments of the token
+    for r in range(1, k):
+        j[:, r] = j[:, r - 1] + (np.asarray(slot)[:, r - 1] < 0)
+    for r in range(k):
+        for t in range(S):
+            if slot[t, r] >= 0 or k + j[t, r] >= E:
+                continue
+            a = ranking[t, k + j[t, r]]
+            if n[a] < C:
+                out[t, r] = n[a]
+                dest[t, r] = a
+                n[a] += 1
+    return dest, out, n
+
+
 def expert_ffn(rows, W1e, W2e) -> np.ndarray:
     """One expert's two-layer ReLU feed-forward network: relu(rows W1e) W2e.
 
@@ -225,11 +268,14 @@ def aux_losses(p, ids, lse, E: int):
     return l_aux, z, f, P
 
 
-def route(logits, k: int, cf: float):
+def route(logits, k: int, cf: float, rerouting: bool = False):
     """Routing of given fp32 logits: everything between the gate GEMM and dispatch.
 
-    Returns a namespace with p, lse, ids, gates, C, slot, cnt, n, l_aux, z.
-    float64 logits (finite-difference checks) are routed without rounding.
+    Returns a namespace with p, lse, ids, gates, C, slot, cnt, n, l_aux, z and
+    dest (the expert serving each assignment: ids, unless `rerouting` gives a
+    dropped assignment a second chance, see `reroute`; then slot and n are the
+    final ones and slot0 the capacity pass's).  float64 logits (finite-difference
+    checks) are routed without rounding.
     """
     logits = np.asarray(logits)
     if logits.dtype != np.float64:
@@ -241,26 +287,32 @@ def route(logits, k: int, cf: float):
     g = normalized_gates(p, ids) if S else np.zeros((0, k))
     slot, cnt = assign_slots(ids, E, C)
     l_aux, z, f, P = aux_losses(p, ids, lse, E)
+    slot0, dest, n = slot, ids, np.minimum(cnt, C)
+    if rerouting:
+        dest, slot, n = reroute(logits, ids, slot0, cnt, C)
     return SimpleNamespace(p=p, lse=lse, ids=ids, gates=g, C=C, slot=slot, cnt=cnt,
-                           n=np.minimum(cnt, C), l_aux=l_aux, z=z, f=f, P=P)
+                           n=n, l_aux=l_aux, z=z, f=f, P=P, dest=dest, slot0=slot0)
 
 
-def forward(x, Wg, bias, W1, W2, k: int, cf: float, round_fp32: bool = True, logits=None):
+def forward(x, Wg, bias, W1, W2, k: int, cf: float, round_fp32: bool = True, logits=None,
+            rerouting: bool = False):
     """The whole layer forward on the CPU (small cases).
 
     Returns the `route` namespace plus logits, the per-expert buffers (xbuf,
     pre-activation hpre, ybuf) and the output y[S, M] (float64).  Given
     `logits` (fp32 [S, E], bias included) the routing uses them instead of
     x . W_g + b, so that a check can hold the discrete routing decisions fixed.
+    With `rerouting`, dropped assignments get their second chance (`reroute`)
+    and are dispatched to and combined from the expert that serves them.
     """
     if logits is None:
         logits = gate_logits(x, Wg, bias, round_fp32)
-    rt = route(logits, k, cf)
+    rt = route(logits, k, cf, rerouting)
     S, E = logits.shape
     C = rt.C
     W1 = _f64(W1)
     W2 = _f64(W2)
-    xbuf = dispatch(x, rt.ids, rt.slot, E, C)
+    xbuf = dispatch(x, rt.dest, rt.slot, E, C)
     ybuf = np.zeros_like(xbuf)
     hpre = np.zeros((E, C, W1.shape[2]))
     for e in range(E):
@@ -270,7 +322,7 @@ def forward(x, Wg, bias, W1, W2, k: int, cf: float, round_fp32: bool = True, log
             hpre[e, :n] = xbuf[e, :n] @ W1[e]
     rt.logits = logits
     rt.xbuf, rt.hpre, rt.ybuf = xbuf, hpre, ybuf
-    rt.y = combine(ybuf, rt.ids, rt.gates, rt.slot)
+    rt.y = combine(ybuf, rt.dest, rt.gates, rt.slot)
     return rt
 
 
