@@ -20,6 +20,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_OOM, MOE
 MOE_F32, MOE_BF16 = 0, 1
 MOE_BWD_SKIP_EMPTY_EXPERTS = 1
 MOE_BUF_X, MOE_BUF_H, MOE_BUF_Y = 0, 1, 2
+MOE_ROUTE_REROUTE = 1
 MOE_NUM_STAGES = 6
 STAGES = ("router", "scan", "dispatch", "ffn1", "ffn2", "combine")
 MOE_NUM_BWD_STAGES = 8
@@ -50,6 +51,8 @@ def _load() -> ctypes.CDLL:
         "moe_get_routing": [P, P, P, P, P, P],
         "moe_route_from_logits": [P, I64, P, P],
         "moe_get_expert_rows": [P, I32, I32, I64, P, P],
+        "moe_set_routing_flags": [P, ctypes.c_uint32],
+        "moe_get_serving_experts": [P, P, P],
         "moe_get_capacity": [P, I64, ctypes.POINTER(I64)],
         "moe_set_profiling": [P, I32],
         "moe_get_stage_times": [P, ctypes.POINTER(ctypes.c_float), I32],
@@ -171,6 +174,14 @@ def moe_route_from_logits(h, S, logits, stream=None) -> None:
 
 def moe_get_expert_rows(h, which, e, nrows, dst, stream=None) -> None:
     _check("moe_get_expert_rows", lib.moe_get_expert_rows(h, which, e, nrows, _ptr(dst), _stream(stream)))
+
+
+def moe_set_routing_flags(h, flags: int) -> None:
+    _check("moe_set_routing_flags", lib.moe_set_routing_flags(h, int(flags)))
+
+
+def moe_get_serving_experts(h, dest, stream=None) -> None:
+    _check("moe_get_serving_experts", lib.moe_get_serving_experts(h, _ptr(dest), _stream(stream)))
 
 
 def moe_get_capacity(h, S) -> int:

@@ -87,6 +87,66 @@ __global__ void __launch_bounds__(kThreads, 4) dispatch_kernel(const T* __restri
   }
 }
 
+// Rerouting: the final slot and serving expert of every choice -- the first pass's
+// slot, or for a dropped choice its offer's slot (off2 + lrank2) when that is below C
+// -- then the row copies, as dispatch_kernel.  x == nullptr: tables only.
+template <typename T, int KM>
+__global__ void __launch_bounds__(kThreads, 4) dispatch_rerouted_kernel(const T* __restrict__ x, int S,
+                                                                        int M, int E, int k, int C,
+                                                                        int64_t Cbuf, int nchunk, Routing R,
+                                                                        T* __restrict__ xbuf) {
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * kThreads) >> 5;
+  const int nv = (int)((int64_t)M * sizeof(T) / 16);
+  pdl_trigger();
+  pdl_wait();                                  // first-pass slots, offers and their offsets complete
+  for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < S; t += warps) {
+    int d = 0, s = -1;
+    if (lane < k) {
+      const int64_t i = (int64_t)t * k + lane;
+      d = R.eidx[i];
+      s = R.slot[i];
+      if (s < 0) {
+        const int a = R.alt[i];
+        if (a >= 0 && a < E) {
+          const int q = R.off2[((int64_t)lane * nchunk + t / kChunk) * E + a] + R.lrank2[i];
+          if (q < C && q < Cbuf) {
+            s = q;
+            d = a;
+          }
+        }
+      }
+      R.slot[i] = s;
+      R.dest[i] = d;
+    }
+    if (x == nullptr) continue;
+    uint4* dst[KM];
+    bool any = false;
+#pragma unroll
+    for (int r = 0; r < KM; ++r) {
+      const int dr = __shfl_sync(0xffffffffu, d, r);
+      const int sr = __shfl_sync(0xffffffffu, s, r);
+      dst[r] = (r < k && sr >= 0) ? reinterpret_cast<uint4*>(xbuf + ((int64_t)dr * Cbuf + sr) * M) : nullptr;
+      any |= dst[r] != nullptr;
+    }
+    if (!any) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)t * M);
+    for (int v0 = lane; v0 < nv; v0 += 32 * kUnroll) {
+      uint4 val[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (v0 + 32 * u < nv) val[u] = ld_nc_v4(src + v0 + 32 * u);
+#pragma unroll
+      for (int r = 0; r < KM; ++r) {
+        if (dst[r] == nullptr) continue;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+          if (v0 + 32 * u < nv) dst[r][v0 + 32 * u] = val[u];
+      }
+    }
+  }
+}
+
 template <typename T>
 struct Vec;
 template <>
@@ -339,6 +399,27 @@ cudaError_t launch_dispatch(const void* x, bool bf16, int S, int M, int E, int k
   else
     dispatch_k<float>(k, x, S, M, E, C, Cbuf, nchunk, R, xbuf, grid, st);
   return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_rerouted(const void* x, bool bf16, int S, int M, int E, int k, int C,
+                                     int64_t Cbuf, const Routing& R, void* xbuf, cudaStream_t st) {
+  const int nchunk = (S + kChunk - 1) / kChunk;
+  const int grid = grid_for(S);
+  auto go = [&](auto tag, auto km) {
+    using T = decltype(tag);
+    constexpr int KM = decltype(km)::value;
+    return launch_pdl(dispatch_rerouted_kernel<T, KM>, dim3(grid), dim3(kThreads), 0, st, (const T*)x, S,
+                      M, E, k, C, Cbuf, nchunk, R, (T*)xbuf);
+  };
+  using I1 = std::integral_constant<int, 1>;
+  using I2 = std::integral_constant<int, 2>;
+  using I4 = std::integral_constant<int, 4>;
+  using I8 = std::integral_constant<int, 8>;
+  if (bf16) {
+    const __nv_bfloat16 b{};
+    return k <= 1 ? go(b, I1{}) : k <= 2 ? go(b, I2{}) : k <= 4 ? go(b, I4{}) : go(b, I8{});
+  }
+  return k <= 1 ? go(0.f, I1{}) : k <= 2 ? go(0.f, I2{}) : k <= 4 ? go(0.f, I4{}) : go(0.f, I8{});
 }
 
 cudaError_t launch_ep_dispatch(const void* x, bool bf16, int S, int M, int E, int k, int C,

@@ -58,6 +58,12 @@ struct Routing {
   float* lse2;       // [nchunk]    per-chunk sum of lse^2
   float* losses;     // [2]  l_aux, z
   unsigned* err;     // device error word
+  // rerouting of dropped choices (a second chance at the token's next-ranked expert)
+  int32_t* dest;     // [S, k]   expert serving each choice (eidx unless rerouted)
+  int32_t* alt;      // [S, k]   expert a dropped choice is offered, -1 if none
+  int32_t* lrank2;   // [S, k]   rank of the offer among same-expert rank-r offers in t's chunk
+  int32_t* hist2;    // [k, nchunk, E] rank-r offers to each expert per chunk
+  int32_t* off2;     // [k, nchunk, E] first free slot of each chunk's offers (kept rows + prefix)
 };
 
 // router.cu
@@ -95,6 +101,19 @@ cudaError_t launch_ep_unpack(const void* recvbuf, bool bf16, int nrows, int M, c
                              unsigned* err, int64_t xrows, cudaStream_t st);
 cudaError_t launch_ep_repack(const void* ybuf, bool bf16, int nrows, int M, const int32_t* rowmap,
                              void* recvbuf, cudaStream_t st);
+// reroute.cu: primary slots, and for each dropped choice the alternative it is offered
+// (the token's next-ranked expert it has not chosen or been offered), with the offers'
+// chunk histograms and local ranks.  Needs the router's logits and the scan's offsets.
+// C: the capacity, at most the rows per expert of the buffers.
+cudaError_t launch_reroute_offers(int S, int E, int k, int C, const Routing& R, cudaStream_t st);
+// scan.cu: offsets of the offers per expert, starting after the rows the first pass
+// kept; nexp becomes the final kept rows per expert.
+cudaError_t launch_reroute_scan(int S, int E, int k, int C, int64_t Cbuf, const Routing& R,
+                                cudaStream_t st);
+// dispatch_combine.cu: final slot and serving expert of every choice, then the row
+// copies (x == nullptr: tables only).
+cudaError_t launch_dispatch_rerouted(const void* x, bool bf16, int S, int M, int E, int k, int C,
+                                     int64_t Cbuf, const Routing& R, void* xbuf, cudaStream_t st);
 // dispatch_combine.cu
 cudaError_t launch_dispatch(const void* x, bool bf16, int S, int M, int E, int k, int C,
                             int64_t Cbuf, const Routing& R, void* xbuf, cudaStream_t st);

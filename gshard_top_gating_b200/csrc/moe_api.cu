@@ -56,6 +56,8 @@ struct moe_layer {
   bool have_forward;
   bool fwd_data;         // the expert buffers hold the last forward's (not a route-only call's)
   bool profiling;
+  uint32_t route_flags;  // MOE_ROUTE_* flags of later forwards
+  bool last_rerouted;    // the last routing call gave dropped choices a second chance
   // backward (moe_enable_backward)
   void* bws;             // the backward's one device allocation
   void* dybuf;           // [E, Cbuf, M] act: dY, then dX_e
@@ -137,6 +139,11 @@ size_t carve(moe_layer* h, char* base) {
   R.lse2 = c.take<float>(nchunk);
   R.losses = c.take<float>(2);
   R.err = c.take<unsigned>(1);
+  R.dest = c.take<int32_t>(S * k);
+  R.alt = c.take<int32_t>(S * k);
+  R.lrank2 = c.take<int32_t>(S * k);
+  R.hist2 = c.take<int32_t>(k * nchunk * E);
+  R.off2 = c.take<int32_t>(k * nchunk * E);
   h->xbuf = c.take<char>((size_t)E * h->Cbuf * h->M * as);
   h->hbuf = c.take<char>((size_t)E * h->Cbuf * h->H * as);
   h->ybuf = c.take<char>((size_t)E * h->Cbuf * h->M * as);
@@ -303,7 +310,13 @@ moe_status moe_get_capacity(moe_handle h, int64_t S, int64_t* C_out) {
 
 int32_t moe_kernels_per_forward(moe_handle h, int64_t S) {
   if (!h || S <= 0) return 0;
-  return 6;
+  return (h->route_flags & MOE_ROUTE_REROUTE) ? 8 : 6;
+}
+
+moe_status moe_set_routing_flags(moe_handle h, uint32_t flags) {
+  if (!h || (flags & ~(uint32_t)MOE_ROUTE_REROUTE)) return MOE_ERR_INVALID_ARG;
+  h->route_flags = flags;
+  return MOE_OK;
 }
 
 }  // extern "C"
@@ -347,8 +360,17 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
   }
   MOE_TRY(mark(1));
   MOE_TRY(launch_scan(iS, h->E, h->k, C, h->Cbuf, R, st));
+  const bool reroute = (h->route_flags & MOE_ROUTE_REROUTE) != 0;
+  h->last_rerouted = reroute;
+  if (reroute) {       // second chance for dropped choices: offers, their scan
+    MOE_TRY(launch_reroute_offers(iS, h->E, h->k, (int)(C < h->Cbuf ? C : h->Cbuf), R, st));
+    MOE_TRY(launch_reroute_scan(iS, h->E, h->k, C, h->Cbuf, R, st));
+  }
   MOE_TRY(mark(2));
-  MOE_TRY(launch_dispatch(x, bf16, iS, iM, h->E, h->k, C, h->Cbuf, R, h->xbuf, st));
+  if (reroute)
+    MOE_TRY(launch_dispatch_rerouted(x, bf16, iS, iM, h->E, h->k, C, h->Cbuf, R, h->xbuf, st));
+  else
+    MOE_TRY(launch_dispatch(x, bf16, iS, iM, h->E, h->k, C, h->Cbuf, R, h->xbuf, st));
   MOE_TRY(mark(3));
   if (bf16) {
     // CTA-pair GEMMs (256-row tiles) when the experts run at capacity, so the
@@ -367,7 +389,9 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
                            h->E, h->Cbuf, iH, iM, false, st));
   }
   MOE_TRY(mark(5));
-  MOE_TRY(launch_combine(h->ybuf, bf16, iS, iM, h->k, h->Cbuf, R, y, st));
+  Routing Rc = R;
+  if (reroute) Rc.eidx = R.dest;     // combine from the expert that served each choice
+  MOE_TRY(launch_combine(h->ybuf, bf16, iS, iM, h->k, h->Cbuf, Rc, y, st));
   MOE_TRY(mark(6));
   return MOE_OK;
 }
@@ -493,6 +517,17 @@ moe_status moe_get_routing(moe_handle h, int32_t* eidx, float* gate, int32_t* sl
   return MOE_OK;
 }
 
+moe_status moe_get_serving_experts(moe_handle h, int32_t* dest, void* stream) {
+  if (!h || !dest) return MOE_ERR_INVALID_ARG;
+  h->last_was_host = false;
+  if (!h->have_forward) return MOE_ERR_STATE;
+  const size_t n = (size_t)h->last_S * h->k;
+  if (n)
+    MOE_TRY(cudaMemcpyAsync(dest, h->last_rerouted ? h->R.dest : h->R.eidx, n * 4, cudaMemcpyDeviceToDevice,
+                            static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
 moe_status moe_route_from_logits(moe_handle h, int64_t S, const float* logits, void* stream) {
   if (!h || S < 0 || S > h->S_max) return MOE_ERR_INVALID_ARG;
   h->last_was_host = false;
@@ -509,6 +544,14 @@ moe_status moe_route_from_logits(moe_handle h, int64_t S, const float* logits, v
   const int C = (int)capacity_of(h->cf, h->k, S, h->E);
   MOE_TRY(launch_route_logits(logits, (int)S, h->E, h->k, h->R, st));
   MOE_TRY(launch_scan((int)S, h->E, h->k, C, h->Cbuf, h->R, st));
+  h->last_rerouted = (h->route_flags & MOE_ROUTE_REROUTE) != 0;
+  if (h->last_rerouted) {
+    MOE_TRY(launch_reroute_offers((int)S, h->E, h->k, (int)(C < h->Cbuf ? C : h->Cbuf), h->R, st));
+    MOE_TRY(launch_reroute_scan((int)S, h->E, h->k, C, h->Cbuf, h->R, st));
+    MOE_TRY(launch_dispatch_rerouted(nullptr, h->act == MOE_BF16, (int)S, (int)h->M, h->E, h->k, C,
+                                     h->Cbuf, h->R, h->xbuf, st));
+    return MOE_OK;
+  }
   // slot pass of the dispatch kernel without moving any row
   MOE_TRY(launch_dispatch(nullptr, h->act == MOE_BF16, (int)S, (int)h->M, h->E, h->k, C, h->Cbuf,
                           h->R, h->xbuf, st));
@@ -621,6 +664,7 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
   if (!h || S < 0 || S > h->S_max) return MOE_ERR_INVALID_ARG;
   h->last_was_host = false;
   if (!h->bws || !h->have_forward || !h->fwd_data || S != h->last_S) return MOE_ERR_STATE;
+  if (h->last_rerouted) return MOE_ERR_UNSUPPORTED;   // the backward of rerouted choices is not built
   if (!dWg || !dW1 || !dW2 || !aligned(dWg, 16) || !aligned(dW1, 16) || !aligned(dW2, 16) ||
       (dbias && !aligned(dbias, 4)))
     return MOE_ERR_INVALID_ARG;

@@ -179,7 +179,38 @@ __global__ void __launch_bounds__(kThreads) ep_scan_kernel(int S, int E, int k, 
   }
 }
 
+// Rerouting: one block per expert.  The offers to e form a rank-major sequence over
+// (r, chunk) like the choices; their slots start after the rows the first pass kept
+// (nexp), and an offer is accepted while its slot is below C.
+__global__ void __launch_bounds__(kThreads) reroute_scan_kernel(int S, int E, int k, int C, int Cbuf,
+                                                                int nchunk, Routing R) {
+  __shared__ int warp_sums[kThreads / 32];
+  const int tid = threadIdx.x, e = blockIdx.x;
+  pdl_trigger();
+  pdl_wait();                                  // offers and first-pass counts complete
+  const int kept = R.nexp[e];
+  const int L = k * nchunk;
+  const int seg = (L + kThreads - 1) / kThreads;
+  const int a = min(L, tid * seg), b = min(L, a + seg);
+  int local = 0;
+  for (int q = a; q < b; ++q) local += R.hist2[(int64_t)q * E + e];
+  int total;
+  int run = kept + block_exclusive_scan(local, warp_sums, total);
+  for (int q = a; q < b; ++q) {
+    R.off2[(int64_t)q * E + e] = run;
+    run += R.hist2[(int64_t)q * E + e];
+  }
+  if (tid == 0) R.nexp[e] = min(kept + total, min(C, Cbuf));
+}
+
 }  // namespace
+
+cudaError_t launch_reroute_scan(int S, int E, int k, int C, int64_t Cbuf, const Routing& R,
+                                cudaStream_t st) {
+  const int nchunk = (S + kChunk - 1) / kChunk;
+  const int cb = Cbuf < 0x7fffffff ? (int)Cbuf : 0x7fffffff;
+  return launch_pdl(reroute_scan_kernel, dim3(E), dim3(kThreads), 0, st, S, E, k, C, cb, nchunk, R);
+}
 
 cudaError_t launch_ep_scan(int S, int E, int k, const Routing& R, double* stats, cudaStream_t st) {
   const int nchunk = (S + kChunk - 1) / kChunk;

@@ -111,6 +111,15 @@ class MoeLayer:
         L.moe_get_expert_rows(self.h, which, e, nrows, out, stream)
         return out
 
+    def set_rerouting(self, on: bool) -> None:
+        """Give dropped choices a second chance at an alternative expert (MOE_ROUTE_REROUTE)."""
+        L.moe_set_routing_flags(self.h, L.MOE_ROUTE_REROUTE if on else 0)
+
+    def serving_experts(self, S: int, stream=None) -> torch.Tensor:
+        dest = torch.empty(S, self.k, dtype=torch.int32, device="cuda")
+        L.moe_get_serving_experts(self.h, dest, stream)
+        return dest
+
     def route_from_logits(self, logits: torch.Tensor, stream=None) -> None:
         L.moe_route_from_logits(self.h, logits.shape[0], logits, stream)
 

@@ -190,6 +190,35 @@ MOE_API moe_status moe_get_capacity(moe_handle h, int64_t S, int64_t* C_out);
 MOE_API moe_status moe_set_profiling(moe_handle h, int32_t enable);
 MOE_API moe_status moe_get_stage_times(moe_handle h, float* ms_host, int32_t n);
 
+/* Flags of moe_set_routing_flags. */
+enum { MOE_ROUTE_REROUTE = 1 };
+
+/*
+ * moe_set_routing_flags -- options of the following forward and route calls (default 0:
+ * a choice over capacity is dropped).
+ * MOE_ROUTE_REROUTE: a dropped choice gets one second chance at an alternative expert
+ * ("GShard: Scaling Giant Neural Networks with Conditional Computation", "Expert
+ * Capacity": overflow tokens are dropped or routed to alternative experts; the rule is
+ * this library's reading).  After the rank-major capacity pass, the token's j-th
+ * dropped choice (in choice-rank order) is offered its (k+j)-th ranked expert (largest
+ * logit among those it neither chose nor was offered, ties to the lower index).  Offers
+ * are taken in the capacity pass's order -- choice rank, then token -- into the room
+ * the pass left (C minus its kept rows), each accepted offer taking the next free slot;
+ * an offer that finds no room stays dropped.  A rerouted choice keeps its gate weight.
+ * moe_get_routing then reports the final slot (at the serving expert) and
+ * moe_get_serving_experts the serving expert.  A forward with this flag launches 8
+ * kernels.  moe_backward of a rerouted forward returns MOE_ERR_UNSUPPORTED.
+ * Returns MOE_ERR_INVALID_ARG for unknown bits.
+ */
+MOE_API moe_status moe_set_routing_flags(moe_handle h, uint32_t flags);
+
+/*
+ * moe_get_serving_experts -- dest_dev [S, k] int32: the expert that serves each choice
+ * of the last forward / route call (the chosen expert unless the choice was rerouted;
+ * for a dropped choice, the chosen one).  Device copy on `stream`.
+ */
+MOE_API moe_status moe_get_serving_experts(moe_handle h, int32_t* dest_dev, void* stream);
+
 /* Number of kernels one moe_forward of S tokens launches. */
 MOE_API int32_t moe_kernels_per_forward(moe_handle h, int64_t S);
 
