@@ -65,7 +65,7 @@ struct moe_ep_layer {
   std::vector<int32_t> plan_host;
   GemmPlan plan1, plan2;
   void* wsplit;
-  CUtensorMap wmap, xmap;
+  CUtensorMap wmap, xmap, xmap64;
   const void* xmap_ptr;
   int64_t xmap_S;
   uint64_t wait_limit_ns;
@@ -320,12 +320,15 @@ moe_status moe_ep_route(moe_ep_handle h, int64_t S, const void* x, double* stats
   }
   const int iS = (int)S, iM = (int)h->M;
   if (h->act == MOE_BF16) {
+    const bool persistent = router_persistent(h->E, iS);
     if (h->xmap_ptr != x || h->xmap_S != S) {
       if (!make_router_xmap(&h->xmap, x, iS, iM, h->E)) return MOE_ERR_CUDA;
+      if (persistent && !make_router_xmap64(&h->xmap64, x, iS, iM)) return MOE_ERR_CUDA;
       h->xmap_ptr = x;
       h->xmap_S = S;
     }
-    EP_TRY(launch_router_tc(h->xmap, h->wmap, h->bias, iS, iM, h->E, h->k, h->R, h->wait_limit_ns, st));
+    EP_TRY(launch_router_tc(h->xmap, persistent ? &h->xmap64 : nullptr, h->wmap, h->bias, iS, iM, h->E,
+                            h->k, h->R, h->wait_limit_ns, st));
   } else {
     EP_TRY(launch_router(x, false, h->Wg, h->bias, iS, iM, h->E, h->k, h->R, st));
   }

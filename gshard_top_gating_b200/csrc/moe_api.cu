@@ -49,7 +49,7 @@ struct moe_layer {
   bool last_was_host;    // the handle's last device work was a moe_forward_host
   GemmPlan plan1, plan2;
   void* wsplit;          // bf16 tokens: W_g split into three bf16 parts [3][EP][M]
-  CUtensorMap wmap, xmap;
+  CUtensorMap wmap, xmap, xmap64;
   const void* xmap_ptr;  // x pointer / S the cached xmap describes
   int64_t xmap_S;
   int64_t last_S;
@@ -349,12 +349,15 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
 
   MOE_TRY(mark(0));
   if (bf16) {
+    const bool persistent = router_persistent(h->E, iS);
     if (h->xmap_ptr != x || h->xmap_S != S) {
       if (!make_router_xmap(&h->xmap, x, iS, iM, h->E)) return MOE_ERR_CUDA;
+      if (persistent && !make_router_xmap64(&h->xmap64, x, iS, iM)) return MOE_ERR_CUDA;
       h->xmap_ptr = x;
       h->xmap_S = S;
     }
-    MOE_TRY(launch_router_tc(h->xmap, h->wmap, h->bias, iS, iM, h->E, h->k, R, h->wait_limit_ns, st));
+    MOE_TRY(launch_router_tc(h->xmap, persistent ? &h->xmap64 : nullptr, h->wmap, h->bias, iS, iM, h->E,
+                             h->k, R, h->wait_limit_ns, st));
   } else {
     MOE_TRY(launch_router(x, bf16, h->Wg, h->bias, iS, iM, h->E, h->k, R, st));
   }

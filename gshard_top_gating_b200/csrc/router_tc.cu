@@ -518,6 +518,419 @@ __global__ void __launch_bounds__(NW * 32, (NW == 8) ? 2 : 1)
   }
 }
 
+// ---------------------------------------------------------------------------------
+// Persistent router (E <= 64, batches that give every SM at least four 64-token chunks).
+//
+// One CTA per SM owns a contiguous range of 64-token chunks (ranges differ by at most
+// one chunk) and walks it in tiles of two chunks (the last tile may be one chunk,
+// loaded as a 64-row box).  Unlike router_tc_kernel, a tile's routing overlaps the
+// next tiles' loads and MMAs:
+//   warp 0       TMA producer over every tile's k-blocks (x tile + three W_g parts)
+//   warp 1       MMA issuer; K-segments alternate between two TMEM accumulators
+//   warps 2..5   fold: each K-segment (lo + mid, + hi) is added into the tile's running
+//                sum, one of two TMEM regions (tiles alternate), and the segment's
+//                accumulator is released at once
+//   warps 6..15  routing group: copies a finished tile's logits from TMEM to shared
+//                memory (plus bias), releases the running-sum region, then routes the
+//                tile exactly as router_tc_kernel does for E <= 64 (a thread per
+//                token), writes the logits and the chunk tables
+// The arithmetic of every logit, probability, gate and table entry is that of
+// router_tc_kernel.  TMEM: two segment accumulators (3*EP columns each) and two
+// running sums (EP each) -- 448 of 512 columns for EP = 64.
+template <int EP>
+struct PCfg {
+  static constexpr int NT = 512;
+  static constexpr int TT = 128;
+  static constexpr uint32_t PART_BYTES = EP * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + 3 * PART_BYTES;
+  static constexpr uint32_t ACC = 3 * EP;                 // one K-segment accumulator
+  static constexpr uint32_t RUN0 = 2 * ACC;               // running sum of tile parity b at RUN0 + b*EP
+  static constexpr uint32_t TMEM_COLS = (2 * ACC + 2 * EP) <= 256 ? 256 : 512;
+  static constexpr uint32_t LD = EP + 1;
+  static constexpr uint32_t L_OFF = 0;                    // logits, then probabilities [TT][EP+1] f32
+  static constexpr uint32_t SEL_OFF = L_OFF + TT * LD * 4;    // chosen experts [TT][8]
+  static constexpr uint32_t H_OFF = SEL_OFF + TT * kMaxK * 4; // running counts [2][8][EP]
+  static constexpr uint32_t LSE_OFF = H_OFF + 2 * kMaxK * EP * 4;   // lse^2 per token [TT]
+  static constexpr uint32_t EPI_BYTES = ((LSE_OFF + TT * 4) + 1023u) & ~1023u;
+  static constexpr uint32_t BAR_BYTES = 256;
+  static constexpr int STAGES_FIT = (int)((227u * 1024u - 1024u - EPI_BYTES - BAR_BYTES) / STAGE_BYTES);
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
+  static_assert(EP <= 64, "the persistent router routes a thread per token (E <= 64)");
+  static_assert(STAGES >= 3, "at least three stages in flight");
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  static_assert(2 * ACC + 2 * EP <= TMEM_COLS, "TMEM columns");
+  static_assert(8u * (2 * STAGES + 9) + 12 <= BAR_BYTES, "barriers, TMEM slot and flags");
+};
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+template <int EP>
+__global__ void __launch_bounds__(512, 1)
+    router_tcp_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmX64,
+                      const __grid_constant__ CUtensorMap tmW, const float* __restrict__ bias, int S, int M,
+                      int E, int k, int nchunk, Routing R, uint64_t limit_ns) {
+  using C = PCfg<EP>;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;
+  unsigned char* gbase = smem_raw + (base - raw_base);
+  unsigned char* gepi = gbase + C::STAGES * C::STAGE_BYTES;
+  float* Ls = reinterpret_cast<float*>(gepi + C::L_OFF);
+  int32_t* sel = reinterpret_cast<int32_t*>(gepi + C::SEL_OFF);
+  int32_t* Hs = reinterpret_cast<int32_t*>(gepi + C::H_OFF);
+  float* lse_t = reinterpret_cast<float*>(gepi + C::LSE_OFF);
+  const uint32_t bar0 = base + C::STAGES * C::STAGE_BYTES + C::EPI_BYTES;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + b); };      // a K-segment is done
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 + b); };  // the fold took it
+  auto lfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 4 + b); };   // a tile's logits are done
+  auto rfree_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 6 + b); };   // its running sum is free
+  const uint32_t done_bar = bar0 + 8u * (2 * C::STAGES + 8);
+  unsigned char* gbar = gepi + C::EPI_BYTES;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbar + 8u * (2 * C::STAGES + 9));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbar + 8u * (2 * C::STAGES + 9) + 4);
+  volatile int* go_flag = reinterpret_cast<volatile int*>(gbar + 8u * (2 * C::STAGES + 9) + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nblk = gridDim.x, blk = blockIdx.x;
+  const int c0 = (int)((int64_t)nchunk * blk / nblk), c1 = (int)((int64_t)nchunk * (blk + 1) / nblk);
+  const int ntiles = (c1 - c0 + 1) / 2;
+  const int KB = M / BK;
+  const int nseg = (KB + kSegBlocks - 1) / kSegBlocks;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 128);             // the four fold warps
+      mbar_init(lfull_bar(b), 128);
+      mbar_init(rfree_bar(b), 1);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmX64);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();          // after the TMEM allocation (see router_tc_kernel)
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, issued = 0, issued_par = 0;
+      bool ok = true;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int ca = c0 + 2 * i;
+        const bool half = ca + 1 >= c1;
+        const int tok0 = ca * kChunk;
+        const uint32_t tx = (half ? 64u : 128u) * BK * 2 + 3 * C::PART_BYTES;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (*abort_flag || !mbar_wait(empty_bar(s), ph ^ 1u, R.err, limit_ns)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const uint32_t sa = base + s * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(full_bar(s), tx);
+          tma_load_2d(sa, half ? (const void*)&tmX64 : (const void*)&tmX, full_bar(s), kb * BK, tok0);
+#pragma unroll
+          for (int part = 0; part < 3; ++part)
+            tma_load_2d(sa + A_BYTES + part * C::PART_BYTES, &tmW, full_bar(s), kb * BK, part * EP);
+          issued |= 1u << s;
+          issued_par = (issued_par & ~(1u << s)) | (ph << s);
+          if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok)
+        for (int q = 0; q < C::STAGES; ++q)
+          if ((issued >> q) & 1u) mbar_wait(full_bar(q), (issued_par >> q) & 1u, R.err, limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, g = 0;
+      bool ok = true;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        for (int kb = 0; kb < KB; ++kb) {
+          const bool seg_first = (kb % kSegBlocks) == 0;
+          const bool seg_last = (kb % kSegBlocks) == kSegBlocks - 1 || kb == KB - 1;
+          const uint32_t buf = g & 1u;
+          if (seg_first) {   // the fold must have taken this accumulator's previous segment
+            if (*abort_flag || !mbar_wait(tempty_bar(buf), ((g >> 1) & 1u) ^ 1u, R.err, limit_ns)) {
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          if (*abort_flag || !mbar_wait(full_bar(s), ph, R.err, limit_ns)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base + s * C::STAGE_BYTES, sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_f16(tmem_base + buf * C::ACC, desc_kmajor_sw128(sa + kk * 32u),
+                       desc_kmajor_sw128(sb + kk * 32u), idesc_router<3 * EP>(), !(seg_first && kk == 0));
+          tc_commit(empty_bar(s));
+          if (seg_last) {
+            tc_commit(tfull_bar(buf));
+            ++g;
+          }
+          if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        tc_commit(done_bar);
+        mbar_wait(done_bar, 0, R.err, limit_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ fold (warps 2..5)
+    const int q = warp & 3;                           // TMEM lanes 32q .. 32q + 31 (= tile rows)
+    const uint32_t tlane = tmem_base + ((uint32_t)(q * 32) << 16);
+    uint32_t g = 0;
+    bool ok = true;
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const int ca = c0 + 2 * i;
+      const int ntok = min((ca + 1 >= c1 ? 1 : 2) * kChunk, S - ca * kChunk);
+      const bool active = q * 32 < ntok;              // warp-uniform: rows past the tile are not read
+      const uint32_t run = tlane + C::RUN0 + (uint32_t)(i & 1) * EP;
+      for (int seg = 0; seg < nseg; ++seg) {
+        const uint32_t buf = g & 1u;
+        bool w = !*abort_flag && mbar_wait(tfull_bar(buf), (g >> 1) & 1u, R.err, limit_ns);
+        if (seg == 0) w = w && mbar_wait(rfree_bar(i & 1), ((i >> 1) & 1) ^ 1, R.err, limit_ns);
+        if (!__all_sync(0xffffffffu, w)) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (active) {
+          const uint32_t acc = tlane + buf * C::ACC;
+#pragma unroll 1
+          for (int c = 0; c < EP / 32; ++c) {
+            uint32_t a[32], b[32];
+            tmem_ld_32x32b_x32(acc + 2 * EP + c * 32, a);       // this segment's x.lo + x.mid, then + x.hi
+            tmem_ld_32x32b_x32(acc + EP + c * 32, b);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(__uint_as_float(a[j]) + __uint_as_float(b[j]));
+            tmem_ld_32x32b_x32(acc + c * 32, b);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(__uint_as_float(a[j]) + __uint_as_float(b[j]));
+            if (seg > 0) {
+              tmem_ld_32x32b_x32(run + c * 32, b);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(__uint_as_float(a[j]) + __uint_as_float(b[j]));
+            }
+            tmem_st_32x32b_x32(run + c * 32, a);
+          }
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        mbar_arrive(tempty_bar(buf));
+        ++g;
+      }
+      if (ok) mbar_arrive(lfull_bar(i & 1));          // the tile's logits (without bias) are in `run`
+    }
+  } else {
+    // ------------------------------------------------------------ routing group (warps 6..15)
+    constexpr int NR = C::NT - 192;                   // 320 threads
+    const int tr = threadIdx.x - 192, wr = tr >> 5;
+    for (int i = 0; i < ntiles; ++i) {
+      const int ca = c0 + 2 * i;
+      const int nch = ca + 1 >= c1 ? 1 : 2;
+      const int tok0 = ca * kChunk;
+      const int ntok = min(nch * kChunk, S - tok0);
+      if (tr == 0)
+        *go_flag = !*abort_flag && mbar_wait(lfull_bar(i & 1), (i >> 1) & 1, R.err, limit_ns);
+      named_bar_sync(1, NR);
+      if (!*go_flag) {
+        if (tr == 0) *abort_flag = 1;
+        break;                                        // uniform: every thread read the same flag
+      }
+      tc_fence_after();
+      if (wr < 4) {                                   // warps 6..9 cover the four TMEM lane groups
+        const int qq = warp & 3, row = qq * 32 + lane;
+        const uint32_t run = tmem_base + ((uint32_t)(qq * 32) << 16) + C::RUN0 + (uint32_t)(i & 1) * EP;
+#pragma unroll 1
+        for (int c = 0; c < EP / 32; ++c) {
+          uint32_t a[32];
+          tmem_ld_32x32b_x32(run + c * 32, a);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int col = c * 32 + j;
+            Ls[row * C::LD + col] = __uint_as_float(a[j]) + ((bias && col < E) ? __ldg(bias + col) : 0.f);
+          }
+        }
+      } else {
+        for (int idx = tr - 128; idx < 2 * kMaxK * EP; idx += NR - 128) Hs[idx] = 0;
+      }
+      tc_fence_before();
+      named_bar_sync(1, NR);
+      if (tr == 0) mbar_arrive(rfree_bar(i & 1));
+      // one thread per token: softmax, lse, top-k (ties to the lower index), gates; the
+      // other warps copy the logits out
+      float mx = 0.f, inv = 0.f;
+      if (tr < C::TT) {
+        const int t = tr;
+        if (t < ntok) {
+          const float* Lr = Ls + t * C::LD;
+          mx = -INFINITY;
+#pragma unroll 8
+          for (int j = 0; j < E; ++j) mx = fmaxf(mx, Lr[j]);
+          float sum = 0.f;
+#pragma unroll 8
+          for (int j = 0; j < E; ++j) sum += expf(Lr[j] - mx);
+          inv = 1.f / sum;
+          const float lse = mx + logf(sum);
+          lse_t[t] = lse * lse;
+          uint64_t taken = 0;
+          int er[kMaxK];
+          float lr[kMaxK];
+#pragma unroll
+          for (int r = 0; r < kMaxK; ++r) {
+            er[r] = 0;
+            lr[r] = 0.f;
+            if (r < k) {
+              float bv = -INFINITY;
+              int bj = -1;
+#pragma unroll 8
+              for (int j = 0; j < E; ++j) {
+                const float v = Lr[j];
+                if (!((taken >> j) & 1ull) && (v > bv || bj < 0)) {
+                  bv = v;
+                  bj = j;
+                }
+              }
+              if (bj < 0) {
+                atomicOr(R.err, DEVERR_BOUNDS);
+                bj = 0;
+              }
+              taken |= 1ull << bj;
+              er[r] = bj;
+              lr[r] = bv;
+            }
+          }
+          float gs = 0.f, gr[kMaxK];
+#pragma unroll
+          for (int r = 0; r < kMaxK; ++r) {
+            gr[r] = (r < k) ? expf(lr[r] - lr[0]) : 0.f;
+            gs += gr[r];
+          }
+          const float ginv = 1.f / gs;
+          const int64_t tok = tok0 + t;
+#pragma unroll
+          for (int r = 0; r < kMaxK; ++r) {
+            if (r < k) {
+              R.eidx[tok * k + r] = er[r];
+              R.gate[tok * k + r] = gr[r] * ginv;
+              sel[t * kMaxK + r] = er[r];
+            }
+          }
+        }
+      } else {
+        for (int idx = tr - C::TT; idx < ntok * E; idx += NR - C::TT) {
+          const int t = idx / E, j = idx - t * E;
+          R.logits[(int64_t)tok0 * E + idx] = Ls[t * C::LD + j];
+        }
+      }
+      named_bar_sync(1, NR);
+      // probabilities in place of the logits (the same exp and scale as the sum above)
+      if (tr < C::TT && tr < ntok) {
+        float* Lr = Ls + tr * C::LD;
+#pragma unroll 8
+        for (int j = 0; j < E; ++j) Lr[j] = expf(Lr[j] - mx) * inv;
+      }
+      named_bar_sync(1, NR);
+      // per-chunk probability sums (tokens in order, four interleaved partial sums) and
+      // lse^2 sums (one warp per chunk, fixed shuffle tree)
+      for (int idx = tr; idx < nch * E; idx += NR) {
+        const int cc = idx / E, j = idx - cc * E;
+        const int t0 = cc * kChunk, t1 = min(t0 + kChunk, ntok);
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        int t = t0;
+        for (; t + 4 <= t1; t += 4) {
+          a0 += Ls[t * C::LD + j];
+          a1 += Ls[(t + 1) * C::LD + j];
+          a2 += Ls[(t + 2) * C::LD + j];
+          a3 += Ls[(t + 3) * C::LD + j];
+        }
+        for (; t < t1; ++t) a0 += Ls[t * C::LD + j];
+        R.psum[(int64_t)(ca + cc) * E + j] = (a0 + a1) + (a2 + a3);
+      }
+      if (wr < nch) {
+        const int t = wr * kChunk + lane;
+        float a = (t < ntok ? lse_t[t] : 0.f) + (t + 32 < ntok ? lse_t[t + 32] : 0.f);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) R.lse2[ca + wr] = a;
+      }
+      // local ranks within each chunk and rank-r histograms (one warp per (chunk, rank))
+      for (int pi = wr; pi < nch * k; pi += NR / 32) {
+        const int cc = pi / k, r = pi - cc * k;
+        int32_t* cnt = Hs + (cc * kMaxK + r) * EP;
+        for (int h = 0; h < kChunk / 32; ++h) {
+          const int t = cc * kChunk + h * 32 + lane;
+          const bool valid = t < ntok;
+          const int e = valid ? sel[t * kMaxK + r] : EP + lane;
+          const unsigned m = __match_any_sync(0xffffffffu, e);
+          if (valid) R.lrank[(int64_t)(tok0 + t) * k + r] = cnt[e] + __popc(m & ((1u << lane) - 1u));
+          __syncwarp();
+          if (valid && lane == __ffs(m) - 1) cnt[e] += __popc(m);
+          __syncwarp();
+        }
+      }
+      named_bar_sync(1, NR);
+      for (int cc = 0; cc < nch; ++cc)
+        for (int idx = tr; idx < k * E; idx += NR) {
+          const int r = idx / E, e = idx - r * E;
+          R.hist[((int64_t)r * nchunk + ca + cc) * E + e] = Hs[(cc * kMaxK + r) * EP + e];
+        }
+      named_bar_sync(1, NR);                          // the tile's smem is reused by the next
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
 // W_g [M, E] fp32 -> three bf16 parts, each [EP, M] (K contiguous), rows >= E zero.
 __global__ void split_gate_kernel(const float* __restrict__ Wg, int M, int E, int EP,
                                   __nv_bfloat16* __restrict__ out) {
@@ -588,6 +1001,19 @@ int sm_count() {
 }
 
 template <int EP>
+cudaError_t launch_persistent(const CUtensorMap& tmX, const CUtensorMap& tmX64, const CUtensorMap& tmW,
+                              const float* bias, int S, int M, int E, int k, const Routing& R,
+                              uint64_t limit_ns, int grid, cudaStream_t st) {
+  using C = PCfg<EP>;
+  auto kern = router_tcp_kernel<EP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int nchunk = (S + kChunk - 1) / kChunk;
+  kern<<<grid, C::NT, C::SMEM, st>>>(tmX, tmX64, tmW, bias, S, M, E, k, nchunk, R, limit_ns);
+  return cudaGetLastError();
+}
+
+template <int EP>
 cudaError_t launch_t(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias, int S, int M,
                      int E, int k, const Routing& R, uint64_t limit_ns, cudaStream_t st) {
   if (router_tokens_per_cta(E, S) == 128)
@@ -623,8 +1049,22 @@ bool make_router_xmap(CUtensorMap* tm, const void* x, int S, int M, int E) {
   return encode_kmajor(tm, x, (uint64_t)M, (uint64_t)S, (uint32_t)router_tokens_per_cta(E, S));
 }
 
-cudaError_t launch_router_tc(const CUtensorMap& tmX, const CUtensorMap& tmW, const float* bias, int S,
-                             int M, int E, int k, const Routing& R, uint64_t limit_ns, cudaStream_t st) {
+bool make_router_xmap64(CUtensorMap* tm, const void* x, int S, int M) {
+  return encode_kmajor(tm, x, (uint64_t)M, (uint64_t)S, 64u);
+}
+
+bool router_persistent(int E, int S) {
+  return router_tc_pad(E) <= 64 && (S + kChunk - 1) / kChunk >= 4 * sm_count();
+}
+
+cudaError_t launch_router_tc(const CUtensorMap& tmX, const CUtensorMap* tmX64, const CUtensorMap& tmW,
+                             const float* bias, int S, int M, int E, int k, const Routing& R,
+                             uint64_t limit_ns, cudaStream_t st) {
+  if (tmX64 && router_persistent(E, S)) {
+    if (router_tc_pad(E) == 32)
+      return launch_persistent<32>(tmX, *tmX64, tmW, bias, S, M, E, k, R, limit_ns, sm_count(), st);
+    return launch_persistent<64>(tmX, *tmX64, tmW, bias, S, M, E, k, R, limit_ns, sm_count(), st);
+  }
   switch (router_tc_pad(E)) {
     case 32: return launch_t<32>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);
     case 64: return launch_t<64>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);
