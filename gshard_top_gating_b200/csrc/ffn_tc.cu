@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
                   int64_t Cbuf, int K, int N, const uint16_t* __restrict__ mask, int64_t row_limit,
-                  uint32_t* __restrict__ bits, unsigned* err, uint64_t limit_ns) {
+                  uint32_t* __restrict__ bits, unsigned* err, uint64_t limit_ns, int rest_only) {
   using C = Cfg<BN>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   int* tile_pre = reinterpret_cast<int*>(misc + 16);                 // [E+1]
   int* mtiles = tile_pre + (kMaxExperts + 1);                        // [E]
-  int* nrows = mtiles + kMaxExperts;                                 // [E]
+  int* rbase = mtiles + kMaxExperts;                                 // [E] first row of the tiles
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NT = N / BN;
@@ -288,8 +288,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int sum = 0;
     for (int e = e0; e < min(E, e0 + per); ++e) {
       const int n = nexp[e];
-      const int m = (n + BM - 1) / BM;
-      nrows[e] = n;
+      // rest_only: the rows after those the CTA-pair kernel takes (256-row tiles up to
+      // 256 * ((n + 127) / 256)), at most 128 of them: one tile or none
+      const int r0 = rest_only ? (n + 127) / 256 * 256 : 0;
+      const int m = (n - r0 + BM - 1) / BM;
+      rbase[e] = r0;
       mtiles[e] = m;
       sum += m * NT;
     }
@@ -320,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       int e, mt, nt;
       for (int tile = blockIdx.x; ok && it.decode(tile, e, mt, nt); tile += gridDim.x) {
-        const int rowA = (int)(e * Cbuf + mt * BM);
+        const int rowA = (int)(e * Cbuf + rbase[e] + mt * BM);
         const int rowB = e * K;
         for (int kb = 0; kb < KB; ++kb) {
           if (*abort_flag || !mbar_wait(empty_bar(s), ph ^ 1u, err, limit_ns)) {
@@ -411,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; it.decode(tile, e, mt, nt); tile += gridDim.x, ++i) {
       const int acc = i & 1;
       const uint32_t aph = (i >> 1) & 1;
-      const int row0 = (int)(e * Cbuf + mt * BM + q * 32);
+      const int row0 = (int)(e * Cbuf + rbase[e] + mt * BM + q * 32);
       const uint16_t* mrow = EPI == kEpiMask ? mask + (int64_t)(row0 + lane) * N + nt * BN : nullptr;
       if (EPI == kEpiMask) {           // bring this row's mask into L2 while the MMAs run
 #pragma unroll
@@ -682,7 +685,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ffn_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
                    int64_t Cbuf, int K, int N, const uint16_t* __restrict__ mask,
-                   uint32_t* __restrict__ bits, unsigned* err, uint64_t limit_ns) {
+                   uint32_t* __restrict__ bits, unsigned* err, uint64_t limit_ns, int leave_rest) {
   using namespace pairk;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -736,7 +739,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int sum = 0;
     for (int e = e0; e < min(E, e0 + per); ++e) {
       const int n = nexp[e];
-      const int m = (n + PM - 1) / PM;
+      // leave_rest: a last block of at most 128 rows is left to the one-CTA kernel
+      const int m = leave_rest ? (n + 127) / PM : (n + PM - 1) / PM;
       nrows[e] = n;
       mtiles[e] = m;
       sum += m * NT;
@@ -1115,19 +1119,19 @@ bool encode_2d(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer,
 
 template <int EPI, bool BKM>
 cudaError_t launch_pair(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint64_t limit_ns,
-                        int num_sms, cudaStream_t st) {
+                        int num_sms, cudaStream_t st, int leave_rest = 0) {
   auto kern = ffn_tc2_kernel<EPI, BKM>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)pairk::SMEM);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(num_sms & ~1), dim3(kThreads), pairk::SMEM, st, p.tmA,
                     BKM ? p.tmB2 : p.tmB, p.tmD, nexp, p.E, p.Cbuf, p.K, p.N,
-                    static_cast<const uint16_t*>(p.mask), p.bits, err, limit_ns);
+                    static_cast<const uint16_t*>(p.mask), p.bits, err, limit_ns, leave_rest);
 }
 
 template <int BN, int EPI, bool BKM>
 cudaError_t launch_t(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint64_t limit_ns,
-                     int num_sms, cudaStream_t st) {
+                     int num_sms, cudaStream_t st, int rest_only = 0) {
   auto kern = ffn_tc_kernel<BN, EPI, BKM>;
   const size_t smem = Cfg<BN>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1135,7 +1139,7 @@ cudaError_t launch_t(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint
   const int64_t row_limit = p.row_limit > 0 ? p.row_limit : (int64_t)p.E * p.Cbuf;
   return launch_pdl(kern, dim3(num_sms), dim3(kThreads), smem, st, p.tmA, p.tmB, p.tmD, nexp, p.E,
                     p.Cbuf, p.K, p.N, static_cast<const uint16_t*>(p.mask), row_limit, p.bits, err,
-                    limit_ns);
+                    limit_ns, rest_only);
 }
 
 template <int BN, int EPI>
@@ -1243,8 +1247,21 @@ bool make_gate_dx_plan(GemmPlan& p, const void* dlb, int64_t S, int EPb, const v
   return true;
 }
 
+template <int EPI>
+cudaError_t launch_mixed(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint64_t limit_ns,
+                         int num_sms, cudaStream_t st) {
+  cudaError_t e = launch_pair<EPI, false>(p, nexp, err, limit_ns, num_sms, st, 1);
+  if (e != cudaSuccess) return e;
+  switch (p.BN) {
+    case 256: return launch_t<256, EPI, false>(p, nexp, err, limit_ns, num_sms, st, 1);
+    case 128: return launch_t<128, EPI, false>(p, nexp, err, limit_ns, num_sms, st, 1);
+    default: return launch_t<64, EPI, false>(p, nexp, err, limit_ns, num_sms, st, 1);
+  }
+}
+
 cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* err,
-                            uint64_t wait_limit_ns, int num_sms, bool want_pair, cudaStream_t st) {
+                            uint64_t wait_limit_ns, int num_sms, bool want_pair, cudaStream_t st,
+                            bool mixed) {
   if (p.kind == kGemmWgrad) {
     if (!p.f32out && p.pair && want_pair) return launch_w2(p, nexp, err, wait_limit_ns, num_sms, st);
     if (p.f32out) {
@@ -1284,6 +1301,13 @@ cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* er
   }
   // forward: ReLU (and the backward's mask bits when a bit buffer is set) or none
   const int epi = p.relu ? (p.bits ? kEpiReluBits : kEpiRelu) : kEpiNone;
+  if (p.pair && mixed && !want_pair && (p.Cbuf % pairk::PM) == 0) {
+    // each expert's 256-row blocks on CTA pairs, a last block of at most 128 rows on
+    // one-CTA tiles: as little padding as 128-row tiles, most rows at the pair rate
+    if (epi == kEpiReluBits) return launch_mixed<kEpiReluBits>(p, nexp, err, wait_limit_ns, num_sms, st);
+    if (epi == kEpiRelu) return launch_mixed<kEpiRelu>(p, nexp, err, wait_limit_ns, num_sms, st);
+    return launch_mixed<kEpiNone>(p, nexp, err, wait_limit_ns, num_sms, st);
+  }
   if (p.pair && want_pair && (p.Cbuf % pairk::PM) == 0) {
     if (epi == kEpiReluBits) return launch_pair<kEpiReluBits, false>(p, nexp, err, wait_limit_ns, num_sms, st);
     if (epi == kEpiRelu) return launch_pair<kEpiRelu, false>(p, nexp, err, wait_limit_ns, num_sms, st);

@@ -163,8 +163,12 @@ bool make_wgrad_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, 
 // B = the router's W_g split [3*EPr, M], D = dx [S, M]
 bool make_gate_dx_plan(GemmPlan& p, const void* dlb, int64_t S, int EPb, const void* wsplit,
                        int EPr, void* dx, int M);
+// want_pair: CTA-pair (256-row) tiles everywhere (experts at capacity).  mixed (forward
+// GEMMs, when want_pair is off): pairs for each expert's 256-row blocks and one-CTA tiles
+// for a last block of at most 128 rows -- two launches.  Otherwise 128-row tiles.
 cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* err,
-                            uint64_t wait_limit_ns, int num_sms, bool want_pair, cudaStream_t st);
+                            uint64_t wait_limit_ns, int num_sms, bool want_pair, cudaStream_t st,
+                            bool mixed = false);
 // backward.cu
 struct BwdArgs {
   int S, M, H, E, k;

@@ -95,6 +95,10 @@ struct moe_layer {
 
 namespace {
 
+// Forward expert GEMMs below capacity: CTA pairs for each expert's 256-row blocks and
+// one-CTA tiles for a last block of at most 128 rows (else 128-row tiles throughout).
+constexpr bool kMixedTiles = true;
+
 size_t act_bytes(moe_dtype a) { return a == MOE_BF16 ? 2 : 4; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -310,7 +314,13 @@ moe_status moe_get_capacity(moe_handle h, int64_t S, int64_t* C_out) {
 
 int32_t moe_kernels_per_forward(moe_handle h, int64_t S) {
   if (!h || S <= 0) return 0;
-  return (h->route_flags & MOE_ROUTE_REROUTE) ? 8 : 6;
+  int n = (h->route_flags & MOE_ROUTE_REROUTE) ? 8 : 6;
+  if (h->act == MOE_BF16 && kMixedTiles && h->Cbuf % 256 == 0) {
+    const int64_t C = capacity_of(h->cf, h->k, S, h->E);
+    const bool saturated = (double)S * h->k / h->E >= (double)C;
+    if (!saturated) n += (h->plan1.pair ? 1 : 0) + (h->plan2.pair ? 1 : 0);   // pair + rest launches
+  }
+  return n;
 }
 
 moe_status moe_set_routing_flags(moe_handle h, uint32_t flags) {
@@ -380,10 +390,13 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
     // rows per expert are close to C and the 256-row padding stays small;
     // otherwise 128-row tiles waste less on partly filled last tiles.
     const bool saturated = (double)S * h->k / h->E >= (double)C;
-    MOE_TRY(launch_ffn_bf16(h->plan1, R.nexp, R.err, h->wait_limit_ns, h->num_sms, saturated, st));
+    // below capacity: pairs for each expert's 256-row blocks, one-CTA tiles for the rest
+    MOE_TRY(launch_ffn_bf16(h->plan1, R.nexp, R.err, h->wait_limit_ns, h->num_sms, saturated, st,
+                            kMixedTiles));
     h->bits_valid = h->plan1.bits != nullptr;
     MOE_TRY(mark(4));
-    MOE_TRY(launch_ffn_bf16(h->plan2, R.nexp, R.err, h->wait_limit_ns, h->num_sms, saturated, st));
+    MOE_TRY(launch_ffn_bf16(h->plan2, R.nexp, R.err, h->wait_limit_ns, h->num_sms, saturated, st,
+                            kMixedTiles));
   } else {
     MOE_TRY(launch_ffn_f32((const float*)h->xbuf, (const float*)h->W1, (float*)h->hbuf, R.nexp,
                            h->E, h->Cbuf, iM, iH, true, st));

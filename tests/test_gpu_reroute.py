@@ -80,7 +80,10 @@ def test_rerouted_forward_matches_oracle(w):
                                lambda e: (run.W1[e].cpu(), run.W2[e].cpu()))
     err = G.rel_err(out.y.float().cpu().numpy(), ref)
     assert err <= G.TOL_Y[w.act], err
-    assert L.moe_kernels_per_forward(run.layer.h, w.S) == 8
+    with_rr = L.moe_kernels_per_forward(run.layer.h, w.S)
+    L.moe_set_routing_flags(run.layer.h, 0)
+    assert with_rr == L.moe_kernels_per_forward(run.layer.h, w.S) + 2     # offers and their scan
+    L.moe_set_routing_flags(run.layer.h, L.MOE_ROUTE_REROUTE)
     # the backward of a rerouted forward is not built
     run.layer.enable_backward()
     run.layer(run.x)
