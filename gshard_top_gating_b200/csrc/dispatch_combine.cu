@@ -147,6 +147,56 @@ __global__ void __launch_bounds__(kThreads, 4) dispatch_rerouted_kernel(const T*
   }
 }
 
+// Top-1 routing with the combine fused into the second expert GEMM: the dispatch also
+// records, for every kept slot, the token that took it and its gate (the GEMM's
+// epilogue stores g * row straight into y[token]), and writes y = 0 for a token whose
+// choice was dropped (no expert row reaches it).
+__global__ void __launch_bounds__(kThreads, 4) dispatch_fused_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                     int S, int M, int E, int C,
+                                                                     int64_t Cbuf, int nchunk, Routing R,
+                                                                     __nv_bfloat16* __restrict__ xbuf,
+                                                                     int32_t* __restrict__ tok,
+                                                                     float* __restrict__ gsc,
+                                                                     __nv_bfloat16* __restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * kThreads) >> 5;
+  const int nv = M * 2 / 16;
+  pdl_trigger();
+  pdl_wait();                                  // routing tables and offsets complete
+  for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < S; t += warps) {
+    int e = 0, s = -1;
+    if (lane == 0) {
+      e = R.eidx[t];
+      int pos = 0x7fffffff;
+      if (e >= 0 && e < E) {
+        pos = R.off[(int64_t)(t / kChunk) * E + e] + R.lrank[t];
+      } else {
+        atomicOr(R.err, DEVERR_BOUNDS);
+      }
+      s = (pos < C && pos < Cbuf) ? pos : -1;
+      R.slot[t] = s;
+      if (s >= 0) {
+        tok[(int64_t)e * Cbuf + s] = t;
+        gsc[(int64_t)e * Cbuf + s] = R.gate[t];
+      }
+    }
+    e = __shfl_sync(0xffffffffu, e, 0);
+    s = __shfl_sync(0xffffffffu, s, 0);
+    uint4* dst = s >= 0 ? reinterpret_cast<uint4*>(xbuf + ((int64_t)e * Cbuf + s) * M)
+                        : reinterpret_cast<uint4*>(y + (int64_t)t * M);
+    const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)t * M);
+    for (int v0 = lane; v0 < nv; v0 += 32 * kUnroll) {
+      uint4 val[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (v0 + 32 * u < nv) val[u] = s >= 0 ? ld_nc_v4(src + v0 + 32 * u) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (v0 + 32 * u < nv) dst[v0 + 32 * u] = val[u];
+    }
+  }
+}
+
 template <typename T>
 struct Vec;
 template <>
@@ -399,6 +449,15 @@ cudaError_t launch_dispatch(const void* x, bool bf16, int S, int M, int E, int k
   else
     dispatch_k<float>(k, x, S, M, E, C, Cbuf, nchunk, R, xbuf, grid, st);
   return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_fused(const void* x, int S, int M, int E, int C, int64_t Cbuf,
+                                  const Routing& R, void* xbuf, int32_t* tok, float* gsc, void* y,
+                                  cudaStream_t st) {
+  const int nchunk = (S + kChunk - 1) / kChunk;
+  return launch_pdl(dispatch_fused_kernel, dim3(grid_for(S)), dim3(kThreads), 0, st,
+                    (const __nv_bfloat16*)x, S, M, E, C, Cbuf, nchunk, R, (__nv_bfloat16*)xbuf, tok, gsc,
+                    (__nv_bfloat16*)y);
 }
 
 cudaError_t launch_dispatch_rerouted(const void* x, bool bf16, int S, int M, int E, int k, int C,

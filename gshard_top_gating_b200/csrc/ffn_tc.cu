@@ -86,7 +86,10 @@ struct TileIter {
 
 // Epilogue modes: plain store, ReLU, or the backward's ReLU mask (keep the
 // accumulator where the first layer's saved output h is > 0, else 0).
-enum { kEpiNone = 0, kEpiRelu = 1, kEpiMask = 2, kEpiF32 = 3, kEpiReluBits = 4, kEpiMaskBits = 5 };
+enum { kEpiNone = 0, kEpiRelu = 1, kEpiMask = 2, kEpiF32 = 3, kEpiReluBits = 4, kEpiMaskBits = 5,
+       kEpiGateY = 6 };
+// kEpiGateY: g * accumulator, rounded to bf16, stored into the layer output row of the
+// token that took the slot (ScatterY), instead of into D.
 // kEpiReluBits: ReLU, and one bit per stored element, set when the stored bf16 value
 // is > 0 (the backward's mask, 1/16 of the bytes of h).  kEpiMaskBits: keep the
 // accumulator where that bit is set.  Bit j of word w of a row covers column 32w + j;
@@ -118,12 +121,60 @@ __device__ __forceinline__ uint32_t positive_bits(const uint4 (&v)[4]) {
 // writes whole 128-byte rows, instead of each thread storing 16 bytes to 32
 // different rows per instruction.  `mrow` (kEpiMask) points at this lane's row of h
 // at the tile's first column; `zero` stores zeros without reading TMEM.
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
 template <int BN, int EPI>
 __device__ __forceinline__ void store_rows(const CUtensorMap* tmD, uint32_t tmem_rows,
                                            uint32_t stage, int row0, int col0, int lane,
                                            const uint16_t* mrow = nullptr, bool zero = false,
                                            uint32_t* brow = nullptr, const uint32_t* bw = nullptr,
-                                           int64_t bstride = 0) {
+                                           int64_t bstride = 0, const ScatterY* sy = nullptr,
+                                           int row_end = 0) {
+  if (EPI == kEpiGateY) {
+    // this lane's row: its token and gate (rows at or past the expert's kept count: none)
+    const int r = row0 + lane;
+    const bool valid = r < row_end;
+    const int tk = valid ? __ldg(sy->tok + r) : -1;
+    const float g = valid ? __ldg(sy->gsc + r) : 0.f;
+    __nv_bfloat16* y = static_cast<__nv_bfloat16*>(sy->y);
+#pragma unroll 1
+    for (int b = 0; b < BN / 64; ++b) {
+      __syncwarp();                            // the previous chunk's staging reads are done
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_rows + b * 64 + h * 32, v);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          pk[j] = pack_bf16x2(g * __uint_as_float(v[2 * j]), g * __uint_as_float(v[2 * j + 1]));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t cc = h * 4 + j;
+          st_shared_v4(stage + lane * 128 + ((cc ^ (lane & 7)) << 4), pk[4 * j], pk[4 * j + 1],
+                       pk[4 * j + 2], pk[4 * j + 3]);
+        }
+      }
+      __syncwarp();
+      // eight lanes per row: each row's 128 bytes go out as one coalesced segment
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int rr = it * 4 + (lane >> 3), c = lane & 7;
+        const int tr = __shfl_sync(0xffffffffu, tk, rr);
+        if (tr >= 0) {
+          const uint4 val = ld_shared_v4(stage + rr * 128 + ((c ^ (rr & 7)) << 4));
+          *reinterpret_cast<uint4*>(y + (int64_t)tr * sy->ldy + col0 + b * 64 + c * 8) = val;
+        }
+      }
+    }
+    return;
+  }
   if (EPI == kEpiF32) {
     // fp32 result: 32 columns (128 bytes) per row per store, same swizzled staging
 #pragma unroll 1
@@ -235,7 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
                   int64_t Cbuf, int K, int N, const uint16_t* __restrict__ mask, int64_t row_limit,
-                  uint32_t* __restrict__ bits, unsigned* err, uint64_t limit_ns, int rest_only) {
+                  uint32_t* __restrict__ bits, unsigned* err, uint64_t limit_ns, int rest_only,
+                  const ScatterY sy) {
   using C = Cfg<BN>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -435,7 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (row0 < row_limit)           // a store box starts inside the tensor (TMA clips its tail)
         store_rows<BN, EPI>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
-                            nt * BN, lane, mrow, false, brow, bw, bstride);
+                            nt * BN, lane, mrow, false, brow, bw, bstride, &sy,
+                            (int)(e * Cbuf) + (EPI == kEpiGateY ? __ldg(nexp + e) : 0));
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
     }
@@ -685,7 +738,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ffn_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
                    int64_t Cbuf, int K, int N, const uint16_t* __restrict__ mask,
-                   uint32_t* __restrict__ bits, unsigned* err, uint64_t limit_ns, int leave_rest) {
+                   uint32_t* __restrict__ bits, unsigned* err, uint64_t limit_ns, int leave_rest,
+                   const ScatterY sy) {
   using namespace pairk;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -876,7 +930,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       store_rows<BN, EPI>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
-                          nt * BN, lane, mrow, false, brow, bw, bstride);
+                          nt * BN, lane, mrow, false, brow, bw, bstride, &sy,
+                          (int)(e * Cbuf) + (EPI == kEpiGateY ? __ldg(nexp + e) : 0));
       tc_fence_before();
       if (leader) mbar_arrive(tempty_bar(acc));
       else mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
@@ -1126,7 +1181,7 @@ cudaError_t launch_pair(const GemmPlan& p, const int32_t* nexp, unsigned* err, u
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(num_sms & ~1), dim3(kThreads), pairk::SMEM, st, p.tmA,
                     BKM ? p.tmB2 : p.tmB, p.tmD, nexp, p.E, p.Cbuf, p.K, p.N,
-                    static_cast<const uint16_t*>(p.mask), p.bits, err, limit_ns, leave_rest);
+                    static_cast<const uint16_t*>(p.mask), p.bits, err, limit_ns, leave_rest, p.sy);
 }
 
 template <int BN, int EPI, bool BKM>
@@ -1139,7 +1194,7 @@ cudaError_t launch_t(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint
   const int64_t row_limit = p.row_limit > 0 ? p.row_limit : (int64_t)p.E * p.Cbuf;
   return launch_pdl(kern, dim3(num_sms), dim3(kThreads), smem, st, p.tmA, p.tmB, p.tmD, nexp, p.E,
                     p.Cbuf, p.K, p.N, static_cast<const uint16_t*>(p.mask), row_limit, p.bits, err,
-                    limit_ns, rest_only);
+                    limit_ns, rest_only, p.sy);
 }
 
 template <int BN, int EPI>
@@ -1299,8 +1354,20 @@ cudaError_t launch_ffn_bf16(const GemmPlan& p, const int32_t* nexp, unsigned* er
         return launch_t<64, kEpiNone, true>(p, nexp, err, wait_limit_ns, num_sms, st);
     }
   }
-  // forward: ReLU (and the backward's mask bits when a bit buffer is set) or none
-  const int epi = p.relu ? (p.bits ? kEpiReluBits : kEpiRelu) : kEpiNone;
+  // forward: ReLU (and the backward's mask bits when a bit buffer is set), none, or the
+  // gate-scaled stores into the layer output
+  const int epi = p.sy.y ? kEpiGateY : (p.relu ? (p.bits ? kEpiReluBits : kEpiRelu) : kEpiNone);
+  if (epi == kEpiGateY) {
+    if (p.pair && mixed && !want_pair && (p.Cbuf % pairk::PM) == 0)
+      return launch_mixed<kEpiGateY>(p, nexp, err, wait_limit_ns, num_sms, st);
+    if (p.pair && want_pair && (p.Cbuf % pairk::PM) == 0)
+      return launch_pair<kEpiGateY, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+    switch (p.BN) {
+      case 256: return launch_t<256, kEpiGateY, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      case 128: return launch_t<128, kEpiGateY, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+      default: return launch_t<64, kEpiGateY, false>(p, nexp, err, wait_limit_ns, num_sms, st);
+    }
+  }
   if (p.pair && mixed && !want_pair && (p.Cbuf % pairk::PM) == 0) {
     // each expert's 256-row blocks on CTA pairs, a last block of at most 128 rows on
     // one-CTA tiles: as little padding as 128-row tiles, most rows at the pair rate

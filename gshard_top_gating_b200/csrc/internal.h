@@ -123,6 +123,11 @@ cudaError_t launch_dispatch_rerouted(const void* x, bool bf16, int S, int M, int
 // dispatch_combine.cu
 cudaError_t launch_dispatch(const void* x, bool bf16, int S, int M, int E, int k, int C,
                             int64_t Cbuf, const Routing& R, void* xbuf, cudaStream_t st);
+// The dispatch of the fused top-1 combine: as launch_dispatch, and every kept slot's token
+// and gate into tok / gsc [E*Cbuf]; a token whose choice was dropped gets y = 0.
+cudaError_t launch_dispatch_fused(const void* x, int S, int M, int E, int C, int64_t Cbuf,
+                                  const Routing& R, void* xbuf, int32_t* tok, float* gsc, void* y,
+                                  cudaStream_t st);
 cudaError_t launch_combine(const void* ybuf, bool bf16, int S, int M, int k, int64_t Cbuf,
                            const Routing& R, void* y, cudaStream_t st);
 // ffn_simt.cu  (fp32 activations)
@@ -130,6 +135,17 @@ cudaError_t launch_ffn_f32(const float* A, const float* B, float* D, const int32
                            int64_t Cbuf, int K, int N, bool relu, cudaStream_t st);
 // ffn_tc.cu  (bf16 activations, tcgen05)
 enum { kGemmFwd = 0, kGemmDgrad = 1, kGemmWgrad = 2 };
+// Gate-scaled stores straight into the layer output (forward FFN2 under top-1 routing):
+// row r of the expert buffers (expert r / Cbuf, slot r % Cbuf) is taken by token tok[r]
+// with gate gsc[r]; its result g * row goes to y[tok[r]] (ldy elements per row).  Rows at
+// or past the expert's kept count are not stored.
+struct ScatterY {
+  const int32_t* tok;   // [E*Cbuf]
+  const float* gsc;     // [E*Cbuf]
+  void* y;              // [S, ldy] bf16, or null: the plain store into D
+  int64_t ldy;
+};
+
 struct GemmPlan {
   // kGemmFwd   D[e,:n_e] = act(A[e,:n_e] . B[e])     A [E*Cbuf, K], B [E*K, N]
   // kGemmDgrad D[e,:n_e] = (A[e,:n_e] . Bt[e]^T) (* [mask > 0])   Bt [E*N, K]
@@ -151,6 +167,7 @@ struct GemmPlan {
   bool f32out;       // kGemmWgrad: D is fp32
   bool skip_zero;    // kGemmWgrad: experts with no kept row leave D[e] untouched (else zeros)
   int64_t row_limit; // rows of D (0 = E*Cbuf): stores of 32-row groups starting past it are skipped
+  ScatterY sy;       // kGemmFwd: with sy.y set, the epilogue stores gate-scaled rows into y instead of D
 };
 bool make_gemm_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, int64_t Cbuf, int K,
                     int N, bool relu);

@@ -57,6 +57,9 @@ struct moe_layer {
   bool fwd_data;         // the expert buffers hold the last forward's (not a route-only call's)
   bool profiling;
   uint32_t route_flags;  // MOE_ROUTE_* flags of later forwards
+  int32_t* slot_tok;     // top-1, fused combine: token of each expert-buffer row [E*Cbuf]
+  float* slot_gate;      // its gate [E*Cbuf]
+  bool last_fused;       // the last forward stored the expert outputs straight into y
   bool last_rerouted;    // the last routing call gave dropped choices a second chance
   // backward (moe_enable_backward)
   void* bws;             // the backward's one device allocation
@@ -94,6 +97,10 @@ struct moe_layer {
 };
 
 namespace {
+
+// Top-1 routing on an inference handle (no backward workspace): the second expert GEMM
+// stores its gate-scaled rows straight into y, and no combine kernel runs.
+bool fuses_combine(const moe_layer* h) { return h->slot_tok != nullptr && !h->bws; }
 
 // Forward expert GEMMs below capacity: CTA pairs for each expert's 256-row blocks and
 // one-CTA tiles for a last block of at most 128 rows (else 128-row tiles throughout).
@@ -156,6 +163,9 @@ size_t carve(moe_layer* h, char* base) {
     h->ystage[b] = c.take<char>((size_t)S * h->M * as);
   }
   h->wsplit = h->act == MOE_BF16 ? c.take<char>((size_t)3 * router_tc_pad(h->E) * h->M * 2) : nullptr;
+  const bool top1 = h->act == MOE_BF16 && k == 1;
+  h->slot_tok = top1 ? c.take<int32_t>((size_t)E * h->Cbuf) : nullptr;
+  h->slot_gate = top1 ? c.take<float>((size_t)E * h->Cbuf) : nullptr;
   return c.off + 256;
 }
 
@@ -314,7 +324,8 @@ moe_status moe_get_capacity(moe_handle h, int64_t S, int64_t* C_out) {
 
 int32_t moe_kernels_per_forward(moe_handle h, int64_t S) {
   if (!h || S <= 0) return 0;
-  int n = (h->route_flags & MOE_ROUTE_REROUTE) ? 8 : 6;
+  const bool reroute = (h->route_flags & MOE_ROUTE_REROUTE) != 0;
+  int n = reroute ? 8 : (fuses_combine(h) ? 5 : 6);
   if (h->act == MOE_BF16 && kMixedTiles && h->Cbuf % 256 == 0) {
     const int64_t C = capacity_of(h->cf, h->k, S, h->E);
     const bool saturated = (double)S * h->k / h->E >= (double)C;
@@ -340,6 +351,7 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
   h->have_forward = true;
   h->fwd_data = true;
   h->bits_valid = false;
+  h->last_fused = false;
   if (h->act == MOE_BF16 && !h->plan1.bits) {
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     // an error (a capture elsewhere in global mode) counts as capturing
@@ -380,7 +392,14 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
     MOE_TRY(launch_reroute_scan(iS, h->E, h->k, C, h->Cbuf, R, st));
   }
   MOE_TRY(mark(2));
-  if (reroute)
+  // top-1 inference: the combine is fused into the second expert GEMM, whose epilogue
+  // stores each row straight into y (the backward needs the expert outputs, so a
+  // handle in training mode keeps the separate combine)
+  const bool fused = fuses_combine(h) && !reroute;
+  h->last_fused = fused;
+  if (fused)
+    MOE_TRY(launch_dispatch_fused(x, iS, iM, h->E, C, h->Cbuf, R, h->xbuf, h->slot_tok, h->slot_gate, y, st));
+  else if (reroute)
     MOE_TRY(launch_dispatch_rerouted(x, bf16, iS, iM, h->E, h->k, C, h->Cbuf, R, h->xbuf, st));
   else
     MOE_TRY(launch_dispatch(x, bf16, iS, iM, h->E, h->k, C, h->Cbuf, R, h->xbuf, st));
@@ -395,8 +414,9 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
                             kMixedTiles));
     h->bits_valid = h->plan1.bits != nullptr;
     MOE_TRY(mark(4));
-    MOE_TRY(launch_ffn_bf16(h->plan2, R.nexp, R.err, h->wait_limit_ns, h->num_sms, saturated, st,
-                            kMixedTiles));
+    GemmPlan p2 = h->plan2;
+    if (fused) p2.sy = ScatterY{h->slot_tok, h->slot_gate, y, h->M};
+    MOE_TRY(launch_ffn_bf16(p2, R.nexp, R.err, h->wait_limit_ns, h->num_sms, saturated, st, kMixedTiles));
   } else {
     MOE_TRY(launch_ffn_f32((const float*)h->xbuf, (const float*)h->W1, (float*)h->hbuf, R.nexp,
                            h->E, h->Cbuf, iM, iH, true, st));
@@ -405,9 +425,11 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
                            h->E, h->Cbuf, iH, iM, false, st));
   }
   MOE_TRY(mark(5));
-  Routing Rc = R;
-  if (reroute) Rc.eidx = R.dest;     // combine from the expert that served each choice
-  MOE_TRY(launch_combine(h->ybuf, bf16, iS, iM, h->k, h->Cbuf, Rc, y, st));
+  if (!fused) {
+    Routing Rc = R;
+    if (reroute) Rc.eidx = R.dest;     // combine from the expert that served each choice
+    MOE_TRY(launch_combine(h->ybuf, bf16, iS, iM, h->k, h->Cbuf, Rc, y, st));
+  }
   MOE_TRY(mark(6));
   return MOE_OK;
 }
@@ -581,6 +603,7 @@ moe_status moe_get_expert_rows(moe_handle h, int32_t which, int32_t e, int64_t n
     return MOE_ERR_INVALID_ARG;
   h->last_was_host = false;
   if (!h->have_forward || !h->fwd_data) return MOE_ERR_STATE;
+  if (which == MOE_BUF_Y && h->last_fused) return MOE_ERR_STATE;   // stored straight into y
   if (nrows == 0) return MOE_OK;
   const size_t as = act_bytes(h->act);
   const int64_t width = which == MOE_BUF_H ? h->H : h->M;
@@ -681,6 +704,7 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
   h->last_was_host = false;
   if (!h->bws || !h->have_forward || !h->fwd_data || S != h->last_S) return MOE_ERR_STATE;
   if (h->last_rerouted) return MOE_ERR_UNSUPPORTED;   // the backward of rerouted choices is not built
+  if (h->last_fused) return MOE_ERR_STATE;            // that forward kept no expert outputs
   if (!dWg || !dW1 || !dW2 || !aligned(dWg, 16) || !aligned(dW1, 16) || !aligned(dW2, 16) ||
       (dbias && !aligned(dbias, 4)))
     return MOE_ERR_INVALID_ARG;

@@ -100,6 +100,9 @@ MOE_API moe_status moe_create(moe_handle* out, int64_t S_max, int64_t M, int64_t
  * x_dev  [S, M] act, row-major (read only).     y_dev  [S, M] act, fully overwritten.
  * A token whose k assignments were all dropped gets y = 0.  S = 0 enqueues no
  * kernel and sets l_aux = z = 0.  No host synchronisation, no allocation.
+ * Top-1 routing (k = 1, bf16) on a handle without moe_enable_backward: the combine is
+ * fused into the second expert GEMM, whose epilogue stores g * row straight into the
+ * token's row of y (the expert-output buffer is not written and no combine kernel runs).
  */
 MOE_API moe_status moe_forward(moe_handle h, int64_t S, const void* x_dev, void* y_dev, void* stream);
 
@@ -173,7 +176,8 @@ enum { MOE_BUF_X = 0,   /* xbuf [E, Cbuf, M] act: the dispatched token rows */
  * act elements.  Row i is the assignment the capacity scan gave slot i of expert
  * e; only rows below n_e = min(cnt[e], C) hold data.  0 <= nrows <= the handle's
  * rows per expert (min(C(S_max), S_max) rounded up to 256).  Device-to-device copy
- * on `stream`.  Returns MOE_ERR_STATE unless the last routing call was a moe_forward.
+ * on `stream`.  Returns MOE_ERR_STATE unless the last routing call was a moe_forward,
+ * and for MOE_BUF_Y after a forward whose combine was fused (top-1 inference).
  */
 MOE_API moe_status moe_get_expert_rows(moe_handle h, int32_t which, int32_t e, int64_t nrows,
                                        void* dst_dev, void* stream);
@@ -416,7 +420,8 @@ MOE_API moe_status moe_enable_backward(moe_handle h);
  *           (experts that kept no token get zeros, or are skipped: see
  *           moe_set_backward_flags).
  * Returns MOE_ERR_STATE unless moe_enable_backward succeeded and the last call
- * that routed on this handle was a moe_forward of S tokens.  Every output
+ * that routed on this handle was a moe_forward of S tokens that kept its expert outputs
+ * (a top-1 forward before moe_enable_backward fuses the combine and keeps none).  Every output
  * pointer must be 16-byte aligned and must not alias the inputs.
  */
 MOE_API moe_status moe_backward(moe_handle h, int64_t S, const void* x_dev, const void* dy_dev,
