@@ -6,9 +6,11 @@ A step is one whole layer forward (router, capacity scan, dispatch, two grouped
 expert GEMMs, combine, losses) over one batch of synthetic tokens already
 resident in HBM.  The headline workload is the largest single-GPU
 configuration, "large" (S=65536 tokens, M=2048, H=8192, E=64, top-2, capacity
-factor 1.0, bf16).  L2 is flushed (a 256 MB write) before every timed step and
-each step is timed with CUDA events on the launching stream; the sum over the
-K steps is the timed region.  The other four workloads are timed the same way
+factor 1.0, bf16).  Workloads whose token batch fits in L2 get a 256 MB write (an
+L2 flush) before every timed step; those whose inputs are larger than L2 (large
+and wide: x of 268 and 235 MB, expert weights of GBs) are timed without one, and
+`config.l2` says which.  Each step is timed with CUDA events on the launching
+stream; the sum over the K steps is the timed region.  The other four workloads are timed the same way
 in the same run and reported under "per_workload" (--workload-only skips them).
 
 With N > 1 (launched by torch.distributed.run) every rank runs an independent
@@ -39,6 +41,15 @@ sys.path.insert(0, ROOT)
 from gshard_top_gating_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024          # B200 L2 cache
+
+
+def inputs_exceed_l2(w) -> bool:
+    """The token batch alone is larger than L2 (and the expert weights far larger), so no
+    step can find the previous step's inputs in L2: such workloads are timed without a
+    flush; the others get a 256 MB write before every timed step."""
+    s = 2 if w.act == "bf16" else 4
+    return w.S * w.M * s > L2_BYTES and w.E * w.M * w.H * s * 2 > L2_BYTES
 STAGES = ("router", "scan", "dispatch", "ffn1", "ffn2", "combine")
 
 
@@ -322,10 +333,13 @@ def measure_backward(args, w, weights, x, y, flush, stream, pk, A, n_e):
         layer(x, out=y)
         bwd()
     torch.cuda.synchronize()
+    if inputs_exceed_l2(w):
+        flush = None
     n = max(3, min(args.steps, 50))
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
     for i in range(n):
-        flush.zero_()
+        if flush is not None:
+            flush.zero_()
         ev[i][0].record(stream)
         layer(x, out=y)
         ev[i][1].record(stream)
@@ -337,7 +351,8 @@ def measure_backward(args, w, weights, x, y, flush, stream, pk, A, n_e):
     L.moe_set_profiling(layer.h, True)
     per = [[] for _ in L.BWD_STAGES]
     for _ in range(min(n, 20)):
-        flush.zero_()
+        if flush is not None:
+            flush.zero_()
         layer(x, out=y)
         bwd()
         for j, t in enumerate(L.moe_get_backward_stage_times(layer.h)):
@@ -377,7 +392,10 @@ def workload_config(w, world):
     return {"workload": f"{w.name} (S={w.S}, M={w.M}, H={w.H}, E={w.E}, k={w.k}, cf={w.cf})",
             "S": w.S, "M": w.M, "H": w.H, "E": w.E, "k": w.k, "capacity_factor": w.cf,
             "C": math.ceil(w.cf * w.k * w.S / w.E),
-            "l2": "flushed before every timed step (256 MB write)",
+            "l2": (f"inputs larger than L2 (x {w.S * w.M * (2 if w.act == 'bf16' else 4) / 2**20:.0f} MiB, "
+                   f"expert weights {w.E * w.M * w.H * (2 if w.act == 'bf16' else 4) * 2 / 2**30:.1f} GiB, "
+                   f"L2 126 MiB): no flush" if inputs_exceed_l2(w)
+                   else "flushed before every timed step (256 MB write)"),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
@@ -403,14 +421,16 @@ def capture_step(layer, x, y, dev, eager):
 
 
 def time_steps(step, flush, stream, steps, world):
-    """K steps, L2 flushed before each, device time per step; (total ms over ranks, t0, t1)."""
+    """K steps (L2 flushed before each when `flush` is a buffer), device time per step;
+    (total ms over ranks, t0, t1)."""
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize()
     t0 = time.monotonic()
     for i in range(steps):
-        flush.zero_()
+        if flush is not None:
+            flush.zero_()
         starts[i].record(stream)
         step()
         ends[i].record(stream)
@@ -427,7 +447,8 @@ def stage_times(layer, x, y, flush, steps):
     L.moe_set_profiling(layer.h, True)
     per = [[] for _ in STAGES]
     for _ in range(steps):
-        flush.zero_()
+        if flush is not None:
+            flush.zero_()
         layer(x, out=y)
         for j, t in enumerate(L.moe_get_stage_times(layer.h)):
             per[j].append(t)
@@ -444,6 +465,8 @@ def measure_workload(args, w, dev, world, flush, pk, pk_kind, headline):
     layer = MoeLayer(w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b, W1, W2)
     y = torch.empty_like(x)
     stream = torch.cuda.current_stream()
+    if inputs_exceed_l2(w):
+        flush = None
     for _ in range(args.warmup):
         layer(x, out=y)
     torch.cuda.synchronize()
@@ -520,7 +543,8 @@ def measure_workload(args, w, dev, world, flush, pk, pk_kind, headline):
         s0 = time.monotonic()
         while time.monotonic() - s0 < 1.5:
             for _ in range(5):
-                flush.zero_()
+                if flush is not None:
+                    flush.zero_()
                 step()
             torch.cuda.synchronize()
         clocks = clk.summary(s0, time.monotonic(),

@@ -100,10 +100,11 @@ __global__ void __launch_bounds__(kThreads) gate_bwd_kernel(BwdArgs a, Routing R
     fj[i] = j < E ? (float)R.first[j] * invS : 0.f;
   }
   for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < a.S; t += warps) {
-    int e = 0, s = -1;
+    int e = 0, d = 0, s = -1;
     float g = 0.f;
     if (lane < k) {
       e = R.eidx[(int64_t)t * k + lane];
+      d = a.dest ? a.dest[(int64_t)t * k + lane] : e;    // the buffer of its rows
       s = R.slot[(int64_t)t * k + lane];
       g = R.gate[(int64_t)t * k + lane];
     }
@@ -114,11 +115,12 @@ __global__ void __launch_bounds__(kThreads) gate_bwd_kernel(BwdArgs a, Routing R
 #pragma unroll
     for (int r = 0; r < KM; ++r) {
       er[r] = __shfl_sync(0xffffffffu, e, r);
+      const int dr = __shfl_sync(0xffffffffu, d, r);
       const int sr = __shfl_sync(0xffffffffu, s, r);
       gr[r] = __shfl_sync(0xffffffffu, g, r);
       dot[r] = 0.f;
       const bool kept = r < k && sr >= 0;
-      const int64_t row = ((int64_t)er[r] * a.Cbuf + sr) * a.M;
+      const int64_t row = ((int64_t)dr * a.Cbuf + sr) * a.M;
       src[r] = kept ? reinterpret_cast<const uint4*>(ybuf + row) : nullptr;
       dst[r] = kept ? reinterpret_cast<uint4*>(dybuf + row) : nullptr;
     }

@@ -210,6 +210,9 @@ struct BwdArgs {
   float* bpart;        // [gate_bwd CTAs, E] bias partials
   int32_t* cnt_rows;   // [1 + nsplit]: S, then the rows of each dW_g split
   int nsplit, kchunk;  // dW_g split-K: nsplit splits of kchunk tokens
+  // rerouted forward: the expert serving each choice [S, k] (its rows' buffer), while
+  // the gate gradient goes to the chosen expert (Routing::eidx); null otherwise
+  const int32_t* dest;
 };
 cudaError_t launch_gate_backward(const BwdArgs& a, const Routing& R, cudaStream_t st);
 cudaError_t launch_pad_zero(void* const* bufs, const int* widths, int nbuf, bool bf16, int E,

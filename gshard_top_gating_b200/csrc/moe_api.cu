@@ -104,7 +104,7 @@ bool fuses_combine(const moe_layer* h) { return h->slot_tok != nullptr && !h->bw
 
 // Forward expert GEMMs below capacity: CTA pairs for each expert's 256-row blocks and
 // one-CTA tiles for a last block of at most 128 rows (else 128-row tiles throughout).
-constexpr bool kMixedTiles = true;
+constexpr bool kMixedTiles = false;
 
 size_t act_bytes(moe_dtype a) { return a == MOE_BF16 ? 2 : 4; }
 
@@ -703,7 +703,6 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
   if (!h || S < 0 || S > h->S_max) return MOE_ERR_INVALID_ARG;
   h->last_was_host = false;
   if (!h->bws || !h->have_forward || !h->fwd_data || S != h->last_S) return MOE_ERR_STATE;
-  if (h->last_rerouted) return MOE_ERR_UNSUPPORTED;   // the backward of rerouted choices is not built
   if (h->last_fused) return MOE_ERR_STATE;            // that forward kept no expert outputs
   if (!dWg || !dW1 || !dW2 || !aligned(dWg, 16) || !aligned(dW1, 16) || !aligned(dW2, 16) ||
       (dbias && !aligned(dbias, 4)))
@@ -746,6 +745,9 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
   a.dx = dx;
   a.dWg = dWg;
   a.dbias = dbias;
+  // a rerouted forward keeps a choice's rows at the expert serving it; its gate, and so
+  // the gate gradient, belongs to the expert it chose
+  a.dest = h->last_rerouted ? h->R.dest : nullptr;
   if (bf16) {
     a.dlb = h->dlb;
     a.EPb = h->EPb;
@@ -767,6 +769,8 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
     }
   }
   const Routing& R = h->R;
+  Routing Rrows = R;                   // row gathers address the serving expert's buffer
+  if (h->last_rerouted) Rrows.eidx = R.dest;
   const bool prof = h->profiling && h->have_events;
   auto mark = [&](int i) -> cudaError_t { return prof ? cudaEventRecord(h->evb[i], st) : cudaSuccess; };
   h->have_backward_times = false;
@@ -816,12 +820,12 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
   if (bf16) {
     const uint64_t lim = h->wait_limit_ns;
     MOE_TRY(launch_ffn_bf16(h->plan_gdx, h->cnt_rows, R.err, lim, h->num_sms, false, st));
-    MOE_TRY(launch_dx_gather(a, R, st));
+    MOE_TRY(launch_dx_gather(a, Rrows, st));
     MOE_TRY(mark(7));
     MOE_TRY(launch_ffn_bf16(h->plan_dwg, h->cnt_rows + 1, R.err, lim, h->num_sms, false, st));
     MOE_TRY(launch_dwg_tc_reduce(a, gate_backward_grid((int)S, h->num_sms), h->num_sms, st));
   } else {
-    MOE_TRY(launch_dx(a, R, st));
+    MOE_TRY(launch_dx(a, Rrows, st));
     MOE_TRY(mark(7));
     MOE_TRY(launch_dwg(a, h->num_sms, st));
   }

@@ -211,7 +211,9 @@ enum { MOE_ROUTE_REROUTE = 1 };
  * an offer that finds no room stays dropped.  A rerouted choice keeps its gate weight.
  * moe_get_routing then reports the final slot (at the serving expert) and
  * moe_get_serving_experts the serving expert.  A forward with this flag launches 8
- * kernels.  moe_backward of a rerouted forward returns MOE_ERR_UNSUPPORTED.
+ * kernels.  moe_backward of a rerouted forward differentiates that forward: a rerouted
+ * choice's rows are at the serving expert, and its gate gradient goes to the expert it
+ * chose (its weight g_r is that expert's normalised gate).
  * Returns MOE_ERR_INVALID_ARG for unknown bits.
  */
 MOE_API moe_status moe_set_routing_flags(moe_handle h, uint32_t flags);

@@ -370,7 +370,7 @@ def z_loss_backward(p, lse, S: int | None = None):
 
 
 def backward(x, Wg, bias, W1, W2, k: int, cf: float, dy, a_aux: float = 0.0, a_z: float = 0.0,
-             round_fp32: bool = True, logits=None):
+             round_fp32: bool = True, logits=None, rerouting: bool = False):
     """Gradients of  L = <dy, y> + a_aux * l_aux + a_z * z  with respect to x, W_g, b, W1, W2.
 
     The routing (expert choice, slots, drops) is piecewise constant and carries
@@ -385,9 +385,11 @@ def backward(x, Wg, bias, W1, W2, k: int, cf: float, dy, a_aux: float = 0.0, a_z
       gate GEMM ([blog] G(x) = Softmax(x . W_g)): dx += dl W_g^T, dW_g = x^T dl, db = sum_t dl.
     Returns a namespace with dx, dWg, dbias, dW1, dW2 (float64), the
     intermediates dl, dgate, dybuf (the expert outputs' gradient) and the
-    forward namespace fwd.  `logits` as in `forward`.
+    forward namespace fwd.  `logits` as in `forward`.  With `rerouting`, a
+    rerouted assignment's rows live at the expert that serves it (dest), while
+    its gate weight -- and so its gradient -- belongs to the expert it chose.
     """
-    rt = forward(x, Wg, bias, W1, W2, k, cf, round_fp32, logits)
+    rt = forward(x, Wg, bias, W1, W2, k, cf, round_fp32, logits, rerouting)
     xf, Wgf, W1f, W2f, dyf = _f64(x), _f64(Wg), _f64(W1), _f64(W2), _f64(dy)
     S, E = rt.logits.shape
     dgate = np.zeros((S, k))
@@ -395,7 +397,7 @@ def backward(x, Wg, bias, W1, W2, k: int, cf: float, dy, a_aux: float = 0.0, a_z
     for r in range(k):
         keep = rt.slot[:, r] >= 0
         t = np.nonzero(keep)[0]
-        e, sl = rt.ids[keep, r], rt.slot[keep, r]
+        e, sl = rt.dest[keep, r], rt.slot[keep, r]
         dgate[t, r] = np.sum(dyf[t] * rt.ybuf[e, sl], axis=1)
         dybuf[e, sl] = rt.gates[t, r][:, None] * dyf[t]
     dW1 = np.zeros_like(W1f)
@@ -409,7 +411,7 @@ def backward(x, Wg, bias, W1, W2, k: int, cf: float, dy, a_aux: float = 0.0, a_z
     dx = np.zeros_like(xf)
     for r in range(k):
         keep = rt.slot[:, r] >= 0
-        dx[keep] += dxbuf[rt.ids[keep, r], rt.slot[keep, r]]
+        dx[keep] += dxbuf[rt.dest[keep, r], rt.slot[keep, r]]
     dl = np.zeros((S, E))
     if S:
         dl += gates_backward(rt.gates, rt.ids, dgate, E)

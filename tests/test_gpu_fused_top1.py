@@ -5,7 +5,7 @@ GEMM's epilogue stores g * row straight into the token's row of y and no combine
 kernel runs.  With one choice the normalised gate is exactly 1, so y must equal,
 bit for bit, the separate-combine path (a handle in training mode), and the
 oracle within the bf16 tolerance; tokens whose choice was dropped get exact zeros.
-The shapes take the one-CTA, CTA-pair and mixed tilings of that GEMM.
+The shapes take the one-CTA and CTA-pair tilings of that GEMM.
 """
 import numpy as np
 import pytest
@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("w", [
-    Workload("t1_mixed", 3000, 256, 512, 16, 1, 1.0, "bf16"),            # below capacity: pairs + rest
+    Workload("t1_below_capacity", 3000, 256, 512, 16, 1, 1.0, "bf16"),   # below capacity
     Workload("t1_pairs", 4096, 256, 256, 8, 1, 0.5, "bf16"),             # at capacity: CTA pairs
     Workload("t1_one_cta", 1000, 192, 128, 8, 1, 1.5, "bf16", skew_bias=True),   # N = 192: one-CTA tiles
     Workload("t1_big", 20000, 1024, 1024, 64, 1, 1.0, "bf16"),

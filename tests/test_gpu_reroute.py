@@ -62,7 +62,7 @@ def test_rerouted_slots_bit_exact_given_logits(S, E, k, cf, skew, ties):
 
 @pytest.mark.parametrize("w", [
     Workload("rr_bf16", 1500, 256, 512, 16, 2, 0.75, "bf16", skew_bias=True),
-    Workload("rr_bf16_top4", 700, 128, 256, 32, 4, 0.6, "bf16"),
+    Workload("rr_bf16_top4", 700, 128, 256, 32, 4, 0.6, "bf16", skew_bias=True),
     Workload("rr_f32", 256, 64, 256, 8, 2, 0.6, "f32", skew_bias=True),
 ], ids=lambda w: w.name)
 def test_rerouted_forward_matches_oracle(w):

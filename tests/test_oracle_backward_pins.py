@@ -12,8 +12,8 @@ import oracle.moe_oracle as M
 EPS = 1e-6
 
 
-def _loss(x, Wg, b, W1, W2, k, cf, dy, a_aux, a_z):
-    rt = M.forward(x, Wg, b, W1, W2, k, cf, round_fp32=False)
+def _loss(x, Wg, b, W1, W2, k, cf, dy, a_aux, a_z, rerouting=False):
+    rt = M.forward(x, Wg, b, W1, W2, k, cf, round_fp32=False, rerouting=rerouting)
     return float(np.sum(dy * rt.y) + a_aux * rt.l_aux + a_z * rt.z)
 
 
@@ -28,7 +28,7 @@ def _case(seed, S, Md, H, E, k, cf, bias=True):
     return x, Wg, b, W1, W2, k, cf, dy
 
 
-def _fd_check(args, a_aux, a_z, grads, n_coords=6, seed=0):
+def _fd_check(args, a_aux, a_z, grads, n_coords=6, seed=0, rerouting=False):
     x, Wg, b, W1, W2, k, cf, dy = args
     rng = np.random.default_rng(seed)
     names = [("x", x, grads.dx), ("Wg", Wg, grads.dWg), ("W1", W1, grads.dW1), ("W2", W2, grads.dW2)]
@@ -39,9 +39,9 @@ def _fd_check(args, a_aux, a_z, grads, n_coords=6, seed=0):
             idx = tuple(rng.integers(0, s) for s in arr.shape)
             orig = arr[idx]
             arr[idx] = orig + EPS
-            lp = _loss(x, Wg, b, W1, W2, k, cf, dy, a_aux, a_z)
+            lp = _loss(x, Wg, b, W1, W2, k, cf, dy, a_aux, a_z, rerouting)
             arr[idx] = orig - EPS
-            lm = _loss(x, Wg, b, W1, W2, k, cf, dy, a_aux, a_z)
+            lm = _loss(x, Wg, b, W1, W2, k, cf, dy, a_aux, a_z, rerouting)
             arr[idx] = orig
             fd = (lp - lm) / (2 * EPS)
             assert abs(fd - g[idx]) <= 2e-6 + 2e-6 * abs(fd), (name, idx, fd, g[idx])
@@ -59,6 +59,21 @@ def test_backward_matches_finite_differences(seed, S, Md, H, E, k, cf):
     for a_aux, a_z in ((0.0, 0.0), (0.7, 0.3)):
         grads = M.backward(x, Wg, b, W1, W2, k, cf, dy, a_aux, a_z, round_fp32=False)
         _fd_check(args, a_aux, a_z, grads, seed=seed)
+
+
+@pytest.mark.parametrize("seed,S,Md,H,E,k,cf", [
+    (11, 12, 5, 6, 5, 2, 0.6),      # dropped choices rerouted, some for good
+    (12, 10, 4, 5, 6, 3, 0.5),      # k = 3: tokens with two dropped choices
+])
+def test_rerouted_backward_matches_finite_differences(seed, S, Md, H, E, k, cf):
+    """With rerouting, rows live at the serving expert and gates at the chosen one."""
+    args = _case(seed, S, Md, H, E, k, cf)
+    x, Wg, b, W1, W2, k, cf, dy = args
+    rt = M.forward(x, Wg, b, W1, W2, k, cf, round_fp32=False, rerouting=True)
+    assert (rt.dest != rt.ids).any(), "the case reroutes something"
+    for a_aux, a_z in ((0.0, 0.0), (0.7, 0.3)):
+        grads = M.backward(x, Wg, b, W1, W2, k, cf, dy, a_aux, a_z, round_fp32=False, rerouting=True)
+        _fd_check(args, a_aux, a_z, grads, seed=seed, rerouting=True)
 
 
 def test_single_expert_backward_is_dense_ffn_backward():
