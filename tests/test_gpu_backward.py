@@ -82,25 +82,33 @@ def _mask_slack(ref, W1, W2, K):
     s_dx = np.zeros((S, M))
     for r in range(fwd.slot.shape[1]):
         keep = fwd.slot[:, r] >= 0
-        s_dx[keep] += s_dxe[fwd.ids[keep, r], fwd.slot[keep, r]]
+        s_dx[keep] += s_dxe[fwd.dest[keep, r], fwd.slot[keep, r]]
     return s_dW1, s_dx
 
 
-def backward_check(w, a_aux=0.7, a_z=0.3, S=None, train=True):
+def backward_check(w, a_aux=0.7, a_z=0.3, S=None, train=True, rerouting=False):
     """train: the backward is enabled before the forward, so FFN1 stores the
-    ReLU mask bits that dP reads; otherwise dP re-reads h."""
+    ReLU mask bits that dP reads; otherwise dP re-reads h.  rerouting: the
+    forward gives dropped choices their second chance (MOE_ROUTE_REROUTE)."""
     run = G.build(w, S=S)
     if train:
         run.layer.enable_backward()
+    if rerouting:
+        run.layer.set_rerouting(True)
     out = G.forward(run)
-    G.check_routing(run, out)
+    if rerouting:
+        rt = O.route(out.logits, w.k, w.cf, rerouting=True)
+        assert np.array_equal(out.slot, rt.slot) and (rt.dest != rt.ids).any()
+        assert np.array_equal(run.layer.serving_experts(run.S).cpu().numpy(), rt.dest)
+    else:
+        G.check_routing(run, out)
     dy = upstream_grad(w, device="cuda", S=run.S)
     g = run.layer.backward(out.x, dy, a_aux, a_z)
     torch.cuda.synchronize()
     L.moe_check(run.layer.h)
     W1, W2 = _np(run.W1), _np(run.W2)
     ref = O.backward(_np(out.x), _np(run.Wg), None if run.b is None else _np(run.b), W1, W2, w.k,
-                     w.cf, _np(dy), a_aux, a_z, logits=out.logits)
+                     w.cf, _np(dy), a_aux, a_z, logits=out.logits, rerouting=rerouting)
     s_dW1, s_dx = _mask_slack(ref, W1, W2, w.M)
     errs = {
         "dx": _excess_err(_np(g["dx"]), ref.dx, s_dx),
@@ -476,4 +484,18 @@ def test_backward_edge_shapes(shape):
     _check_all(errs, act)
     if E == 1:
         assert np.abs(_np(g["dWg"])).max() <= 1e-6 * np.abs(_np(g["dx"])).max()
+    run.layer.close()
+
+
+@pytest.mark.parametrize("w", [
+    Workload("bwd_rr_bf16", 900, 128, 256, 16, 2, 0.6, "bf16", skew_bias=True),
+    Workload("bwd_rr_bf16_k3", 500, 256, 128, 12, 3, 0.5, "bf16", skew_bias=True),
+    Workload("bwd_rr_f32", 300, 64, 128, 8, 2, 0.6, "f32", skew_bias=True),
+], ids=lambda w: w.name)
+def test_backward_of_rerouted_forward(w):
+    """Rows of a rerouted choice sit at the serving expert; its gate gradient goes to
+    the expert it chose (oracle `backward(..., rerouting=True)`)."""
+    run, out, g, ref, errs = backward_check(w, rerouting=True)
+    print(f"\n{w.name}: {errs}")
+    _check_all(errs, w.act)
     run.layer.close()
