@@ -655,6 +655,9 @@ def _sized_runs(sample, budget_s, S, probe=64, max_passes=20):
     c = sample.run(probe) / probe
     ntok = int(max(probe, min(S, budget_s / max(c, 1e-9))))
     dt = sample.run(ntok)
+    if dt < 0.5 * budget_s and ntok < S:        # the probe's fixed costs overstated a token's cost
+        ntok = int(min(S, ntok * budget_s / max(dt, 1e-9)))
+        dt = sample.run(ntok)
     reps = 1
     if ntok == S:
         more = max(0, min(max_passes - 1, int((budget_s - dt) / max(dt, 1e-9))))
