@@ -98,3 +98,35 @@ def test_ep_rejects_a_plan_from_inconsistent_stats():
         bad = np.stack([st, st]); bad[1, 0] += 0.5
         layer.dispatch(bad, x[:128].contiguous())
     layer.close()
+
+
+def test_ep_forward_dist_one_rank_nccl():
+    """The torch.distributed driver (all-gather of stats, two all_to_all_single) in a
+    one-rank NCCL group equals the one-device layer; no rank waits on another."""
+    import os
+    import socket
+    import torch.distributed as dist
+    from datetime import timedelta
+    from gshard_top_gating_b200.ep import ep_forward_dist
+    w = Workload("ep_dist1", 1024, 256, 256, 16, 2, 1.0, "bf16")
+    x, Wg, b, W1, W2 = make_inputs(w, device="cuda")
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True, timeout=timedelta(seconds=30))
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1, timeout=timedelta(seconds=60),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        layer = EPMoeLayer(1, 0, w.S, w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b, W1, W2)
+        y = ep_forward_dist(layer, x)
+        one = MoeLayer(w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b, W1, W2)
+        y1 = one(x)
+        torch.cuda.synchronize()
+        assert torch.equal(y, y1)
+        la, za = layer.aux_loss()
+        lb, zb = one.aux_loss()
+        assert abs(la - lb) <= 1e-5 * lb and abs(za - zb) <= 1e-5 * zb
+        one.close()
+        layer.close()
+    finally:
+        dist.destroy_process_group()
