@@ -327,7 +327,7 @@ moe_status moe_ep_route(moe_ep_handle h, int64_t S, const void* x, double* stats
       h->xmap_ptr = x;
       h->xmap_S = S;
     }
-    EP_TRY(launch_router_tc(h->xmap, persistent ? &h->xmap64 : nullptr, h->wmap, h->bias, iS, iM, h->E,
+    EP_TRY(launch_router_tc(h->xmap, persistent ? &h->xmap64 : nullptr, x, h->wmap, h->bias, iS, iM, h->E,
                             h->k, h->R, h->wait_limit_ns, st));
   } else {
     EP_TRY(launch_router(x, false, h->Wg, h->bias, iS, iM, h->E, h->k, h->R, st));

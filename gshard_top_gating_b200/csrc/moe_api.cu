@@ -378,7 +378,7 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
       h->xmap_ptr = x;
       h->xmap_S = S;
     }
-    MOE_TRY(launch_router_tc(h->xmap, persistent ? &h->xmap64 : nullptr, h->wmap, h->bias, iS, iM, h->E,
+    MOE_TRY(launch_router_tc(h->xmap, persistent ? &h->xmap64 : nullptr, x, h->wmap, h->bias, iS, iM, h->E,
                              h->k, R, h->wait_limit_ns, st));
   } else {
     MOE_TRY(launch_router(x, bf16, h->Wg, h->bias, iS, iM, h->E, h->k, R, st));

@@ -525,29 +525,29 @@ __global__ void __launch_bounds__(NW * 32, (NW == 8) ? 2 : 1)
 // one chunk) and walks it in tiles of two chunks (the last tile may be one chunk,
 // loaded as a 64-row box).  Unlike router_tc_kernel, a tile's routing overlaps the
 // next tiles' loads and MMAs:
-//   warp 0       TMA producer of the token tiles (x ring, from DRAM)
-//   warp 6       TMA producer of the three W_g parts (W ring, from L2)
+//   warp 0       TMA producer over every tile's k-blocks (x tile + three W_g parts)
 //   warp 1       MMA issuer; K-segments alternate between two TMEM accumulators
 //   warps 2..5   fold: each K-segment (lo + mid, + hi) is added into the tile's running
 //                sum, one of two TMEM regions (tiles alternate), and the segment's
 //                accumulator is released at once
-//   warps 7..15  routing group: copies a finished tile's logits from TMEM to shared
+//   warps 6..15  routing group: copies a finished tile's logits from TMEM to shared
 //                memory (plus bias), releases the running-sum region, then routes the
 //                tile exactly as router_tc_kernel does for E <= 64 (a thread per
 //                token), writes the logits and the chunk tables
 // The arithmetic of every logit, probability, gate and table entry is that of
 // router_tc_kernel.  TMEM: two segment accumulators (3*EP columns each) and two
-// running sums (EP each) -- 448 of 512 columns for EP = 64.  The token tiles come from
-// DRAM and the gate parts from L2, so they travel in separate rings: a deep x ring keeps
-// enough bytes of x in flight for DRAM's latency, a shallow W ring enough for L2's.
+// running sums (EP each) -- 448 of 512 columns for EP = 64.
+// A tile's TMA boxes read 128 bytes of each token row per k-block, rows 2M bytes
+// apart; from DRAM that pattern wastes much of each page it opens.  So while tile i
+// is multiplied, the producer brings tile i+1's token rows into L2 as whole
+// contiguous rows (a bulk prefetch of a few rows per k-block), and tile i+1's boxes
+// then come from L2.
 template <int EP>
 struct PCfg {
   static constexpr int NT = 512;
   static constexpr int TT = 128;
   static constexpr uint32_t PART_BYTES = EP * BK * 2;
-  static constexpr uint32_t W_BYTES = 3 * PART_BYTES;     // one W ring stage
-  static constexpr int XS = EP == 64 ? 6 : 8;             // x ring stages (16 KB each)
-  static constexpr int WS = EP == 64 ? 3 : 4;             // W ring stages
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + 3 * PART_BYTES;
   static constexpr uint32_t ACC = 3 * EP;                 // one K-segment accumulator
   static constexpr uint32_t RUN0 = 2 * ACC;               // running sum of tile parity b at RUN0 + b*EP
   static constexpr uint32_t TMEM_COLS = (2 * ACC + 2 * EP) <= 256 ? 256 : 512;
@@ -557,15 +557,15 @@ struct PCfg {
   static constexpr uint32_t H_OFF = SEL_OFF + TT * kMaxK * 4; // running counts [2][8][EP]
   static constexpr uint32_t LSE_OFF = H_OFF + 2 * kMaxK * EP * 4;   // lse^2 per token [TT]
   static constexpr uint32_t EPI_BYTES = ((LSE_OFF + TT * 4) + 1023u) & ~1023u;
-  static constexpr uint32_t BAR_BYTES = 512;
-  static constexpr uint32_t RING_BYTES = XS * A_BYTES + WS * W_BYTES;
-  static constexpr int NBAR = 2 * XS + 2 * WS + 9;
-  static constexpr size_t SMEM = 1024 + (size_t)RING_BYTES + EPI_BYTES + BAR_BYTES;
+  static constexpr uint32_t BAR_BYTES = 256;
+  static constexpr int STAGES_FIT = (int)((227u * 1024u - 1024u - EPI_BYTES - BAR_BYTES) / STAGE_BYTES);
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
   static_assert(EP <= 64, "the persistent router routes a thread per token (E <= 64)");
-  static_assert(W_BYTES % 1024 == 0, "W stages stay 1024-aligned (128-byte swizzle)");
+  static_assert(STAGES >= 3, "at least three stages in flight");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
   static_assert(2 * ACC + 2 * EP <= TMEM_COLS, "TMEM columns");
-  static_assert(8u * NBAR + 12 <= BAR_BYTES, "barriers, TMEM slot and flags");
+  static_assert(8u * (2 * STAGES + 9) + 12 <= BAR_BYTES, "barriers, TMEM slot and flags");
 };
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
@@ -575,35 +575,31 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 template <int EP>
 __global__ void __launch_bounds__(512, 1)
     router_tcp_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmX64,
-                      const __grid_constant__ CUtensorMap tmW, const float* __restrict__ bias, int S, int M,
-                      int E, int k, int nchunk, Routing R, uint64_t limit_ns) {
+                      const __grid_constant__ CUtensorMap tmW, const __nv_bfloat16* __restrict__ xraw,
+                      const float* __restrict__ bias, int S, int M, int E, int k, int nchunk, Routing R,
+                      uint64_t limit_ns) {
   using C = PCfg<EP>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t base = (raw_base + 1023u) & ~1023u;
   unsigned char* gbase = smem_raw + (base - raw_base);
-  unsigned char* gepi = gbase + C::RING_BYTES;
-  const uint32_t wring = base + C::XS * A_BYTES;                  // W ring after the x ring
+  unsigned char* gepi = gbase + C::STAGES * C::STAGE_BYTES;
   float* Ls = reinterpret_cast<float*>(gepi + C::L_OFF);
   int32_t* sel = reinterpret_cast<int32_t*>(gepi + C::SEL_OFF);
   int32_t* Hs = reinterpret_cast<int32_t*>(gepi + C::H_OFF);
   float* lse_t = reinterpret_cast<float*>(gepi + C::LSE_OFF);
-  const uint32_t bar0 = base + C::RING_BYTES + C::EPI_BYTES;
-  constexpr int XS = C::XS, WS = C::WS;
-  auto xfull_bar = [&](int s) { return bar0 + 8u * s; };
-  auto xempty_bar = [&](int s) { return bar0 + 8u * (XS + s); };
-  auto wfull_bar = [&](int s) { return bar0 + 8u * (2 * XS + s); };
-  auto wempty_bar = [&](int s) { return bar0 + 8u * (2 * XS + WS + s); };
-  constexpr int B0 = 2 * XS + 2 * WS;
-  auto tfull_bar = [&](int b) { return bar0 + 8u * (B0 + b); };      // a K-segment is done
-  auto tempty_bar = [&](int b) { return bar0 + 8u * (B0 + 2 + b); };  // the fold took it
-  auto lfull_bar = [&](int b) { return bar0 + 8u * (B0 + 4 + b); };   // a tile's logits are done
-  auto rfree_bar = [&](int b) { return bar0 + 8u * (B0 + 6 + b); };   // its running sum is free
-  const uint32_t done_bar = bar0 + 8u * (B0 + 8);
+  const uint32_t bar0 = base + C::STAGES * C::STAGE_BYTES + C::EPI_BYTES;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + b); };      // a K-segment is done
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 + b); };  // the fold took it
+  auto lfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 4 + b); };   // a tile's logits are done
+  auto rfree_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 6 + b); };   // its running sum is free
+  const uint32_t done_bar = bar0 + 8u * (2 * C::STAGES + 8);
   unsigned char* gbar = gepi + C::EPI_BYTES;
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbar + 8u * C::NBAR);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbar + 8u * C::NBAR + 4);
-  volatile int* go_flag = reinterpret_cast<volatile int*>(gbar + 8u * C::NBAR + 8);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbar + 8u * (2 * C::STAGES + 9));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbar + 8u * (2 * C::STAGES + 9) + 4);
+  volatile int* go_flag = reinterpret_cast<volatile int*>(gbar + 8u * (2 * C::STAGES + 9) + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nblk = gridDim.x, blk = blockIdx.x;
@@ -613,13 +609,9 @@ __global__ void __launch_bounds__(512, 1)
   const int nseg = (KB + kSegBlocks - 1) / kSegBlocks;
 
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < XS; ++s) {
-      mbar_init(xfull_bar(s), 1);
-      mbar_init(xempty_bar(s), 1);
-    }
-    for (int s = 0; s < WS; ++s) {
-      mbar_init(wfull_bar(s), 1);
-      mbar_init(wempty_bar(s), 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
@@ -644,11 +636,9 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem_base = *tmem_slot;
   pdl_trigger();          // after the TMEM allocation (see router_tc_kernel)
 
-  if (warp == 0 || warp == 6) {
-    // ------------------------------------------------------------ TMA producers: x (warp 0), W (warp 6)
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const bool xs_role = warp == 0;
-      const int NS = xs_role ? XS : WS;
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_par = 0;
       bool ok = true;
@@ -656,42 +646,44 @@ __global__ void __launch_bounds__(512, 1)
         const int ca = c0 + 2 * i;
         const bool half = ca + 1 >= c1;
         const int tok0 = ca * kChunk;
+        const uint32_t tx = (half ? 64u : 128u) * BK * 2 + 3 * C::PART_BYTES;
+        // the next tile's rows, a slice per k-block, into L2 as whole rows
+        const int cn = ca + 2;
+        const int ntok_next = i + 1 < ntiles ? min((cn + 1 >= c1 ? 1 : 2) * kChunk, S - cn * kChunk) : 0;
+        const int rows_per_kb = (ntok_next + KB - 1) / KB;
         for (int kb = 0; kb < KB; ++kb) {
-          const uint32_t eb = xs_role ? xempty_bar(s) : wempty_bar(s);
-          const uint32_t fb = xs_role ? xfull_bar(s) : wfull_bar(s);
-          if (*abort_flag || !mbar_wait(eb, ph ^ 1u, R.err, limit_ns)) {
+          const int r0 = kb * rows_per_kb, r1 = min(ntok_next, r0 + rows_per_kb);
+          if (r1 > r0)
+            bulk_prefetch_l2(xraw + (int64_t)(cn * kChunk + r0) * M, (uint32_t)((r1 - r0) * M * 2));
+          if (*abort_flag || !mbar_wait(empty_bar(s), ph ^ 1u, R.err, limit_ns)) {
             *abort_flag = 1;
             ok = false;
             break;
           }
-          if (xs_role) {
-            mbar_arrive_expect_tx(fb, (half ? 64u : 128u) * BK * 2);
-            tma_load_2d(base + s * A_BYTES, half ? (const void*)&tmX64 : (const void*)&tmX, fb, kb * BK, tok0);
-          } else {
-            mbar_arrive_expect_tx(fb, C::W_BYTES);
+          const uint32_t sa = base + s * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(full_bar(s), tx);
+          tma_load_2d(sa, half ? (const void*)&tmX64 : (const void*)&tmX, full_bar(s), kb * BK, tok0);
 #pragma unroll
-            for (int part = 0; part < 3; ++part)
-              tma_load_2d(wring + s * C::W_BYTES + part * C::PART_BYTES, &tmW, fb, kb * BK, part * EP);
-          }
+          for (int part = 0; part < 3; ++part)
+            tma_load_2d(sa + A_BYTES + part * C::PART_BYTES, &tmW, full_bar(s), kb * BK, part * EP);
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
-          if (++s == NS) {
+          if (++s == C::STAGES) {
             s = 0;
             ph ^= 1u;
           }
         }
       }
       if (!ok)
-        for (int q = 0; q < NS; ++q)
-          if ((issued >> q) & 1u)
-            mbar_wait(xs_role ? xfull_bar(q) : wfull_bar(q), (issued_par >> q) & 1u, R.err, limit_ns);
+        for (int q = 0; q < C::STAGES; ++q)
+          if ((issued >> q) & 1u) mbar_wait(full_bar(q), (issued_par >> q) & 1u, R.err, limit_ns);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int xs = 0, ws = 0;
-      uint32_t xph = 0, wph = 0, g = 0;
+      int s = 0;
+      uint32_t ph = 0, g = 0;
       bool ok = true;
       for (int i = 0; i < ntiles && ok; ++i) {
         for (int kb = 0; kb < KB; ++kb) {
@@ -706,31 +698,25 @@ __global__ void __launch_bounds__(512, 1)
             }
             tc_fence_after();
           }
-          if (*abort_flag || !mbar_wait(xfull_bar(xs), xph, R.err, limit_ns) ||
-              !mbar_wait(wfull_bar(ws), wph, R.err, limit_ns)) {
+          if (*abort_flag || !mbar_wait(full_bar(s), ph, R.err, limit_ns)) {
             *abort_flag = 1;
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = base + xs * A_BYTES, sb = wring + ws * C::W_BYTES;
+          const uint32_t sa = base + s * C::STAGE_BYTES, sb = sa + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             tc_mma_f16(tmem_base + buf * C::ACC, desc_kmajor_sw128(sa + kk * 32u),
                        desc_kmajor_sw128(sb + kk * 32u), idesc_router<3 * EP>(), !(seg_first && kk == 0));
-          tc_commit(xempty_bar(xs));
-          tc_commit(wempty_bar(ws));
+          tc_commit(empty_bar(s));
           if (seg_last) {
             tc_commit(tfull_bar(buf));
             ++g;
           }
-          if (++xs == XS) {
-            xs = 0;
-            xph ^= 1u;
-          }
-          if (++ws == WS) {
-            ws = 0;
-            wph ^= 1u;
+          if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
           }
         }
       }
@@ -792,9 +778,9 @@ __global__ void __launch_bounds__(512, 1)
       if (ok) mbar_arrive(lfull_bar(i & 1));          // the tile's logits (without bias) are in `run`
     }
   } else {
-    // ------------------------------------------------------------ routing group (warps 7..15)
-    constexpr int NR = C::NT - 224;                   // 288 threads
-    const int tr = threadIdx.x - 224, wr = tr >> 5;
+    // ------------------------------------------------------------ routing group (warps 6..15)
+    constexpr int NR = C::NT - 192;                   // 320 threads
+    const int tr = threadIdx.x - 192, wr = tr >> 5;
     for (int i = 0; i < ntiles; ++i) {
       const int ca = c0 + 2 * i;
       const int nch = ca + 1 >= c1 ? 1 : 2;
@@ -808,7 +794,7 @@ __global__ void __launch_bounds__(512, 1)
         break;                                        // uniform: every thread read the same flag
       }
       tc_fence_after();
-      if (wr < 4) {                                   // warps 7..10 cover the four TMEM lane groups
+      if (wr < 4) {                                   // warps 6..9 cover the four TMEM lane groups
         const int qq = warp & 3, row = qq * 32 + lane;
         const uint32_t run = tmem_base + ((uint32_t)(qq * 32) << 16) + C::RUN0 + (uint32_t)(i & 1) * EP;
 #pragma unroll 1
@@ -1029,14 +1015,15 @@ int sm_count() {
 
 template <int EP>
 cudaError_t launch_persistent(const CUtensorMap& tmX, const CUtensorMap& tmX64, const CUtensorMap& tmW,
-                              const float* bias, int S, int M, int E, int k, const Routing& R,
+                              const void* x, const float* bias, int S, int M, int E, int k, const Routing& R,
                               uint64_t limit_ns, int grid, cudaStream_t st) {
   using C = PCfg<EP>;
   auto kern = router_tcp_kernel<EP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int nchunk = (S + kChunk - 1) / kChunk;
-  kern<<<grid, C::NT, C::SMEM, st>>>(tmX, tmX64, tmW, bias, S, M, E, k, nchunk, R, limit_ns);
+  kern<<<grid, C::NT, C::SMEM, st>>>(tmX, tmX64, tmW, static_cast<const __nv_bfloat16*>(x), bias, S, M, E,
+                                     k, nchunk, R, limit_ns);
   return cudaGetLastError();
 }
 
@@ -1084,13 +1071,13 @@ bool router_persistent(int E, int S) {
   return router_tc_pad(E) <= 64 && (S + kChunk - 1) / kChunk >= 4 * sm_count();
 }
 
-cudaError_t launch_router_tc(const CUtensorMap& tmX, const CUtensorMap* tmX64, const CUtensorMap& tmW,
-                             const float* bias, int S, int M, int E, int k, const Routing& R,
-                             uint64_t limit_ns, cudaStream_t st) {
-  if (tmX64 && router_persistent(E, S)) {
+cudaError_t launch_router_tc(const CUtensorMap& tmX, const CUtensorMap* tmX64, const void* x,
+                             const CUtensorMap& tmW, const float* bias, int S, int M, int E, int k,
+                             const Routing& R, uint64_t limit_ns, cudaStream_t st) {
+  if (tmX64 && x && router_persistent(E, S)) {
     if (router_tc_pad(E) == 32)
-      return launch_persistent<32>(tmX, *tmX64, tmW, bias, S, M, E, k, R, limit_ns, sm_count(), st);
-    return launch_persistent<64>(tmX, *tmX64, tmW, bias, S, M, E, k, R, limit_ns, sm_count(), st);
+      return launch_persistent<32>(tmX, *tmX64, tmW, x, bias, S, M, E, k, R, limit_ns, sm_count(), st);
+    return launch_persistent<64>(tmX, *tmX64, tmW, x, bias, S, M, E, k, R, limit_ns, sm_count(), st);
   }
   switch (router_tc_pad(E)) {
     case 32: return launch_t<32>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);

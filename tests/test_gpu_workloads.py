@@ -38,7 +38,8 @@ def _expert_rows_check(run, out, rt, e):
     got_x = run.layer.expert_rows(L.MOE_BUF_X, e, n)
     assert torch.equal(got_x, xs), "dispatched rows"
     W1e, W2e = run.W1[e].cpu(), run.W2[e].cpu()
-    h_ref = np.maximum(O._f64(xs.cpu()) @ O._f64(W1e), 0.0)
+    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+    h_ref = np.maximum(f64(xs) @ f64(W1e), 0.0)
     y_ref = O.expert_ffn(xs.cpu(), W1e, W2e)
     e_h = G.rel_err(run.layer.expert_rows(L.MOE_BUF_H, e, n).float().cpu().numpy(), h_ref)
     e_y = G.rel_err(run.layer.expert_rows(L.MOE_BUF_Y, e, n).float().cpu().numpy(), y_ref)
