@@ -93,12 +93,6 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int c0, int
                : "memory");
 }
 
-// Bring `bytes` (a multiple of 16; p 16-byte aligned) of contiguous global memory into L2.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
-               : "memory");
-}
-
 // Shared -> global tile store through a tensor map; completes asynchronously (bulk group).
 __device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int c0, int c1) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(

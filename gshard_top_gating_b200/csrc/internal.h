@@ -81,7 +81,7 @@ bool make_router_xmap64(CUtensorMap* tm, const void* x, int S, int M);
 // whether S tokens with E experts take the persistent router (E <= 64 and at least four
 // 64-token chunks per SM), which needs the 64-row x map as well
 bool router_persistent(int E, int S);
-// x: the token rows (the persistent router prefetches the next tile's rows into L2)
+// x: the token rows themselves (unused by the current kernels; the maps describe them)
 cudaError_t launch_router_tc(const CUtensorMap& tmX, const CUtensorMap* tmX64, const void* x,
                              const CUtensorMap& tmW, const float* bias, int S, int M, int E, int k,
                              const Routing& R, uint64_t limit_ns, cudaStream_t st);

@@ -537,11 +537,6 @@ __global__ void __launch_bounds__(NW * 32, (NW == 8) ? 2 : 1)
 // The arithmetic of every logit, probability, gate and table entry is that of
 // router_tc_kernel.  TMEM: two segment accumulators (3*EP columns each) and two
 // running sums (EP each) -- 448 of 512 columns for EP = 64.
-// A tile's TMA boxes read 128 bytes of each token row per k-block, rows 2M bytes
-// apart; from DRAM that pattern wastes much of each page it opens.  So while tile i
-// is multiplied, the producer brings tile i+1's token rows into L2 as whole
-// contiguous rows (a bulk prefetch of a few rows per k-block), and tile i+1's boxes
-// then come from L2.
 template <int EP>
 struct PCfg {
   static constexpr int NT = 512;
@@ -575,9 +570,8 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 template <int EP>
 __global__ void __launch_bounds__(512, 1)
     router_tcp_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmX64,
-                      const __grid_constant__ CUtensorMap tmW, const __nv_bfloat16* __restrict__ xraw,
-                      const float* __restrict__ bias, int S, int M, int E, int k, int nchunk, Routing R,
-                      uint64_t limit_ns) {
+                      const __grid_constant__ CUtensorMap tmW, const float* __restrict__ bias, int S, int M,
+                      int E, int k, int nchunk, Routing R, uint64_t limit_ns) {
   using C = PCfg<EP>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -647,14 +641,7 @@ __global__ void __launch_bounds__(512, 1)
         const bool half = ca + 1 >= c1;
         const int tok0 = ca * kChunk;
         const uint32_t tx = (half ? 64u : 128u) * BK * 2 + 3 * C::PART_BYTES;
-        // the next tile's rows, a slice per k-block, into L2 as whole rows
-        const int cn = ca + 2;
-        const int ntok_next = i + 1 < ntiles ? min((cn + 1 >= c1 ? 1 : 2) * kChunk, S - cn * kChunk) : 0;
-        const int rows_per_kb = (ntok_next + KB - 1) / KB;
         for (int kb = 0; kb < KB; ++kb) {
-          const int r0 = kb * rows_per_kb, r1 = min(ntok_next, r0 + rows_per_kb);
-          if (r1 > r0)
-            bulk_prefetch_l2(xraw + (int64_t)(cn * kChunk + r0) * M, (uint32_t)((r1 - r0) * M * 2));
           if (*abort_flag || !mbar_wait(empty_bar(s), ph ^ 1u, R.err, limit_ns)) {
             *abort_flag = 1;
             ok = false;
@@ -1015,15 +1002,14 @@ int sm_count() {
 
 template <int EP>
 cudaError_t launch_persistent(const CUtensorMap& tmX, const CUtensorMap& tmX64, const CUtensorMap& tmW,
-                              const void* x, const float* bias, int S, int M, int E, int k, const Routing& R,
+                              const float* bias, int S, int M, int E, int k, const Routing& R,
                               uint64_t limit_ns, int grid, cudaStream_t st) {
   using C = PCfg<EP>;
   auto kern = router_tcp_kernel<EP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int nchunk = (S + kChunk - 1) / kChunk;
-  kern<<<grid, C::NT, C::SMEM, st>>>(tmX, tmX64, tmW, static_cast<const __nv_bfloat16*>(x), bias, S, M, E,
-                                     k, nchunk, R, limit_ns);
+  kern<<<grid, C::NT, C::SMEM, st>>>(tmX, tmX64, tmW, bias, S, M, E, k, nchunk, R, limit_ns);
   return cudaGetLastError();
 }
 
@@ -1074,10 +1060,11 @@ bool router_persistent(int E, int S) {
 cudaError_t launch_router_tc(const CUtensorMap& tmX, const CUtensorMap* tmX64, const void* x,
                              const CUtensorMap& tmW, const float* bias, int S, int M, int E, int k,
                              const Routing& R, uint64_t limit_ns, cudaStream_t st) {
-  if (tmX64 && x && router_persistent(E, S)) {
+  (void)x;
+  if (tmX64 && router_persistent(E, S)) {
     if (router_tc_pad(E) == 32)
-      return launch_persistent<32>(tmX, *tmX64, tmW, x, bias, S, M, E, k, R, limit_ns, sm_count(), st);
-    return launch_persistent<64>(tmX, *tmX64, tmW, x, bias, S, M, E, k, R, limit_ns, sm_count(), st);
+      return launch_persistent<32>(tmX, *tmX64, tmW, bias, S, M, E, k, R, limit_ns, sm_count(), st);
+    return launch_persistent<64>(tmX, *tmX64, tmW, bias, S, M, E, k, R, limit_ns, sm_count(), st);
   }
   switch (router_tc_pad(E)) {
     case 32: return launch_t<32>(tmX, tmW, bias, S, M, E, k, R, limit_ns, st);
