@@ -14,6 +14,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "losses.cuh"
 
 namespace moe {
 
@@ -230,16 +231,24 @@ struct Vec<float> {
   }
 };
 
+// loss_blocks = 1: the grid's last block computes the auxiliary losses instead of
+// combining tokens (the router's partials are long complete by then).
 template <typename T, int KM>
 __global__ void __launch_bounds__(kThreads, KM >= 8 ? 3 : 4) combine_kernel(const T* __restrict__ ybuf, int S, int M,
                                                               int k, int64_t Cbuf, Routing R,
-                                                              T* __restrict__ y) {
+                                                              T* __restrict__ y, int loss_blocks, int E,
+                                                              int nchunk) {
+  static_assert(kThreads == kLossThreads, "the loss block runs with the combine's block size");
   const int lane = threadIdx.x & 31;
-  const int warps = (gridDim.x * kThreads) >> 5;
+  const int warps = ((gridDim.x - loss_blocks) * kThreads) >> 5;
   const int nv = (int)((int64_t)M * sizeof(T) / 16);
   constexpr int U = KM >= 4 ? 1 : 2;          // 16-byte vectors per lane per step
   pdl_trigger();
   pdl_wait();                                  // expert outputs complete
+  if (loss_blocks && blockIdx.x == gridDim.x - 1) {
+    aux_loss_block(S, E, nchunk, R);
+    return;
+  }
   for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < S; t += warps) {
     int e = 0, s = -1;
     float g = 0.f;
@@ -415,9 +424,10 @@ void dispatch_t(const void* x, int S, int M, int E, int k, int C, int64_t Cbuf, 
 
 template <typename T, int KM>
 void combine_t(const void* ybuf, int S, int M, int k, int64_t Cbuf, const Routing& R, void* y,
-               int grid, cudaStream_t st) {
-  launch_pdl(combine_kernel<T, KM>, dim3(grid), dim3(kThreads), 0, st, (const T*)ybuf, S, M, k, Cbuf,
-             R, (T*)y);
+               int grid, cudaStream_t st, int loss_blocks, int E) {
+  const int nchunk = (S + kChunk - 1) / kChunk;
+  launch_pdl(combine_kernel<T, KM>, dim3(grid + loss_blocks), dim3(kThreads), 0, st, (const T*)ybuf, S, M,
+             k, Cbuf, R, (T*)y, loss_blocks, E, nchunk);
 }
 
 template <typename T>
@@ -431,11 +441,11 @@ void dispatch_k(int k, const void* x, int S, int M, int E, int C, int64_t Cbuf, 
 
 template <typename T>
 void combine_k(int k, const void* ybuf, int S, int M, int64_t Cbuf, const Routing& R, void* y,
-               int grid, cudaStream_t st) {
-  if (k <= 1) combine_t<T, 1>(ybuf, S, M, k, Cbuf, R, y, grid, st);
-  else if (k <= 2) combine_t<T, 2>(ybuf, S, M, k, Cbuf, R, y, grid, st);
-  else if (k <= 4) combine_t<T, 4>(ybuf, S, M, k, Cbuf, R, y, grid, st);
-  else combine_t<T, 8>(ybuf, S, M, k, Cbuf, R, y, grid, st);
+               int grid, cudaStream_t st, int loss_blocks, int E) {
+  if (k <= 1) combine_t<T, 1>(ybuf, S, M, k, Cbuf, R, y, grid, st, loss_blocks, E);
+  else if (k <= 2) combine_t<T, 2>(ybuf, S, M, k, Cbuf, R, y, grid, st, loss_blocks, E);
+  else if (k <= 4) combine_t<T, 4>(ybuf, S, M, k, Cbuf, R, y, grid, st, loss_blocks, E);
+  else combine_t<T, 8>(ybuf, S, M, k, Cbuf, R, y, grid, st, loss_blocks, E);
 }
 
 }  // namespace
@@ -522,12 +532,13 @@ cudaError_t launch_ep_repack(const void* ybuf, bool bf16, int nrows, int M, cons
 }
 
 cudaError_t launch_combine(const void* ybuf, bool bf16, int S, int M, int k, int64_t Cbuf,
-                           const Routing& R, void* y, cudaStream_t st) {
+                           const Routing& R, void* y, cudaStream_t st, bool with_losses, int E) {
   const int grid = grid_for(S);
+  const int lb = with_losses ? 1 : 0;
   if (bf16)
-    combine_k<__nv_bfloat16>(k, ybuf, S, M, Cbuf, R, y, grid, st);
+    combine_k<__nv_bfloat16>(k, ybuf, S, M, Cbuf, R, y, grid, st, lb, E);
   else
-    combine_k<float>(k, ybuf, S, M, Cbuf, R, y, grid, st);
+    combine_k<float>(k, ybuf, S, M, Cbuf, R, y, grid, st, lb, E);
   return cudaGetLastError();
 }
 

@@ -116,7 +116,9 @@ __device__ __forceinline__ uint32_t positive_bits(const uint4 (&v)[4]) {
 // Epilogue of one warp's 32 accumulator rows x BN columns: TMEM -> bf16 (+ReLU or
 // mask) -> a 4 KB staging tile in shared memory laid out as the store tensor map's
 // 128-byte swizzle (row r, 16-byte chunk c at r*128 + ((c ^ (r % 8)) * 16)) -> one TMA
-// store per 64 columns.  Rows past n_e land in the expert's own padding rows (rows
+// store per 64 columns, under an L2 evict-first policy: a GEMM's output is far larger
+// than L2 and read by the next kernel, so it should not push out the operand strips
+// that this kernel's other tiles are about to read again.  Rows past n_e land in the expert's own padding rows (rows
 // per expert are a multiple of 128), which nothing reads as data.  The TMA engine
 // writes whole 128-byte rows, instead of each thread storing 16 bytes to 32
 // different rows per instruction.  `mrow` (kEpiMask) points at this lane's row of h
@@ -196,7 +198,7 @@ __device__ __forceinline__ void store_rows(const CUtensorMap* tmD, uint32_t tmem
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_store_2d(tmD, stage, col0 + b * 32, row0);
+        tma_store_2d_hint(tmD, stage, col0 + b * 32, row0, l2_policy_evict_first());
         bulk_commit();
       }
     }
@@ -272,7 +274,7 @@ __device__ __forceinline__ void store_rows(const CUtensorMap* tmD, uint32_t tmem
     fence_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(tmD, stage, col0 + b * 64, row0);
+      tma_store_2d_hint(tmD, stage, col0 + b * 64, row0, l2_policy_evict_first());
       bulk_commit();
     }
   }

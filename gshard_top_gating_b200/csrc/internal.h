@@ -86,7 +86,9 @@ cudaError_t launch_router_tc(const CUtensorMap& tmX, const CUtensorMap* tmX64, c
                              const CUtensorMap& tmW, const float* bias, int S, int M, int E, int k,
                              const Routing& R, uint64_t limit_ns, cudaStream_t st);
 // scan.cu
-cudaError_t launch_scan(int S, int E, int k, int C, int64_t Cbuf, const Routing& R, cudaStream_t st);
+// with_losses: one more block computes the auxiliary losses (else the combine does)
+cudaError_t launch_scan(int S, int E, int k, int C, int64_t Cbuf, const Routing& R, cudaStream_t st,
+                        bool with_losses = true);
 // scan.cu, expert parallelism: per-rank scan of one rank's tokens.  off[r][c][e] gets the
 // exclusive prefix of hist[r][.][e] over chunks; stats (doubles, ep_stats_len(E, k)):
 // [r*E + e] rank-r demand of expert e, [k*E + j] sum over tokens of p_tj,
@@ -129,8 +131,10 @@ cudaError_t launch_dispatch(const void* x, bool bf16, int S, int M, int E, int k
 cudaError_t launch_dispatch_fused(const void* x, int S, int M, int E, int C, int64_t Cbuf,
                                   const Routing& R, void* xbuf, int32_t* tok, float* gsc, void* y,
                                   cudaStream_t st);
+// with_losses: one more block computes the auxiliary losses (E experts) beside the combine
 cudaError_t launch_combine(const void* ybuf, bool bf16, int S, int M, int k, int64_t Cbuf,
-                           const Routing& R, void* y, cudaStream_t st);
+                           const Routing& R, void* y, cudaStream_t st, bool with_losses = false,
+                           int E = 0);
 // ffn_simt.cu  (fp32 activations)
 cudaError_t launch_ffn_f32(const float* A, const float* B, float* D, const int32_t* nexp, int E,
                            int64_t Cbuf, int K, int N, bool relu, cudaStream_t st);

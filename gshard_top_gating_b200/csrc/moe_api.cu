@@ -384,18 +384,20 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
     MOE_TRY(launch_router(x, bf16, h->Wg, h->bias, iS, iM, h->E, h->k, R, st));
   }
   MOE_TRY(mark(1));
-  MOE_TRY(launch_scan(iS, h->E, h->k, C, h->Cbuf, R, st));
   const bool reroute = (h->route_flags & MOE_ROUTE_REROUTE) != 0;
+  // top-1 inference: the combine is fused into the second expert GEMM, whose epilogue
+  // stores each row straight into y (the backward needs the expert outputs, so a
+  // handle in training mode keeps the separate combine)
+  const bool fused = fuses_combine(h) && !reroute;
+  // the losses are computed beside the combine, off the dispatch's critical path, or in
+  // the scan when no combine kernel runs
+  MOE_TRY(launch_scan(iS, h->E, h->k, C, h->Cbuf, R, st, fused));
   h->last_rerouted = reroute;
   if (reroute) {       // second chance for dropped choices: offers, their scan
     MOE_TRY(launch_reroute_offers(iS, h->E, h->k, (int)(C < h->Cbuf ? C : h->Cbuf), R, st));
     MOE_TRY(launch_reroute_scan(iS, h->E, h->k, C, h->Cbuf, R, st));
   }
   MOE_TRY(mark(2));
-  // top-1 inference: the combine is fused into the second expert GEMM, whose epilogue
-  // stores each row straight into y (the backward needs the expert outputs, so a
-  // handle in training mode keeps the separate combine)
-  const bool fused = fuses_combine(h) && !reroute;
   h->last_fused = fused;
   if (fused)
     MOE_TRY(launch_dispatch_fused(x, iS, iM, h->E, C, h->Cbuf, R, h->xbuf, h->slot_tok, h->slot_gate, y, st));
@@ -428,7 +430,7 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
   if (!fused) {
     Routing Rc = R;
     if (reroute) Rc.eidx = R.dest;     // combine from the expert that served each choice
-    MOE_TRY(launch_combine(h->ybuf, bf16, iS, iM, h->k, h->Cbuf, Rc, y, st));
+    MOE_TRY(launch_combine(h->ybuf, bf16, iS, iM, h->k, h->Cbuf, Rc, y, st, true, h->E));
   }
   MOE_TRY(mark(6));
   return MOE_OK;

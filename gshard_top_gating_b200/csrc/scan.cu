@@ -15,6 +15,7 @@
 // Partials are summed in a fixed order in double, so results are deterministic.
 #include "common.cuh"
 #include "internal.h"
+#include "losses.cuh"
 
 namespace moe {
 
@@ -47,23 +48,10 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int& 
   return before + x - v;
 }
 
-__device__ __forceinline__ double block_sum_f64(double v, double* sm) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if (lane == 0) sm[warp] = v;
-  __syncthreads();
-  double s = 0.0;
-#pragma unroll
-  for (int w = 0; w < kThreads / 32; ++w) s += sm[w];
-  __syncthreads();
-  return s;
-}
-
 __global__ void __launch_bounds__(kThreads) scan_kernel(int S, int E, int k, int C, int Cbuf,
                                                         int nchunk, Routing R) {
+  static_assert(kThreads == kLossThreads, "the loss block runs with the scan's block size");
   __shared__ int warp_sums[kThreads / 32];
-  __shared__ double dsum[kThreads / 32];
   const int tid = threadIdx.x;
   pdl_trigger();
   pdl_wait();                                  // router tables complete
@@ -86,43 +74,8 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(int S, int E, int k, int
     }
     return;
   }
-  // block E: auxiliary losses.  G threads share each expert column j, thread
-  // (j, g) summing chunks g, g+G, ...; the G partials are then added in order.
-  __shared__ double part_P[kThreads];
-  __shared__ long long part_f[kThreads];
-  const int G = E >= kThreads ? 1 : kThreads / E;
-  if (tid < E * G) {
-    const int j = tid % E, g = tid / E;
-    double P = 0.0;
-    long long f = 0;
-    for (int c = g; c < nchunk; c += G) {
-      P += (double)R.psum[(int64_t)c * E + j];
-      f += R.hist[(int64_t)c * E + j];          // rank-0 plane of hist: first choices
-    }
-    part_P[tid] = P;
-    part_f[tid] = f;
-  }
-  __syncthreads();
-  double term = 0.0;
-  for (int j = tid; j < E; j += kThreads) {
-    double P = 0.0;
-    long long f = 0;
-    for (int g = 0; g < G; ++g) {
-      P += part_P[g * E + j];
-      f += part_f[g * E + j];
-    }
-    term += (double)f * P;
-    R.first[j] = (int32_t)f;                   // kept for the backward's d l_aux / d logits
-  }
-  const double fp = block_sum_f64(term, dsum);
-  double zl = 0.0;
-  for (int c = tid; c < nchunk; c += kThreads) zl += (double)R.lse2[c];
-  const double zs = block_sum_f64(zl, dsum);
-  if (tid == 0) {
-    const double Sd = (double)S;
-    R.losses[0] = (float)((double)E * fp / (Sd * Sd));
-    R.losses[1] = (float)(zs / Sd);
-  }
+  // block E (launched when no combine kernel follows): the auxiliary losses
+  aux_loss_block(S, E, nchunk, R);
 }
 
 // Expert parallelism: the scan of one rank's own tokens.  Block e (< E): for every
@@ -217,10 +170,12 @@ cudaError_t launch_ep_scan(int S, int E, int k, const Routing& R, double* stats,
   return launch_pdl(ep_scan_kernel, dim3(E + 1), dim3(kThreads), 0, st, S, E, k, nchunk, R, stats);
 }
 
-cudaError_t launch_scan(int S, int E, int k, int C, int64_t Cbuf, const Routing& R, cudaStream_t st) {
+cudaError_t launch_scan(int S, int E, int k, int C, int64_t Cbuf, const Routing& R, cudaStream_t st,
+                        bool with_losses) {
   const int nchunk = (S + kChunk - 1) / kChunk;
   const int cb = Cbuf < 0x7fffffff ? (int)Cbuf : 0x7fffffff;
-  return launch_pdl(scan_kernel, dim3(E + 1), dim3(kThreads), 0, st, S, E, k, C, cb, nchunk, R);
+  return launch_pdl(scan_kernel, dim3(E + (with_losses ? 1 : 0)), dim3(kThreads), 0, st, S, E, k, C, cb,
+                    nchunk, R);
 }
 
 }  // namespace moe
