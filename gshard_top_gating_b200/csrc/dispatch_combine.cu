@@ -231,8 +231,9 @@ struct Vec<float> {
   }
 };
 
-// loss_blocks = 1: the grid's last block computes the auxiliary losses instead of
-// combining tokens (the router's partials are long complete by then).
+// loss_blocks = 1: the grid's first block computes the auxiliary losses instead of
+// combining tokens (the router's partials are long complete by then); being first,
+// it is resident from the start and runs beside the token blocks.
 template <typename T, int KM>
 __global__ void __launch_bounds__(kThreads, KM >= 8 ? 3 : 4) combine_kernel(const T* __restrict__ ybuf, int S, int M,
                                                               int k, int64_t Cbuf, Routing R,
@@ -241,15 +242,16 @@ __global__ void __launch_bounds__(kThreads, KM >= 8 ? 3 : 4) combine_kernel(cons
   static_assert(kThreads == kLossThreads, "the loss block runs with the combine's block size");
   const int lane = threadIdx.x & 31;
   const int warps = ((gridDim.x - loss_blocks) * kThreads) >> 5;
+  const int blk = blockIdx.x - loss_blocks;    // this block's index among the token blocks
   const int nv = (int)((int64_t)M * sizeof(T) / 16);
   constexpr int U = KM >= 4 ? 1 : 2;          // 16-byte vectors per lane per step
   pdl_trigger();
   pdl_wait();                                  // expert outputs complete
-  if (loss_blocks && blockIdx.x == gridDim.x - 1) {
+  if (blk < 0) {
     aux_loss_block(S, E, nchunk, R);
     return;
   }
-  for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < S; t += warps) {
+  for (int t = (blk * kThreads + threadIdx.x) >> 5; t < S; t += warps) {
     int e = 0, s = -1;
     float g = 0.f;
     if (lane < k) {
