@@ -535,8 +535,10 @@ cudaError_t launch_ep_repack(const void* ybuf, bool bf16, int nrows, int M, cons
 
 cudaError_t launch_combine(const void* ybuf, bool bf16, int S, int M, int k, int64_t Cbuf,
                            const Routing& R, void* y, cudaStream_t st, bool with_losses, int E) {
-  const int grid = grid_for(S);
+  // with the loss block, one token block fewer: grid_for fills the SMs' resident slots
+  // exactly, and a block past them would run alone after the others
   const int lb = with_losses ? 1 : 0;
+  const int grid = grid_for(S) > 1 ? grid_for(S) - lb : grid_for(S);
   if (bf16)
     combine_k<__nv_bfloat16>(k, ybuf, S, M, Cbuf, R, y, grid, st, lb, E);
   else

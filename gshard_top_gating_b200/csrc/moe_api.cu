@@ -106,6 +106,11 @@ bool fuses_combine(const moe_layer* h) { return h->slot_tok != nullptr && !h->bw
 // one-CTA tiles for a last block of at most 128 rows (else 128-row tiles throughout).
 constexpr bool kMixedTiles = false;
 
+// Token rows x model width from which the combine (which moves about 3 bytes per element)
+// outlasts the loss block, so summing the losses beside it costs nothing; below that the
+// scan keeps them (measured: beside the skewed workload's 12 us combine, 16 us).
+constexpr double kLossBesideCombine = 33554432.0;
+
 size_t act_bytes(moe_dtype a) { return a == MOE_BF16 ? 2 : 4; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -389,9 +394,10 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
   // stores each row straight into y (the backward needs the expert outputs, so a
   // handle in training mode keeps the separate combine)
   const bool fused = fuses_combine(h) && !reroute;
-  // the losses are computed beside the combine, off the dispatch's critical path, or in
-  // the scan when no combine kernel runs
-  MOE_TRY(launch_scan(iS, h->E, h->k, C, h->Cbuf, R, st, fused));
+  // the losses are summed beside a long combine, off the dispatch's critical path;
+  // beside a short one (or without one) they stay in the scan
+  const bool loss_in_combine = !fused && (double)S * h->M >= kLossBesideCombine;
+  MOE_TRY(launch_scan(iS, h->E, h->k, C, h->Cbuf, R, st, !loss_in_combine));
   h->last_rerouted = reroute;
   if (reroute) {       // second chance for dropped choices: offers, their scan
     MOE_TRY(launch_reroute_offers(iS, h->E, h->k, (int)(C < h->Cbuf ? C : h->Cbuf), R, st));
@@ -430,7 +436,7 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
   if (!fused) {
     Routing Rc = R;
     if (reroute) Rc.eidx = R.dest;     // combine from the expert that served each choice
-    MOE_TRY(launch_combine(h->ybuf, bf16, iS, iM, h->k, h->Cbuf, Rc, y, st, true, h->E));
+    MOE_TRY(launch_combine(h->ybuf, bf16, iS, iM, h->k, h->Cbuf, Rc, y, st, loss_in_combine, h->E));
   }
   MOE_TRY(mark(6));
   return MOE_OK;
