@@ -307,7 +307,7 @@ def measure_copies(args, x, xh, yh, stream):
             "h2d_GBps": round(nbytes / h2d / 1e6, 1), "d2h_GBps": round(nbytes / d2h / 1e6, 1)}
 
 
-def measure_backward(args, w, weights, x, y, flush, stream, pk, A, n_e):
+def measure_backward(args, w, weights, x, y, flush, stream, pk, pk_kind, A, n_e):
     """One training step = moe_forward + moe_backward of the same tokens, device-timed.
 
     On a handle of its own, in training mode from its first forward (the backward
@@ -379,7 +379,7 @@ def measure_backward(args, w, weights, x, y, flush, stream, pk, A, n_e):
         "expert_gemm_TFLOP/s": round(4 * 2.0 * A * w.M * w.H / (ffn / 1e3) / 1e12, 1) if ffn > 0 else None,
         "roofline": {"bound": b_, "kernel": dom, "achieved": round(ach, 2), "peak": peak, "unit": unit,
                      "frac": round(ach / peak, 4),
-                     "peak_source": "measured, burst" if b_ == "tensor" else "measured",
+                     "peak_source": f"{pk_kind}, burst" if b_ == "tensor" else pk_kind,
                      "frac_of_sustained": (round(ach / pk["bf16_tflops_sustained"], 4)
                                            if b_ == "tensor" and pk.get("bf16_tflops_sustained") else None)},
         "stages": stages,
@@ -557,7 +557,7 @@ def measure_workload(args, w, dev, world, flush, pk, pk_kind, headline):
                   "ms_per_step": round(e2e_ms / args.steps, 4), "copies_alone": copies}
     out["clocks"] = clocks
     out["train_step"] = (None if args.no_backward
-                         else measure_backward(args, w, (Wg, b, W1, W2), x, y, flush, stream, pk, A, n_e))
+                         else measure_backward(args, w, (Wg, b, W1, W2), x, y, flush, stream, pk, pk_kind, A, n_e))
     layer.close()
     out["_inputs"] = (x, Wg, b, W1, W2)
     return out
