@@ -73,6 +73,9 @@ def _load() -> ctypes.CDLL:
         "moe_ep_route": [P, I64, P, P, P],
         "moe_ep_dispatch": [P, P, P, P, P, P, P],
         "moe_ep_experts": [P, P, P],
+        "moe_ep_experts_phase": [P, P, I32, P],
+        "moe_ep_set_phases": [P, I32],
+        "moe_ep_phase_plan": [I32, I32, I32, I32, D, P, P, I32, P, P, P],
         "moe_ep_combine": [P, P, P, P],
         "moe_ep_aux_loss": [P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)],
         "moe_ep_get_routing": [P, P, P, P, P, P, P],
@@ -292,15 +295,40 @@ def moe_ep_route(h, S, x, stats, stream=None) -> None:
     _check("moe_ep_route", lib.moe_ep_route(h, S, _ptr(x), _ptr(stats), _stream(stream)))
 
 
-def moe_ep_dispatch(h, stats_all, x, sendbuf, G, stream=None):
-    """stats_all: numpy float64 [G, stats_len]; returns (send_rows[G], recv_rows[G]) int64."""
+def moe_ep_dispatch(h, stats_all, x, sendbuf, G, stream=None, phases=1):
+    """stats_all: numpy float64 [G, stats_len]; returns (send_rows, recv_rows) int64, each
+    [G] with one phase or [phases, G] (the handle's phase count must be `phases`)."""
     import numpy as np
     st = np.ascontiguousarray(stats_all, dtype=np.float64)
-    send = np.zeros(G, dtype=np.int64)
-    recv = np.zeros(G, dtype=np.int64)
+    send = np.zeros(phases * G, dtype=np.int64)
+    recv = np.zeros(phases * G, dtype=np.int64)
     _check("moe_ep_dispatch", lib.moe_ep_dispatch(h, _np_ptr(st), _ptr(x), _ptr(sendbuf), _np_ptr(send),
                                                   _np_ptr(recv), _stream(stream)))
-    return send, recv
+    if phases == 1:
+        return send, recv
+    return send.reshape(phases, G), recv.reshape(phases, G)
+
+
+def moe_ep_set_phases(h, phases: int) -> None:
+    _check("moe_ep_set_phases", lib.moe_ep_set_phases(h, phases))
+
+
+def moe_ep_experts_phase(h, recvbuf, phase: int, stream=None) -> None:
+    _check("moe_ep_experts_phase", lib.moe_ep_experts_phase(h, _ptr(recvbuf), phase, _stream(stream)))
+
+
+def moe_ep_phase_plan(G, g, E, k, capacity_factor, counts, S, phases):
+    """Per-phase row counts of rank g: (send_rows[phases, G], recv_rows[phases, G], split[E])."""
+    import numpy as np
+    cnt = np.ascontiguousarray(counts, dtype=np.int64)
+    Sv = np.ascontiguousarray(S, dtype=np.int64)
+    send = np.zeros((phases, G), dtype=np.int64)
+    recv = np.zeros((phases, G), dtype=np.int64)
+    split = np.zeros(E, dtype=np.int64)
+    _check("moe_ep_phase_plan", lib.moe_ep_phase_plan(G, g, E, k, float(capacity_factor), _np_ptr(cnt),
+                                                      _np_ptr(Sv), phases, _np_ptr(send), _np_ptr(recv),
+                                                      _np_ptr(split)))
+    return send, recv, split
 
 
 def moe_ep_experts(h, recvbuf, stream=None) -> None:

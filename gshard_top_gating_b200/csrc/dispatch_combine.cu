@@ -299,8 +299,10 @@ __global__ void __launch_bounds__(kThreads, KM >= 8 ? 3 : 4) combine_kernel(cons
 // Expert parallelism, sending side: the global rank-major slot of each of the rank's
 // choices is base[r][e] (all earlier ranks' and earlier choice ranks' demand of e, from
 // the exchanged counts) plus the rank-local position off[r][c][e] + lrank.  Kept rows go
-// to the send buffer, where each (expert, rank r) run of this rank's kept choices starts
-// at soff[r][e]; a run's kept choices are a prefix of it, so row = soff + local position.
+// to the send buffer.  A run (this rank's kept choices of rank r at expert e) is a prefix
+// of its choices; its first a0[r][e] rows travel in phase 0 from soff0[r][e], the rest in
+// phase 1 from soff1[r][e] (soff = [soff0 | soff1 | a0], each [k][E]; with one phase,
+// a0 covers the whole run).
 template <typename T, int KM>
 __global__ void __launch_bounds__(kThreads, 4) ep_dispatch_kernel(const T* __restrict__ x, int S, int M,
                                                                   int E, int k, int C, int nchunk,
@@ -320,10 +322,12 @@ __global__ void __launch_bounds__(kThreads, 4) ep_dispatch_kernel(const T* __res
       int s = -1;
       if (e >= 0 && e < E) {
         const int local = R.off[((int64_t)lane * nchunk + t / kChunk) * E + e] + R.lrank[(int64_t)t * k + lane];
-        const int g = base[lane * E + e] + local;
+        const int i = lane * E + e;
+        const int g = base[i] + local;
         if (g < C) {
           s = g;
-          sp = soff[lane * E + e] + local;
+          const int a = soff[2 * k * E + i];
+          sp = local < a ? soff[i] + local : soff[k * E + i] + (local - a);
         }
       } else {
         atomicOr(R.err, DEVERR_BOUNDS);

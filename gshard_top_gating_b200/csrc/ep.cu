@@ -28,6 +28,15 @@
 //   [caller]         all-to-all back (the same counts, reversed)
 //   moe_ep_combine   y[t] = sum_{r kept} g_r * (returned row of (t, r)), r ascending, fp32
 // The losses use the gathered stats: f_j and P_j over the whole batch.
+//
+// Two phases (moe_ep_set_phases): each expert's slots are split at
+//     split_e = 256 * floor((n_e + 256) / 512)   (about half, a whole number of GEMM tiles),
+// slots below it travel in phase 0 and the rest in phase 1.  The send and receive buffers
+// hold the phase-0 rows first, each phase ordered as above, and each phase has its own
+// row counts per peer, so a caller can exchange phase 1 while the experts compute phase 0
+// (moe_ep_experts_phase) and return phase 0 while they compute phase 1.  The rows, their
+// slots and every output are those of the one-phase forward: a GEMM tile never straddles
+// the split.
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
@@ -59,9 +68,13 @@ struct moe_ep_layer {
   void* xbuf;
   void* hbuf;
   void* ybuf;
-  int32_t* plan_dev;     // base [k][E] | soff [k][E] | seg_start [nseg] | seg_dst [nseg] | nexp [El]
+  // base [k][E] | soff0 [k][E] | soff1 [k][E] | a0 [k][E] | seg_start [2][nseg] |
+  // seg_dst [2][nseg] | nexp [2][El] | rowb [2][El]   (per phase: segments, rows, first row)
+  int32_t* plan_dev;
   int32_t* rowmap;       // [El * Cbuf] expert row of each received row
-  int nseg;
+  int nseg;              // received segments per phase: G * El * k
+  int phases;            // 1 or 2
+  int64_t recv_off[2], recv_cnt[2];   // each phase's rows in the receive buffer
   std::vector<int32_t> plan_host;
   GemmPlan plan1, plan2;
   void* wsplit;
@@ -108,6 +121,10 @@ struct Carver {
   }
 };
 
+size_t plan_ints(const moe_ep_layer* h) {
+  return (size_t)4 * h->k * h->E + 4 * (size_t)h->nseg + 4 * (size_t)h->El;
+}
+
 size_t carve(moe_ep_layer* h, char* base) {
   Carver c{base};
   const int64_t S = h->S_max, E = h->E, k = h->k;
@@ -132,7 +149,7 @@ size_t carve(moe_ep_layer* h, char* base) {
   h->xbuf = c.take<char>((size_t)h->El * h->Cbuf * h->M * as);
   h->hbuf = c.take<char>((size_t)h->El * h->Cbuf * h->H * as);
   h->ybuf = c.take<char>((size_t)h->El * h->Cbuf * h->M * as);
-  h->plan_dev = c.take<int32_t>((size_t)2 * k * E + 2 * h->nseg + h->El);
+  h->plan_dev = c.take<int32_t>(plan_ints(h));
   h->rowmap = c.take<int32_t>((size_t)h->El * h->Cbuf);
   h->wsplit = h->act == MOE_BF16 ? c.take<char>((size_t)3 * router_tc_pad(h->E) * h->M * 2) : nullptr;
   return c.off + 256;
@@ -142,10 +159,16 @@ size_t carve(moe_ep_layer* h, char* base) {
 struct Plan {
   int64_t C = 0, S_total = 0;
   std::vector<int64_t> base, kept;           // [G][k][E]
-  std::vector<int64_t> send_rows, recv_rows; // [G]
+  std::vector<int64_t> n, split;             // [E] kept rows of each expert, first phase-1 slot
+  std::vector<int64_t> a0;                   // [G][k][E] leading rows of each run in phase 0
+  std::vector<int64_t> send_rows, recv_rows; // [phases][G]
 };
 
-moe_status make_plan(int G, int g, int E, int k, double cf, const int64_t* cnt, const int64_t* S, Plan& p) {
+int64_t phase_split(int64_t n, int phases) { return phases == 2 ? 256 * ((n + 256) / 512) : n; }
+
+moe_status make_plan(int G, int g, int E, int k, double cf, const int64_t* cnt, const int64_t* S, Plan& p,
+                     int phases = 1) {
+  if (phases != 1 && phases != 2) return MOE_ERR_INVALID_ARG;
   if (G < 1 || g < 0 || g >= G || E < 1 || k < 1 || k > E || (E % G) || !cnt || !S ||
       !(cf > 0.0) || !isfinite(cf))
     return MOE_ERR_INVALID_ARG;
@@ -179,15 +202,32 @@ moe_status make_plan(int G, int g, int E, int k, double cf, const int64_t* cnt, 
         run += cnt[i];
       }
   }
-  p.send_rows.assign(G, 0);
-  p.recv_rows.assign(G, 0);
+  p.n.assign(E, 0);
+  p.split.assign(E, 0);
+  for (int e = 0; e < E; ++e) {
+    for (int q = 0; q < G; ++q)
+      for (int r = 0; r < k; ++r) p.n[e] += p.kept[((size_t)q * k + r) * E + e];
+    p.split[e] = phase_split(p.n[e], phases);
+  }
+  p.a0.assign(n, 0);
   for (int q = 0; q < G; ++q)
     for (int r = 0; r < k; ++r)
       for (int e = 0; e < E; ++e) {
-        const int64_t v = p.kept[((size_t)q * k + r) * E + e];
-        if (q == g) p.send_rows[e / El] += v;          // to the rank that holds expert e
-        if (e / El == g) p.recv_rows[q] += v;          // from rank q, for one of our experts
+        const size_t i = ((size_t)q * k + r) * E + e;
+        const int64_t a = p.split[e] - p.base[i];      // the run's slots below the split
+        p.a0[i] = a <= 0 ? 0 : (a < p.kept[i] ? a : p.kept[i]);
       }
+  p.send_rows.assign((size_t)phases * G, 0);
+  p.recv_rows.assign((size_t)phases * G, 0);
+  for (int ph = 0; ph < phases; ++ph)
+    for (int q = 0; q < G; ++q)
+      for (int r = 0; r < k; ++r)
+        for (int e = 0; e < E; ++e) {
+          const size_t i = ((size_t)q * k + r) * E + e;
+          const int64_t v = ph == 0 ? p.a0[i] : p.kept[i] - p.a0[i];
+          if (q == g) p.send_rows[(size_t)ph * G + e / El] += v;   // to the rank that holds expert e
+          if (e / El == g) p.recv_rows[(size_t)ph * G + q] += v;   // from rank q, for one of our experts
+        }
   return MOE_OK;
 }
 
@@ -209,6 +249,19 @@ moe_status moe_ep_plan(int32_t G, int32_t g, int32_t E, int32_t k, double capaci
   if (recv_rows_host) memcpy(recv_rows_host, p.recv_rows.data(), G * sizeof(int64_t));
   if (base_host) memcpy(base_host, p.base.data(), p.base.size() * sizeof(int64_t));
   if (kept_host) memcpy(kept_host, p.kept.data(), p.kept.size() * sizeof(int64_t));
+  return MOE_OK;
+}
+
+moe_status moe_ep_phase_plan(int32_t G, int32_t g, int32_t E, int32_t k, double capacity_factor,
+                             const int64_t* counts_host, const int64_t* S_host, int32_t phases,
+                             int64_t* send_rows_host, int64_t* recv_rows_host, int64_t* split_host) {
+  Plan p;
+  const moe_status s = make_plan(G, g, E, k, capacity_factor, counts_host, S_host, p, phases);
+  if (s != MOE_OK) return s;
+  const size_t n = (size_t)phases * G;
+  if (send_rows_host) memcpy(send_rows_host, p.send_rows.data(), n * sizeof(int64_t));
+  if (recv_rows_host) memcpy(recv_rows_host, p.recv_rows.data(), n * sizeof(int64_t));
+  if (split_host) memcpy(split_host, p.split.data(), (size_t)E * sizeof(int64_t));
   return MOE_OK;
 }
 
@@ -251,6 +304,7 @@ moe_status moe_ep_create(moe_ep_handle* out, int32_t G, int32_t g, int64_t S_max
   h->W2 = W2_local;
   h->Cbuf = Cbuf;
   h->nseg = G * h->El * k;
+  h->phases = 1;
   h->wait_limit_ns = 2000000000ull;
   cudaError_t ce = cudaGetDevice(&h->device);
   if (ce == cudaSuccess) ce = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
@@ -267,7 +321,7 @@ moe_status moe_ep_create(moe_ep_handle* out, int32_t G, int32_t g, int64_t S_max
   }
   carve(h, static_cast<char*>(h->ws));
   ce = cudaMemset(h->R.err, 0, sizeof(unsigned));
-  if (ce == cudaSuccess) ce = cudaMemset(h->plan_dev, 0, ((size_t)2 * k * E + 2 * h->nseg + h->El) * 4);
+  if (ce == cudaSuccess) ce = cudaMemset(h->plan_dev, 0, plan_ints(h) * 4);
   if (ce != cudaSuccess) {
     cudaFree(h->ws);
     delete h;
@@ -285,8 +339,16 @@ moe_status moe_ep_create(moe_ep_handle* out, int32_t G, int32_t g, int64_t S_max
       return MOE_ERR_CUDA;
     }
   }
-  h->plan_host.assign((size_t)2 * k * E + 2 * h->nseg + h->El, 0);
+  h->plan_host.assign(plan_ints(h), 0);
   *out = h;
+  return MOE_OK;
+}
+
+moe_status moe_ep_set_phases(moe_ep_handle h, int32_t phases) {
+  if (!h || (phases != 1 && phases != 2)) return MOE_ERR_INVALID_ARG;
+  if (phases == 2 && h->act != MOE_BF16) return MOE_ERR_UNSUPPORTED;   // the FFMA GEMMs take no row base
+  h->phases = phases;
+  h->planned = h->computed = false;
   return MOE_OK;
 }
 
@@ -356,51 +418,70 @@ moe_status moe_ep_dispatch(moe_ep_handle h, const double* stats_all_host, const 
   }
   if (Sv[h->g] != h->S) return MOE_ERR_INVALID_ARG;
   Plan p;
-  moe_status s = make_plan(G, h->g, E, k, h->cf, cnt.data(), Sv.data(), p);
+  moe_status s = make_plan(G, h->g, E, k, h->cf, cnt.data(), Sv.data(), p, h->phases);
   if (s != MOE_OK) return s;
   if (p.S_total > h->S_total_max) return MOE_ERR_INVALID_ARG;
   if (h->S > 0 && (!x || !sendbuf || !aligned(x, 16) || !aligned(sendbuf, 16))) return MOE_ERR_INVALID_ARG;
 
-  // device tables: base and send offsets of this rank's runs, the received segments, the
-  // local experts' kept rows
+  // device tables: base, send offsets (per phase) and phase-0 lengths of this rank's runs;
+  // per phase, the received segments and the local experts' rows
+  const size_t kE = (size_t)k * E;
   int32_t* base = h->plan_host.data();
-  int32_t* soff = base + (size_t)k * E;
-  int32_t* seg_start = soff + (size_t)k * E;
-  int32_t* seg_dst = seg_start + h->nseg;
-  int32_t* nexp = seg_dst + h->nseg;
+  int32_t* soff0 = base + kE;
+  int32_t* soff1 = soff0 + kE;
+  int32_t* a0 = soff1 + kE;
+  int32_t* seg_start = a0 + kE;                // [2][nseg]
+  int32_t* seg_dst = seg_start + 2 * (size_t)h->nseg;
+  int32_t* nexp = seg_dst + 2 * (size_t)h->nseg;   // [2][El]
+  int32_t* rowb = nexp + 2 * (size_t)El;
   int64_t pos = 0;
-  for (int e = 0; e < E; ++e)                  // destination ranks ascend with e
-    for (int r = 0; r < k; ++r) {
-      const size_t i = ((size_t)h->g * k + r) * E + e;
-      base[r * E + e] = (int32_t)p.base[i];
-      soff[r * E + e] = (int32_t)pos;
-      pos += p.kept[i];
-    }
-  int64_t rpos = 0;
-  for (int q = 0; q < G; ++q)                  // arrival order: source rank, expert, choice rank
-    for (int el = 0; el < El; ++el)
+  for (int ph = 0; ph < h->phases; ++ph)       // phase 0 rows first; destination ranks ascend with e
+    for (int e = 0; e < E; ++e)
       for (int r = 0; r < k; ++r) {
-        const int e = h->g * El + el;
-        const size_t i = ((size_t)q * k + r) * E + e;
-        const int sq = (q * El + el) * k + r;
-        seg_start[sq] = (int32_t)rpos;
-        seg_dst[sq] = (int32_t)((int64_t)el * h->Cbuf + p.base[i]);
-        rpos += p.kept[i];
+        const size_t i = ((size_t)h->g * k + r) * E + e;
+        if (ph == 0) {
+          base[r * E + e] = (int32_t)p.base[i];
+          a0[r * E + e] = (int32_t)p.a0[i];
+          soff0[r * E + e] = (int32_t)pos;
+          soff1[r * E + e] = 0;
+          pos += p.a0[i];
+        } else {
+          soff1[r * E + e] = (int32_t)pos;
+          pos += p.kept[i] - p.a0[i];
+        }
       }
-  for (int el = 0; el < El; ++el) {
-    int64_t n = 0;
+  int64_t rpos_all = 0;
+  for (int ph = 0; ph < h->phases; ++ph) {     // arrival order in a phase: source rank, expert, choice rank
+    int64_t rpos = 0;
     for (int q = 0; q < G; ++q)
-      for (int r = 0; r < k; ++r) n += p.kept[((size_t)q * k + r) * E + h->g * El + el];
-    nexp[el] = (int32_t)n;
+      for (int el = 0; el < El; ++el)
+        for (int r = 0; r < k; ++r) {
+          const int e = h->g * El + el;
+          const size_t i = ((size_t)q * k + r) * E + e;
+          const size_t sq = (size_t)ph * h->nseg + ((size_t)q * El + el) * k + r;
+          const int64_t lead = ph == 0 ? 0 : p.a0[i];
+          seg_start[sq] = (int32_t)rpos;
+          seg_dst[sq] = (int32_t)((int64_t)el * h->Cbuf + p.base[i] + lead);
+          rpos += ph == 0 ? p.a0[i] : p.kept[i] - p.a0[i];
+        }
+    h->recv_off[ph] = rpos_all;
+    h->recv_cnt[ph] = rpos;
+    rpos_all += rpos;
+    for (int el = 0; el < El; ++el) {
+      const int e = h->g * El + el;
+      nexp[(size_t)ph * El + el] = (int32_t)(ph == 0 ? p.split[e] : p.n[e] - p.split[e]);
+      rowb[(size_t)ph * El + el] = (int32_t)(ph == 0 ? 0 : p.split[e]);
+    }
   }
+  const int64_t rpos = rpos_all;
   // from pageable memory: the call returns once the table is staged, so the host copy
   // may be rewritten by the next dispatch
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   EP_TRY(cudaMemcpyAsync(h->plan_dev, h->plan_host.data(), h->plan_host.size() * sizeof(int32_t),
                          cudaMemcpyHostToDevice, st));
-  for (int q = 0; q < G; ++q) {
-    send_rows_host[q] = p.send_rows[q];
-    recv_rows_host[q] = p.recv_rows[q];
+  for (size_t i = 0; i < (size_t)h->phases * G; ++i) {
+    send_rows_host[i] = p.send_rows[i];
+    recv_rows_host[i] = p.recv_rows[i];
   }
   h->C = p.C;
   h->S_total = p.S_total;
@@ -424,37 +505,68 @@ moe_status moe_ep_dispatch(moe_ep_handle h, const double* stats_all_host, const 
   h->computed = false;
   if (h->S == 0) return MOE_OK;
   EP_TRY(launch_ep_dispatch(x, h->act == MOE_BF16, (int)h->S, (int)h->M, E, k, (int)p.C, h->R,
-                            h->plan_dev, h->plan_dev + (size_t)k * E, h->spos, sendbuf, st));
+                            h->plan_dev, h->plan_dev + kE, h->spos, sendbuf, st));
   return MOE_OK;
 }
+
+namespace {
+
+// One phase: its received rows into the experts' slots, the two GEMMs over its slot
+// ranges, the outputs back over its received rows.
+moe_status experts_phase(moe_ep_layer* h, void* recvbuf, int ph, cudaStream_t st) {
+  const bool bf16 = h->act == MOE_BF16;
+  const int k = h->k, E = h->E, El = h->El;
+  const size_t kE = (size_t)k * E;
+  const int32_t* seg_start = h->plan_dev + 4 * kE + (size_t)ph * h->nseg;
+  const int32_t* seg_dst = h->plan_dev + 4 * kE + 2 * (size_t)h->nseg + (size_t)ph * h->nseg;
+  const int32_t* nexp = h->plan_dev + 4 * kE + 4 * (size_t)h->nseg + (size_t)ph * El;
+  const int32_t* rowb = h->plan_dev + 4 * kE + 4 * (size_t)h->nseg + 2 * (size_t)El + (size_t)ph * El;
+  const size_t as = act_bytes(h->act);
+  char* rb = static_cast<char*>(recvbuf) + (size_t)h->recv_off[ph] * h->M * as;
+  int32_t* rowmap = h->rowmap + h->recv_off[ph];
+  const int nrows = (int)h->recv_cnt[ph];
+  EP_TRY(launch_ep_unpack(rb, bf16, nrows, (int)h->M, seg_start, seg_dst, h->nseg, rowmap, h->xbuf, h->R.err,
+                          (int64_t)El * h->Cbuf, st));
+  if (bf16) {
+    // CTA-pair (256-row) tiles when the batch's experts run at capacity, the rule of
+    // the one-device layer on the same batch
+    const bool pair = (double)h->S_total * h->k / E >= (double)h->C;
+    GemmPlan p1 = h->plan1, p2 = h->plan2;
+    p1.row_base = p2.row_base = rowb;
+    EP_TRY(launch_ffn_bf16(p1, nexp, h->R.err, h->wait_limit_ns, h->num_sms, pair, st));
+    EP_TRY(launch_ffn_bf16(p2, nexp, h->R.err, h->wait_limit_ns, h->num_sms, pair, st));
+  } else {                                     // one phase only (moe_ep_set_phases)
+    EP_TRY(launch_ffn_f32((const float*)h->xbuf, (const float*)h->W1, (float*)h->hbuf, nexp, El, h->Cbuf,
+                          (int)h->M, (int)h->H, true, st));
+    EP_TRY(launch_ffn_f32((const float*)h->hbuf, (const float*)h->W2, (float*)h->ybuf, nexp, El, h->Cbuf,
+                          (int)h->H, (int)h->M, false, st));
+  }
+  EP_TRY(launch_ep_repack(h->ybuf, bf16, nrows, (int)h->M, rowmap, rb, st));
+  return MOE_OK;
+}
+
+}  // namespace
 
 moe_status moe_ep_experts(moe_ep_handle h, void* recvbuf, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   if (!h->planned) return MOE_ERR_STATE;
   if (h->recv_total > 0 && (!recvbuf || !aligned(recvbuf, 16))) return MOE_ERR_INVALID_ARG;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool bf16 = h->act == MOE_BF16;
-  const int k = h->k, E = h->E;
-  const int32_t* seg_start = h->plan_dev + (size_t)2 * k * E;
-  const int32_t* seg_dst = seg_start + h->nseg;
-  const int32_t* nexp = seg_dst + h->nseg;
-  EP_TRY(launch_ep_unpack(recvbuf, bf16, (int)h->recv_total, (int)h->M, seg_start, seg_dst, h->nseg,
-                          h->rowmap, h->xbuf, h->R.err, (int64_t)h->El * h->Cbuf, st));
-  if (bf16) {
-    // CTA-pair (256-row) tiles when the batch's experts run at capacity, the rule of
-    // the one-device layer on the same batch
-    const bool pair = (double)h->S_total * h->k / E >= (double)h->C;
-    EP_TRY(launch_ffn_bf16(h->plan1, nexp, h->R.err, h->wait_limit_ns, h->num_sms, pair, st));
-    EP_TRY(launch_ffn_bf16(h->plan2, nexp, h->R.err, h->wait_limit_ns, h->num_sms, pair, st));
-  } else {
-    EP_TRY(launch_ffn_f32((const float*)h->xbuf, (const float*)h->W1, (float*)h->hbuf, nexp, h->El, h->Cbuf,
-                          (int)h->M, (int)h->H, true, st));
-    EP_TRY(launch_ffn_f32((const float*)h->hbuf, (const float*)h->W2, (float*)h->ybuf, nexp, h->El, h->Cbuf,
-                          (int)h->H, (int)h->M, false, st));
+  for (int ph = 0; ph < h->phases; ++ph) {
+    const moe_status s = experts_phase(h, recvbuf, ph, static_cast<cudaStream_t>(stream));
+    if (s != MOE_OK) return s;
   }
-  EP_TRY(launch_ep_repack(h->ybuf, bf16, (int)h->recv_total, (int)h->M, h->rowmap, recvbuf, st));
   h->computed = true;
   return MOE_OK;
+}
+
+moe_status moe_ep_experts_phase(moe_ep_handle h, void* recvbuf, int32_t phase, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (!h->planned) return MOE_ERR_STATE;
+  if (phase < 0 || phase >= h->phases) return MOE_ERR_INVALID_ARG;
+  if (h->recv_cnt[phase] > 0 && (!recvbuf || !aligned(recvbuf, 16))) return MOE_ERR_INVALID_ARG;
+  const moe_status s = experts_phase(h, recvbuf, phase, static_cast<cudaStream_t>(stream));
+  if (s == MOE_OK && phase == h->phases - 1) h->computed = true;
+  return s;
 }
 
 moe_status moe_ep_combine(moe_ep_handle h, const void* sendbuf, void* y, void* stream) {

@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
                   int64_t Cbuf, int K, int N, const uint16_t* __restrict__ mask, int64_t row_limit,
                   uint32_t* __restrict__ bits, unsigned* err, uint64_t limit_ns, int rest_only,
-                  const ScatterY sy) {
+                  const ScatterY sy, const int32_t* __restrict__ row_base) {
   using C = Cfg<BN>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // 256 * ((n + 127) / 256)), at most 128 of them: one tile or none
       const int r0 = rest_only ? (n + 127) / 256 * 256 : 0;
       const int m = (n - r0 + BM - 1) / BM;
-      rbase[e] = r0;
+      rbase[e] = r0 + (row_base ? row_base[e] : 0);   // row_base: the tiles start at that row
       mtiles[e] = m;
       sum += m * NT;
     }
@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (row0 < row_limit)           // a store box starts inside the tensor (TMA clips its tail)
         store_rows<BN, EPI>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
                             nt * BN, lane, mrow, false, brow, bw, bstride, &sy,
-                            (int)(e * Cbuf) + (EPI == kEpiGateY ? __ldg(nexp + e) : 0));
+                            (int)(e * Cbuf) + (EPI == kEpiGateY ? rbase[e] + __ldg(nexp + e) : 0));
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
     }
@@ -726,7 +726,7 @@ constexpr int STAGES = 6;
 constexpr uint32_t TMEM_COLS = 2 * BN;                    // double-buffered accumulator
 constexpr uint32_t STAGING = 4 * 4096;                   // one 32 x 64 bf16 store tile per epilogue warp
 constexpr size_t SMEM =
-    1024 + (size_t)STAGES * STAGE_BYTES + STAGING + 512 + 16 + 4 * (3 * kMaxExperts + 1);
+    1024 + (size_t)STAGES * STAGE_BYTES + STAGING + 512 + 16 + 4 * (4 * kMaxExperts + 1);
 constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;            // shared::cluster address -> rank 0
 static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 static_assert(SMEM + 1024 + 80 * 1024 > 228 * 1024, "a GEMM CTA must own its SM (as Cfg)");
@@ -741,7 +741,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmD, const int32_t* __restrict__ nexp, int E,
                    int64_t Cbuf, int K, int N, const uint16_t* __restrict__ mask,
                    uint32_t* __restrict__ bits, unsigned* err, uint64_t limit_ns, int leave_rest,
-                   const ScatterY sy) {
+                   const ScatterY sy, const int32_t* __restrict__ row_base) {
   using namespace pairk;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -760,6 +760,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   int* tile_pre = reinterpret_cast<int*>(misc + 16);
   int* mtiles = tile_pre + (kMaxExperts + 1);
   int* nrows = mtiles + kMaxExperts;
+  int* rbase = nrows + kMaxExperts;      // [E] first row of each expert's tiles
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -798,6 +799,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // leave_rest: a last block of at most 128 rows is left to the one-CTA kernel
       const int m = leave_rest ? (n + 127) / PM : (n + PM - 1) / PM;
       nrows[e] = n;
+      rbase[e] = row_base ? row_base[e] : 0;   // row_base: the tiles start at that row
       mtiles[e] = m;
       sum += m * NT;
     }
@@ -828,7 +830,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool ok = true;
       int e, mt, nt;
       for (int tile = pair; ok && it.decode(tile, e, mt, nt); tile += npairs) {
-        const int rowA = (int)(e * Cbuf + mt * PM + rank * (PM / 2));
+        const int rowA = (int)(e * Cbuf + rbase[e] + mt * PM + rank * (PM / 2));
         const int rowB = e * K;
         const int colB = nt * BN + rank * (BN / 2);
         for (int kb = 0; kb < KB; ++kb) {
@@ -916,7 +918,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int tile = pair; it.decode(tile, e, mt, nt); tile += npairs, ++i) {
       const int acc = i & 1;
       const uint32_t aph = (i >> 1) & 1;
-      const int row0 = (int)(e * Cbuf + mt * PM + (int)rank * (PM / 2) + q * 32);
+      const int row0 = (int)(e * Cbuf + rbase[e] + mt * PM + (int)rank * (PM / 2) + q * 32);
       const uint16_t* mrow = EPI == kEpiMask ? mask + (int64_t)(row0 + lane) * N + nt * BN : nullptr;
       const int64_t bstride = (int64_t)E * Cbuf;
       uint32_t* brow = (EPI == kEpiReluBits || EPI == kEpiMaskBits)
@@ -933,7 +935,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       store_rows<BN, EPI>(&tmD, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, stage, row0,
                           nt * BN, lane, mrow, false, brow, bw, bstride, &sy,
-                          (int)(e * Cbuf) + (EPI == kEpiGateY ? __ldg(nexp + e) : 0));
+                          (int)(e * Cbuf) + (EPI == kEpiGateY ? rbase[e] + __ldg(nexp + e) : 0));
       tc_fence_before();
       if (leader) mbar_arrive(tempty_bar(acc));
       else mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
@@ -1183,7 +1185,7 @@ cudaError_t launch_pair(const GemmPlan& p, const int32_t* nexp, unsigned* err, u
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(num_sms & ~1), dim3(kThreads), pairk::SMEM, st, p.tmA,
                     BKM ? p.tmB2 : p.tmB, p.tmD, nexp, p.E, p.Cbuf, p.K, p.N,
-                    static_cast<const uint16_t*>(p.mask), p.bits, err, limit_ns, leave_rest, p.sy);
+                    static_cast<const uint16_t*>(p.mask), p.bits, err, limit_ns, leave_rest, p.sy, p.row_base);
 }
 
 template <int BN, int EPI, bool BKM>
@@ -1196,7 +1198,7 @@ cudaError_t launch_t(const GemmPlan& p, const int32_t* nexp, unsigned* err, uint
   const int64_t row_limit = p.row_limit > 0 ? p.row_limit : (int64_t)p.E * p.Cbuf;
   return launch_pdl(kern, dim3(num_sms), dim3(kThreads), smem, st, p.tmA, p.tmB, p.tmD, nexp, p.E,
                     p.Cbuf, p.K, p.N, static_cast<const uint16_t*>(p.mask), row_limit, p.bits, err,
-                    limit_ns, rest_only, p.sy);
+                    limit_ns, rest_only, p.sy, p.row_base);
 }
 
 template <int BN, int EPI>

@@ -173,6 +173,8 @@ struct GemmPlan {
   bool skip_zero;    // kGemmWgrad: experts with no kept row leave D[e] untouched (else zeros)
   int64_t row_limit; // rows of D (0 = E*Cbuf): stores of 32-row groups starting past it are skipped
   ScatterY sy;       // kGemmFwd: with sy.y set, the epilogue stores gate-scaled rows into y instead of D
+  const int32_t* row_base;  // kGemmFwd / kGemmDgrad: [E] device, expert e's rows start at row_base[e]
+                            // (its n_e rows are [row_base[e], row_base[e] + n_e)); null = 0
 };
 bool make_gemm_plan(GemmPlan& p, const void* A, const void* B, void* D, int E, int64_t Cbuf, int K,
                     int N, bool relu);

@@ -1,6 +1,7 @@
 """Expert-parallel layer forward over G ranks (marshalling and byte movement only).
 
-    layer = EPMoeLayer(G, g, S_max, S_total_max, M, H, E, k, cf, Wg, bias, W1_local, W2_local)
+    layer = EPMoeLayer(G, g, S_max, S_total_max, M, H, E, k, cf, Wg, bias, W1_local, W2_local,
+                       phases=2)
     y = ep_forward_dist(layer, x)            # one process per GPU, torch.distributed (NCCL)
     ys = ep_forward_local(layers, xs)        # G ranks emulated in one process on one device
 
@@ -14,7 +15,10 @@ module only moves bytes between the library's four steps:
     experts -> all-to-all back -> combine
 
 The exchange sizes come from the library's plan: rank g sends send_rows[d] rows
-to rank d and receives recv_rows[q] rows from rank q.
+to rank d and receives recv_rows[q] rows from rank q.  With two phases (bf16) each
+exchange is split in two by expert slot, so that the second half travels while the
+experts compute the first, and the first half returns while they compute the second;
+the result is bit for bit the one-phase forward's.
 """
 from __future__ import annotations
 
@@ -28,7 +32,7 @@ class EPMoeLayer:
     """One rank's share of the layer: the whole gate, E/G experts, its buffers."""
 
     def __init__(self, G, g, S_max, S_total_max, M, H, E, k, capacity_factor, Wg, gate_bias,
-                 W1_local, W2_local):
+                 W1_local, W2_local, phases: int = 1):
         act = W1_local.dtype
         if act not in (torch.float32, torch.bfloat16):
             raise TypeError("expert weights must be float32 or bfloat16")
@@ -43,6 +47,9 @@ class EPMoeLayer:
         self._keep = (Wg, gate_bias, W1_local, W2_local)
         self.h = L.moe_ep_create(G, g, S_max, S_total_max, M, H, E, k, capacity_factor, act, Wg, gate_bias,
                                  W1_local, W2_local)
+        self.phases = phases
+        if phases != 1:
+            L.moe_ep_set_phases(self.h, phases)
         dev = W1_local.device
         ns, nr = L.moe_ep_buffer_rows(self.h)
         self.sendbuf = torch.empty(max(ns, 1), M, dtype=act, device=dev)
@@ -60,11 +67,24 @@ class EPMoeLayer:
         return self.stats
 
     def dispatch(self, stats_all: np.ndarray, x: torch.Tensor, stream=None):
-        self.send_rows, self.recv_rows = L.moe_ep_dispatch(self.h, stats_all, x, self.sendbuf, self.G, stream)
+        """Returns (send_rows, recv_rows), each [phases, G]."""
+        send, recv = L.moe_ep_dispatch(self.h, stats_all, x, self.sendbuf, self.G, stream, self.phases)
+        self.send_rows = send.reshape(self.phases, self.G)
+        self.recv_rows = recv.reshape(self.phases, self.G)
         return self.send_rows, self.recv_rows
 
     def experts(self, stream=None) -> None:
         L.moe_ep_experts(self.h, self.recvbuf, stream)
+
+    def experts_phase(self, phase: int, stream=None) -> None:
+        L.moe_ep_experts_phase(self.h, self.recvbuf, phase, stream)
+
+    def phase_rows(self, phase: int):
+        """(send_off, send_rows[G], recv_off, recv_rows[G]) of one phase: the phase's
+        region of each buffer starts after the earlier phases' rows."""
+        so = int(self.send_rows[:phase].sum())
+        ro = int(self.recv_rows[:phase].sum())
+        return so, self.send_rows[phase], ro, self.recv_rows[phase]
 
     def combine(self, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
         y = out if out is not None else torch.empty(self.S, self.M, dtype=self.act, device=self.sendbuf.device)
@@ -101,43 +121,75 @@ def _offsets(rows) -> np.ndarray:
     return np.concatenate([[0], np.cumsum(np.asarray(rows, dtype=np.int64))])
 
 
+def _exchange(layers, phase, back=False):
+    """One phase's all-to-all between emulated ranks (device-to-device copies)."""
+    G = len(layers)
+    for q in range(G):
+        sq, send_q, _, _ = layers[q].phase_rows(phase)
+        soff = sq + _offsets(send_q)
+        for d in range(G):
+            _, _, rd, recv_d = layers[d].phase_rows(phase)
+            roff = rd + _offsets(recv_d)
+            n = int(send_q[d])
+            assert n == int(recv_d[q]), "send and receive counts of a pair disagree"
+            if n:
+                src = layers[q].sendbuf[soff[d]:soff[d] + n]
+                dst = layers[d].recvbuf[roff[q]:roff[q] + n]
+                if back:
+                    src.copy_(dst)
+                else:
+                    dst.copy_(src)
+
+
 def ep_forward_local(layers, xs, outs=None):
     """G ranks of one layer emulated in one process (all on one device): every exchange
-    is one device-to-device copy per (source, destination) block.  Returns the outputs."""
-    G = len(layers)
+    is one device-to-device copy per (source, destination) block, phase by phase, in the
+    order a rank takes them (the experts of phase p run after its rows arrived, the
+    return of phase p after its experts).  Returns the outputs."""
     stats = [layer.route(x) for layer, x in zip(layers, xs)]
     stats_all = torch.stack(stats).cpu().numpy()                     # the all-gather
-    plans = [layer.dispatch(stats_all, x) for layer, x in zip(layers, xs)]
-    soff = [_offsets(send) for send, _ in plans]
-    roff = [_offsets(recv) for _, recv in plans]
-    for q in range(G):                                               # the all-to-all
-        for d in range(G):
-            n = int(plans[q][0][d])
-            assert n == int(plans[d][1][q]), "send and receive counts of a pair disagree"
-            if n:
-                layers[d].recvbuf[roff[d][q]:roff[d][q] + n].copy_(layers[q].sendbuf[soff[q][d]:soff[q][d] + n])
-    for layer in layers:
-        layer.experts()
-    for q in range(G):                                               # the all-to-all back
-        for d in range(G):
-            n = int(plans[q][0][d])
-            if n:
-                layers[q].sendbuf[soff[q][d]:soff[q][d] + n].copy_(layers[d].recvbuf[roff[d][q]:roff[d][q] + n])
+    for layer, x in zip(layers, xs):
+        layer.dispatch(stats_all, x)
+    phases = layers[0].phases
+    for p in range(phases):
+        _exchange(layers, p)                                         # the all-to-all of phase p
+        for layer in layers:
+            layer.experts_phase(p)
+        _exchange(layers, p, back=True)                              # and back
     return [layer.combine(None if outs is None else outs[i]) for i, layer in enumerate(layers)]
 
 
 def ep_forward_dist(layer: EPMoeLayer, x: torch.Tensor, group=None, out=None) -> torch.Tensor:
-    """One rank's forward in a torch.distributed job of G ranks (one per GPU)."""
+    """One rank's forward in a torch.distributed job of G ranks (one per GPU).
+
+    With two phases the exchanges run asynchronously on the process group's stream:
+    phase 1's rows travel while the experts compute phase 0, and phase 0's outputs
+    return while they compute phase 1.  A collective starts after the work already
+    queued on the current stream; `wait()` queues the current stream behind it."""
     import torch.distributed as dist
     G = layer.G
     stats = layer.route(x)
     gathered = torch.empty(G, stats.numel(), dtype=stats.dtype, device=stats.device)
     dist.all_gather_into_tensor(gathered, stats, group=group)
-    send, recv = layer.dispatch(gathered.cpu().numpy(), x)
-    ns, nr = int(send.sum()), int(recv.sum())
-    dist.all_to_all_single(layer.recvbuf[:nr], layer.sendbuf[:ns], [int(v) for v in recv],
-                           [int(v) for v in send], group=group)
-    layer.experts()
-    dist.all_to_all_single(layer.sendbuf[:ns], layer.recvbuf[:nr], [int(v) for v in send],
-                           [int(v) for v in recv], group=group)
+    layer.dispatch(gathered.cpu().numpy(), x)
+
+    def a2a(phase, back):
+        so, send, ro, recv = layer.phase_rows(phase)
+        s_buf = layer.sendbuf[so:so + int(send.sum())]
+        r_buf = layer.recvbuf[ro:ro + int(recv.sum())]
+        send_l, recv_l = [int(v) for v in send], [int(v) for v in recv]
+        if back:
+            return dist.all_to_all_single(s_buf, r_buf, send_l, recv_l, group=group, async_op=True)
+        return dist.all_to_all_single(r_buf, s_buf, recv_l, send_l, group=group, async_op=True)
+
+    there = [a2a(0, False)]
+    back = []
+    for p in range(layer.phases):
+        if p + 1 < layer.phases:
+            there.append(a2a(p + 1, False))                          # the next phase travels ...
+        there[p].wait()
+        layer.experts_phase(p)                                       # ... while this one computes
+        back.append(a2a(p, True))
+    for w in back:
+        w.wait()
     return layer.combine(out)

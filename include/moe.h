@@ -296,6 +296,19 @@ MOE_API moe_status moe_assign_slots_noalloc(int64_t S, int32_t E, int32_t k, int
  * the receiver gets each source's rows in that order, source after source, and
  * moe_ep_experts writes each expert output over the row it came from, so the second
  * exchange is the first one reversed.
+ *
+ * Two phases (moe_ep_set_phases, bf16): the exchanges split in two, so that they can
+ * overlap the expert GEMMs -- send phase 1 while the experts compute phase 0, return
+ * phase 0 while they compute phase 1.  Each expert's slots are split at
+ * split_e = 256 * floor((n_e + 256) / 512) (n_e its kept rows over the batch): slots
+ * below it travel in phase 0, the rest in phase 1.  Both buffers hold all phase-0 rows
+ * first, then all phase-1 rows, each phase ordered as above, and the row counts per
+ * peer come per phase ([2][G], phase-major).  One forward with overlap:
+ *   moe_ep_route; all-gather; moe_ep_dispatch -> send_rows[2][G], recv_rows[2][G]
+ *   exchange phase 0;  [exchange phase 1 | moe_ep_experts_phase(0)]
+ *   [return phase 0 | moe_ep_experts_phase(1)];  return phase 1;  moe_ep_combine
+ * Every GEMM tile lies within one phase, so rows, slots and outputs are bit for bit
+ * those of the one-phase forward.
  */
 typedef struct moe_ep_layer* moe_ep_handle;
 
@@ -319,6 +332,16 @@ MOE_API moe_status moe_ep_plan(int32_t G, int32_t g, int32_t E, int32_t k, doubl
                                int64_t* kept_host);
 
 /*
+ * moe_ep_phase_plan -- per-phase row counts of rank g (host arithmetic, as moe_ep_plan):
+ * send_rows_host / recv_rows_host [phases][G] (phase-major) and, optional, split_host [E]
+ * (the first phase-1 slot of each expert; n_e with one phase).  phases: 1 or 2, else
+ * MOE_ERR_INVALID_ARG; invalid counts as moe_ep_plan.
+ */
+MOE_API moe_status moe_ep_phase_plan(int32_t G, int32_t g, int32_t E, int32_t k, double capacity_factor,
+                                     const int64_t* counts_host, const int64_t* S_host, int32_t phases,
+                                     int64_t* send_rows_host, int64_t* recv_rows_host, int64_t* split_host);
+
+/*
  * moe_ep_create -- rank g's handle.  S_max: most tokens this rank routes in a forward;
  * S_total_max: most tokens of a batch over all ranks (sizes the expert buffers).
  * Wg_dev [M, E] and gate_bias_dev [E] (or NULL) as in moe_create; W1_local_dev
@@ -335,22 +358,34 @@ MOE_API moe_status moe_ep_destroy(moe_ep_handle h);
 /* Rows the caller's buffers need: send buffer S_max*k, receive buffer E/G * min(C, S_total_max). */
 MOE_API moe_status moe_ep_buffer_rows(moe_ep_handle h, int64_t* send_rows_max, int64_t* recv_rows_max);
 
+/* Exchanges in 1 (default) or 2 phases for the forwards that follow (see above).  Two
+ * phases need bf16 activations (MOE_ERR_UNSUPPORTED otherwise); a forward in progress
+ * must start again from moe_ep_dispatch. */
+MOE_API moe_status moe_ep_set_phases(moe_ep_handle h, int32_t phases);
+
 /* Step 1: router and the rank's own scan on S tokens (x_dev [S, M] act); writes the
  * rank's stats (moe_ep_stats_len doubles, 8-byte aligned device memory) on `stream`. */
 MOE_API moe_status moe_ep_route(moe_ep_handle h, int64_t S, const void* x_dev, double* stats_dev,
                                 void* stream);
 
 /* Step 2: stats_all_host [G][moe_ep_stats_len] (every rank's stats, rank order) ->
- * plan, send_rows_host / recv_rows_host [G], and the kept rows of x_dev (the same x as
- * step 1) packed into sendbuf_dev (>= sum(send_rows) rows).  Host arithmetic, then
- * one table upload and one kernel on `stream`. */
+ * plan, send_rows_host / recv_rows_host [phases][G], and the kept rows of x_dev (the
+ * same x as step 1) packed into sendbuf_dev (>= sum(send_rows) rows).  Host arithmetic,
+ * then one table upload and one kernel on `stream`. */
 MOE_API moe_status moe_ep_dispatch(moe_ep_handle h, const double* stats_all_host, const void* x_dev,
                                    void* sendbuf_dev, int64_t* send_rows_host, int64_t* recv_rows_host,
                                    void* stream);
 
 /* Step 3: the received rows (recvbuf_dev, sum(recv_rows) rows) into the local experts'
- * slots, both expert GEMMs, and each expert output written over its received row. */
+ * slots, both expert GEMMs, and each expert output written over its received row
+ * (every phase, in order). */
 MOE_API moe_status moe_ep_experts(moe_ep_handle h, void* recvbuf_dev, void* stream);
+
+/* Step 3 for one phase (0 <= phase < phases): the phase's received rows (its region of
+ * recvbuf_dev: after the sum of the earlier phases' recv_rows) through the experts, the
+ * outputs written over them.  Needs only that phase's rows to have arrived.
+ * MOE_ERR_INVALID_ARG for a phase out of range. */
+MOE_API moe_status moe_ep_experts_phase(moe_ep_handle h, void* recvbuf_dev, int32_t phase, void* stream);
 
 /* Step 4: y_dev [S, M] act from the returned rows in sendbuf_dev (fully overwritten;
  * a token whose choices were all dropped gets 0). */

@@ -4,7 +4,11 @@ each computes its plan with the library's moe_ep_plan (no GPU, no device call).
 The plan must keep the one-device meaning of capacity over the whole batch: every
 run's first global slot and kept rows are what the oracle's rank-major capacity
 rule (`assign_slots`) gives on the concatenated batch, and what rank q sends to
-rank d is exactly what rank d expects from rank q.
+rank d is exactly what rank d expects from rank q.  The two-phase plan
+(moe_ep_phase_plan) splits each expert's slots at 256 * floor((n_e + 256) / 512):
+per phase, what rank q sends to rank d is what d expects from q, both equal the
+oracle's kept choices on each side of the split, and the phases add up to the
+one-phase plan.
 """
 import os
 import socket
@@ -30,6 +34,7 @@ CASES = {
     "ragged": ((17, 0, 90, 33), 16, 2, 1.25, 2, 0.0),
     "top4_skewed": ((40, 40, 40, 40), 16, 4, 0.75, 3, 2.5),
     "top8_of_32": ((25, 31, 0, 70), 32, 8, 1.0, 4, 1.0),
+    "big": ((700, 900, 800, 600), 8, 2, 1.25, 5, 0.5),        # n_e up to C = 938: both phases non-empty
 }
 
 
@@ -64,13 +69,19 @@ def _worker(rank, world, port, case, q):
         # what rank d receives from this rank must be what this rank sends to d
         got = torch.zeros(world, dtype=torch.int64)
         dist.all_to_all_single(got, torch.from_numpy(send.copy()))
-        q.put((rank, C, send, recv, base, kept, got.numpy(), counts, S))
+        send2, recv2, split = L.moe_ep_phase_plan(world, rank, E, k, cf, counts, S, 2)
+        got2 = []
+        for ph in range(2):                    # the same check for each phase's exchange
+            g2 = torch.zeros(world, dtype=torch.int64)
+            dist.all_to_all_single(g2, torch.from_numpy(send2[ph].copy()))
+            got2.append(g2.numpy())
+        q.put((rank, C, send, recv, base, kept, got.numpy(), counts, S, send2, recv2, split, np.stack(got2)))
     finally:
         dist.destroy_process_group()
 
 
 @pytest.mark.parametrize("world,case", [(2, "even"), (4, "even"), (4, "ragged"), (4, "top4_skewed"),
-                                        (4, "top8_of_32"), (2, "top8_of_32")])
+                                        (4, "top8_of_32"), (2, "top8_of_32"), (4, "big"), (2, "big")])
 def test_exchange_plan_matches_the_one_device_capacity_rule(world, case):
     ctx = mp.get_context("spawn")
     qu = ctx.Queue()
@@ -92,7 +103,21 @@ def test_exchange_plan_matches_the_one_device_capacity_rule(world, case):
     pos, _ = O.assign_slots(ids, E, S_tot * k + 1)        # positions with nothing dropped
     El = E // world
     owner = np.repeat(np.arange(len(S_all)), S_all)
-    for rank, C_got, send, recv, base, kept, got, counts, S in res:
+    n_e = np.minimum(cnt_tot, C)
+    split_ref = 256 * ((n_e + 256) // 512)
+    assert np.all(split_ref <= n_e)
+    for rank, C_got, send, recv, base, kept, got, counts, S, send2, recv2, split, got2 in res:
+        assert np.array_equal(split, split_ref)
+        # per phase: the exchange is consistent, matches the oracle's kept choices on
+        # each side of the split, and the two phases add up to the one-phase plan
+        assert np.array_equal(got2, recv2)
+        assert np.array_equal(send2.sum(axis=0), send) and np.array_equal(recv2.sum(axis=0), recv)
+        ph_of = np.where(slot >= 0, (slot >= split_ref[np.clip(ids, 0, E - 1)]).astype(int), -1)
+        for ph in range(2):
+            for d in range(world):
+                e_d = (ids // El == d)
+                assert send2[ph, d] == int(np.sum((ph_of == ph) & e_d & (owner == rank)[:, None]))
+                assert recv2[ph, d] == int(np.sum((ph_of == ph) & (ids // El == rank) & (owner == d)[:, None]))
         assert C_got == C
         assert np.array_equal(S, S_all)
         # what every rank d sends here (exchanged by gloo) is what this rank expects from d
@@ -131,3 +156,8 @@ def test_plan_rejects_inconsistent_counts():
         L.moe_ep_plan(2, 0, 3, 1, 1.0, np.zeros((2, 1, 3)), [0, 0])   # E not a multiple of G
     with pytest.raises(L.MoeError):
         L.moe_ep_plan(2, 2, 2, 1, 1.0, counts, [3, 3])             # g out of range
+    with pytest.raises(L.MoeError) as ei:
+        L.moe_ep_phase_plan(2, 0, 2, 1, 1.0, counts, [3, 3], 3)   # one or two phases only
+    assert ei.value.status == L.MOE_ERR_INVALID_ARG
+    send1, recv1, split1 = L.moe_ep_phase_plan(2, 0, 2, 1, 1.0, counts, [3, 3], 1)
+    assert send1.tolist() == [[2, 1]] and recv1.tolist() == [[2, 0]] and split1.tolist() == [2, 3]

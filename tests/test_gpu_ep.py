@@ -84,6 +84,50 @@ def test_ep_emulated_ranks_equal_one_device(w, shards):
         layer.close()
 
 
+PHASE_CASES = [
+    # experts at capacity (C = 2560, n_e about 2048): both phases non-empty, CTA-pair tiles
+    (Workload("ep2_sat", 8192, 256, 512, 8, 2, 1.25, "bf16"), (3000, 1000, 2500, 1692)),
+    (Workload("ep2_sat_full", 4096, 256, 256, 8, 2, 1.0, "bf16"), (2048, 2048)),
+    # below capacity, one-CTA tiles; some experts above 256 rows, some below
+    (Workload("ep2_skewed", 4096, 128, 256, 16, 2, 2.0, "bf16", skew_bias=True), (1000, 1100, 996, 1000)),
+    # n_e about 128: every row in phase 1, phase 0 empty
+    (Workload("ep2_top8", 1024, 128, 256, 64, 8, 1.25, "bf16"), (128,) * 8),
+]
+
+
+@pytest.mark.parametrize("w,shards", PHASE_CASES, ids=[c[0].name for c in PHASE_CASES])
+def test_ep_two_phases_equal_one_phase_bit_for_bit(w, shards):
+    """Exchanges in two phases (split by expert slot, so that they can overlap the
+    expert GEMMs) give the one-phase forward's routing, outputs and losses exactly."""
+    G = len(shards)
+    x, Wg, b, W1, W2 = make_inputs(w, device="cuda")
+    El = w.E // G
+    cuts = np.cumsum((0,) + shards)
+    xs = [x[cuts[g]:cuts[g + 1]].contiguous() for g in range(G)]
+    Ws = [(W1[g * El:(g + 1) * El].contiguous(), W2[g * El:(g + 1) * El].contiguous()) for g in range(G)]
+    res = {}
+    for phases in (1, 2):
+        layers = [EPMoeLayer(G, g, max(shards[g], 1), w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b, *Ws[g],
+                             phases=phases) for g in range(G)]
+        ys = ep_forward_local(layers, xs)
+        torch.cuda.synchronize()
+        parts = [layer.routing() for layer in layers]
+        res[phases] = (torch.cat(ys), torch.cat([p[0] for p in parts]), torch.cat([p[2] for p in parts]),
+                       [layer.aux_loss() for layer in layers], [layer.send_rows for layer in layers])
+        for layer in layers:
+            layer.close()
+    y1, e1, s1, a1, _ = res[1]
+    y2, e2, s2, a2, send2 = res[2]
+    assert torch.equal(e1, e2) and torch.equal(s1, s2)
+    assert torch.equal(y1, y2)
+    assert a1 == a2
+    moved0 = sum(int(s[0].sum()) for s in send2)
+    moved1 = sum(int(s[1].sum()) for s in send2)
+    print(f"\n{w.name}: rows in phase 0 / 1: {moved0} / {moved1}")
+    if w.name.startswith("ep2_sat"):
+        assert moved0 > 0 and moved1 > 0
+
+
 def test_ep_rejects_a_plan_from_inconsistent_stats():
     w = Workload("ep_bad", 256, 64, 64, 8, 2, 1.0, "bf16")
     x, Wg, b, W1, W2 = make_inputs(w, device="cuda")
@@ -100,6 +144,29 @@ def test_ep_rejects_a_plan_from_inconsistent_stats():
     layer.close()
 
 
+def test_ep_phase_arguments():
+    from gshard_top_gating_b200 import _lib as L
+    w = Workload("ep_args", 256, 64, 64, 8, 2, 1.0, "f32")
+    x, Wg, b, W1, W2 = make_inputs(w, device="cuda")
+    layer = EPMoeLayer(2, 0, 128, 256, w.M, w.H, w.E, w.k, w.cf, Wg, b, W1[:4].contiguous(), W2[:4].contiguous())
+    with pytest.raises(L.MoeError) as ei:      # the FFMA GEMMs take no row base: one phase only
+        L.moe_ep_set_phases(layer.h, 2)
+    assert ei.value.status == L.MOE_ERR_UNSUPPORTED
+    for bad in (0, 3):
+        with pytest.raises(L.MoeError) as ei:
+            L.moe_ep_set_phases(layer.h, bad)
+        assert ei.value.status == L.MOE_ERR_INVALID_ARG
+    with pytest.raises(L.MoeError) as ei:      # no plan yet
+        layer.experts_phase(0)
+    assert ei.value.status == L.MOE_ERR_STATE
+    st = layer.route(x[:128].contiguous()).cpu().numpy()
+    layer.dispatch(np.stack([st, st]), x[:128].contiguous())
+    with pytest.raises(L.MoeError) as ei:      # phase out of range
+        layer.experts_phase(1)
+    assert ei.value.status == L.MOE_ERR_INVALID_ARG
+    layer.close()
+
+
 def test_ep_forward_dist_one_rank_nccl():
     """The torch.distributed driver (all-gather of stats, two all_to_all_single) in a
     one-rank NCCL group equals the one-device layer; no rank waits on another."""
@@ -108,7 +175,7 @@ def test_ep_forward_dist_one_rank_nccl():
     import torch.distributed as dist
     from datetime import timedelta
     from gshard_top_gating_b200.ep import ep_forward_dist
-    w = Workload("ep_dist1", 1024, 256, 256, 16, 2, 1.0, "bf16")
+    w = Workload("ep_dist1", 4096, 256, 256, 8, 2, 1.0, "bf16")      # n_e about 1024: both phases used
     x, Wg, b, W1, W2 = make_inputs(w, device="cuda")
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -117,16 +184,17 @@ def test_ep_forward_dist_one_rank_nccl():
     dist.init_process_group("nccl", store=store, rank=0, world_size=1, timeout=timedelta(seconds=60),
                             device_id=torch.device("cuda", torch.cuda.current_device()))
     try:
-        layer = EPMoeLayer(1, 0, w.S, w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b, W1, W2)
-        y = ep_forward_dist(layer, x)
         one = MoeLayer(w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b, W1, W2)
         y1 = one(x)
-        torch.cuda.synchronize()
-        assert torch.equal(y, y1)
-        la, za = layer.aux_loss()
         lb, zb = one.aux_loss()
-        assert abs(la - lb) <= 1e-5 * lb and abs(za - zb) <= 1e-5 * zb
+        for phases in (1, 2):                  # two phases: asynchronous exchanges per phase
+            layer = EPMoeLayer(1, 0, w.S, w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b, W1, W2, phases=phases)
+            y = ep_forward_dist(layer, x)
+            torch.cuda.synchronize()
+            assert torch.equal(y, y1), phases
+            la, za = layer.aux_loss()
+            assert abs(la - lb) <= 1e-5 * lb and abs(za - zb) <= 1e-5 * zb
+            layer.close()
         one.close()
-        layer.close()
     finally:
         dist.destroy_process_group()
