@@ -74,6 +74,9 @@ def _load() -> ctypes.CDLL:
         "moe_ep_dispatch": [P, P, P, P, P, P, P],
         "moe_ep_experts": [P, P, P],
         "moe_ep_experts_phase": [P, P, I32, P],
+        "moe_ep_set_peers": [P, P],
+        "moe_ep_dispatch_to_peers": [P, P, P, P, P, P],
+        "moe_ep_combine_from_peers": [P, P, P],
         "moe_ep_set_phases": [P, I32],
         "moe_ep_phase_plan": [I32, I32, I32, I32, D, P, P, I32, P, P, P],
         "moe_ep_combine": [P, P, P, P],
@@ -307,6 +310,30 @@ def moe_ep_dispatch(h, stats_all, x, sendbuf, G, stream=None, phases=1):
     if phases == 1:
         return send, recv
     return send.reshape(phases, G), recv.reshape(phases, G)
+
+
+def moe_ep_set_peers(h, recv_ptrs) -> None:
+    """recv_ptrs: G device addresses (ints) of every rank's receive buffer, or None."""
+    if recv_ptrs is None:
+        _check("moe_ep_set_peers", lib.moe_ep_set_peers(h, None))
+        return
+    arr = (ctypes.c_void_p * len(recv_ptrs))(*[int(p) for p in recv_ptrs])
+    _check("moe_ep_set_peers", lib.moe_ep_set_peers(h, ctypes.cast(arr, ctypes.c_void_p)))
+
+
+def moe_ep_dispatch_to_peers(h, stats_all, x, G, stream=None):
+    """As moe_ep_dispatch, rows stored straight into the owners' receive buffers."""
+    import numpy as np
+    st = np.ascontiguousarray(stats_all, dtype=np.float64)
+    send = np.zeros(G, dtype=np.int64)
+    recv = np.zeros(G, dtype=np.int64)
+    _check("moe_ep_dispatch_to_peers", lib.moe_ep_dispatch_to_peers(h, _np_ptr(st), _ptr(x), _np_ptr(send),
+                                                                    _np_ptr(recv), _stream(stream)))
+    return send, recv
+
+
+def moe_ep_combine_from_peers(h, y, stream=None) -> None:
+    _check("moe_ep_combine_from_peers", lib.moe_ep_combine_from_peers(h, _ptr(y), _stream(stream)))
 
 
 def moe_ep_set_phases(h, phases: int) -> None:

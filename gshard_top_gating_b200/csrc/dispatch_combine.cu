@@ -238,7 +238,8 @@ template <typename T, int KM>
 __global__ void __launch_bounds__(kThreads, KM >= 8 ? 3 : 4) combine_kernel(const T* __restrict__ ybuf, int S, int M,
                                                               int k, int64_t Cbuf, Routing R,
                                                               T* __restrict__ y, int loss_blocks, int E,
-                                                              int nchunk) {
+                                                              int nchunk, const EpPeer* __restrict__ peers,
+                                                              int El) {
   static_assert(kThreads == kLossThreads, "the loss block runs with the combine's block size");
   const int lane = threadIdx.x & 31;
   const int warps = ((gridDim.x - loss_blocks) * kThreads) >> 5;
@@ -266,9 +267,16 @@ __global__ void __launch_bounds__(kThreads, KM >= 8 ? 3 : 4) combine_kernel(cons
       const int er = __shfl_sync(0xffffffffu, e, r);
       const int sr = __shfl_sync(0xffffffffu, s, r);
       gr[r] = __shfl_sync(0xffffffffu, g, r);
-      srcs[r] = (r < k && sr >= 0)
-                    ? reinterpret_cast<const uint4*>(ybuf + ((int64_t)er * Cbuf + sr) * M)
-                    : nullptr;
+      const T* row = nullptr;
+      if (r < k && sr >= 0) {
+        if (peers) {                           // the owner's receive buffer (expert parallelism)
+          const EpPeer p = peers[er / El];
+          row = static_cast<const T*>(p.base) + ((int64_t)sr + p.delta) * M;
+        } else {
+          row = ybuf + ((int64_t)er * Cbuf + sr) * M;
+        }
+      }
+      srcs[r] = reinterpret_cast<const uint4*>(row);
     }
     uint4* dst = reinterpret_cast<uint4*>(y + (int64_t)t * M);
     for (int v0 = lane; v0 < nv; v0 += 32 * U) {
@@ -309,16 +317,18 @@ __global__ void __launch_bounds__(kThreads, 4) ep_dispatch_kernel(const T* __res
                                                                   Routing R, const int32_t* __restrict__ base,
                                                                   const int32_t* __restrict__ soff,
                                                                   int32_t* __restrict__ spos,
-                                                                  T* __restrict__ sendbuf) {
+                                                                  T* __restrict__ sendbuf,
+                                                                  const EpPeer* __restrict__ peers, int El) {
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * kThreads) >> 5;
   const int nv = (int)((int64_t)M * sizeof(T) / 16);
   pdl_trigger();
   pdl_wait();                                  // local offsets and the exchanged plan complete
   for (int t = (blockIdx.x * kThreads + threadIdx.x) >> 5; t < S; t += warps) {
-    int sp = -1;
+    int sp = -1, ev = 0;
     if (lane < k) {
       const int e = R.eidx[(int64_t)t * k + lane];
+      ev = e;
       int s = -1;
       if (e >= 0 && e < E) {
         const int local = R.off[((int64_t)lane * nchunk + t / kChunk) * E + e] + R.lrank[(int64_t)t * k + lane];
@@ -341,7 +351,17 @@ __global__ void __launch_bounds__(kThreads, 4) ep_dispatch_kernel(const T* __res
 #pragma unroll
     for (int r = 0; r < KM; ++r) {
       const int pr = __shfl_sync(0xffffffffu, sp, r);
-      dst[r] = (r < k && pr >= 0) ? reinterpret_cast<uint4*>(sendbuf + (int64_t)pr * M) : nullptr;
+      const int er = __shfl_sync(0xffffffffu, ev, r);
+      T* row = nullptr;
+      if (r < k && pr >= 0) {
+        if (peers) {                           // straight into the owner's receive buffer
+          const EpPeer p = peers[er / El];
+          row = static_cast<T*>(p.base) + ((int64_t)pr + p.delta) * M;
+        } else {
+          row = sendbuf + (int64_t)pr * M;
+        }
+      }
+      dst[r] = reinterpret_cast<uint4*>(row);
       any |= dst[r] != nullptr;
     }
     if (!any) continue;                        // every choice dropped: the row is not sent
@@ -430,10 +450,10 @@ void dispatch_t(const void* x, int S, int M, int E, int k, int C, int64_t Cbuf, 
 
 template <typename T, int KM>
 void combine_t(const void* ybuf, int S, int M, int k, int64_t Cbuf, const Routing& R, void* y,
-               int grid, cudaStream_t st, int loss_blocks, int E) {
+               int grid, cudaStream_t st, int loss_blocks, int E, const EpPeer* peers, int El) {
   const int nchunk = (S + kChunk - 1) / kChunk;
   launch_pdl(combine_kernel<T, KM>, dim3(grid + loss_blocks), dim3(kThreads), 0, st, (const T*)ybuf, S, M,
-             k, Cbuf, R, (T*)y, loss_blocks, E, nchunk);
+             k, Cbuf, R, (T*)y, loss_blocks, E, nchunk, peers, El);
 }
 
 template <typename T>
@@ -447,11 +467,11 @@ void dispatch_k(int k, const void* x, int S, int M, int E, int C, int64_t Cbuf, 
 
 template <typename T>
 void combine_k(int k, const void* ybuf, int S, int M, int64_t Cbuf, const Routing& R, void* y,
-               int grid, cudaStream_t st, int loss_blocks, int E) {
-  if (k <= 1) combine_t<T, 1>(ybuf, S, M, k, Cbuf, R, y, grid, st, loss_blocks, E);
-  else if (k <= 2) combine_t<T, 2>(ybuf, S, M, k, Cbuf, R, y, grid, st, loss_blocks, E);
-  else if (k <= 4) combine_t<T, 4>(ybuf, S, M, k, Cbuf, R, y, grid, st, loss_blocks, E);
-  else combine_t<T, 8>(ybuf, S, M, k, Cbuf, R, y, grid, st, loss_blocks, E);
+               int grid, cudaStream_t st, int loss_blocks, int E, const EpPeer* peers, int El) {
+  if (k <= 1) combine_t<T, 1>(ybuf, S, M, k, Cbuf, R, y, grid, st, loss_blocks, E, peers, El);
+  else if (k <= 2) combine_t<T, 2>(ybuf, S, M, k, Cbuf, R, y, grid, st, loss_blocks, E, peers, El);
+  else if (k <= 4) combine_t<T, 4>(ybuf, S, M, k, Cbuf, R, y, grid, st, loss_blocks, E, peers, El);
+  else combine_t<T, 8>(ybuf, S, M, k, Cbuf, R, y, grid, st, loss_blocks, E, peers, El);
 }
 
 }  // namespace
@@ -499,14 +519,15 @@ cudaError_t launch_dispatch_rerouted(const void* x, bool bf16, int S, int M, int
 
 cudaError_t launch_ep_dispatch(const void* x, bool bf16, int S, int M, int E, int k, int C,
                                const Routing& R, const int32_t* base, const int32_t* soff,
-                               int32_t* spos, void* sendbuf, cudaStream_t st) {
+                               int32_t* spos, void* sendbuf, cudaStream_t st, const EpPeer* peers,
+                               int El) {
   const int nchunk = (S + kChunk - 1) / kChunk;
   const int grid = grid_for(S);
   auto go = [&](auto tag, auto km) {
     using T = decltype(tag);
     constexpr int KM = decltype(km)::value;
     return launch_pdl(ep_dispatch_kernel<T, KM>, dim3(grid), dim3(kThreads), 0, st, (const T*)x, S, M, E,
-                      k, C, nchunk, R, base, soff, spos, (T*)sendbuf);
+                      k, C, nchunk, R, base, soff, spos, (T*)sendbuf, peers, El);
   };
   using I1 = std::integral_constant<int, 1>;
   using I2 = std::integral_constant<int, 2>;
@@ -538,15 +559,16 @@ cudaError_t launch_ep_repack(const void* ybuf, bool bf16, int nrows, int M, cons
 }
 
 cudaError_t launch_combine(const void* ybuf, bool bf16, int S, int M, int k, int64_t Cbuf,
-                           const Routing& R, void* y, cudaStream_t st, bool with_losses, int E) {
+                           const Routing& R, void* y, cudaStream_t st, bool with_losses, int E,
+                           const EpPeer* peers, int El) {
   // with the loss block, one token block fewer: grid_for fills the SMs' resident slots
   // exactly, and a block past them would run alone after the others
   const int lb = with_losses ? 1 : 0;
   const int grid = grid_for(S) > 1 ? grid_for(S) - lb : grid_for(S);
   if (bf16)
-    combine_k<__nv_bfloat16>(k, ybuf, S, M, Cbuf, R, y, grid, st, lb, E);
+    combine_k<__nv_bfloat16>(k, ybuf, S, M, Cbuf, R, y, grid, st, lb, E, peers, El);
   else
-    combine_k<float>(k, ybuf, S, M, Cbuf, R, y, grid, st, lb, E);
+    combine_k<float>(k, ybuf, S, M, Cbuf, R, y, grid, st, lb, E, peers, El);
   return cudaGetLastError();
 }
 

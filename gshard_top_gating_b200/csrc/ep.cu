@@ -29,6 +29,13 @@
 //   moe_ep_combine   y[t] = sum_{r kept} g_r * (returned row of (t, r)), r ascending, fp32
 // The losses use the gathered stats: f_j and P_j over the whole batch.
 //
+// Over peer memory (moe_ep_set_peers, moe_ep_dispatch_to_peers, moe_ep_combine_from_peers):
+// the pack writes each kept row straight into its owner's receive buffer, at the row the
+// all-to-all would have put it, and the combine reads each expert output from there, so
+// neither exchange is a separate step.  The caller maps the buffers and orders the ranks
+// (every rank's dispatch before any rank's experts, every rank's experts before any
+// combine, every combine before the next dispatch).
+//
 // Two phases (moe_ep_set_phases): each expert's slots are split at
 //     split_e = 256 * floor((n_e + 256) / 512)   (about half, a whole number of GEMM tiles),
 // slots below it travel in phase 0 and the rest in phase 1.  The send and receive buffers
@@ -75,6 +82,9 @@ struct moe_ep_layer {
   int nseg;              // received segments per phase: G * El * k
   int phases;            // 1 or 2
   int64_t recv_off[2], recv_cnt[2];   // each phase's rows in the receive buffer
+  EpPeer* peers_dev;     // [G] every rank's receive buffer and this rank's row offset in it
+  std::vector<void*> peer_ptrs;       // [G] set by moe_ep_set_peers (empty: not set)
+  std::vector<EpPeer> peers_host;
   std::vector<int32_t> plan_host;
   GemmPlan plan1, plan2;
   void* wsplit;
@@ -151,6 +161,7 @@ size_t carve(moe_ep_layer* h, char* base) {
   h->ybuf = c.take<char>((size_t)h->El * h->Cbuf * h->M * as);
   h->plan_dev = c.take<int32_t>(plan_ints(h));
   h->rowmap = c.take<int32_t>((size_t)h->El * h->Cbuf);
+  h->peers_dev = c.take<EpPeer>((size_t)h->G);
   h->wsplit = h->act == MOE_BF16 ? c.take<char>((size_t)3 * router_tc_pad(h->E) * h->M * 2) : nullptr;
   return c.off + 256;
 }
@@ -398,10 +409,17 @@ moe_status moe_ep_route(moe_ep_handle h, int64_t S, const void* x, double* stats
   return MOE_OK;
 }
 
-moe_status moe_ep_dispatch(moe_ep_handle h, const double* stats_all_host, const void* x, void* sendbuf,
-                           int64_t* send_rows_host, int64_t* recv_rows_host, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// moe_ep_dispatch (sendbuf) and moe_ep_dispatch_to_peers (to_peers: the owners' receive
+// buffers set by moe_ep_set_peers).
+moe_status dispatch_impl(moe_ep_layer* h, const double* stats_all_host, const void* x, void* sendbuf,
+                         bool to_peers, int64_t* send_rows_host, int64_t* recv_rows_host, void* stream) {
   if (!h || !stats_all_host || !send_rows_host || !recv_rows_host) return MOE_ERR_INVALID_ARG;
   if (!h->routed) return MOE_ERR_STATE;
+  if (to_peers && (h->peer_ptrs.empty() || h->phases != 1)) return MOE_ERR_STATE;
   const int G = h->G, E = h->E, k = h->k, El = h->El, L = ep_stats_len(E, k);
   // the gathered counts must be exact non-negative integers, and this rank's must be its own
   std::vector<int64_t> cnt((size_t)G * k * E), Sv(G);
@@ -421,7 +439,8 @@ moe_status moe_ep_dispatch(moe_ep_handle h, const double* stats_all_host, const 
   moe_status s = make_plan(G, h->g, E, k, h->cf, cnt.data(), Sv.data(), p, h->phases);
   if (s != MOE_OK) return s;
   if (p.S_total > h->S_total_max) return MOE_ERR_INVALID_ARG;
-  if (h->S > 0 && (!x || !sendbuf || !aligned(x, 16) || !aligned(sendbuf, 16))) return MOE_ERR_INVALID_ARG;
+  if (h->S > 0 && (!x || !aligned(x, 16) || (!to_peers && (!sendbuf || !aligned(sendbuf, 16)))))
+    return MOE_ERR_INVALID_ARG;
 
   // device tables: base, send offsets (per phase) and phase-0 lengths of this rank's runs;
   // per phase, the received segments and the local experts' rows
@@ -479,6 +498,25 @@ moe_status moe_ep_dispatch(moe_ep_handle h, const double* stats_all_host, const 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   EP_TRY(cudaMemcpyAsync(h->plan_dev, h->plan_host.data(), h->plan_host.size() * sizeof(int32_t),
                          cudaMemcpyHostToDevice, st));
+  if (to_peers) {
+    // rank d receives, source after source, rows[q][d] from each rank q; this rank's rows for
+    // d start there after the earlier sources', and in this rank's send order after its
+    // rows for the earlier destinations
+    std::vector<int64_t> rows((size_t)G * G, 0);
+    for (int q = 0; q < G; ++q)
+      for (int r = 0; r < k; ++r)
+        for (int e = 0; e < E; ++e) rows[(size_t)q * G + e / El] += p.kept[((size_t)q * k + r) * E + e];
+    h->peers_host.assign(G, EpPeer{nullptr, 0});
+    int64_t send_start = 0;
+    for (int d = 0; d < G; ++d) {
+      int64_t arrive = 0;
+      for (int q = 0; q < h->g; ++q) arrive += rows[(size_t)q * G + d];
+      h->peers_host[d] = EpPeer{h->peer_ptrs[d], arrive - send_start};
+      send_start += rows[(size_t)h->g * G + d];
+    }
+    EP_TRY(cudaMemcpyAsync(h->peers_dev, h->peers_host.data(), (size_t)G * sizeof(EpPeer),
+                           cudaMemcpyHostToDevice, st));
+  }
   for (size_t i = 0; i < (size_t)h->phases * G; ++i) {
     send_rows_host[i] = p.send_rows[i];
     recv_rows_host[i] = p.recv_rows[i];
@@ -505,7 +543,48 @@ moe_status moe_ep_dispatch(moe_ep_handle h, const double* stats_all_host, const 
   h->computed = false;
   if (h->S == 0) return MOE_OK;
   EP_TRY(launch_ep_dispatch(x, h->act == MOE_BF16, (int)h->S, (int)h->M, E, k, (int)p.C, h->R,
-                            h->plan_dev, h->plan_dev + kE, h->spos, sendbuf, st));
+                            h->plan_dev, h->plan_dev + kE, h->spos, sendbuf, st,
+                            to_peers ? h->peers_dev : nullptr, El));
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_ep_dispatch(moe_ep_handle h, const double* stats_all_host, const void* x, void* sendbuf,
+                           int64_t* send_rows_host, int64_t* recv_rows_host, void* stream) {
+  return dispatch_impl(h, stats_all_host, x, sendbuf, false, send_rows_host, recv_rows_host, stream);
+}
+
+moe_status moe_ep_set_peers(moe_ep_handle h, const void* const* recv_bufs_host) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (!recv_bufs_host) {                       // back to the caller's exchanges
+    h->peer_ptrs.clear();
+    return MOE_OK;
+  }
+  for (int d = 0; d < h->G; ++d)
+    if (!recv_bufs_host[d] || !aligned(recv_bufs_host[d], 16)) return MOE_ERR_INVALID_ARG;
+  h->peer_ptrs.resize(h->G);
+  for (int d = 0; d < h->G; ++d) h->peer_ptrs[d] = const_cast<void*>(recv_bufs_host[d]);
+  h->planned = h->computed = false;
+  return MOE_OK;
+}
+
+moe_status moe_ep_dispatch_to_peers(moe_ep_handle h, const double* stats_all_host, const void* x,
+                                    int64_t* send_rows_host, int64_t* recv_rows_host, void* stream) {
+  return dispatch_impl(h, stats_all_host, x, nullptr, true, send_rows_host, recv_rows_host, stream);
+}
+
+moe_status moe_ep_combine_from_peers(moe_ep_handle h, void* y, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (!h->planned || h->peer_ptrs.empty()) return MOE_ERR_STATE;
+  if (h->S == 0) return MOE_OK;
+  if (!y || !aligned(y, 16)) return MOE_ERR_INVALID_ARG;
+  Routing R2 = h->R;
+  R2.slot = h->spos;
+  EP_TRY(launch_combine(nullptr, h->act == MOE_BF16, (int)h->S, (int)h->M, h->k, 0, R2, y,
+                        static_cast<cudaStream_t>(stream), false, 0, h->peers_dev, h->El));
   return MOE_OK;
 }
 

@@ -95,6 +95,13 @@ cudaError_t launch_scan(int S, int E, int k, int C, int64_t Cbuf, const Routing&
 // [k*E + E] sum of lse^2, [k*E + E + 1] the rank's token count S.
 inline int ep_stats_len(int E, int k) { return k * E + E + 2; }
 cudaError_t launch_ep_scan(int S, int E, int k, const Routing& R, double* stats, cudaStream_t st);
+// Expert parallelism over peer memory: rank d's receive buffer as this GPU addresses it,
+// and the row at which this rank's rows for d start there minus the row at which they
+// start in this rank's send order (row in d's buffer = send row + delta).
+struct EpPeer {
+  void* base;
+  int64_t delta;
+};
 // dispatch_combine.cu, expert parallelism (one rank's side of the two exchanges):
 //   ep_dispatch: slot[t][r] = base[r][e] + off[r][c][e] + lrank (global rank-major slot),
 //     kept iff < C; a kept row goes to sendbuf[soff[r][e] + off + lrank] (runs ordered by
@@ -102,9 +109,12 @@ cudaError_t launch_ep_scan(int S, int E, int k, const Routing& R, double* stats,
 //   ep_unpack: received row j of segment q (starts seg_start[q], sorted) goes to expert row
 //     seg_dst[q] + (j - seg_start[q]); rowmap[j] records it
 //   ep_repack: recvbuf[j] = ybuf[rowmap[j]] (the expert outputs go back in arrival order)
+// peers (device [G], or null): each kept row goes straight to its owner's receive buffer
+// (rank e / El) instead of into sendbuf
 cudaError_t launch_ep_dispatch(const void* x, bool bf16, int S, int M, int E, int k, int C,
                                const Routing& R, const int32_t* base, const int32_t* soff,
-                               int32_t* spos, void* sendbuf, cudaStream_t st);
+                               int32_t* spos, void* sendbuf, cudaStream_t st,
+                               const EpPeer* peers = nullptr, int El = 1);
 cudaError_t launch_ep_unpack(const void* recvbuf, bool bf16, int nrows, int M, const int32_t* seg_start,
                              const int32_t* seg_dst, int nseg, int32_t* rowmap, void* xbuf,
                              unsigned* err, int64_t xrows, cudaStream_t st);
@@ -132,9 +142,11 @@ cudaError_t launch_dispatch_fused(const void* x, int S, int M, int E, int C, int
                                   const Routing& R, void* xbuf, int32_t* tok, float* gsc, void* y,
                                   cudaStream_t st);
 // with_losses: one more block computes the auxiliary losses (E experts) beside the combine
+// peers (device [G], or null): the row of choice (t, r) is read from its owner's receive
+// buffer, peers[e / El].base + (slot + peers[e / El].delta) rows, instead of ybuf
 cudaError_t launch_combine(const void* ybuf, bool bf16, int S, int M, int k, int64_t Cbuf,
                            const Routing& R, void* y, cudaStream_t st, bool with_losses = false,
-                           int E = 0);
+                           int E = 0, const EpPeer* peers = nullptr, int El = 1);
 // ffn_simt.cu  (fp32 activations)
 cudaError_t launch_ffn_f32(const float* A, const float* B, float* D, const int32_t* nexp, int E,
                            int64_t Cbuf, int K, int N, bool relu, cudaStream_t st);

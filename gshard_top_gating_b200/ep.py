@@ -19,6 +19,12 @@ to rank d and receives recv_rows[q] rows from rank q.  With two phases (bf16) ea
 exchange is split in two by expert slot, so that the second half travels while the
 experts compute the first, and the first half returns while they compute the second;
 the result is bit for bit the one-phase forward's.
+
+Over peer memory (`set_peers` with every rank's receive buffer as this GPU addresses it)
+the pack kernel stores each kept row straight into its owner's receive buffer and the
+combine reads the expert outputs from there: neither all-to-all is a separate step
+(`ep_forward_local_peers` on one device; `ep_forward_dist_peers` across processes, with
+the caller mapping the buffers).
 """
 from __future__ import annotations
 
@@ -32,7 +38,7 @@ class EPMoeLayer:
     """One rank's share of the layer: the whole gate, E/G experts, its buffers."""
 
     def __init__(self, G, g, S_max, S_total_max, M, H, E, k, capacity_factor, Wg, gate_bias,
-                 W1_local, W2_local, phases: int = 1):
+                 W1_local, W2_local, phases: int = 1, recvbuf: torch.Tensor | None = None):
         act = W1_local.dtype
         if act not in (torch.float32, torch.bfloat16):
             raise TypeError("expert weights must be float32 or bfloat16")
@@ -53,7 +59,12 @@ class EPMoeLayer:
         dev = W1_local.device
         ns, nr = L.moe_ep_buffer_rows(self.h)
         self.sendbuf = torch.empty(max(ns, 1), M, dtype=act, device=dev)
-        self.recvbuf = torch.empty(max(nr, 1), M, dtype=act, device=dev)
+        if recvbuf is not None:              # e.g. a buffer the other ranks can map
+            if recvbuf.dtype != act or recvbuf.dim() != 2 or recvbuf.shape[1] != M or recvbuf.shape[0] < nr:
+                raise ValueError("recvbuf must be [>= receive rows, M] of the activation dtype")
+            self.recvbuf = recvbuf
+        else:
+            self.recvbuf = torch.empty(max(nr, 1), M, dtype=act, device=dev)
         self.stats = torch.zeros(L.moe_ep_stats_len(E, k), dtype=torch.float64, device=dev)
         self.S = 0
         self.send_rows = self.recv_rows = None
@@ -75,6 +86,21 @@ class EPMoeLayer:
 
     def experts(self, stream=None) -> None:
         L.moe_ep_experts(self.h, self.recvbuf, stream)
+
+    # the peer-memory forms
+    def set_peers(self, recv_ptrs) -> None:
+        """recv_ptrs: every rank's receive buffer address as this GPU sees it (rank order)."""
+        L.moe_ep_set_peers(self.h, recv_ptrs)
+
+    def dispatch_to_peers(self, stats_all: np.ndarray, x: torch.Tensor, stream=None):
+        send, recv = L.moe_ep_dispatch_to_peers(self.h, stats_all, x, self.G, stream)
+        self.send_rows, self.recv_rows = send.reshape(1, self.G), recv.reshape(1, self.G)
+        return self.send_rows, self.recv_rows
+
+    def combine_from_peers(self, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        y = out if out is not None else torch.empty(self.S, self.M, dtype=self.act, device=self.recvbuf.device)
+        L.moe_ep_combine_from_peers(self.h, y, stream)
+        return y
 
     def experts_phase(self, phase: int, stream=None) -> None:
         L.moe_ep_experts_phase(self.h, self.recvbuf, phase, stream)
@@ -157,6 +183,47 @@ def ep_forward_local(layers, xs, outs=None):
             layer.experts_phase(p)
         _exchange(layers, p, back=True)                              # and back
     return [layer.combine(None if outs is None else outs[i]) for i, layer in enumerate(layers)]
+
+
+def ep_forward_local_peers(layers, xs, outs=None):
+    """G ranks emulated in one process on one device, over "peer memory": every rank's
+    receive buffer is a buffer of this device, so the pack writes into the owners'
+    buffers and the combine reads from them exactly as it would over NVLink.  Every
+    rank's step finishes before any rank's next (one stream).  Returns the outputs."""
+    ptrs = [layer.recvbuf.data_ptr() for layer in layers]
+    for layer in layers:
+        layer.set_peers(ptrs)
+    stats = [layer.route(x) for layer, x in zip(layers, xs)]
+    stats_all = torch.stack(stats).cpu().numpy()
+    for layer, x in zip(layers, xs):
+        layer.dispatch_to_peers(stats_all, x)
+    for layer in layers:
+        layer.experts()
+    return [layer.combine_from_peers(None if outs is None else outs[i]) for i, layer in enumerate(layers)]
+
+
+def ep_forward_dist_peers(layer: EPMoeLayer, x: torch.Tensor, group=None, out=None) -> torch.Tensor:
+    """One rank's forward over peer memory in a torch.distributed job: `layer.set_peers`
+    must already hold every rank's receive buffer as this GPU maps it (CUDA IPC or
+    symmetric memory; `layer.recvbuf` is this rank's).  The ranks meet at a barrier
+    after each step whose writes the others read."""
+    import torch.distributed as dist
+
+    def fence():
+        torch.cuda.current_stream().synchronize()
+        dist.barrier(group=group)
+
+    G = layer.G
+    stats = layer.route(x)
+    gathered = torch.empty(G, stats.numel(), dtype=stats.dtype, device=stats.device)
+    dist.all_gather_into_tensor(gathered, stats, group=group)
+    layer.dispatch_to_peers(gathered.cpu().numpy(), x)
+    fence()                                  # every rank's rows are in their owners' buffers
+    layer.experts()
+    fence()                                  # every expert output is in place
+    y = layer.combine_from_peers(out)
+    fence()                                  # no rank reads a buffer the next forward rewrites
+    return y
 
 
 def ep_forward_dist(layer: EPMoeLayer, x: torch.Tensor, group=None, out=None) -> torch.Tensor:

@@ -309,6 +309,18 @@ MOE_API moe_status moe_assign_slots_noalloc(int64_t S, int32_t E, int32_t k, int
  *   [return phase 0 | moe_ep_experts_phase(1)];  return phase 1;  moe_ep_combine
  * Every GEMM tile lies within one phase, so rows, slots and outputs are bit for bit
  * those of the one-phase forward.
+ *
+ * Over peer memory (moe_ep_set_peers): when every rank's receive buffer is mapped on
+ * every GPU (CUDA IPC, symmetric memory), moe_ep_dispatch_to_peers packs each kept row
+ * straight into its owner's receive buffer at the row the all-to-all would have put it
+ * (stores over NVLink, no send buffer), and moe_ep_combine_from_peers reads each expert
+ * output from the owner's buffer, where moe_ep_experts wrote it.  Both exchanges become
+ * part of those kernels.  The caller orders the ranks:
+ *   moe_ep_route; all-gather; moe_ep_dispatch_to_peers   [every rank done, writes visible]
+ *   moe_ep_experts(own receive buffer)                   [every rank done]
+ *   moe_ep_combine_from_peers                            [every rank done before the next
+ *                                                         forward's dispatch]
+ * e.g. a stream synchronise and a barrier of the ranks at each bracket.  One phase only.
  */
 typedef struct moe_ep_layer* moe_ep_handle;
 
@@ -390,6 +402,22 @@ MOE_API moe_status moe_ep_experts_phase(moe_ep_handle h, void* recvbuf_dev, int3
 /* Step 4: y_dev [S, M] act from the returned rows in sendbuf_dev (fully overwritten;
  * a token whose choices were all dropped gets 0). */
 MOE_API moe_status moe_ep_combine(moe_ep_handle h, const void* sendbuf_dev, void* y_dev, void* stream);
+
+/* The receive buffer of every rank, as this GPU addresses it (recv_bufs_host [G] device
+ * pointers, 16-byte aligned, each of moe_ep_buffer_rows' receive rows; entry g is this
+ * rank's own), for the peer-memory forms below.  NULL forgets them.  Host only. */
+MOE_API moe_status moe_ep_set_peers(moe_ep_handle h, const void* const* recv_bufs_host);
+
+/* Step 2 over peer memory: as moe_ep_dispatch, with each kept row stored into its
+ * owner's receive buffer instead of a send buffer.  MOE_ERR_STATE without peers or with
+ * two phases. */
+MOE_API moe_status moe_ep_dispatch_to_peers(moe_ep_handle h, const double* stats_all_host, const void* x_dev,
+                                            int64_t* send_rows_host, int64_t* recv_rows_host, void* stream);
+
+/* Step 4 over peer memory: y_dev [S, M] act, each kept choice's expert output read from
+ * its owner's receive buffer (same sum and rounding as moe_ep_combine).  MOE_ERR_STATE
+ * before moe_ep_dispatch_to_peers. */
+MOE_API moe_status moe_ep_combine_from_peers(moe_ep_handle h, void* y_dev, void* stream);
 
 /* l_aux and z of the whole batch, from the stats given to the last moe_ep_dispatch (host). */
 MOE_API moe_status moe_ep_aux_loss(moe_ep_handle h, float* l_aux_host, float* z_loss_host);

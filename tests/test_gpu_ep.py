@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import oracle as O
-from gshard_top_gating_b200.ep import EPMoeLayer, ep_forward_local
+from gshard_top_gating_b200.ep import EPMoeLayer, ep_forward_local, ep_forward_local_peers
 from gshard_top_gating_b200.inputs import Workload, make_inputs
 from gshard_top_gating_b200.layer import MoeLayer
 from tests import gpu_helpers as Gh
@@ -128,6 +128,68 @@ def test_ep_two_phases_equal_one_phase_bit_for_bit(w, shards):
         assert moved0 > 0 and moved1 > 0
 
 
+@pytest.mark.parametrize("w,shards", CASES, ids=[c[0].name for c in CASES])
+def test_ep_over_peer_memory_equals_the_all_to_all(w, shards):
+    """The pack storing rows straight into the owners' receive buffers and the combine
+    reading them there (one device standing in for peer memory) give the all-to-all
+    forward's routing, outputs and losses bit for bit."""
+    G = len(shards)
+    x, Wg, b, W1, W2 = make_inputs(w, device="cuda")
+    El = w.E // G
+    cuts = np.cumsum((0,) + shards)
+    xs = [x[cuts[g]:cuts[g + 1]].contiguous() for g in range(G)]
+    Ws = [(W1[g * El:(g + 1) * El].contiguous(), W2[g * El:(g + 1) * El].contiguous()) for g in range(G)]
+    res = []
+    for fwd in (ep_forward_local, ep_forward_local_peers):
+        layers = [EPMoeLayer(G, g, max(shards[g], 1), w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b, *Ws[g])
+                  for g in range(G)]
+        for _ in range(2):                     # twice: the second forward reuses every buffer
+            ys = fwd(layers, xs)
+        torch.cuda.synchronize()
+        parts = [layer.routing() for layer in layers]
+        res.append((torch.cat(ys), torch.cat([p[0] for p in parts]), torch.cat([p[2] for p in parts]),
+                    [layer.aux_loss() for layer in layers]))
+        for layer in layers:
+            layer.close()
+    (y1, e1, s1, a1), (y2, e2, s2, a2) = res
+    assert torch.equal(e1, e2) and torch.equal(s1, s2)
+    assert torch.equal(y1, y2)
+    assert a1 == a2
+
+
+def test_ep_peer_memory_arguments():
+    from gshard_top_gating_b200 import _lib as L
+    w = Workload("ep_peer_args", 256, 64, 64, 8, 2, 1.0, "bf16")
+    x, Wg, b, W1, W2 = make_inputs(w, device="cuda")
+    layer = EPMoeLayer(2, 0, 128, 256, w.M, w.H, w.E, w.k, w.cf, Wg, b, W1[:4].contiguous(), W2[:4].contiguous())
+    st = layer.route(x[:128].contiguous()).cpu().numpy()
+    stats = np.stack([st, st])
+    with pytest.raises(L.MoeError) as ei:      # no peers set
+        layer.dispatch_to_peers(stats, x[:128].contiguous())
+    assert ei.value.status == L.MOE_ERR_STATE
+    other = torch.empty_like(layer.recvbuf)
+    with pytest.raises(L.MoeError) as ei:      # a null or misaligned buffer
+        layer.set_peers([layer.recvbuf.data_ptr(), 0])
+    assert ei.value.status == L.MOE_ERR_INVALID_ARG
+    with pytest.raises(L.MoeError) as ei:
+        layer.set_peers([layer.recvbuf.data_ptr(), other.data_ptr() + 2])
+    assert ei.value.status == L.MOE_ERR_INVALID_ARG
+    layer.set_peers([layer.recvbuf.data_ptr(), other.data_ptr()])
+    with pytest.raises(L.MoeError) as ei:      # nothing planned yet
+        layer.combine_from_peers()
+    assert ei.value.status == L.MOE_ERR_STATE
+    layer.dispatch_to_peers(stats, x[:128].contiguous())
+    layer.experts()
+    layer.combine_from_peers()
+    L.moe_ep_set_phases(layer.h, 2)            # peers take one phase
+    layer.route(x[:128].contiguous())
+    with pytest.raises(L.MoeError) as ei:
+        layer.dispatch_to_peers(stats, x[:128].contiguous())
+    assert ei.value.status == L.MOE_ERR_STATE
+    torch.cuda.synchronize()
+    layer.close()
+
+
 def test_ep_rejects_a_plan_from_inconsistent_stats():
     w = Workload("ep_bad", 256, 64, 64, 8, 2, 1.0, "bf16")
     x, Wg, b, W1, W2 = make_inputs(w, device="cuda")
@@ -195,6 +257,14 @@ def test_ep_forward_dist_one_rank_nccl():
             la, za = layer.aux_loss()
             assert abs(la - lb) <= 1e-5 * lb and abs(za - zb) <= 1e-5 * zb
             layer.close()
+        # over peer memory: one rank's own receive buffer is its only peer
+        from gshard_top_gating_b200.ep import ep_forward_dist_peers
+        layer = EPMoeLayer(1, 0, w.S, w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b, W1, W2)
+        layer.set_peers([layer.recvbuf.data_ptr()])
+        y = ep_forward_dist_peers(layer, x)
+        torch.cuda.synchronize()
+        assert torch.equal(y, y1)
+        layer.close()
         one.close()
     finally:
         dist.destroy_process_group()
