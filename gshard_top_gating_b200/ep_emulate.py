@@ -1,6 +1,7 @@
 """Expert-parallel forward of one workload, G ranks emulated on one GPU, timed per rank.
 
     python -m gshard_top_gating_b200.ep_emulate --workload large --ranks 8 --phases 2
+    python -m gshard_top_gating_b200.ep_emulate --workload large --ranks 8 --peers --check
 
 Each rank is its own library handle with S/G tokens and E/G experts, as in
 `ep.ep_forward_local`.  The ranks run one after another on one device, so each
@@ -8,9 +9,10 @@ rank's kernels are timed alone with CUDA events: route (router and per-rank scan
 dispatch (plan upload and pack), the experts of each phase (unpack, both grouped
 GEMMs, repack) and combine.  The exchanges between ranks are device copies here and
 are not timed; the JSON line reports the rows and bytes each rank would send and
-receive per phase, from which a transport's time follows.  The routing, slots and
-outputs are those of the one-device layer on the whole batch (tests/test_gpu_ep.py).
-Needs a GPU.
+receive per phase, from which a transport's time follows.  With --peers the pack
+writes into the owners' receive buffers and the combine reads from them (every buffer
+on the one device stands in for a peer's).  --check compares the concatenated output
+with the one-device layer's on the whole batch, bit for bit.  Needs a GPU.
 """
 from __future__ import annotations
 
@@ -22,6 +24,7 @@ import torch
 
 from .ep import EPMoeLayer, _exchange
 from .inputs import WORKLOADS, make_inputs
+from .layer import MoeLayer
 
 
 def main() -> None:
@@ -31,7 +34,11 @@ def main() -> None:
     ap.add_argument("--ranks", type=int, default=8)
     ap.add_argument("--phases", type=int, choices=(1, 2), default=2)
     ap.add_argument("--reps", type=int, default=5)
+    ap.add_argument("--peers", action="store_true", help="pack and combine over peer memory (one phase)")
+    ap.add_argument("--check", action="store_true", help="compare with the one-device layer, bit for bit")
     args = ap.parse_args()
+    if args.peers:
+        args.phases = 1
     w = WORKLOADS[args.workload]
     G = args.ranks
     if w.E % G or w.S % G:
@@ -44,6 +51,10 @@ def main() -> None:
                          phases=args.phases) for g in range(G)]
     xs = [x[g * Sg:(g + 1) * Sg].contiguous() for g in range(G)]
     ys = [torch.empty_like(xg) for xg in xs]
+    if args.peers:
+        ptrs = [layer.recvbuf.data_ptr() for layer in layers]
+        for layer in layers:
+            layer.set_peers(ptrs)
 
     def timed(fn):
         a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -59,15 +70,23 @@ def main() -> None:
         for g, layer in enumerate(layers):
             ev["route"][g] = timed(lambda: layer.route(xs[g]))
         stats_all = torch.stack([layer.stats for layer in layers]).cpu().numpy()
-        for g, layer in enumerate(layers):
-            ev["dispatch"][g] = timed(lambda: layer.dispatch(stats_all, xs[g]))
-        for p in range(args.phases):
-            _exchange(layers, p)
+        if args.peers:
             for g, layer in enumerate(layers):
-                ev[f"experts_phase{p}"][g] = timed(lambda: layer.experts_phase(p))
-            _exchange(layers, p, back=True)
-        for g, layer in enumerate(layers):
-            ev["combine"][g] = timed(lambda: layer.combine(ys[g]))
+                ev["dispatch"][g] = timed(lambda: layer.dispatch_to_peers(stats_all, xs[g]))
+            for g, layer in enumerate(layers):
+                ev["experts_phase0"][g] = timed(lambda: layer.experts())
+            for g, layer in enumerate(layers):
+                ev["combine"][g] = timed(lambda: layer.combine_from_peers(ys[g]))
+        else:
+            for g, layer in enumerate(layers):
+                ev["dispatch"][g] = timed(lambda: layer.dispatch(stats_all, xs[g]))
+            for p in range(args.phases):
+                _exchange(layers, p)
+                for g, layer in enumerate(layers):
+                    ev[f"experts_phase{p}"][g] = timed(lambda: layer.experts_phase(p))
+                _exchange(layers, p, back=True)
+            for g, layer in enumerate(layers):
+                ev["combine"][g] = timed(lambda: layer.combine(ys[g]))
         torch.cuda.synchronize()
         if rep:
             for s in stages:
@@ -88,9 +107,19 @@ def main() -> None:
                                          for p in range(args.phases)],
         })
     compute = {s: round(max(med[s]), 4) for s in stages}
+    check = None
+    if args.check:
+        one = MoeLayer(w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b, W1, W2)
+        y1 = one(x)
+        torch.cuda.synchronize()
+        y = torch.cat(ys)
+        check = {"bitwise_equal_to_one_device": bool(torch.equal(y, y1)),
+                 "max_abs_diff": float((y.float() - y1.float()).abs().max())}
+        one.close()
     print(json.dumps({
         "workload": f"{w.name} (S={w.S}, M={w.M}, H={w.H}, E={w.E}, k={w.k}, cf={w.cf})",
-        "ranks": G, "phases": args.phases, "tokens_per_rank": Sg, "experts_per_rank": El,
+        "ranks": G, "phases": args.phases, "transport": "peer memory" if args.peers else "all-to-all",
+        "tokens_per_rank": Sg, "experts_per_rank": El, "check": check,
         "slowest_rank_ms": compute, "slowest_rank_compute_ms": round(sum(compute.values()), 4),
         "per_rank": per_rank,
     }))
