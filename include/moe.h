@@ -52,7 +52,7 @@ extern "C" {
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1,   /* a null, misaligned or out-of-range argument */
-  MOE_ERR_UNSUPPORTED = 2,   /* valid but outside what this build handles (e.g. E > 256) */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid but outside what the library handles (e.g. E > 256) */
   MOE_ERR_CUDA = 3,          /* a CUDA runtime / driver call failed, or a device fault */
   MOE_ERR_OOM = 4,           /* device workspace allocation failed */
   MOE_ERR_STATE = 5,         /* call out of order (e.g. aux loss before any forward) */
