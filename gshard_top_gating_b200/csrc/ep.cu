@@ -85,6 +85,7 @@ struct moe_ep_layer {
   EpPeer* peers_dev;     // [G] every rank's receive buffer and this rank's row offset in it
   std::vector<void*> peer_ptrs;       // [G] set by moe_ep_set_peers (empty: not set)
   std::vector<EpPeer> peers_host;
+  bool to_peers;         // the last dispatch wrote into the peers' buffers
   std::vector<int32_t> plan_host;
   GemmPlan plan1, plan2;
   void* wsplit;
@@ -541,6 +542,7 @@ moe_status dispatch_impl(moe_ep_layer* h, const double* stats_all_host, const vo
   h->z = p.S_total ? zs / Sd : 0.0;
   h->planned = true;
   h->computed = false;
+  h->to_peers = to_peers;
   if (h->S == 0) return MOE_OK;
   EP_TRY(launch_ep_dispatch(x, h->act == MOE_BF16, (int)h->S, (int)h->M, E, k, (int)p.C, h->R,
                             h->plan_dev, h->plan_dev + kE, h->spos, sendbuf, st,
@@ -578,7 +580,7 @@ moe_status moe_ep_dispatch_to_peers(moe_ep_handle h, const double* stats_all_hos
 
 moe_status moe_ep_combine_from_peers(moe_ep_handle h, void* y, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
-  if (!h->planned || h->peer_ptrs.empty()) return MOE_ERR_STATE;
+  if (!h->planned || !h->to_peers || h->peer_ptrs.empty()) return MOE_ERR_STATE;
   if (h->S == 0) return MOE_OK;
   if (!y || !aligned(y, 16)) return MOE_ERR_INVALID_ARG;
   Routing R2 = h->R;
@@ -650,7 +652,7 @@ moe_status moe_ep_experts_phase(moe_ep_handle h, void* recvbuf, int32_t phase, v
 
 moe_status moe_ep_combine(moe_ep_handle h, const void* sendbuf, void* y, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
-  if (!h->planned) return MOE_ERR_STATE;
+  if (!h->planned || h->to_peers) return MOE_ERR_STATE;   // rows went to the peers: combine_from_peers
   if (h->S == 0) return MOE_OK;
   if (!y || !aligned(y, 16) || (h->send_total > 0 && (!sendbuf || !aligned(sendbuf, 16))))
     return MOE_ERR_INVALID_ARG;

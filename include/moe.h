@@ -416,7 +416,7 @@ MOE_API moe_status moe_ep_dispatch_to_peers(moe_ep_handle h, const double* stats
 
 /* Step 4 over peer memory: y_dev [S, M] act, each kept choice's expert output read from
  * its owner's receive buffer (same sum and rounding as moe_ep_combine).  MOE_ERR_STATE
- * before moe_ep_dispatch_to_peers. */
+ * unless the last dispatch was moe_ep_dispatch_to_peers (and moe_ep_combine after one). */
 MOE_API moe_status moe_ep_combine_from_peers(moe_ep_handle h, void* y_dev, void* stream);
 
 /* l_aux and z of the whole batch, from the stats given to the last moe_ep_dispatch (host). */

@@ -180,7 +180,14 @@ def test_ep_peer_memory_arguments():
     assert ei.value.status == L.MOE_ERR_STATE
     layer.dispatch_to_peers(stats, x[:128].contiguous())
     layer.experts()
+    with pytest.raises(L.MoeError) as ei:      # the rows went to the peers' buffers
+        layer.combine()
+    assert ei.value.status == L.MOE_ERR_STATE
     layer.combine_from_peers()
+    layer.dispatch(stats, x[:128].contiguous())
+    with pytest.raises(L.MoeError) as ei:      # and now to the send buffer
+        layer.combine_from_peers()
+    assert ei.value.status == L.MOE_ERR_STATE
     L.moe_ep_set_phases(layer.h, 2)            # peers take one phase
     layer.route(x[:128].contiguous())
     with pytest.raises(L.MoeError) as ei:
