@@ -16,6 +16,8 @@
 
 #include <new>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/moe.h"
 #include "common.cuh"
 #include "internal.h"
@@ -349,6 +351,29 @@ moe_status moe_set_routing_flags(moe_handle h, uint32_t flags) {
 
 namespace {
 
+// NVTX ranges on the host timeline: one around a forward or backward, one per stage
+// around its launches (header-only NVTX: without a tool attached, each push or pop
+// is a call that returns at once).
+struct NvtxStages {
+  const char* (*name)(int32_t);
+  int n, open = -1;
+  NvtxStages(const char* top, const char* (*name_)(int32_t), int n_) : name(name_), n(n_) {
+    nvtxRangePushA(top);
+  }
+  void stage(int i) {
+    if (open >= 0) nvtxRangePop();
+    open = -1;
+    if (i < n) {
+      nvtxRangePushA(name(i));
+      open = i;
+    }
+  }
+  ~NvtxStages() {
+    if (open >= 0) nvtxRangePop();
+    nvtxRangePop();
+  }
+};
+
 moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStream_t st) {
   if (!h || S < 0 || S > h->S_max) return MOE_ERR_INVALID_ARG;
   if (S > 0 && (!x || !y || !aligned(x, 16) || !aligned(y, 16))) return MOE_ERR_INVALID_ARG;
@@ -372,7 +397,11 @@ moe_status forward_impl(moe_handle h, int64_t S, const void* x, void* y, cudaStr
   const int iS = (int)S, iM = (int)h->M, iH = (int)h->H;
   const Routing& R = h->R;
   const bool prof = h->profiling && h->have_events;
-  auto mark = [&](int i) -> cudaError_t { return prof ? cudaEventRecord(h->ev[i], st) : cudaSuccess; };
+  NvtxStages nv("moe_forward", moe_stage_name, MOE_NUM_STAGES);
+  auto mark = [&](int i) -> cudaError_t {
+    nv.stage(i);
+    return prof ? cudaEventRecord(h->ev[i], st) : cudaSuccess;
+  };
 
   MOE_TRY(mark(0));
   if (bf16) {
@@ -780,7 +809,11 @@ moe_status moe_backward(moe_handle h, int64_t S, const void* x, const void* dy, 
   Routing Rrows = R;                   // row gathers address the serving expert's buffer
   if (h->last_rerouted) Rrows.eidx = R.dest;
   const bool prof = h->profiling && h->have_events;
-  auto mark = [&](int i) -> cudaError_t { return prof ? cudaEventRecord(h->evb[i], st) : cudaSuccess; };
+  NvtxStages nv("moe_backward", moe_backward_stage_name, MOE_NUM_BWD_STAGES);
+  auto mark = [&](int i) -> cudaError_t {
+    nv.stage(i);
+    return prof ? cudaEventRecord(h->evb[i], st) : cudaSuccess;
+  };
   h->have_backward_times = false;
   MOE_TRY(mark(0));
   MOE_TRY(launch_gate_backward(a, R, st));
