@@ -93,3 +93,49 @@ def test_null_handle_calls_are_rejected(L):
     assert L.lib.moe_backward(None, 1, FAKE, FAKE, 0.0, 0.0, FAKE, FAKE, None, FAKE, FAKE, None) == 1
     assert L.lib.moe_kernels_per_backward(None, 10) == 0
     assert L.lib.moe_set_backward_flags(None, 0) == 1
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "moe.h"
+
+/* A C11 caller of the boundary: host-only entry points, no device work. */
+int main(void) {
+    /* G = 2 ranks, k = 1, E = 2: rank 0 chose experts {0,0,1}, rank 1 {1,1,1} */
+    const int64_t counts[4] = {2, 1, 0, 3}, S[2] = {3, 3};
+    int64_t C = 0, send[2], recv[2], send2[4], recv2[4], split[2];
+    if (moe_ep_stats_len(2, 1) != 1 * 2 + 2 + 2) return 1;
+    if (moe_ep_plan(2, 0, 2, 1, 1.0, counts, S, &C, send, recv, NULL, NULL) != MOE_OK) return 2;
+    if (C != 3 || send[0] != 2 || send[1] != 1 || recv[0] != 2 || recv[1] != 0) return 3;
+    if (moe_ep_phase_plan(2, 0, 2, 1, 1.0, counts, S, 2, send2, recv2, split) != MOE_OK) return 4;
+    if (send2[0] + send2[2] != send[0] || send2[1] + send2[3] != send[1]) return 5;
+    if (moe_ep_plan(2, 0, 2, 1, 1.0, counts, S, NULL, NULL, NULL, NULL, NULL) != MOE_OK) return 6;
+    if (moe_create(NULL, 1, 64, 64, 2, 1, 1.0, MOE_BF16, NULL, NULL, NULL, NULL) != MOE_ERR_INVALID_ARG)
+        return 7;
+    if (strlen(moe_status_string(MOE_ERR_TIMEOUT)) == 0) return 8;
+    printf("ok %lld\n", (long long)C);
+    return 0;
+}
+"""
+
+
+def test_header_is_c11_and_links_from_c(tmp_path):
+    """A plain C11 program compiles against include/moe.h with warnings as errors, links
+    against the library and runs its host-only entry points."""
+    import shutil
+    from gshard_top_gating_b200 import _lib
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "caller.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    libname = os.path.basename(_lib.LIB_PATH)
+    subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), os.path.join(libdir, libname), f"-Wl,-rpath,{libdir}"],
+                   check=True, capture_output=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    assert out.stdout.strip() == "ok 3"
