@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemm g, Routing R) {
   for (int q = 0; q < 4; ++q) {
     const int i = i0 + ty * 4 + q;
     if (i >= rows) continue;
-    if (EPI == kSgDx) {
+    if constexpr (EPI == kSgDx) {
       // dx[t] = acc + sum over kept choices of the expert-side gradient rows
       const TD* dxe = static_cast<const TD*>(g.dxe);
       float add[4] = {0.f, 0.f, 0.f, 0.f};
@@ -458,16 +458,16 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemm g, Routing R) {
         const int j = j0 + tx * 4 + w;
         if (j < g.cols) D[(int64_t)i * g.d_i + j] = static_cast<TD>(add[w] + acc[q][w]);
       }
-      continue;
-    }
+    } else {
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const int j = j0 + tx * 4 + w;
-      if (j >= g.cols) continue;
-      const int64_t o = (int64_t)z * g.d_z + (int64_t)i * g.d_i + j;
-      float v = acc[q][w];
-      if (EPI == kSgMask) v = g.mask[o] > 0.f ? v : 0.f;
-      D[o] = static_cast<TD>(v);
+      for (int w = 0; w < 4; ++w) {
+        const int j = j0 + tx * 4 + w;
+        if (j >= g.cols) continue;
+        const int64_t o = (int64_t)z * g.d_z + (int64_t)i * g.d_i + j;
+        float v = acc[q][w];
+        if (EPI == kSgMask) v = g.mask[o] > 0.f ? v : 0.f;
+        D[o] = static_cast<TD>(v);
+      }
     }
   }
 }

@@ -202,7 +202,6 @@ template <typename T>
 struct Vec;
 template <>
 struct Vec<__nv_bfloat16> {
-  static constexpr int N = 8;
   __device__ static void load_fma(float (&a)[8], const uint4& u, float g) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -218,7 +217,6 @@ struct Vec<__nv_bfloat16> {
 };
 template <>
 struct Vec<float> {
-  static constexpr int N = 4;
   __device__ static void load_fma(float (&a)[8], const uint4& u, float g) {
     a[0] = fmaf(g, __uint_as_float(u.x), a[0]);
     a[1] = fmaf(g, __uint_as_float(u.y), a[1]);
