@@ -447,6 +447,77 @@ def test_backward_large_sampled():
     torch.cuda.empty_cache()
 
 
+def test_backward_wide_sampled():
+    """The wide workload at full size (top-8 of 256 experts, 7168-wide rows, one-CTA
+    backward kernels): 16 rows of dW2[e] and 16 columns of dW1[e] for four experts, and
+    dx of eight tokens with all their kept choices (up to 64 experts), each from the
+    oracle's step functions one expert at a time."""
+    w = WORKLOADS["wide"]
+    run = G.build(w)
+    run.layer.enable_backward()
+    out = G.forward(run)
+    rt = G.check_routing(run, out)
+    dy = upstream_grad(w, device="cuda")
+    a_aux, a_z = 0.01, 0.001
+    g = run.layer.backward(out.x, dy, a_aux, a_z)
+    torch.cuda.synchronize()
+    S, E, k, M, H = w.S, w.E, w.k, w.M, w.H
+    rng = np.random.default_rng(13)
+    toks = np.sort(rng.choice(S, 8, replace=False))
+    used = sorted(set(int(e) for t in toks for r in range(k) if rt.slot[t, r] >= 0 for e in [rt.ids[t, r]]))
+    sample_e = sorted(rng.choice(used, 4, replace=False).tolist())
+    xs = _np(out.x[torch.as_tensor(toks, device="cuda")])
+    dys = _np(dy[torch.as_tensor(toks, device="cuda")])
+    dgate = np.zeros((len(toks), k))
+    dxe = np.zeros((len(toks), M))
+    slack = np.zeros((len(toks), M))
+    errs = {}
+    for e in used:
+        W1e, W2e = _np(run.W1[e]), _np(run.W2[e])
+        for i, t in enumerate(toks):                  # this expert's share of the sampled tokens' dx
+            for r in range(k):
+                if rt.slot[t, r] < 0 or rt.ids[t, r] != e:
+                    continue
+                pre = xs[i] @ W1e
+                dgate[i, r] = dys[i] @ (np.maximum(pre, 0.0) @ W2e)
+                dq = (rt.gates[t, r] * dys[i]) @ W2e.T
+                amb = np.abs(pre) <= M * 2.0 ** -23 * (np.abs(xs[i]) @ np.abs(W1e))
+                dxe[i] += (dq * (pre > 0)) @ W1e.T
+                slack[i] += (np.abs(dq) * amb) @ np.abs(W1e).T
+        if e not in sample_e:
+            continue
+        sel = [(t, r) for r in range(k) for t in np.nonzero((rt.ids[:, r] == e) & (rt.slot[:, r] >= 0))[0]]
+        sel.sort(key=lambda tr: rt.slot[tr[0], tr[1]])
+        ts = np.array([t for t, _ in sel])
+        rs = np.array([r for _, r in sel])
+        xr = _np(out.x[torch.as_tensor(ts, device="cuda")])
+        dY = rt.gates[ts, rs][:, None] * _np(dy[torch.as_tensor(ts, device="cuda")])
+        cols = rng.choice(H, 16, replace=False)
+        pre_c = xr @ W1e[:, cols]
+        ref2 = np.maximum(pre_c, 0.0).T @ dY
+        got2 = _np(g["dW2"][e])[cols]
+        errs[f"dW2[{e}] rows"] = _excess_err(got2, ref2)
+        errs[f"fro dW2[{e}] rows"] = _fro_err(got2, ref2)
+        dq = dY @ W2e[cols].T
+        amb = np.abs(pre_c) <= M * 2.0 ** -23 * (np.abs(xr) @ np.abs(W1e[:, cols]))
+        ref1 = xr.T @ (dq * (pre_c > 0))
+        got1 = _np(g["dW1"][e])[:, cols]
+        errs[f"dW1[{e}] cols"] = _excess_err(got1, ref1, np.abs(xr).T @ (np.abs(dq) * amb))
+        errs[f"fro dW1[{e}] cols"] = _fro_err(got1, ref1)
+    dl = O.gates_backward(rt.gates[toks], rt.ids[toks], dgate, E)
+    dl += a_aux * O.aux_loss_backward(rt.p[toks], rt.f, E, S=S)
+    dl += a_z * O.z_loss_backward(rt.p[toks], rt.lse[toks], S=S)
+    ref_dx = dxe + dl @ _np(run.Wg).T
+    got_dx = _np(g["dx"][torch.as_tensor(toks, device="cuda")])
+    errs["dx"] = _excess_err(got_dx, ref_dx, slack)
+    errs["fro dx"] = _fro_err(got_dx, ref_dx)
+    print(f"\nwide backward errors ({len(toks)} tokens over {len(used)} experts): {errs}")
+    _check_all(errs, "bf16")
+    run.layer.close()
+    del run
+    torch.cuda.empty_cache()
+
+
 def test_backward_stage_times():
     """With profiling on, the backward records its eight stages."""
     w = Workload("prof", 512, 256, 256, 8, 2, 1.25, "bf16", seed=35)
