@@ -197,6 +197,33 @@ def test_ep_peer_memory_arguments():
     layer.close()
 
 
+def test_ep_large_workload_over_eight_ranks_bit_exact():
+    """The large workload (65536 tokens, 64 experts at capacity) split over 8 emulated
+    ranks, in all three forms (all-to-all with one and two phases, peer memory), gives
+    the one-device layer's output bit for bit."""
+    from gshard_top_gating_b200.inputs import WORKLOADS
+    w = WORKLOADS["large"]
+    G = 8
+    x, Wg, b, W1, W2 = make_inputs(w, device="cuda")
+    one = MoeLayer(w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b, W1, W2)
+    y1 = one(x)
+    torch.cuda.synchronize()
+    one.close()
+    El, Sg = w.E // G, w.S // G
+    xs = [x[g * Sg:(g + 1) * Sg].contiguous() for g in range(G)]
+    for phases, fwd in ((1, ep_forward_local), (2, ep_forward_local), (1, ep_forward_local_peers)):
+        layers = [EPMoeLayer(G, g, Sg, w.S, w.M, w.H, w.E, w.k, w.cf, Wg, b,
+                             W1[g * El:(g + 1) * El].contiguous(), W2[g * El:(g + 1) * El].contiguous(),
+                             phases=phases) for g in range(G)]
+        ys = fwd(layers, xs)
+        torch.cuda.synchronize()
+        assert torch.equal(torch.cat(ys), y1), (phases, fwd.__name__)
+        for layer in layers:
+            layer.close()
+        del layers, ys
+        torch.cuda.empty_cache()
+
+
 def test_ep_rejects_a_plan_from_inconsistent_stats():
     w = Workload("ep_bad", 256, 64, 64, 8, 2, 1.0, "bf16")
     x, Wg, b, W1, W2 = make_inputs(w, device="cuda")
