@@ -30,6 +30,7 @@ CASES = [
     (Workload("ep_skewed", 1536, 128, 256, 32, 2, 1.25, "bf16", skew_bias=True), (400, 0, 600, 536)),
     (Workload("ep_sat", 4096, 256, 256, 8, 2, 1.0, "bf16"), (2048, 2048)),      # experts at capacity
     (Workload("ep_f32", 256, 64, 256, 8, 2, 1.25, "f32"), (100, 156)),
+    (Workload("ep_g3_k3", 1500, 128, 256, 24, 3, 1.25, "bf16"), (500, 700, 300)),   # odd G, k = 3
 ]
 
 
@@ -92,6 +93,8 @@ PHASE_CASES = [
     (Workload("ep2_skewed", 4096, 128, 256, 16, 2, 2.0, "bf16", skew_bias=True), (1000, 1100, 996, 1000)),
     # n_e about 128: every row in phase 1, phase 0 empty
     (Workload("ep2_top8", 1024, 128, 256, 64, 8, 1.25, "bf16"), (128,) * 8),
+    # odd G, k = 3, some experts past the split
+    (Workload("ep2_g3_k3", 6000, 128, 256, 12, 3, 1.0, "bf16"), (2500, 1000, 2500)),
 ]
 
 
