@@ -1,5 +1,6 @@
 /*
- * moe.h -- C ABI of a single-GPU GShard Mixture-of-Experts layer, forward and backward (B200, sm_100a).
+ * moe.h -- C ABI of a GShard Mixture-of-Experts layer on B200 (sm_100a): the layer on one GPU,
+ * forward and backward, and its expert-parallel forward over G GPUs (moe_ep_*).
  *
  * The layer (sources: "GShard: Scaling Giant Neural Networks with Conditional
  * Computation", section "Mixture-of-Experts Implementation" and its "Expert
