@@ -367,7 +367,8 @@ def measure_backward(args, w, weights, x, y, flush, stream, pk, pk_kind, A, n_e)
     n_active = int((n_e > 0).sum().item())
     algo = algorithmic_bwd(w, A, n_active, pad_rows, nsplit)
     stages = {nm: stage_entry(algo[nm], stage_ms[nm], pk) for nm in L.BWD_STAGES if stage_ms[nm] > 0}
-    dom = max(stage_ms, key=lambda k_: stage_ms[k_])
+    timed = {k_: t for k_, t in stage_ms.items() if algo[k_][0] != "latency"}
+    dom = max(timed, key=lambda k_: timed[k_])
     b_, ach, peak, unit = stage_roof(algo[dom], stage_ms[dom] / 1e3, pk)
     ffn = sum(stage_ms[k_] for k_ in ("dW2", "dP", "dW1", "dX_e"))
     launches = n * (L.moe_kernels_per_forward(layer.h, w.S) + L.moe_kernels_per_backward(layer.h, w.S))
@@ -496,7 +497,9 @@ def measure_workload(args, w, dev, world, flush, pk, pk_kind, headline):
     algo = algorithmic(w, A, n_active)
     stages = {n: stage_entry(algo[n], stage_ms[n], pk) for n in STAGES if stage_ms[n] > 0}
     if w.act == "bf16":
-        dom = max(stage_ms, key=lambda n: stage_ms[n])
+        # the dominant stage among those with a roofline (a latency-bound stage has none)
+        timed = {n: t for n, t in stage_ms.items() if algo[n][0] != "latency"}
+        dom = max(timed, key=lambda n: timed[n])
         bound, achieved, peak, unit = stage_roof(algo[dom], stage_ms[dom] / 1e3, pk)
         roof = {"bound": bound, "kernel": dom, "achieved": round(achieved, 2), "peak": peak,
                 "unit": unit, "frac": round(achieved / peak, 4), "traffic": ncu_traffic(dom, w.name),
